@@ -1,0 +1,215 @@
+"""fp64 CPU oracle for banded sparse self-attention -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import this package.  The product
+path (the CUDA library and its Python binding) never imports, links or runs it,
+and the two share no code: the oracle is plain C (``swa_oracle.c``) compiled
+with gcc and OpenMP, reached through ctypes from here.
+
+What it computes, and from which passage of the pages, is stated function by
+function in ``swa_oracle.c``.  Every function is pinned by the ``-m "not gpu"``
+tests in ``tests/test_oracle_pins.py`` (brute force, worked example, closed
+cases, the bucket threshold table).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "swa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``liboracle.so`` next to its source (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", _LIB, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            P, I, I64, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
+            lib.oracle_forward.argtypes = [I, I, I, I, I, P, P, P, P, I, P, P, I, I, P, P, P, I, P,
+                                           D, P, I64, P, P, P]
+            lib.oracle_forward.restype = I
+            lib.oracle_dense_bruteforce.argtypes = [I, I, I, I, I, P, P, P, P, I, P, P, I, I, P, P,
+                                                    P, I, P, D, P, P]
+            lib.oracle_dense_bruteforce.restype = I
+            lib.oracle_key_counts.argtypes = [I, I, I, P, I, I, P, P, I, P, P]
+            lib.oracle_key_counts.restype = I
+            lib.oracle_key_list.argtypes = [I, I, I, P, I, P, P, I, P, I, I, I, P]
+            lib.oracle_key_list.restype = I
+            lib.oracle_relative_bucket.argtypes = [I]
+            lib.oracle_relative_bucket.restype = I
+            lib.oracle_expand_side_bias.argtypes = [I, I, I, P, P]
+            lib.oracle_expand_side_bias.restype = I
+            lib.oracle_side_aggregate.argtypes = [I, I, I, I, I, P, P, P]
+            lib.oracle_side_aggregate.restype = I
+            lib.oracle_num_threads.argtypes = []
+            lib.oracle_num_threads.restype = I
+            _lib = lib
+    return _lib
+
+
+def _f32(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor: widen exactly (bf16/fp32 -> fp32)
+        import torch
+        x = x.detach().to("cpu", torch.float32).numpy()
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def _i32(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().numpy()
+    return np.ascontiguousarray(x, dtype=np.int32)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _per_head(x, Hq):
+    a = np.asarray(x, dtype=np.int32).reshape(-1)
+    if a.size == 1:
+        a = np.full(Hq, int(a[0]), dtype=np.int32)
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise RuntimeError(f"oracle {what} failed with code {rc}")
+
+
+class Problem:
+    """One attention problem, widened to fp32 host arrays (exact for bf16/fp32)."""
+
+    def __init__(self, q, k, v, *, window, dilation=1, causal=False, global_idx=None,
+                 side_k=None, side_v=None, side_block=16, bias=None, valid_len=None, scale=None):
+        self.q, self.k, self.v = _f32(q), _f32(k), _f32(v)
+        self.B, self.Hq, self.n, self.D = self.q.shape
+        self.Hkv = self.k.shape[1]
+        self.window = _per_head(window, self.Hq)
+        self.dilation = _per_head(dilation, self.Hq)
+        self.causal = int(bool(causal))
+        self.global_idx = _i32(global_idx)
+        self.g = 0 if self.global_idx is None else int(self.global_idx.shape[-1])
+        if self.g == 0:
+            self.global_idx = None
+        self.side_k, self.side_v = _f32(side_k), _f32(side_v)
+        self.S = 0 if self.side_k is None else int(self.side_k.shape[2])
+        self.side_block = int(side_block) if self.S else 0
+        self.bias = _f32(bias)
+        self.valid_len = _i32(valid_len)
+        self.scale = float(scale) if scale is not None else 1.0 / np.sqrt(self.D)
+
+    def _common(self):
+        return (self.B, self.Hq, self.Hkv, self.n, self.D, _ptr(self.q), _ptr(self.k), _ptr(self.v),
+                _ptr(self.global_idx), self.g, _ptr(self.side_k), _ptr(self.side_v), self.S,
+                self.side_block, _ptr(self.bias), _ptr(self.window), _ptr(self.dilation),
+                self.causal, _ptr(self.valid_len), self.scale)
+
+    def forward(self, rows=None):
+        """fp64 (out, lse, count).  ``rows``: flat row ids (b*Hq+h)*n+i, or None for all.
+
+        Without ``rows`` the results are shaped [B,Hq,n,D] / [B,Hq,n]; with rows they
+        are [len(rows), D] / [len(rows)].
+        """
+        lib = _load()
+        if rows is None:
+            total = self.B * self.Hq * self.n
+            rp = None
+        else:
+            rows = np.ascontiguousarray(rows, dtype=np.int64)
+            total = rows.size
+            rp = _ptr(rows)
+        out = np.empty((total, self.D), dtype=np.float64)
+        lse = np.empty(total, dtype=np.float64)
+        cnt = np.empty(total, dtype=np.int64)
+        _check(lib.oracle_forward(*self._common(), rp, total, _ptr(out), _ptr(lse), _ptr(cnt)),
+               "forward")
+        if rows is None:
+            return (out.reshape(self.B, self.Hq, self.n, self.D), lse.reshape(self.B, self.Hq, self.n),
+                    cnt.reshape(self.B, self.Hq, self.n))
+        return out, lse, cnt
+
+    def dense_bruteforce(self):
+        lib = _load()
+        out = np.empty((self.B, self.Hq, self.n, self.D), dtype=np.float64)
+        lse = np.empty((self.B, self.Hq, self.n), dtype=np.float64)
+        _check(lib.oracle_dense_bruteforce(*self._common(), _ptr(out), _ptr(lse)), "dense")
+        return out, lse
+
+
+def key_counts(B, Hq, n, *, window, dilation=1, causal=False, global_idx=None, S=0,
+               valid_len=None):
+    """|K(i)| + S per row, [B,Hq,n] int64 (0 for padded rows)."""
+    lib = _load()
+    gi = _i32(global_idx)
+    g = 0 if gi is None else int(gi.shape[-1])
+    vl = _i32(valid_len)
+    cnt = np.empty((B, Hq, n), dtype=np.int64)
+    _check(lib.oracle_key_counts(B, Hq, n, _ptr(gi) if g else None, g, S,
+                                 _ptr(_per_head(window, Hq)), _ptr(_per_head(dilation, Hq)),
+                                 int(bool(causal)), _ptr(vl), _ptr(cnt)), "key_counts")
+    return cnt
+
+
+def key_list(B, Hq, n, b, h, i, *, window, dilation=1, causal=False, global_idx=None,
+             valid_len=None):
+    """The explicit key set K(i) (ascending, no side keys) of one row."""
+    lib = _load()
+    gi = _i32(global_idx)
+    g = 0 if gi is None else int(gi.shape[-1])
+    vl = _i32(valid_len)
+    keys = np.empty(max(n, 1), dtype=np.int32)
+    w, d = _per_head(window, Hq), _per_head(dilation, Hq)
+    nk = lib.oracle_key_list(B, Hq, n, _ptr(gi) if g else None, g, _ptr(w), _ptr(d),
+                             int(bool(causal)), _ptr(vl), b, h, i, _ptr(keys))
+    if nk < 0:
+        raise MemoryError("oracle key_list")
+    return keys[:nk].copy()
+
+
+def relative_bucket(delta: int) -> int:
+    return int(_load().oracle_relative_bucket(int(delta)))
+
+
+def expand_side_bias(table, S: int, nblk: int):
+    """[Hq,32] bucket table -> [Hq, S + nblk - 1] fp32 side-bias table."""
+    t = _f32(table)
+    Hq = t.shape[0]
+    out = np.empty((Hq, S + nblk - 1), dtype=np.float32)
+    _check(_load().oracle_expand_side_bias(Hq, S, nblk, _ptr(t), _ptr(out)), "expand_side_bias")
+    return out
+
+
+def side_aggregate(x, block: int, valid_len=None):
+    """Block means [B,H,n,D] -> [B,H,n//block,D] (fp64)."""
+    a = _f32(x)
+    B, H, n, D = a.shape
+    vl = _i32(valid_len)
+    out = np.empty((B, H, n // block, D), dtype=np.float64)
+    _check(_load().oracle_side_aggregate(B, H, n, D, block, _ptr(a), _ptr(vl), _ptr(out)),
+           "side_aggregate")
+    return out
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())

@@ -1,0 +1,319 @@
+"""Pins of the fp64 oracle against things other than itself (CPU only).
+
+* brute force: an independent dense-mask statement of the same attention, on a
+  grid of tiny problems (values <= 1e-12, supports exact via one-hot V);
+* the worked window example of the BigBird notes (tests/golden);
+* closed cases: window >= n is full (or causal) softmax attention from torch;
+  global rows are full-attention rows; weights sum to one; outputs stay in the
+  convex hull of the attended V rows; padded rows are exactly zero; q = 0 gives
+  the plain mean over the key set (a cardinality check); dilation d equals d
+  independent residue problems; GQA equals MHA with replicated K/V; side keys
+  merge with the window part through the logsumexp identity;
+* attended-pair counts against the closed forms of the LongT5 complexity
+  statements O(l*r) and O(l*(r + l/k));
+* the T5 bucket function against its threshold table and a float-log
+  evaluation of the textbook formula.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(shape, rng):
+    return rng.standard_normal(shape).astype(np.float32)
+
+
+def _problem(oracle_mod, rng, B, Hq, Hkv, n, D, r, d, causal, g, pad, S=0, kb=4, bias=False):
+    q = _rand((B, Hq, n, D), rng)
+    k = _rand((B, Hkv, n, D), rng)
+    v = _rand((B, Hkv, n, D), rng)
+    V = max(n - pad, 0)
+    gi = None
+    if g and V > 0:
+        g = min(g, V)
+        gi = np.stack([np.sort(rng.choice(V, g, replace=False)) for _ in range(B)]).astype(np.int32)
+    sk = sv = bt = None
+    if S:
+        sk = _rand((B, Hkv, S, D), rng)
+        sv = _rand((B, Hkv, S, D), rng)
+        if bias:
+            nblk = (n + kb - 1) // kb
+            bt = _rand((Hq, S + nblk - 1), rng)
+    vl = np.full(B, V, np.int32) if pad else None
+    return oracle_mod.Problem(q, k, v, window=r, dilation=d, causal=causal, global_idx=gi,
+                              side_k=sk, side_v=sv, side_block=kb, bias=bt, valid_len=vl)
+
+
+def _assert_close_lse(a, b, tol):
+    assert np.array_equal(np.isneginf(a), np.isneginf(b))
+    m = ~np.isneginf(a)
+    if m.any():
+        assert np.max(np.abs(a[m] - b[m])) <= tol
+
+
+def test_worked_window_example(oracle_mod):
+    with open(os.path.join(GOLDEN, "bigbird_window_example.txt")) as f:
+        rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
+    for n, r, pos, attended in rows:
+        n, r, pos = int(n), int(r), int(pos)
+        expect = [int(x) - 1 for x in attended.split(",")]
+        keys = oracle_mod.key_list(1, 1, n, 0, 0, pos - 1, window=r)
+        assert keys.tolist() == expect
+
+
+def test_oracle_matches_dense_bruteforce_grid(oracle_mod):
+    rng = np.random.default_rng(7)
+    cases = 0
+    for n in (1, 2, 3, 5, 8, 13, 21, 33, 40):
+        for r, d, causal, g, pad in itertools.product((0, 1, 2, 5), (1, 2, 3), (0, 1), (0, 1, 3),
+                                                      (0, 1, 3)):
+            if rng.random() > 0.22:   # a seeded third of the grid keeps the run short
+                continue
+            S = int(rng.integers(0, 3)) * 2
+            G = int(rng.choice([1, 2]))
+            p = _problem(oracle_mod, rng, 2, 2 * G, 2, n, 8, r, d, causal, g, pad, S=S, kb=4,
+                         bias=bool(S and rng.random() < 0.7))
+            o, lse, _ = p.forward()
+            od, lsed = p.dense_bruteforce()
+            assert np.max(np.abs(o - od)) <= 1e-12
+            _assert_close_lse(lse, lsed, 1e-12)
+            cases += 1
+    assert cases > 150
+
+
+def test_support_exact_onehot_v(oracle_mod):
+    """V = identity rows -> o_i is the weight row; zero pattern must agree exactly."""
+    rng = np.random.default_rng(11)
+    for (n, r, d, causal, g, pad) in [(24, 2, 1, 0, 2, 3), (24, 3, 2, 0, 3, 0), (24, 4, 3, 1, 0, 2),
+                                      (17, 1, 1, 1, 0, 0), (24, 0, 1, 0, 1, 5)]:
+        p = _problem(oracle_mod, rng, 1, 2, 2, n, n, r, d, causal, g, pad)
+        p.v = np.ascontiguousarray(np.broadcast_to(np.eye(n, dtype=np.float32), p.v.shape))
+        o, _, cnt = p.forward()
+        od, _ = p.dense_bruteforce()
+        assert np.array_equal(o > 0, od > 0)
+        assert np.array_equal((o > 0).sum(-1), cnt)   # no side keys: count = |K(i)|
+
+
+def test_window_covering_sequence_is_full_attention(oracle_mod):
+    rng = np.random.default_rng(3)
+    n, D = 37, 16
+    for causal in (0, 1):
+        p = _problem(oracle_mod, rng, 2, 4, 2, n, D, n, 1, causal, 0, 0)
+        o, _, _ = p.forward()
+        q = torch.from_numpy(p.q).double()
+        k = torch.from_numpy(p.k).double().repeat_interleave(2, dim=1)
+        v = torch.from_numpy(p.v).double().repeat_interleave(2, dim=1)
+        ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=bool(causal))
+        assert np.max(np.abs(o - ref.numpy())) <= 1e-12
+    # dilation with r*d >= n but d > 1 is not full attention: only the residue class
+    p = _problem(oracle_mod, rng, 1, 1, 1, n, D, n, 2, 0, 0, 0)
+    _, _, cnt = p.forward()
+    assert cnt[0, 0, 0] == (n + 1) // 2
+
+
+def test_global_rows_are_full_attention_rows(oracle_mod):
+    rng = np.random.default_rng(5)
+    n, D, pad = 50, 16, 6
+    p = _problem(oracle_mod, rng, 2, 2, 2, n, D, 3, 2, 0, 4, pad)
+    o, lse, _ = p.forward()
+    V = n - pad
+    q = torch.from_numpy(p.q).double()[..., :V, :]
+    k = torch.from_numpy(p.k).double()[..., :V, :]
+    v = torch.from_numpy(p.v).double()[..., :V, :]
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v)
+    s = torch.einsum("bhid,bhjd->bhij", q, k) * p.scale
+    ref_lse = torch.logsumexp(s, -1)
+    for b in range(2):
+        for i in p.global_idx[b]:
+            assert np.max(np.abs(o[b, :, i] - ref.numpy()[b, :, i])) <= 1e-12
+            assert np.max(np.abs(lse[b, :, i] - ref_lse.numpy()[b, :, i])) <= 1e-12
+
+
+def test_weights_sum_to_one_and_convex_hull(oracle_mod):
+    rng = np.random.default_rng(9)
+    p = _problem(oracle_mod, rng, 2, 4, 2, 64, 16, 5, 2, 0, 3, 7, S=4, kb=8, bias=True)
+    ones = p.v.copy()
+    p.v = np.ones_like(p.v)
+    sv = p.side_v
+    p.side_v = np.ones_like(p.side_v)
+    o, _, cnt = p.forward()
+    valid = cnt > 0
+    assert np.max(np.abs(o[valid] - 1.0)) <= 1e-13
+    p.v, p.side_v = ones, sv
+    o, _, _ = p.forward()
+    for b, h, i in itertools.product(range(2), range(4), range(64)):
+        if not valid[b, h, i]:
+            continue
+        keys = oracle_mod.key_list(2, 4, 64, b, h, i, window=p.window, dilation=p.dilation,
+                                   global_idx=p.global_idx, valid_len=p.valid_len)
+        rows = np.concatenate([p.v[b, h // 2, keys], p.side_v[b, h // 2]], 0)
+        assert np.all(o[b, h, i] <= rows.max(0) + 1e-12)
+        assert np.all(o[b, h, i] >= rows.min(0) - 1e-12)
+
+
+def test_padded_rows_exact_zero(oracle_mod):
+    rng = np.random.default_rng(13)
+    p = _problem(oracle_mod, rng, 2, 2, 2, 30, 8, 3, 1, 0, 2, 9, S=2, kb=4, bias=True)
+    o, lse, cnt = p.forward()
+    assert np.all(o[:, :, 21:] == 0.0)
+    assert np.all(np.isneginf(lse[:, :, 21:]))
+    assert np.all(cnt[:, :, 21:] == 0)
+    assert np.all(np.isfinite(o))
+    assert np.all(np.isfinite(lse[:, :, :21]))
+
+
+def test_zero_query_gives_mean_over_key_set(oracle_mod):
+    rng = np.random.default_rng(17)
+    p = _problem(oracle_mod, rng, 1, 2, 2, 40, 8, 4, 3, 0, 3, 2, S=3, kb=8)
+    p.q = np.zeros_like(p.q)
+    o, lse, cnt = p.forward()
+    for h, i in itertools.product(range(2), range(38)):
+        keys = oracle_mod.key_list(1, 2, 40, 0, h, i, window=p.window, dilation=p.dilation,
+                                   global_idx=p.global_idx, valid_len=p.valid_len)
+        rows = np.concatenate([p.v[0, h, keys], p.side_v[0, h]], 0).astype(np.float64)
+        assert rows.shape[0] == cnt[0, h, i]
+        assert np.max(np.abs(o[0, h, i] - rows.mean(0))) <= 1e-13
+        assert abs(lse[0, h, i] - math.log(cnt[0, h, i])) <= 1e-13
+
+
+def test_dilation_equals_residue_subproblems(oracle_mod):
+    rng = np.random.default_rng(19)
+    n, D, r = 41, 8, 3
+    for d, causal in [(2, 0), (3, 0), (3, 1), (5, 0)]:
+        p = _problem(oracle_mod, rng, 1, 1, 1, n, D, r, d, causal, 0, 0)
+        o, lse, _ = p.forward()
+        for c in range(d):
+            idx = np.arange(c, n, d)
+            sub = oracle_mod.Problem(p.q[:, :, idx], p.k[:, :, idx], p.v[:, :, idx], window=r,
+                                     dilation=1, causal=causal, scale=p.scale)
+            os_, ls_, _ = sub.forward()
+            assert np.max(np.abs(o[:, :, idx] - os_)) <= 1e-14
+            assert np.max(np.abs(lse[:, :, idx] - ls_)) <= 1e-14
+
+
+def test_gqa_equals_replicated_mha(oracle_mod):
+    rng = np.random.default_rng(23)
+    p = _problem(oracle_mod, rng, 2, 6, 2, 29, 8, 2, 1, 0, 2, 3, S=2, kb=4, bias=True)
+    o, lse, _ = p.forward()
+    rep = oracle_mod.Problem(p.q, np.repeat(p.k, 3, axis=1), np.repeat(p.v, 3, axis=1),
+                             window=p.window, dilation=p.dilation, global_idx=p.global_idx,
+                             side_k=np.repeat(p.side_k, 3, axis=1), side_v=np.repeat(p.side_v, 3, axis=1),
+                             side_block=4, bias=p.bias, valid_len=p.valid_len)
+    o2, lse2, _ = rep.forward()
+    assert np.max(np.abs(o - o2)) == 0.0
+    _assert_close_lse(lse, lse2, 0.0)
+
+
+def test_side_keys_merge_by_logsumexp(oracle_mod):
+    """attn(K(i) U S) == lse-merge(attn(K(i)), attn(S)); the side part computed with
+    torch over the bias column the LongT5 side bias names (memory block - query block)."""
+    rng = np.random.default_rng(29)
+    n, D, S, kb = 48, 8, 6, 8
+    p = _problem(oracle_mod, rng, 1, 2, 2, n, D, 3, 1, 0, 0, 0, S=S, kb=kb, bias=True)
+    o, lse, _ = p.forward()
+    nos = oracle_mod.Problem(p.q, p.k, p.v, window=p.window, dilation=p.dilation)
+    o1, l1, _ = nos.forward()
+    q = torch.from_numpy(p.q).double()
+    sk = torch.from_numpy(p.side_k).double()
+    sv = torch.from_numpy(p.side_v).double()
+    s = torch.einsum("bhid,bhsd->bhis", q, sk) * p.scale
+    nblk = n // kb
+    bias = torch.from_numpy(p.bias).double()
+    i = torch.arange(n)[:, None]
+    sig = torch.arange(S)[None, :]
+    col = sig - i // kb + nblk - 1
+    s = s + bias[:, col][None]
+    l2 = torch.logsumexp(s, -1).numpy()
+    o2 = torch.einsum("bhis,bhsd->bhid", torch.softmax(s, -1), sv).numpy()
+    m = np.maximum(l1, l2)
+    w1, w2 = np.exp(l1 - m), np.exp(l2 - m)
+    merged = (o1 * w1[..., None] + o2 * w2[..., None]) / (w1 + w2)[..., None]
+    assert np.max(np.abs(o - merged)) <= 1e-12
+    assert np.max(np.abs(lse - (m + np.log(w1 + w2)))) <= 1e-12
+
+
+def test_pair_counts_match_complexity_closed_forms(oracle_mod):
+    # LongT5 Local: each token sees r on each side: sum |W(i)| = n(2r+1) - r(r+1) for n > r
+    n, r = 1000, 127
+    cnt = oracle_mod.key_counts(1, 1, n, window=r)
+    assert cnt.sum() == n * (2 * r + 1) - r * (r + 1)
+    # Transient-Global adds every one of the S = n/k block summaries to every row
+    cnt = oracle_mod.key_counts(1, 1, n, window=r, S=n // 16)
+    assert cnt.sum() == n * (2 * r + 1) - r * (r + 1) + n * (n // 16)
+    # causal window of 512 keys (r = 511) including self
+    n, r = 3000, 511
+    cnt = oracle_mod.key_counts(1, 1, n, window=r, causal=True)
+    assert cnt.sum() == n * (r + 1) - r * (r + 1) // 2
+    assert cnt[0, 0, -1] == 512
+
+
+def test_local_keys_inside_three_block_context(oracle_mod):
+    """LongT5 local attention splits into blocks of block_len = r + 1 and attends inside
+    the 3-block context (previous, own, next): every window key must lie there."""
+    n, r = 1024, 127
+    bl = r + 1
+    for i in (0, 1, 127, 128, 500, 1023):
+        keys = oracle_mod.key_list(1, 1, n, 0, 0, i, window=r)
+        blk = i // bl
+        assert keys.min() >= max(0, (blk - 1) * bl)
+        assert keys.max() < min(n, (blk + 2) * bl)
+        assert len(keys) <= 3 * bl
+
+
+def test_bucket_threshold_table(oracle_mod):
+    with open(os.path.join(GOLDEN, "t5_bucket_thresholds.txt")) as f:
+        rows = [tuple(map(int, l.split())) for l in f if l.strip() and not l.startswith("#")]
+    for a in range(8):
+        assert oracle_mod.relative_bucket(-a) == a
+        assert oracle_mod.relative_bucket(a) == (16 + a if a else 0)
+    for bucket, first in rows:
+        assert oracle_mod.relative_bucket(-first) == bucket
+        assert oracle_mod.relative_bucket(-(first - 1)) == bucket - 1
+        assert oracle_mod.relative_bucket(first) == bucket + 16
+    for a in (128, 129, 1000, 100000):
+        assert oracle_mod.relative_bucket(-a) == 15
+        assert oracle_mod.relative_bucket(a) == 31
+
+
+def test_bucket_matches_float_log_formula(oracle_mod):
+    """Textbook T5 bucket with the log in fp32 (as the reference library evaluates it)."""
+    a = np.arange(1, 2048, dtype=np.int64)
+    af = a.astype(np.float32)
+    large = 8 + (np.log(af / np.float32(8)) / np.float32(math.log(128 / 8)) * np.float32(8)).astype(np.int64)
+    expect = np.where(a < 8, a, np.minimum(large, 15))
+    got = np.array([oracle_mod.relative_bucket(-int(x)) for x in a])
+    assert np.array_equal(got, expect)
+    got_pos = np.array([oracle_mod.relative_bucket(int(x)) for x in a])
+    assert np.array_equal(got_pos, expect + 16)
+
+
+def test_expand_side_bias_columns(oracle_mod):
+    table = np.arange(2 * 32, dtype=np.float32).reshape(2, 32)
+    S, nblk = 5, 7
+    out = oracle_mod.expand_side_bias(table, S, nblk)
+    assert out.shape == (2, S + nblk - 1)
+    # column c holds delta = c - (nblk - 1): delta 0 -> bucket 0, +1 -> 17, -1 -> 1
+    assert out[1, nblk - 1] == 32 + 0
+    assert out[1, nblk] == 32 + 17
+    assert out[1, nblk - 2] == 32 + 1
+    assert out[0, 0] == oracle_mod.relative_bucket(-(nblk - 1))
+
+
+def test_side_aggregate_block_means(oracle_mod):
+    rng = np.random.default_rng(31)
+    x = _rand((2, 3, 64, 4), rng)
+    out = oracle_mod.side_aggregate(x, 16)
+    ref = x.astype(np.float64).reshape(2, 3, 4, 16, 4).mean(3)
+    assert np.max(np.abs(out - ref)) <= 1e-15
+    # padding tokens belong to no block; a trailing partial block joins the previous one
+    ramp = np.broadcast_to(np.arange(70, dtype=np.float32)[None, None, :, None], (1, 1, 70, 2)).copy()
+    out = oracle_mod.side_aggregate(ramp, 16, valid_len=np.array([60], np.int32))
+    assert out.shape == (1, 1, 4, 2)
+    assert out[0, 0, 0, 0] == 7.5
+    assert out[0, 0, 3, 0] == np.mean(np.arange(48, 60))
