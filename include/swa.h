@@ -1,0 +1,157 @@
+/*
+ * swa.h -- C ABI of the banded sparse self-attention library (libswa.so) for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (forward pass, one call).  For every batch b, query
+ * head h (KV head h / (Hq/Hkv)) and query position i < valid_len[b]:
+ *   - the key set K(i) is the sliding window W(i) = { i + d*t : -r <= t <= r }
+ *     (causal: -r <= t <= 0) clipped to [0, valid_len[b]), with r = window[h] and
+ *     d = dilation[h] -- "精读笔记：Big Bird" §3.2.1 (query i attends i-w/2 .. i+w/2),
+ *     the Longformer page §二 (dilated window: skip tokens inside the window), and
+ *     SWAN-GPT §3.3(1) (fixed 512-key causal window in the SWA-RoPE layers);
+ *   - united, as a set, with the global positions global_idx[b][:]; a global query
+ *     instead attends every valid key (BigBird §3.2.3, internal/ITC global tokens;
+ *     Longformer page §二 global attention);
+ *   - plus every side key s in [0, S) of the LongT5 Transient-Global attention
+ *     ("LongT5 长序列模型完全指南": Transient-Global block summaries as extra keys,
+ *     with a global relative-position bias added to their scores);
+ *   score = scale * <q_i, k_j>  (+ bias[h][s - floor(i / side_block) + nblk - 1] on
+ *   side keys, nblk = ceil(seq_len / side_block)); o_i = softmax(scores) . V;
+ *   lse_i = natural-log logsumexp of the scores.  Padded query rows
+ *   (i >= valid_len[b]) give o = 0 and lse = -inf; padded keys are never attended.
+ *
+ * Layouts: every tensor is row-major and contiguous.
+ *   q, out      [B, Hq,  n, D]      dtype of the plan (bf16 or fp32)
+ *   k, v        [B, Hkv, n, D]
+ *   side_k/v    [B, Hkv, S, D]
+ *   bias        [Hq, S + nblk - 1]  fp32
+ *   lse         [B, Hq, n]          fp32
+ *   global_idx  [B, g]              int32, each row strictly increasing, < valid_len[b]
+ *   valid_len   [B]                 int32 (trailing padding), or NULL for "no padding"
+ *
+ * Ownership: the caller owns every tensor.  The plan owns its workspace
+ * (allocated by swa_plan_create, freed by swa_plan_destroy).  swa_forward neither
+ * allocates nor synchronises (except in SWA_DEBUG_CHECKS mode) and never aborts
+ * the process: every failure is a returned status.
+ *
+ * Threads and streams: one plan may be used by one stream at a time (its
+ * workspace is reused by every forward).
+ */
+#ifndef SWA_H_
+#define SWA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct swa_plan_s* swa_plan_t;
+
+typedef enum {
+  SWA_OK = 0,
+  SWA_ERR_INVALID_ARG = 1,   /* a null/misaligned pointer, a bad size or value */
+  SWA_ERR_UNSUPPORTED = 2,   /* valid request outside what the kernels implement */
+  SWA_ERR_CUDA = 3,          /* a CUDA runtime/driver call or launch failed */
+  SWA_ERR_OOM = 4,           /* workspace allocation failed */
+  SWA_ERR_TIMEOUT = 5,       /* a bounded device-side wait expired (kernel returned early) */
+  SWA_ERR_DEVICE_CHECK = 6   /* a device-side precondition check failed (debug mode) */
+} swa_status;
+
+typedef enum { SWA_BF16 = 0, SWA_FP32 = 1 } swa_dtype;
+
+/* Plan flags. */
+#define SWA_DEBUG_CHECKS 1u  /* check global_idx on the device and synchronise after
+                                each forward, reporting device errors as a status */
+
+typedef struct {
+  int batch;           /* B >= 1 */
+  int seq_len;         /* n >= 1 */
+  int num_q_heads;     /* Hq >= 1, <= 128 */
+  int num_kv_heads;    /* Hkv >= 1, Hq % Hkv == 0 */
+  int head_dim;        /* D: 64 or 128 */
+  swa_dtype dtype;     /* element type of q, k, v, side_k, side_v, out */
+  int max_global;      /* largest g any forward will pass (0: no global tokens) */
+  int num_side;        /* S >= 0 side keys per (batch, KV head) */
+  int side_block;      /* k > 0 when num_side > 0: query block size of the side bias */
+  float scale;         /* score scale; 0 selects 1/sqrt(head_dim) */
+  unsigned flags;      /* SWA_DEBUG_CHECKS */
+} swa_plan_desc;
+
+/* Validate the descriptor and allocate the plan and its device workspace on the
+ * current CUDA device.  Returns SWA_ERR_INVALID_ARG for a null argument or a
+ * value out of range, SWA_ERR_UNSUPPORTED for head_dim not in {64, 128},
+ * SWA_ERR_OOM when the workspace cannot be allocated. */
+swa_status swa_plan_create(swa_plan_t* out_plan, const swa_plan_desc* desc);
+
+/* One forward pass, enqueued on `stream` (a cudaStream_t; NULL = legacy default).
+ *   q, k, v       device, required, 16-byte aligned
+ *   global_idx    device [B, num_global] or NULL when num_global == 0;
+ *                 0 <= num_global <= max_global
+ *   side_k/v      device [B, Hkv, S, D], required when num_side > 0, else ignored
+ *   bias          device [Hq, S + nblk - 1] fp32, or NULL (no bias)
+ *   window        HOST [Hq] one-sided radius r >= 0 per query head
+ *   dilation      HOST [Hq] d >= 1 per query head, or NULL (all 1)
+ *   causal        0 or 1
+ *   valid_len     device [B], or NULL (= seq_len)
+ *   out           device [B, Hq, n, D], plan dtype, required
+ *   lse           device [B, Hq, n] fp32, or NULL
+ * Returns SWA_ERR_INVALID_ARG for a null required pointer, a pointer not 16-byte
+ * aligned, window < 0, dilation < 1, num_global out of range; SWA_ERR_UNSUPPORTED
+ * for causal together with num_global > 0, or more than 16 distinct
+ * (dilation, residue) classes; SWA_ERR_CUDA when a launch fails.  In
+ * SWA_DEBUG_CHECKS mode it also synchronises and returns SWA_ERR_DEVICE_CHECK
+ * (bad global_idx) or SWA_ERR_TIMEOUT.  Global-index preconditions are NOT
+ * checked outside debug mode. */
+swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void* v,
+                       const int32_t* global_idx, int num_global, const void* side_k,
+                       const void* side_v, const float* bias, const int32_t* window,
+                       const int32_t* dilation, int causal, const int32_t* valid_len, void* out,
+                       float* lse, void* stream);
+
+/* Synchronise `stream` and read (then clear) the plan's device error word:
+ * SWA_ERR_TIMEOUT if a bounded wait expired in any kernel since the last check,
+ * SWA_ERR_DEVICE_CHECK if a precondition check failed, SWA_ERR_CUDA if the
+ * stream reports an error, else SWA_OK. */
+swa_status swa_plan_check(swa_plan_t plan, void* stream);
+
+/* Release the workspace and the plan (NULL is accepted). */
+swa_status swa_plan_destroy(swa_plan_t plan);
+
+/* Bytes of device workspace the plan holds. */
+size_t swa_plan_workspace_bytes(swa_plan_t plan);
+
+/* Number of kernel launches the most recent swa_forward enqueued. */
+int swa_plan_last_launches(swa_plan_t plan);
+
+/* Static, human-readable name of a status. */
+const char* swa_status_string(swa_status s);
+
+/* Transient-Global side keys / values: out[b,h,s,:] = mean of x[b,h,j,:] over the
+ * tokens j of block s = [s*k, s*k + k) that are below valid_len[b]; the S =
+ * floor(n / k) blocks cover the sequence, a trailing partial block joining the
+ * last one; a block with no valid token is zero ("LongT5 长序列模型完全指南",
+ * Transient-Global: tokens of each k-block are summed and normalised into one
+ * global token; padding tokens belong to no block).  Device pointers, x [B,H,n,D],
+ * out [B,H,floor(n/k),D], dtype bf16 or fp32, accumulation in fp32. */
+swa_status swa_side_aggregate(const void* x, void* out, int batch, int heads, int seq_len,
+                              int head_dim, int block, const int32_t* valid_len, swa_dtype dtype,
+                              void* stream);
+
+/* Host helper: T5 bidirectional relative-position bucket (32 buckets, max
+ * distance 128) of delta = memory block - query block ("LongT5 长序列模型完全指南",
+ * 相对位置编码 section and the LongT5Config defaults). */
+int swa_relative_bucket(int delta);
+
+/* Host helper: expand a per-head 32-bucket table [Hq][32] into the side-bias
+ * table [Hq][S + nblk - 1] that swa_forward reads, column c holding the bucket of
+ * delta = c - (nblk - 1).  Host pointers. */
+swa_status swa_expand_side_bias(int num_q_heads, int num_side, int nblk, const float* table,
+                                float* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWA_H_ */

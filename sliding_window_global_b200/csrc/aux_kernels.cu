@@ -1,0 +1,323 @@
+// aux_kernels.cu -- the non-tensor-core kernels of the library:
+//   * gather of the global rows (q, k, v at the global positions) into dense
+//     [B*H, gpad, D] buffers that the tensor-core kernel loads by TMA;
+//   * logsumexp merge of the split global-row partials, overwriting the rows of
+//     global queries (BigBird notes §3.2.3: a global token attends over the whole
+//     sequence);
+//   * the fp32 CUDA-core path (one warp per query row, online softmax) used for
+//     fp32 inputs, where bf16 tensor-core products cannot meet fp32 accuracy;
+//   * the Transient-Global block-mean aggregation that builds side keys/values
+//     (LongT5 guide, Transient-Global: block summaries of k tokens);
+//   * a device-side check of the global-index precondition.
+#include <cuda_bf16.h>
+
+#include "swa_kernels.h"
+
+namespace swa {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f(float x);
+template <>
+__device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// ------------------------------------------------------------------ gather
+// dst[bh, e, :] = src[bh', global_idx[b, e], :] for e < g, zeros for g <= e < gpad.
+__global__ void gather_rows_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                   const int32_t* __restrict__ gidx, int H, int n, int g, int gpad,
+                                   int row_vecs, int B) {
+  const size_t total = (size_t)B * H * gpad * row_vecs;
+  for (size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x; t < total;
+       t += (size_t)gridDim.x * blockDim.x) {
+    int x = (int)(t % row_vecs);
+    size_t r = t / row_vecs;
+    int e = (int)(r % gpad);
+    size_t bh = r / gpad;
+    int b = (int)(bh / H);
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (e < g) {
+      int pos = gidx[(size_t)b * g + e];
+      v = src[(bh * n + pos) * row_vecs + x];
+    }
+    dst[t] = v;
+  }
+}
+
+// ------------------------------------------------------------------ merge
+// One warp per global row: o = sum_s w_s o_s / sum_s w_s, w_s = exp(lse_s - max).
+template <typename T, int D>
+__global__ void merge_global_rows_kernel(AttnParams p) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int rows = p.B * p.Hq * p.g;
+  if (warp >= rows) return;
+  const int e = warp % p.g;
+  const int bh = warp / p.g;
+  const int b = bh / p.Hq;
+  const size_t stride = (size_t)p.B * p.Hq * p.gpad;
+  const size_t base = (size_t)bh * p.gpad + e;
+  float m = -INFINITY;
+  for (int s = 0; s < p.nsplit; ++s) m = fmaxf(m, p.part_lse[s * stride + base]);
+  constexpr int PER = D / 32;
+  float acc[PER];
+#pragma unroll
+  for (int x = 0; x < PER; ++x) acc[x] = 0.f;
+  float wsum = 0.f;
+  if (m > -INFINITY) {
+    for (int s = 0; s < p.nsplit; ++s) {
+      float ls = p.part_lse[s * stride + base];
+      if (ls == -INFINITY) continue;
+      float wgt = __expf(ls - m);
+      wsum += wgt;
+      const float* po = p.part_o + (s * stride + base) * D;
+#pragma unroll
+      for (int x = 0; x < PER; ++x) acc[x] += wgt * po[lane + 32 * x];
+    }
+  }
+  const int pos = p.global_idx[(size_t)b * p.g + e];
+  const size_t off = (size_t)bh * p.n + pos;
+  T* o = static_cast<T*>(p.out) + off * D;
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+  for (int x = 0; x < PER; ++x) o[lane + 32 * x] = from_f<T>(acc[x] * inv);
+  if (lane == 0 && p.lse) p.lse[off] = wsum > 0.f ? m + __logf(wsum) : -INFINITY;
+}
+
+// ------------------------------------------------------------------ fp32 CUDA-core path
+// One warp per query row.  Keys are enumerated in the order: window keys, global
+// keys (masked when already inside the window), side keys; a global query row
+// instead walks every valid key, then the side keys.  32 keys per step: each lane
+// scores one key, the warp updates the running max / sum with shuffles, and each
+// lane accumulates D/32 output columns.
+template <typename T, int D>
+__global__ void simt_attn_kernel(AttnParams p, const T* __restrict__ q, const T* __restrict__ k,
+                                 const T* __restrict__ v, const T* __restrict__ side_k,
+                                 const T* __restrict__ side_v) {
+  constexpr int PER = D / 32;
+  __shared__ float sq[4][D];
+  const int wib = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const size_t row = (size_t)blockIdx.x * 4 + wib;
+  if (row >= (size_t)p.B * p.Hq * p.n) return;
+  const int i = (int)(row % p.n);
+  const int h = (int)((row / p.n) % p.Hq);
+  const int b = (int)(row / ((size_t)p.n * p.Hq));
+  const int hk = h / p.G;
+  int V = p.valid_len ? p.valid_len[b] : p.n;
+  if (V > p.n) V = p.n;
+  T* orow = static_cast<T*>(p.out) + row * D;
+  if (i >= V) {
+#pragma unroll
+    for (int x = 0; x < PER; ++x) orow[lane + 32 * x] = from_f<T>(0.f);
+    if (lane == 0 && p.lse) p.lse[row] = -INFINITY;
+    return;
+  }
+  const T* qi = q + row * D;
+#pragma unroll
+  for (int x = 0; x < PER; ++x) sq[wib][lane + 32 * x] = to_f<T>(qi[lane + 32 * x]);
+  __syncwarp();
+  const int r = p.window[h], d = p.cls[p.class_base[h]].d;
+  const int32_t* gl = p.g ? p.global_idx + (size_t)b * p.g : nullptr;
+  bool is_global = false;
+  for (int t = 0; t < p.g; ++t) is_global |= (gl[t] == i);
+  int t_lo = max(-r, -(i / d));
+  int t_hi = p.causal ? 0 : min(r, (V - 1 - i) / d);
+  const int nwin = is_global ? V : (t_hi - t_lo + 1);
+  const int ngl = is_global ? 0 : p.g;
+  const int total = nwin + ngl + p.S;
+  const T* kb = k + ((size_t)b * p.Hkv + hk) * p.n * D;
+  const T* vb = v + ((size_t)b * p.Hkv + hk) * p.n * D;
+  const T* skb = p.S ? side_k + ((size_t)b * p.Hkv + hk) * p.S * D : nullptr;
+  const T* svb = p.S ? side_v + ((size_t)b * p.Hkv + hk) * p.S * D : nullptr;
+  const float scale = p.scale_log2 * 0.6931471805599453f;  // natural-log scale
+  const int qblk = p.S ? i / p.side_block : 0;
+  float m = -INFINITY, l = 0.f;
+  float acc[PER];
+#pragma unroll
+  for (int x = 0; x < PER; ++x) acc[x] = 0.f;
+  for (int base = 0; base < total; base += 32) {
+    const int idx = base + lane;
+    float s = -INFINITY;
+    const T* krow = nullptr;
+    const T* vrow = nullptr;
+    float bb = 0.f;
+    if (idx < nwin) {
+      int j = is_global ? idx : i + d * (t_lo + idx);
+      krow = kb + (size_t)j * D;
+      vrow = vb + (size_t)j * D;
+    } else if (idx < nwin + ngl) {
+      int j = gl[idx - nwin];
+      int diff = i - j;
+      bool inwin = (p.causal ? (diff >= 0 && diff <= r * d) : (abs(diff) <= r * d)) && (diff % d == 0);
+      if (!inwin && j < V) {
+        krow = kb + (size_t)j * D;
+        vrow = vb + (size_t)j * D;
+      }
+    } else if (idx < total) {
+      int sg = idx - nwin - ngl;
+      krow = skb + (size_t)sg * D;
+      vrow = svb + (size_t)sg * D;
+      if (p.bias) bb = p.bias[(size_t)h * (p.S + p.nblk - 1) + sg - qblk + p.nblk - 1];
+    }
+    if (krow) {
+      float dotv = 0.f;
+#pragma unroll 8
+      for (int x = 0; x < D; ++x) dotv = fmaf(sq[wib][x], to_f<T>(krow[x]), dotv);
+      s = dotv * scale + bb;
+    }
+    float cmax = s;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+    const float m_new = fmaxf(m, cmax);
+    if (m_new == -INFINITY) continue;
+    const float alpha = (m == -INFINITY) ? 0.f : expf(m - m_new);
+    const float pr = (s == -INFINITY) ? 0.f : expf(s - m_new);
+    float psum = pr;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
+    l = l * alpha + psum;
+    m = m_new;
+#pragma unroll
+    for (int x = 0; x < PER; ++x) acc[x] *= alpha;
+    for (int src = 0; src < 32; ++src) {
+      const float ps = __shfl_sync(0xffffffffu, pr, src);
+      const T* vr = reinterpret_cast<const T*>(
+          __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(vrow), src));
+      if (ps != 0.f) {
+#pragma unroll
+        for (int x = 0; x < PER; ++x) acc[x] = fmaf(ps, to_f<T>(vr[lane + 32 * x]), acc[x]);
+      }
+    }
+  }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+  for (int x = 0; x < PER; ++x) orow[lane + 32 * x] = from_f<T>(acc[x] * inv);
+  if (lane == 0 && p.lse) p.lse[row] = l > 0.f ? m + logf(l) : -INFINITY;
+}
+
+// ------------------------------------------------------------------ side aggregation
+// out[b,h,s,:] = mean of x[b,h,j,:] over block s (j < valid_len); a trailing
+// partial block joins the last full block; an empty block gives zeros.
+template <typename T>
+__global__ void side_aggregate_kernel(const T* __restrict__ x, T* __restrict__ out, int B, int H,
+                                      int n, int D, int kb, const int32_t* __restrict__ valid_len) {
+  const int S = n / kb;
+  const size_t total = (size_t)B * H * S * D;
+  for (size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x; t < total;
+       t += (size_t)gridDim.x * blockDim.x) {
+    int col = (int)(t % D);
+    size_t r = t / D;
+    int s = (int)(r % S);
+    size_t bh = r / S;
+    int b = (int)(bh / H);
+    int V = valid_len ? min(valid_len[b], n) : n;
+    int lo = s * kb;
+    int hi = (s == S - 1) ? n : lo + kb;
+    hi = min(hi, V);
+    float acc = 0.f;
+    for (int j = lo; j < hi; ++j) acc += to_f<T>(x[(bh * n + j) * D + col]);
+    int cnt = hi > lo ? hi - lo : 0;
+    out[t] = from_f<T>(cnt ? acc / (float)cnt : 0.f);
+  }
+}
+
+// ------------------------------------------------------------------ precondition check
+// global_idx rows must be strictly increasing and inside [0, valid_len).
+__global__ void check_globals_kernel(const int32_t* __restrict__ gidx, int g, int B, int n,
+                                     const int32_t* __restrict__ valid_len, int* err) {
+  int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= B * g) return;
+  int b = t / g, e = t % g;
+  int V = valid_len ? min(valid_len[b], n) : n;
+  int pos = gidx[t];
+  bool bad = pos < 0 || pos >= V || (e > 0 && gidx[t - 1] >= pos);
+  if (bad) atomicOr(err, kDevErrCheck);
+}
+
+}  // namespace
+
+cudaError_t launch_gather_globals(const AttnParams& p, const void* q, const void* k, const void* v,
+                                  void* gq, void* gk, void* gv, int elem_bytes, cudaStream_t s) {
+  const int row_vecs = p.D * elem_bytes / 16;
+  const int threads = 256;
+  auto blocks = [&](size_t total) { return (int)min((total + threads - 1) / threads, (size_t)4096); };
+  size_t tq = (size_t)p.B * p.Hq * p.gpad * row_vecs;
+  size_t tk = (size_t)p.B * p.Hkv * p.gpad * row_vecs;
+  gather_rows_kernel<<<blocks(tq), threads, 0, s>>>(static_cast<const uint4*>(q), static_cast<uint4*>(gq),
+                                                    p.global_idx, p.Hq, p.n, p.g, p.gpad, row_vecs, p.B);
+  gather_rows_kernel<<<blocks(tk), threads, 0, s>>>(static_cast<const uint4*>(k), static_cast<uint4*>(gk),
+                                                    p.global_idx, p.Hkv, p.n, p.g, p.gpad, row_vecs, p.B);
+  gather_rows_kernel<<<blocks(tk), threads, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(gv),
+                                                    p.global_idx, p.Hkv, p.n, p.g, p.gpad, row_vecs, p.B);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge_global_rows(const AttnParams& p, int bf16_out, cudaStream_t s) {
+  const int rows = p.B * p.Hq * p.g;
+  const int threads = 256;
+  const int blocks = (rows * 32 + threads - 1) / threads;
+  if (bf16_out) {
+    if (p.D == 64) merge_global_rows_kernel<__nv_bfloat16, 64><<<blocks, threads, 0, s>>>(p);
+    else merge_global_rows_kernel<__nv_bfloat16, 128><<<blocks, threads, 0, s>>>(p);
+  } else {
+    if (p.D == 64) merge_global_rows_kernel<float, 64><<<blocks, threads, 0, s>>>(p);
+    else merge_global_rows_kernel<float, 128><<<blocks, threads, 0, s>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_simt(const AttnParams& p, const void* q, const void* k, const void* v,
+                        const void* side_k, const void* side_v, int bf16, cudaStream_t s) {
+  const size_t rows = (size_t)p.B * p.Hq * p.n;
+  const unsigned blocks = (unsigned)((rows + 3) / 4);
+  if (bf16) {
+    using T = __nv_bfloat16;
+    if (p.D == 64)
+      simt_attn_kernel<T, 64><<<blocks, 128, 0, s>>>(p, (const T*)q, (const T*)k, (const T*)v,
+                                                      (const T*)side_k, (const T*)side_v);
+    else
+      simt_attn_kernel<T, 128><<<blocks, 128, 0, s>>>(p, (const T*)q, (const T*)k, (const T*)v,
+                                                       (const T*)side_k, (const T*)side_v);
+  } else {
+    using T = float;
+    if (p.D == 64)
+      simt_attn_kernel<T, 64><<<blocks, 128, 0, s>>>(p, (const T*)q, (const T*)k, (const T*)v,
+                                                      (const T*)side_k, (const T*)side_v);
+    else
+      simt_attn_kernel<T, 128><<<blocks, 128, 0, s>>>(p, (const T*)q, (const T*)k, (const T*)v,
+                                                       (const T*)side_k, (const T*)side_v);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_check_globals(const AttnParams& p, cudaStream_t s) {
+  const int t = p.B * p.g;
+  if (t == 0) return cudaSuccess;
+  check_globals_kernel<<<(t + 255) / 256, 256, 0, s>>>(p.global_idx, p.g, p.B, p.n, p.valid_len, p.err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_side_aggregate(const void* x, void* out, int B, int H, int n, int D, int kb,
+                                  const int32_t* valid_len, int bf16, cudaStream_t s) {
+  const size_t total = (size_t)B * H * (n / kb) * D;
+  const int threads = 256;
+  const int blocks = (int)min((total + threads - 1) / threads, (size_t)8192);
+  if (bf16)
+    side_aggregate_kernel<__nv_bfloat16><<<blocks, threads, 0, s>>>(
+        (const __nv_bfloat16*)x, (__nv_bfloat16*)out, B, H, n, D, kb, valid_len);
+  else
+    side_aggregate_kernel<float><<<blocks, threads, 0, s>>>((const float*)x, (float*)out, B, H, n, D, kb,
+                                                            valid_len);
+  return cudaGetLastError();
+}
+
+}  // namespace swa

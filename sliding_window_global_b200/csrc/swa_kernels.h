@@ -1,0 +1,70 @@
+// swa_kernels.h -- parameter blocks shared by the host runtime (swa_api.cu) and
+// the device kernels.  Internal to the library; the public C ABI is
+// include/swa.h.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace swa {
+
+constexpr int kTile = 128;           // query rows per tile and keys per KV tile
+constexpr int kMaxClasses = 16;      // distinct (dilation, residue) classes per forward
+constexpr int kMaxHeads = 128;       // query heads per plan
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
+
+// Bits of the device error word.
+constexpr int kDevErrTimeout = 1;    // a bounded wait expired
+constexpr int kDevErrCheck = 2;      // a device-side precondition check failed
+
+// Residue class: positions c, c+d, c+2d, ... of one dilation value d.
+struct ResidueClass {
+  int d, c, n_c;                     // dilation, residue, rows in the class
+};
+
+struct AttnParams {
+  // Tensor maps (3-D: x = head_dim, y = row, z = batch*head plane).  Band maps are
+  // per residue class: base + c*row, row stride d*row.
+  CUtensorMap mq[kMaxClasses];
+  CUtensorMap mk[kMaxClasses];
+  CUtensorMap mv[kMaxClasses];
+  CUtensorMap mgq, mgk, mgv;         // gathered global rows [B*H, gpad, D]
+  CUtensorMap msk, msv;              // side keys / values [B*Hkv, S, D]
+  ResidueClass cls[kMaxClasses];
+
+  int B, Hq, Hkv, n, D, G;           // G = Hq / Hkv
+  int g, gpad, S, side_block, nblk, causal;
+  int dense_class;                   // class id of (d = 1, c = 0): all rows, for global rows
+  float scale_log2;                  // softmax scale * log2(e)
+
+  const int32_t* valid_len;          // [B] or nullptr (= n)
+  const int32_t* global_idx;         // [B, g] or nullptr
+  const float* bias;                 // [Hq, S + nblk - 1] or nullptr
+  void* out;                         // [B, Hq, n, D], input dtype
+  float* lse;                        // [B, Hq, n] or nullptr
+  float* part_o;                     // global-row partials [nsplit, B*Hq, gpad, D]
+  float* part_lse;                   // [nsplit, B*Hq, gpad]
+  int nsplit_keys, split_keys, nsplit;  // global-row key splits (+1 for side keys)
+  int* err;                          // device error word
+
+  int window[kMaxHeads];
+  int class_base[kMaxHeads];         // class id of (dilation[h], c = 0)
+  int tiles[kMaxHeads];              // query tiles of head h over all its residues
+};
+
+// Launchers (each returns the launch's cudaError_t).
+cudaError_t launch_band_tc(const AttnParams& p, int max_tiles, cudaStream_t s);
+cudaError_t launch_global_rows_tc(const AttnParams& p, cudaStream_t s);
+cudaError_t launch_gather_globals(const AttnParams& p, const void* q, const void* k,
+                                  const void* v, void* gq, void* gk, void* gv, int elem_bytes,
+                                  cudaStream_t s);
+cudaError_t launch_merge_global_rows(const AttnParams& p, int bf16_out, cudaStream_t s);
+cudaError_t launch_simt(const AttnParams& p, const void* q, const void* k, const void* v,
+                        const void* side_k, const void* side_v, int bf16, cudaStream_t s);
+cudaError_t launch_check_globals(const AttnParams& p, cudaStream_t s);
+cudaError_t launch_side_aggregate(const void* x, void* out, int B, int H, int n, int D, int kb,
+                                  const int32_t* valid_len, int bf16, cudaStream_t s);
+size_t band_tc_smem_bytes(int D);
+
+}  // namespace swa

@@ -49,6 +49,12 @@ class Workload:
     rope: bool = False              # rotate q and k with RoPE (base 10000, all dims)
     seed: int = 0
 
+    def __post_init__(self):
+        if len(self.window) != self.q_heads or len(self.dilation) != self.q_heads:
+            raise ValueError(f"{self.name}: window/dilation need one value per query head")
+        if self.q_heads % self.kv_heads:
+            raise ValueError(f"{self.name}: q_heads must be a multiple of kv_heads")
+
     @property
     def torch_dtype(self):
         return torch.float32 if self.dtype == "fp32" else torch.bfloat16
@@ -91,8 +97,9 @@ WORKLOADS = {
 SMALL = {
     "longformer_tiny": WORKLOADS["longformer_tiny"],
     "longformer_base": dataclasses.replace(WORKLOADS["longformer_base"], name="longformer_base_small",
-                                           seq_len=1000, window=_heads(100, 12), num_global=16,
-                                           padding=77, q_heads=4, kv_heads=4, seed=2002),
+                                           seq_len=1000, window=_heads(100, 4), dilation=_heads(1, 4),
+                                           num_global=16, padding=77, q_heads=4, kv_heads=4,
+                                           seed=2002),
     "dilated": dataclasses.replace(WORKLOADS["dilated"], name="dilated_small", seq_len=1111,
                                    q_heads=4, kv_heads=4, window=_heads(70, 4),
                                    dilation=(1, 1, 2, 3), num_global=5, seed=2003),

@@ -1,0 +1,187 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs.
+
+* every workload at a reduced size (several tiles and a ragged tail), full output;
+* every workload at full size on sampled rows, plus whole-output properties;
+* edge cases: r = 0, window covering the sequence, ragged n, one valid row, g > 128,
+  side counts that are not a tile multiple, causal + dilation, GQA;
+* exact support: with V = identity rows the output row is the weight row, so every
+  key outside K(i) must come back exactly 0 and every key inside it positive.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sliding_window_global_b200 import workloads
+from tests import helpers
+
+pytestmark = pytest.mark.gpu
+
+
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def _check_workload(w, seed_inp=None):
+    inp = helpers.host_problem(w, seed_inp)
+    dinp = helpers.to_dev(inp)
+    out, lse, plan = helpers.run_gpu(w, dinp)
+    assert plan.check() == 0
+    ref_o, ref_l, _ = helpers.oracle_problem(w, inp).forward()
+    return helpers.compare(out.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_l, w.dtype, w.name)
+
+
+@pytest.mark.parametrize("name", list(workloads.SMALL))
+def test_small_workloads_full_output(name):
+    _need_gpu()
+    _check_workload(workloads.SMALL[name])
+
+
+@pytest.mark.parametrize("name", list(workloads.WORKLOADS))
+def test_full_size_sampled_rows(name):
+    _need_gpu()
+    w = workloads.WORKLOADS[name]
+    inp = helpers.host_problem(w)
+    dinp = helpers.to_dev(inp)
+    out, lse, plan = helpers.run_gpu(w, dinp)
+    assert plan.check() == 0
+    rows = helpers.sample_rows(w, inp, 1500 if w.seq_len * w.q_heads < 10**6 else 600)
+    ref_o, ref_l, _ = helpers.oracle_problem(w, inp).forward(rows)
+    o = out.reshape(-1, w.head_dim)[torch.from_numpy(rows).cuda()].float().cpu().numpy()
+    l = lse.reshape(-1)[torch.from_numpy(rows).cuda()].cpu().numpy()
+    helpers.compare(o, l, ref_o, ref_l, w.dtype, name)
+    # whole-output properties at full size
+    assert bool(torch.isfinite(out.float()).all())
+    if w.padding:
+        V = w.valid_len
+        assert bool((out[:, :, V:] == 0).all())
+        assert bool(torch.isneginf(lse[:, :, V:]).all())
+        assert bool(torch.isfinite(lse[:, :, :V]).all())
+
+
+def _small(base, **kw):
+    return dataclasses.replace(workloads.SMALL[base], **kw)
+
+
+EDGE = [
+    ("r0", _small("longformer_base", window=(0,) * 4, num_global=0, global_mode="none")),
+    ("full_window", _small("longformer_base", window=(5000,) * 4, num_global=0, global_mode="none")),
+    ("full_window_causal", _small("swan_swa", window=(5000,) * 8)),
+    ("one_valid_row", _small("longformer_base", padding=999, num_global=1)),
+    ("many_globals", _small("dilated", num_global=150, seq_len=700)),
+    ("globals_only_pad", _small("longformer_base", padding=500)),
+    ("side_not_tile_multiple", _small("longt5_tglobal", seq_len=1600, side_block=16)),
+    ("side_block_7", _small("longt5_tglobal", seq_len=777, side_block=7, padding=20)),
+    ("causal_dilated", _small("swan_swa", dilation=(1, 2, 3, 4, 1, 2, 3, 4), window=(40,) * 8)),
+    ("gqa_d64", _small("swan_swa", head_dim=64, q_heads=6, kv_heads=2, window=(130,) * 6,
+                       dilation=(1,) * 6)),
+    ("noncausal_d128", _small("swan_swa", causal=False, window=(200,) * 8)),
+    ("batch3_tiny_n", _small("dilated", batch=3, seq_len=77, window=(9,) * 4, num_global=3)),
+    ("n_one", _small("longformer_base", seq_len=1, padding=0, num_global=0, global_mode="none")),
+    ("fp32_gqa_side", dataclasses.replace(workloads.SMALL["longt5_tglobal"], dtype="fp32",
+                                          q_heads=4, kv_heads=2, window=(20,) * 4,
+                                          dilation=(1, 2, 1, 2), seq_len=300)),
+    ("fp32_globals_pad", dataclasses.replace(workloads.SMALL["longformer_base"], dtype="fp32",
+                                             seq_len=400, padding=33, num_global=7)),
+]
+
+
+@pytest.mark.parametrize("name,w", EDGE, ids=[e[0] for e in EDGE])
+def test_edge_cases(name, w):
+    _need_gpu()
+    _check_workload(w)
+
+
+SUPPORT = [
+    # (n, D, r, dilation, causal, g, padding)
+    (128, 128, 5, 1, False, 0, 0),
+    (128, 128, 7, 2, False, 3, 9),
+    (120, 128, 4, 3, True, 0, 5),
+    (128, 128, 40, 1, True, 0, 0),
+    (64, 64, 3, 1, False, 2, 0),
+    (64, 64, 2, 2, False, 0, 7),
+    (100, 128, 0, 1, False, 4, 0),
+]
+
+
+@pytest.mark.parametrize("n,D,r,d,causal,g,pad", SUPPORT)
+def test_support_exact(n, D, r, d, causal, g, pad):
+    """V = identity rows: o_i[j] = weight of key j -> zero exactly off K(i), > 0 on it."""
+    _need_gpu()
+    from sliding_window_global_b200 import Plan
+    gen = torch.Generator("cpu").manual_seed(n * 1000 + r * 10 + d)
+    B, H = 2, 2
+    q = torch.randn((B, H, n, D), generator=gen).to(torch.bfloat16)
+    k = torch.randn((B, H, n, D), generator=gen).to(torch.bfloat16)
+    v = torch.zeros((B, H, n, D))
+    v[:, :, torch.arange(n), torch.arange(n)] = 1.0
+    v = v.to(torch.bfloat16)
+    V = n - pad
+    gl = None
+    if g:
+        gl = torch.stack([torch.sort(torch.randperm(V, generator=gen)[:g]).values for _ in range(B)])
+        gl = gl.to(torch.int32)
+    vl = torch.full((B,), V, dtype=torch.int32) if pad else None
+    plan = Plan(B, n, H, H, D, torch.bfloat16, max_global=g)
+    out, _ = plan.forward(q.cuda(), k.cuda(), v.cuda(), window=r, dilation=d, causal=causal,
+                          global_idx=None if gl is None else gl.cuda(),
+                          valid_len=None if vl is None else vl.cuda())
+    o = out.float().cpu().numpy()
+    for b in range(B):
+        for h in range(H):
+            for i in range(n):
+                keys = oracle.key_list(B, H, n, b, h, i, window=r, dilation=d, causal=causal,
+                                       global_idx=None if gl is None else gl.numpy(),
+                                       valid_len=None if vl is None else vl.numpy())
+                inside = np.zeros(n, bool)
+                inside[keys] = True
+                row = o[b, h, i, :n]
+                assert np.all(row[~inside] == 0.0), (b, h, i)
+                assert np.all(row[inside] > 0.0), (b, h, i)
+
+
+def test_side_aggregate_matches_oracle():
+    _need_gpu()
+    from sliding_window_global_b200 import side_aggregate
+    gen = torch.Generator("cpu").manual_seed(5)
+    x = torch.randn((2, 3, 1000, 64), generator=gen).to(torch.bfloat16)
+    vl = torch.tensor([1000, 937], dtype=torch.int32)
+    got = side_aggregate(x.cuda(), 16, vl.cuda()).float().cpu().numpy()
+    ref = oracle.side_aggregate(x, 16, vl.numpy())
+    # the device rounds an fp32 mean to bf16: within one bf16 ulp of the fp64 mean
+    ulp = np.abs(ref) * 2.0 ** -7 + 1e-30
+    assert np.all(np.abs(got - ref) <= ulp)
+
+
+def test_debug_mode_flags_bad_global_index():
+    """A global index out of [0, valid_len) is a precondition failure that debug mode
+    reports as a status (the kernels never read it: the check runs first)."""
+    _need_gpu()
+    from sliding_window_global_b200 import Plan, SwaError
+    w = workloads.SMALL["longformer_base"]
+    inp = helpers.to_dev(helpers.host_problem(w))
+    plan = Plan(w.batch, w.seq_len, w.q_heads, w.kv_heads, w.head_dim, torch.bfloat16,
+                max_global=4, debug=True)
+    bad = torch.tensor([[3, 2, 5, 9]], dtype=torch.int32, device="cuda")  # not increasing
+    with pytest.raises(SwaError) as e:
+        plan.forward(inp["q"], inp["k"], inp["v"], window=inp["window"], global_idx=bad,
+                     valid_len=inp["valid_len"])
+    assert e.value.status == 6
+    good = torch.tensor([[2, 3, 5, 9]], dtype=torch.int32, device="cuda")
+    plan.forward(inp["q"], inp["k"], inp["v"], window=inp["window"], global_idx=good,
+                 valid_len=inp["valid_len"])
+    assert plan.check() == 0
+
+
+def test_repeat_calls_deterministic_and_launch_count():
+    _need_gpu()
+    w = workloads.SMALL["dilated"]
+    dinp = helpers.to_dev(helpers.host_problem(w))
+    o1, l1, plan = helpers.run_gpu(w, dinp)
+    o2, l2, _ = helpers.run_gpu(w, dinp, plan=plan)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert plan.last_launches == 6   # gather x3, band, global rows, merge
