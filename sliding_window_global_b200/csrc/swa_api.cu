@@ -268,10 +268,10 @@ swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void
       }
     }
     p.class_base[h] = base;
-    int tiles = 0;
-    for (int c = 0; c < std::min(dh, n); ++c) tiles += (p.cls[base + c].n_c + kTile - 1) / kTile;
-    p.tiles[h] = tiles;
-    max_tiles = std::max(max_tiles, tiles);
+    int units = 0;   // pairs of 128-row query tiles, per residue class
+    for (int c = 0; c < std::min(dh, n); ++c) units += ((p.cls[base + c].n_c + kTile - 1) / kTile + 1) / 2;
+    p.tiles[h] = units;
+    max_tiles = std::max(max_tiles, units);
   }
   if (st == SWA_OK && num_global > 0) {
     p.dense_class = -1;
@@ -316,6 +316,8 @@ swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void
                           (uint64_t)p.B * p.Hkv, dd * row, (uint64_t)n * row);
       ok = ok && make_map(&p.mv[c], static_cast<const char*>(v) + cc * row, D, nc,
                           (uint64_t)p.B * p.Hkv, dd * row, (uint64_t)n * row);
+      ok = ok && make_map(&p.mo[c], static_cast<const char*>(out) + cc * row, D, nc, (uint64_t)p.B * Hq,
+                          dd * row, (uint64_t)n * row);
     }
     if (ok && num_global > 0) {
       p.part_o = plan->part_o;

@@ -29,6 +29,7 @@ struct AttnParams {
   CUtensorMap mq[kMaxClasses];
   CUtensorMap mk[kMaxClasses];
   CUtensorMap mv[kMaxClasses];
+  CUtensorMap mo[kMaxClasses];       // out, same class views as mq
   CUtensorMap mgq, mgk, mgv;         // gathered global rows [B*H, gpad, D]
   CUtensorMap msk, msv;              // side keys / values [B*Hkv, S, D]
   ResidueClass cls[kMaxClasses];
@@ -50,11 +51,11 @@ struct AttnParams {
 
   int window[kMaxHeads];
   int class_base[kMaxHeads];         // class id of (dilation[h], c = 0)
-  int tiles[kMaxHeads];              // query tiles of head h over all its residues
+  int tiles[kMaxHeads];              // two-tile query units of head h over all its residues
 };
 
 // Launchers (each returns the launch's cudaError_t).
-cudaError_t launch_band_tc(const AttnParams& p, int max_tiles, cudaStream_t s);
+cudaError_t launch_band_tc(const AttnParams& p, int max_units, cudaStream_t s);
 cudaError_t launch_global_rows_tc(const AttnParams& p, cudaStream_t s);
 cudaError_t launch_gather_globals(const AttnParams& p, const void* q, const void* k,
                                   const void* v, void* gq, void* gk, void* gv, int elem_bytes,
