@@ -41,6 +41,7 @@ struct swa_plan_s {
   float* part_o;
   float* part_lse;
   int last_launches;
+  int num_sms;         // persistent grid size
 };
 
 namespace {
@@ -118,7 +119,8 @@ swa_status swa_plan_create(swa_plan_t* out_plan, const swa_plan_desc* d) {
   swa_plan_s* p = new (std::nothrow) swa_plan_s();
   if (!p) return SWA_ERR_OOM;
   p->desc = *d;
-  if (cudaGetDevice(&p->device) != cudaSuccess) {
+  if (cudaGetDevice(&p->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, p->device) != cudaSuccess) {
     delete p;
     return SWA_ERR_CUDA;
   }
@@ -350,11 +352,12 @@ swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void
       }
     }
     if (ce == cudaSuccess) {
-      ce = swa::launch_band_tc(p, max_tiles, s);
+      p.max_units = max_tiles;
+      ce = swa::launch_band_tc(p, plan->num_sms, s);
       ++launches;
     }
     if (ce == cudaSuccess && num_global > 0) {
-      ce = swa::launch_global_rows_tc(p, s);
+      ce = swa::launch_global_rows_tc(p, plan->num_sms, s);
       ++launches;
       if (ce == cudaSuccess) {
         ce = swa::launch_merge_global_rows(p, 1, s);

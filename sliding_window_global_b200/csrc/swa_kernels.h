@@ -47,6 +47,7 @@ struct AttnParams {
   float* part_o;                     // global-row partials [nsplit, B*Hq, gpad, D]
   float* part_lse;                   // [nsplit, B*Hq, gpad]
   int nsplit_keys, split_keys, nsplit;  // global-row key splits (+1 for side keys)
+  int max_units;                     // largest tiles[h]
   int* err;                          // device error word
 
   int window[kMaxHeads];
@@ -55,8 +56,8 @@ struct AttnParams {
 };
 
 // Launchers (each returns the launch's cudaError_t).
-cudaError_t launch_band_tc(const AttnParams& p, int max_units, cudaStream_t s);
-cudaError_t launch_global_rows_tc(const AttnParams& p, cudaStream_t s);
+cudaError_t launch_band_tc(const AttnParams& p, int num_sms, cudaStream_t s);
+cudaError_t launch_global_rows_tc(const AttnParams& p, int num_sms, cudaStream_t s);
 cudaError_t launch_gather_globals(const AttnParams& p, const void* q, const void* k,
                                   const void* v, void* gq, void* gk, void* gv, int elem_bytes,
                                   cudaStream_t s);
