@@ -87,6 +87,7 @@ struct Cfg {
 struct Work {
   bool valid;           // the unit id names real work
   int b, h, hk, cls, d, c, r;
+  int hx[2];            // query head of tile A, B (equal unless heads are paired)
   int u0[2];            // first row (class coordinates / global slot) of tile A, B
   int rows[2];          // rows that exist
   int nvalid[2];        // rows below the valid length / below g
@@ -101,26 +102,33 @@ struct Work {
 
 template <int MODE>
 __device__ __forceinline__ int total_units(const AttnParams& p) {
-  return MODE == 0 ? p.max_units * p.B * p.Hq : p.nsplit * (p.gpad / kTile) * p.B * p.Hq;
+  return MODE == 0 ? p.max_units * p.B * (p.pair_heads ? p.Hq / 2 : p.Hq)
+                   : p.nsplit * (p.gpad / kTile) * p.B * p.Hq;
 }
 
 template <int MODE>
 __device__ __forceinline__ void decode_work(const AttnParams& p, int unit_id, Work& w) {
   if (MODE == 0) {
-    const int BH = p.B * p.Hq;
+    // unit ids run over (unit, batch, head or head pair), heads fastest
+    const int hunits = p.pair_heads ? p.Hq / 2 : p.Hq;
+    const int BH = p.B * hunits;
     const int bh = unit_id % BH;
     int unit = unit_id / BH;
-    w.b = bh / p.Hq;
-    w.h = bh % p.Hq;
-    w.valid = unit < p.tiles[w.h];             // p.tiles holds two-tile units per head
+    w.b = bh / hunits;
+    w.h = p.pair_heads ? 2 * (bh % hunits) : bh % hunits;
+    w.hx[0] = w.h;
+    w.hx[1] = p.pair_heads ? w.h + 1 : w.h;
+    w.valid = unit < p.tiles[w.h];
     w.hk = w.h / p.G;
     w.r = p.window[w.h];
     const int base = p.class_base[w.h];
     w.d = p.cls[base].d;
+    const int nres = p.cls[base].nres;
+    const int per_unit = p.pair_heads ? 1 : 2;           // row tiles per unit and class
     int c = 0;
-    for (; c < w.d - 1; ++c) {
+    for (; c < nres - 1; ++c) {
       const int tc = (p.cls[base + c].n_c + kTile - 1) / kTile;
-      const int uc = (tc + 1) / 2;
+      const int uc = (tc + per_unit - 1) / per_unit;
       if (unit < uc) break;
       unit -= uc;
     }
@@ -133,7 +141,7 @@ __device__ __forceinline__ void decode_work(const AttnParams& p, int unit_id, Wo
     w.split = 0;
     w.key_end = 0;
     for (int x = 0; x < 2; ++x) {
-      w.u0[x] = unit * 2 * kTile + x * kTile;
+      w.u0[x] = p.pair_heads ? unit * kTile : unit * 2 * kTile + x * kTile;
       w.rows[x] = w.valid ? max(0, min(kTile, nc - w.u0[x])) : 0;
       w.nvalid[x] = max(0, min(w.rows[x], w.Vc - w.u0[x]));
       w.active[x] = w.nvalid[x] > 0;
@@ -155,6 +163,7 @@ __device__ __forceinline__ void decode_work(const AttnParams& p, int unit_id, Wo
     const int bh = rest / gtiles;
     w.b = bh / p.Hq;
     w.h = bh % p.Hq;
+    w.hx[0] = w.hx[1] = w.h;
     w.hk = w.h / p.G;
     w.r = 0;
     w.d = 1;
@@ -285,7 +294,7 @@ __device__ __forceinline__ float row_max128(const float (&x)[kTile]) {
 // ------------------------------------------------------------------ output rows
 __device__ __forceinline__ size_t out_row(const AttnParams& p, const Work& w, int x, int row) {
   const int pos = w.c + w.d * (w.u0[x] + row);
-  return (size_t)(w.b * p.Hq + w.h) * p.n + pos;
+  return (size_t)(w.b * p.Hq + w.hx[x]) * p.n + pos;
 }
 
 template <int D>
@@ -375,9 +384,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         decode_work<MODE>(p, uid, w);
         if (!w.active[0]) continue;
         const CUtensorMap* mq = (MODE == 0) ? &p.mq[w.cls] : &p.mgq;
-        const int qz = w.b * p.Hq + w.h;
         const int kz = w.b * p.Hkv + w.hk;
         for (int x = 0; x < 2 && ok; ++x) {
+          const int qz = w.b * p.Hq + w.hx[x];
           if (!w.active[x]) continue;
           if (qloads[x] > 0 &&
               !mbar_wait_bounded(&q_empty[x], (qloads[x] - 1) & 1, abort_v, kWaitLimitNs)) {
@@ -597,10 +606,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         if (j < w.nband) {
           const int kv0 = w.band_lo + j * kTile;
           const int lo_t = klo - kv0, hi_t = khi - kv0;
-          const bool interior = (lo_t <= 0) && (hi_t >= kTile);
-          if (!__all_sync(0xffffffffu, interior)) {
+          // boundary tiles: most cut only one side of the band (window start or
+          // causal diagonal), which costs one compare and one select per score
+          const bool cut_lo = __any_sync(0xffffffffu, lo_t > 0);
+          const bool cut_hi = __any_sync(0xffffffffu, hi_t < kTile);
+          if (cut_lo && cut_hi) {
 #pragma unroll
             for (int e = 0; e < kTile; ++e) s[e] = (e >= lo_t && e < hi_t) ? s[e] : -INFINITY;
+          } else if (cut_lo) {
+#pragma unroll
+            for (int e = 0; e < kTile; ++e) s[e] = (e >= lo_t) ? s[e] : -INFINITY;
+          } else if (cut_hi) {
+#pragma unroll
+            for (int e = 0; e < kTile; ++e) s[e] = (e < hi_t) ? s[e] : -INFINITY;
           }
           tmax = row_max128(s) * sl2;
           raw = true;
@@ -726,7 +744,42 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const bool has = row_valid && l > 0.f;
       const float inv = has ? 1.f / l : 0.f;
       const float lse_v = has ? (m + __log2f(l)) * kLn2 : -INFINITY;
-      if (MODE == 0) {
+      if (MODE == 0 && !has_bias) {
+        // Coalesced store: 32-column chunks staged in shared memory (the side-bias
+        // area, unused without bias; two 8 KB buffers per group, 64-byte swizzle)
+        // and written by TMA; rows beyond the class end are clipped by the map.
+        uint8_t* stage = reinterpret_cast<uint8_t*>(sBias) + x * 2 * 8192;
+        if (row == 0) tma_store_wait_read<0>();          // previous unit's stores have read
+        named_barrier_sync(1 + x, 128);
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint8_t* buf = stage + (ch & 1) * 8192;
+          if (ch >= 2) {
+            if (row == 0) tma_store_wait_read<1>();      // the store of chunk ch-2 has read buf
+            named_barrier_sync(1 + x, 128);
+          }
+          uint32_t rr[32];
+          tmem_ld32(o_addr + ch * 32, rr);
+          tmem_wait_ld_dep(rr);
+          uint8_t* rbase = buf + row * 64;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 0]) * inv, __uint_as_float(rr[q4 * 8 + 1]) * inv);
+            v.y = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 2]) * inv, __uint_as_float(rr[q4 * 8 + 3]) * inv);
+            v.z = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 4]) * inv, __uint_as_float(rr[q4 * 8 + 5]) * inv);
+            v.w = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 6]) * inv, __uint_as_float(rr[q4 * 8 + 7]) * inv);
+            *reinterpret_cast<uint4*>(rbase + ((q4 ^ ((row >> 1) & 3)) << 4)) = v;
+          }
+          fence_proxy_async_smem();
+          named_barrier_sync(1 + x, 128);
+          if (row == 0) {
+            tma_store_3d(&p.mo[w.cls], buf, ch * 32, w.u0[x], w.b * p.Hq + w.hx[x]);
+            tma_store_commit();
+          }
+        }
+        if (row < w.rows[x] && p.lse) p.lse[out_row(p, w, x, row)] = lse_v;
+      } else if (MODE == 0) {
         const size_t off = out_row(p, w, x, row);
         uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + off * D);
 #pragma unroll
@@ -769,6 +822,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
   }
 
+  if (warp < 8 && (tid & 127) == 0) tma_store_wait_read<0>();   // staged stores have read smem
   tc_fence_before();
   __syncthreads();
   if (abort_flag) {

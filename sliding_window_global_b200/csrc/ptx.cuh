@@ -115,6 +115,17 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
       : "memory");
 }
 
+// Close the current bulk async-group (TMA stores issued by this thread).
+__device__ __forceinline__ void tma_store_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until at most N of this thread's bulk async-groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void tma_store_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
 // Close the current bulk async-group and wait until all of this thread's bulk
 // stores have completed.
 __device__ __forceinline__ void tma_store_commit_and_wait() {

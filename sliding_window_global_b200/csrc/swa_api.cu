@@ -69,17 +69,20 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D bf16 map: x = D (box 64, 128-byte swizzle), y = rows (box 128), z = planes (box 1).
+// 3-D bf16 map: x = D, y = rows (box 128), z = planes (box 1).  Loads use a box
+// of 64 columns with the 128-byte swizzle (the tcgen05 operand layout); output
+// stores use a box of 32 columns with the 64-byte swizzle (the staging layout).
 bool make_map(CUtensorMap* m, const void* base, int D, uint64_t rows, uint64_t planes,
-              uint64_t row_stride_bytes, uint64_t plane_stride_bytes) {
+              uint64_t row_stride_bytes, uint64_t plane_stride_bytes, bool store_box = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn || rows == 0 || planes == 0) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, rows, planes};
   cuuint64_t strides[2] = {row_stride_bytes, plane_stride_bytes};
-  cuuint32_t box[3] = {64, (cuuint32_t)kTile, 1};
+  cuuint32_t box[3] = {store_box ? 32u : 64u, (cuuint32_t)kTile, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  store_box ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -248,7 +251,6 @@ swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void
   p.err = plan->err;
 
   // residue classes: one per (distinct dilation value, residue)
-  std::vector<int> dvals;
   int nclass = 0;
   int max_tiles = 0;
   swa_status st = SWA_OK;
@@ -266,14 +268,32 @@ swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void
         p.cls[nclass].d = dh;
         p.cls[nclass].c = c;
         p.cls[nclass].n_c = (n - c + dh - 1) / dh;
+        p.cls[nclass].nres = need;
         ++nclass;
       }
     }
     p.class_base[h] = base;
-    int units = 0;   // pairs of 128-row query tiles, per residue class
-    for (int c = 0; c < std::min(dh, n); ++c) units += ((p.cls[base + c].n_c + kTile - 1) / kTile + 1) / 2;
-    p.tiles[h] = units;
-    max_tiles = std::max(max_tiles, units);
+  }
+  // Work units: two 128-row query tiles.  When query heads come in GQA pairs with
+  // the same window and dilation (and no per-head side bias), a unit is the same
+  // rows of two heads that share one KV head; otherwise it is two consecutive
+  // row tiles of one head.
+  if (st == SWA_OK) {
+    bool pair = (p.G % 2 == 0) && !(d.num_side > 0 && bias);
+    for (int h = 0; pair && h < Hq; h += 2)
+      pair = window[h] == window[h + 1] && p.class_base[h] == p.class_base[h + 1];
+    p.pair_heads = pair ? 1 : 0;
+    for (int h = 0; h < Hq; ++h) {
+      const int base = p.class_base[h];
+      const int dh = p.cls[base].d;
+      int units = 0;
+      for (int c = 0; c < std::min(dh, n); ++c) {
+        const int tiles = (p.cls[base + c].n_c + kTile - 1) / kTile;
+        units += pair ? tiles : (tiles + 1) / 2;
+      }
+      p.tiles[h] = units;
+      max_tiles = std::max(max_tiles, units);
+    }
   }
   if (st == SWA_OK && num_global > 0) {
     p.dense_class = -1;
@@ -285,6 +305,7 @@ swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void
         p.cls[nclass].d = 1;
         p.cls[nclass].c = 0;
         p.cls[nclass].n_c = n;
+        p.cls[nclass].nres = 1;
         p.dense_class = nclass++;
       }
     }
@@ -318,8 +339,8 @@ swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void
                           (uint64_t)p.B * p.Hkv, dd * row, (uint64_t)n * row);
       ok = ok && make_map(&p.mv[c], static_cast<const char*>(v) + cc * row, D, nc,
                           (uint64_t)p.B * p.Hkv, dd * row, (uint64_t)n * row);
-      ok = ok && make_map(&p.mo[c], static_cast<const char*>(out) + cc * row, D, nc, (uint64_t)p.B * Hq,
-                          dd * row, (uint64_t)n * row);
+      ok = ok && make_map(&p.mo[c], static_cast<char*>(out) + cc * row, D, nc, (uint64_t)p.B * Hq,
+                          dd * row, (uint64_t)n * row, true);
     }
     if (ok && num_global > 0) {
       p.part_o = plan->part_o;

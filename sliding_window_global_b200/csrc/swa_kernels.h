@@ -21,6 +21,7 @@ constexpr int kDevErrCheck = 2;      // a device-side precondition check failed
 // Residue class: positions c, c+d, c+2d, ... of one dilation value d.
 struct ResidueClass {
   int d, c, n_c;                     // dilation, residue, rows in the class
+  int nres;                          // classes of this dilation: min(d, n)
 };
 
 struct AttnParams {
@@ -29,7 +30,7 @@ struct AttnParams {
   CUtensorMap mq[kMaxClasses];
   CUtensorMap mk[kMaxClasses];
   CUtensorMap mv[kMaxClasses];
-  CUtensorMap mo[kMaxClasses];       // out, same class views as mq
+  CUtensorMap mo[kMaxClasses];       // out, same class views as mq (32-column store boxes)
   CUtensorMap mgq, mgk, mgv;         // gathered global rows [B*H, gpad, D]
   CUtensorMap msk, msv;              // side keys / values [B*Hkv, S, D]
   ResidueClass cls[kMaxClasses];
@@ -48,11 +49,12 @@ struct AttnParams {
   float* part_lse;                   // [nsplit, B*Hq, gpad]
   int nsplit_keys, split_keys, nsplit;  // global-row key splits (+1 for side keys)
   int max_units;                     // largest tiles[h]
+  int pair_heads;                    // units pair heads 2m, 2m+1 (same rows) instead of row tiles
   int* err;                          // device error word
 
   int window[kMaxHeads];
   int class_base[kMaxHeads];         // class id of (dilation[h], c = 0)
-  int tiles[kMaxHeads];              // two-tile query units of head h over all its residues
+  int tiles[kMaxHeads];              // work units of head h (of head pair h/2 when pairing)
 };
 
 // Launchers (each returns the launch's cudaError_t).
