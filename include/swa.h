@@ -150,6 +150,39 @@ int swa_relative_bucket(int delta);
 swa_status swa_expand_side_bias(int num_q_heads, int num_side, int nblk, const float* table,
                                 float* out);
 
+/* ---------------------------------------------------------------------------
+ * Allocation-free forward pass.  (An addition of this library: the pages
+ * describe nothing like it.)
+ *
+ * For callers that cannot allocate memory when they run the attention: code
+ * under a fixed memory budget or inside a host framework that owns all device
+ * memory, real-time paths where allocating (and the synchronisation that a
+ * device allocation can imply) is not allowed, and plug-ins that cannot keep a
+ * plan object alive.  swa_forward_noalloc takes the plan descriptor directly and
+ * runs the same kernels as swa_forward; it calls no cudaMalloc, cudaFree or any
+ * other allocating routine, on the device or on the host.
+ *
+ * Its scratch memory (device error word, gathered global rows, split partials
+ * of the global query rows) is one static device array of
+ * SWA_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until the
+ * process exits.  The first call on a device looks up that array's device
+ * address (cudaGetSymbolAddress, with the device current); make that first call
+ * before any stream capture on the device.  Problems whose scratch would exceed
+ * the limit -- only bf16 calls with global tokens need more than the error word
+ * -- return SWA_ERR_UNSUPPORTED without launching anything.  All calls share the
+ * array: each clears the error word and rewrites the rest before reading it, but
+ * calls that overlap on the GPU (unordered streams or threads) race on it.
+ * Arguments, layouts and the other statuses are those of swa_plan_create plus
+ * swa_forward (desc: the plan descriptor; stream: a cudaStream_t).
+ * ------------------------------------------------------------------------- */
+#define SWA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+swa_status swa_forward_noalloc(const swa_plan_desc* desc, const void* q, const void* k,
+                               const void* v, const int32_t* global_idx, int num_global,
+                               const void* side_k, const void* side_v, const float* bias,
+                               const int32_t* window, const int32_t* dilation, int causal,
+                               const int32_t* valid_len, void* out, float* lse, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

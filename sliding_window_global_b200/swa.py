@@ -29,7 +29,7 @@ SWA_DEBUG_CHECKS = 1
 EXPORTS = (
     "swa_plan_create", "swa_forward", "swa_plan_check", "swa_plan_destroy",
     "swa_plan_workspace_bytes", "swa_plan_last_launches", "swa_status_string",
-    "swa_side_aggregate", "swa_relative_bucket", "swa_expand_side_bias",
+    "swa_side_aggregate", "swa_relative_bucket", "swa_expand_side_bias", "swa_forward_noalloc",
 )
 
 
@@ -82,6 +82,9 @@ def load_library():
         lib.swa_relative_bucket.restype = I
         lib.swa_expand_side_bias.argtypes = [I, I, I, P, P]
         lib.swa_expand_side_bias.restype = I
+        lib.swa_forward_noalloc.argtypes = [ctypes.POINTER(PlanDesc), P, P, P, P, I, P, P, P, P, P, I,
+                                            P, P, P, P]
+        lib.swa_forward_noalloc.restype = I
         _lib = lib
         return lib
 
