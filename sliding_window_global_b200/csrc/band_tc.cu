@@ -76,11 +76,18 @@ struct Cfg {
   static constexpr uint32_t kVOff = kKOff + NS * kTileBytes;
   static constexpr uint32_t kBiasOff = kVOff + NS * kTileBytes;  // 4 shifted copies
   static constexpr uint32_t kBarOff = kBiasOff + 4 * kBiasCopy * 4;
-  static constexpr int kNumBars = 2 + 2 + 3 * NS + 2 + 2 + 2;
+  static constexpr int kNumBars = 2 + 2 + 3 * NS + 2 + 2 + 2 + 2 + 2;
   static constexpr uint32_t kSmemBytes = kBarOff + kNumBars * 8 + 1024;
-  static constexpr uint32_t kTmemCols = 512;                    // S_A | S_B | O_A | O_B
+  // TMEM columns.  D = 128: S_A | S_B | O_A | O_B, P written over S.  D = 64 has
+  // room for separate P buffers (S_A | S_B | P_A | P_B | O_A | O_B), so the next
+  // S can be computed while the softmax of the current one still runs.
+  static constexpr bool kSepP = (D == 64);
+  static constexpr uint32_t kTmemCols = 512;
   __host__ __device__ static constexpr uint32_t s_col(int x) { return x ? 128u : 0u; }
-  __host__ __device__ static constexpr uint32_t o_col(int x) { return 256u + (x ? D : 0); }
+  __host__ __device__ static constexpr uint32_t p_col(int x) { return kSepP ? 256u + 64u * x : s_col(x); }
+  __host__ __device__ static constexpr uint32_t o_col(int x) {
+    return kSepP ? 384u + 64u * x : 256u + (x ? D : 0);
+  }
 };
 
 // ------------------------------------------------------------------ work description
@@ -337,6 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   uint64_t* s_full = kv_empty + NS;       // [2]
   uint64_t* p_full = s_full + 2;          // [2]
   uint64_t* o_full = p_full + 2;          // [2]
+  uint64_t* s_free = o_full + 2;          // [2] S read into registers (separate-P layout)
+  uint64_t* pv_done = s_free + 2;         // [2] a PV finished: P buffer free, O updated
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ int sGpos[2 * kTile];        // positions of the current global tile, per group
@@ -354,6 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_init(&s_full[x], 1);
       mbar_init(&p_full[x], kTile);
       mbar_init(&o_full[x], 1);
+      mbar_init(&s_free[x], kTile);
+      mbar_init(&pv_done[x], 1);
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(&k_full[s], 1);
@@ -425,6 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const uint32_t v_base = smem_u32(sV);
       int qwaits[2] = {0, 0};
       int pwaits[2] = {0, 0};
+      int nqk[2] = {0, 0};                          // QKs issued per tile buffer (kernel-wide)
       int kv = 0;
       bool ok = true;
       for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
@@ -442,6 +454,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         auto issue_qk = [&](int x, int j) -> bool {
           const int g = kv + j;
           if (!mbar_wait_bounded(&k_full[g % NS], (g / NS) & 1, abort_v, kWaitLimitNs)) return false;
+          // separate-P layout: S_x is rewritten only after the softmax read the last one
+          if (C::kSepP && nqk[x] > 0 &&
+              !mbar_wait_bounded(&s_free[x], (nqk[x] - 1) & 1, abort_v, kWaitLimitNs))
+            return false;
+          ++nqk[x];
           tc_fence_after();
           const uint32_t qt = q_base + x * C::kTileBytes;
           const uint32_t kt = k_base + (g % NS) * C::kTileBytes;
@@ -467,6 +484,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           const int st = g % NS;
           for (int x = 0; x < 2 && ok; ++x)
             if (uses(w, x, j) && issued[x] < j) ok = issue_qk(x, j);
+          if (C::kSepP) {
+            // the next S of each tile as soon as its softmax has read the current one
+            for (int x = 0; x < 2 && ok; ++x)
+              if (uses(w, x, j) && uses(w, x, j + 1) && issued[x] == j) ok = issue_qk(x, j + 1);
+          }
           if (!ok) break;
           if (!mbar_wait_bounded(&v_full[st], (g / NS) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
           const uint32_t vt = v_base + st * C::kTileBytes;
@@ -477,11 +499,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < kTile / 16; ++kk)
-              umma_ts(tmem + C::o_col(x), tmem + C::s_col(x) + kk * 8,
+              umma_ts(tmem + C::o_col(x), tmem + C::p_col(x) + kk * 8,
                       sdesc_sw128(vt + kk * 2048, kSub, 1024), idesc_pv, (npv[x] > 0 || kk > 0) ? 1u : 0u);
             ++npv[x];
+            if (C::kSepP) umma_commit(&pv_done[x]);
             if (j == last[x]) umma_commit(&o_full[x]);
-            else if (uses(w, x, j + 1)) ok = issue_qk(x, j + 1);
+            else if (!C::kSepP && uses(w, x, j + 1)) ok = issue_qk(x, j + 1);
           }
           umma_commit(&kv_empty[st]);
         }
@@ -497,7 +520,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const int row = tid & 127;                 // TMEM lane == row in the tile
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t s_addr = lane_base + C::s_col(x);
+    const uint32_t p_addr = lane_base + C::p_col(x);
     const uint32_t o_addr = lane_base + C::o_col(x);
+    int pw = 0;                                // P buffers written (separate-P layout)
     const float sl2 = p.scale_log2;
     int it = 0;                                // S/P tiles handled so far (barrier phase)
     int oc = 0;                                // units finished (o_full phase)
@@ -594,6 +619,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           tmem_ld32(s_addr + ch * 32, *reinterpret_cast<uint32_t(*)[32]>(xr + ch * 32));
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(xr + ch * 32));
+        if (C::kSepP) {
+          tc_fence_before();
+          mbar_arrive(&s_free[x]);             // the MMA warp may compute the next S now
+        }
         float s[kTile];
 #pragma unroll
         for (int e = 0; e < kTile; ++e) s[e] = __uint_as_float(xr[e]);
@@ -685,6 +714,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         const float neg_m = (m == -INFINITY) ? 0.f : -m;
         const float mul = raw ? sl2 : 1.f;
+        if (C::kSepP && pw > 0) {
+          // the previous PV has read P_x and updated O_x
+          if (!mbar_wait_bounded(&pv_done[x], (pw - 1) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+        }
         float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
         // P = 2^(t - m) as bf16, written back over the S columns 16 at a time (the
         // columns of chunk c only hold S values already read into registers)
@@ -711,12 +745,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             pk[q / 2] = pack_bf16x2(a0, a1);
             pk[q / 2 + 1] = pack_bf16x2(a2, a3);
           }
-          tmem_st16(s_addr + ch * 16, pk);
+          tmem_st16(p_addr + ch * 16, pk);
         }
         l += (acc0 + acc1) + (acc2 + acc3);
         if (rescale && iu > 0) {
-          // O_x is stable: its previous PV was issued before this S, and MMAs
-          // complete in order.
+          // O_x is stable: with P over S its previous PV was issued before this S
+          // and MMAs complete in order; with separate P the wait above saw it done.
 #pragma unroll
           for (int ch = 0; ch < D / 32; ++ch) {
             uint32_t rr[32];
@@ -730,6 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[x]);
+        ++pw;
         ++it;
         ++iu;
       }
