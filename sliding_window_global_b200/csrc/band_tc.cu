@@ -632,9 +632,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // Masked entries become -inf.
         float tmax;
         bool raw = false;
+        uint32_t live = 0xFu;                  // 32-column chunks with any allowed key in the warp
         if (j < w.nband) {
           const int kv0 = w.band_lo + j * kTile;
           const int lo_t = klo - kv0, hi_t = khi - kv0;
+          live = 0;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch)
+            if (__any_sync(0xffffffffu, lo_t < 32 * ch + 32 && hi_t > 32 * ch)) live |= 1u << ch;
           // boundary tiles: most cut only one side of the band (window start or
           // causal diagonal), which costs one compare and one select per score
           const bool cut_lo = __any_sync(0xffffffffu, lo_t > 0);
@@ -697,6 +702,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           if (!__all_sync(0xffffffffu, lim >= kTile)) {
 #pragma unroll
             for (int e = 0; e < kTile; ++e) s[e] = e < lim ? s[e] : -INFINITY;
+            live = 0;
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch)
+              if (__any_sync(0xffffffffu, 32 * ch < lim)) live |= 1u << ch;
           }
           tmax = row_max128(s);
         }
@@ -725,6 +734,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           uint32_t pk[16];
+          if (!(live & (1u << ch))) {
+            // every key of this chunk is masked for every row of the warp: P = 0
+#pragma unroll
+            for (int q = 0; q < 16; ++q) pk[q] = 0u;
+            tmem_st16(p_addr + ch * 16, pk);
+            continue;
+          }
 #pragma unroll
           for (int q = 0; q < 32; q += 4) {
             const int e = ch * 32 + q;

@@ -82,6 +82,13 @@ EDGE = [
     ("noncausal_d128", _small("swan_swa", causal=False, window=(200,) * 8)),
     ("batch3_tiny_n", _small("dilated", batch=3, seq_len=77, window=(9,) * 4, num_global=3)),
     ("n_one", _small("longformer_base", seq_len=1, padding=0, num_global=0, global_mode="none")),
+    # GQA head pairs on one KV head (a unit = the same rows of two heads)
+    ("pair_dilated_globals", _small("swan_swa", causal=False, window=(60,) * 8,
+                                    dilation=(1, 1, 2, 2, 3, 3, 1, 1), num_global=6,
+                                    global_mode="random", padding=41)),
+    ("pair_side_no_bias", _small("longt5_tglobal", q_heads=4, kv_heads=2, window=(127,) * 4,
+                                 dilation=(1,) * 4, side_bias=False)),
+    ("pair_d64_ragged", _small("swan_swa", head_dim=64, seq_len=333, window=(90,) * 8)),
     ("fp32_gqa_side", dataclasses.replace(workloads.SMALL["longt5_tglobal"], dtype="fp32",
                                           q_heads=4, kv_heads=2, window=(20,) * 4,
                                           dilation=(1, 2, 1, 2), seq_len=300)),
