@@ -76,7 +76,7 @@ struct Cfg {
   static constexpr uint32_t kVOff = kKOff + NS * kTileBytes;
   static constexpr uint32_t kBiasOff = kVOff + NS * kTileBytes;  // 4 shifted copies
   static constexpr uint32_t kBarOff = kBiasOff + 4 * kBiasCopy * 4;
-  static constexpr int kNumBars = 2 + 2 + 3 * NS + 2 + 2 + 2 + 2 + 2;
+  static constexpr int kNumBars = 2 + 2 + 3 * NS + 2 + 2 + 2 + 2 + 2 + 2;
   static constexpr uint32_t kSmemBytes = kBarOff + kNumBars * 8 + 1024;
   // TMEM columns.  D = 128: S_A | S_B | O_A | O_B, P written over S.  D = 64 has
   // room for separate P buffers (S_A | S_B | P_A | P_B | O_A | O_B), so the next
@@ -346,6 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   uint64_t* o_full = p_full + 2;          // [2]
   uint64_t* s_free = o_full + 2;          // [2] S read into registers (separate-P layout)
   uint64_t* pv_done = s_free + 2;         // [2] a PV finished: P buffer free, O updated
+  uint64_t* p_half = pv_done + 2;         // [2] P of keys 0-63 written (P-over-S layout)
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ int sGpos[2 * kTile];        // positions of the current global tile, per group
@@ -365,6 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_init(&o_full[x], 1);
       mbar_init(&s_free[x], kTile);
       mbar_init(&pv_done[x], 1);
+      mbar_init(&p_half[x], kTile);
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(&k_full[s], 1);
@@ -494,11 +496,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           const uint32_t vt = v_base + st * C::kTileBytes;
           for (int x = 0; x < 2 && ok; ++x) {
             if (!uses(w, x, j)) continue;
+            if (!C::kSepP) {
+              // P over S: the first half of P (keys 0-63) is published early, so the
+              // PV over it overlaps the exponentials of the second half
+              if (!mbar_wait_bounded(&p_half[x], pwaits[x] & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < kTile / 32; ++kk)
+                umma_ts(tmem + C::o_col(x), tmem + C::p_col(x) + kk * 8,
+                        sdesc_sw128(vt + kk * 2048, kSub, 1024), idesc_pv, (npv[x] > 0 || kk > 0) ? 1u : 0u);
+            }
             if (!mbar_wait_bounded(&p_full[x], pwaits[x] & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
             ++pwaits[x];
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < kTile / 16; ++kk)
+            for (int kk = C::kSepP ? 0 : kTile / 32; kk < kTile / 16; ++kk)
               umma_ts(tmem + C::o_col(x), tmem + C::p_col(x) + kk * 8,
                       sdesc_sw128(vt + kk * 2048, kSub, 1024), idesc_pv, (npv[x] > 0 || kk > 0) ? 1u : 0u);
             ++npv[x];
@@ -728,9 +740,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           if (!mbar_wait_bounded(&pv_done[x], (pw - 1) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
           tc_fence_after();
         }
+        if (!C::kSepP && rescale && iu > 0) {
+          // P over S: O_x must be rescaled before the first half of P is published.
+          // It is stable: its previous PV was issued before this S and MMAs complete
+          // in order.  (16 columns at a time: the scores are still live in registers.)
+#pragma unroll 1
+          for (int ch = 0; ch < D / 16; ++ch) {
+            uint32_t rr[16];
+            tmem_ld16(o_addr + ch * 16, rr);
+            tmem_wait_ld_dep16(rr);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
+            tmem_st16(o_addr + ch * 16, rr);
+          }
+        }
         float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-        // P = 2^(t - m) as bf16, written back over the S columns 16 at a time (the
-        // columns of chunk c only hold S values already read into registers)
+        // P = 2^(t - m) as bf16, written 16 columns at a time (over S: the columns of
+        // chunk c only hold S values already read into registers)
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           uint32_t pk[16];
@@ -738,35 +764,38 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             // every key of this chunk is masked for every row of the warp: P = 0
 #pragma unroll
             for (int q = 0; q < 16; ++q) pk[q] = 0u;
-            tmem_st16(p_addr + ch * 16, pk);
-            continue;
-          }
+          } else {
 #pragma unroll
-          for (int q = 0; q < 32; q += 4) {
-            const int e = ch * 32 + q;
-            float a0, a1, a2, a3;
-            ffma2(a0, a1, s[e], s[e + 1], mul, mul, neg_m, neg_m);
-            ffma2(a2, a3, s[e + 2], s[e + 3], mul, mul, neg_m, neg_m);
-            if (q < kEmuPer32) {
-              exp2_poly2(a0, a1, a0, a1);
-              exp2_poly2(a2, a3, a2, a3);
-            } else {
-              a0 = ex2_approx(a0);
-              a1 = ex2_approx(a1);
-              a2 = ex2_approx(a2);
-              a3 = ex2_approx(a3);
+            for (int q = 0; q < 32; q += 4) {
+              const int e = ch * 32 + q;
+              float a0, a1, a2, a3;
+              ffma2(a0, a1, s[e], s[e + 1], mul, mul, neg_m, neg_m);
+              ffma2(a2, a3, s[e + 2], s[e + 3], mul, mul, neg_m, neg_m);
+              if (q < kEmuPer32) {
+                exp2_poly2(a0, a1, a0, a1);
+                exp2_poly2(a2, a3, a2, a3);
+              } else {
+                a0 = ex2_approx(a0);
+                a1 = ex2_approx(a1);
+                a2 = ex2_approx(a2);
+                a3 = ex2_approx(a3);
+              }
+              fadd2(acc0, acc1, acc0, acc1, a0, a1);
+              fadd2(acc2, acc3, acc2, acc3, a2, a3);
+              pk[q / 2] = pack_bf16x2(a0, a1);
+              pk[q / 2 + 1] = pack_bf16x2(a2, a3);
             }
-            fadd2(acc0, acc1, acc0, acc1, a0, a1);
-            fadd2(acc2, acc3, acc2, acc3, a2, a3);
-            pk[q / 2] = pack_bf16x2(a0, a1);
-            pk[q / 2 + 1] = pack_bf16x2(a2, a3);
           }
           tmem_st16(p_addr + ch * 16, pk);
+          if (!C::kSepP && ch == 1) {
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&p_half[x]);
+          }
         }
         l += (acc0 + acc1) + (acc2 + acc3);
-        if (rescale && iu > 0) {
-          // O_x is stable: with P over S its previous PV was issued before this S
-          // and MMAs complete in order; with separate P the wait above saw it done.
+        if (C::kSepP && rescale && iu > 0) {
+          // separate P: the wait on the previous PV above saw O_x updated
 #pragma unroll
           for (int ch = 0; ch < D / 32; ++ch) {
             uint32_t rr[32];
