@@ -48,6 +48,10 @@ def _load():
             lib.oracle_dense_bruteforce.argtypes = [I, I, I, I, I, P, P, P, P, I, P, P, I, I, P, P,
                                                     P, I, P, D, P, P]
             lib.oracle_dense_bruteforce.restype = I
+            lib.oracle_forward_ex.argtypes = lib.oracle_forward.argtypes + [P, I]
+            lib.oracle_forward_ex.restype = I
+            lib.oracle_dense_bruteforce_ex.argtypes = lib.oracle_dense_bruteforce.argtypes + [P, I]
+            lib.oracle_dense_bruteforce_ex.restype = I
             lib.oracle_key_counts.argtypes = [I, I, I, P, I, I, P, P, I, P, P]
             lib.oracle_key_counts.restype = I
             lib.oracle_key_list.argtypes = [I, I, I, P, I, P, P, I, P, I, I, I, P]
@@ -101,7 +105,10 @@ class Problem:
     """One attention problem, widened to fp32 host arrays (exact for bf16/fp32)."""
 
     def __init__(self, q, k, v, *, window, dilation=1, causal=False, global_idx=None,
-                 side_k=None, side_v=None, side_block=16, bias=None, valid_len=None, scale=None):
+                 side_k=None, side_v=None, side_block=16, bias=None, valid_len=None, scale=None,
+                 local_bias=None):
+        """``local_bias``: optional [Hq, 2R+1] table added to window keys of non-global
+        rows at column (j - i) + R (R inferred from the table width)."""
         self.q, self.k, self.v = _f32(q), _f32(k), _f32(v)
         self.B, self.Hq, self.n, self.D = self.q.shape
         self.Hkv = self.k.shape[1]
@@ -118,6 +125,13 @@ class Problem:
         self.bias = _f32(bias)
         self.valid_len = _i32(valid_len)
         self.scale = float(scale) if scale is not None else 1.0 / np.sqrt(self.D)
+        self.local_bias = _f32(local_bias)
+        self.local_radius = 0
+        if self.local_bias is not None:
+            width = self.local_bias.shape[-1]
+            if self.local_bias.shape != (self.Hq, width) or width % 2 == 0:
+                raise ValueError("local_bias must be [Hq, 2R+1]")
+            self.local_radius = (width - 1) // 2
 
     def _common(self):
         return (self.B, self.Hq, self.Hkv, self.n, self.D, _ptr(self.q), _ptr(self.k), _ptr(self.v),
@@ -142,8 +156,8 @@ class Problem:
         out = np.empty((total, self.D), dtype=np.float64)
         lse = np.empty(total, dtype=np.float64)
         cnt = np.empty(total, dtype=np.int64)
-        _check(lib.oracle_forward(*self._common(), rp, total, _ptr(out), _ptr(lse), _ptr(cnt)),
-               "forward")
+        _check(lib.oracle_forward_ex(*self._common(), rp, total, _ptr(out), _ptr(lse), _ptr(cnt),
+                                     _ptr(self.local_bias), self.local_radius), "forward")
         if rows is None:
             return (out.reshape(self.B, self.Hq, self.n, self.D), lse.reshape(self.B, self.Hq, self.n),
                     cnt.reshape(self.B, self.Hq, self.n))
@@ -153,7 +167,8 @@ class Problem:
         lib = _load()
         out = np.empty((self.B, self.Hq, self.n, self.D), dtype=np.float64)
         lse = np.empty((self.B, self.Hq, self.n), dtype=np.float64)
-        _check(lib.oracle_dense_bruteforce(*self._common(), _ptr(out), _ptr(lse)), "dense")
+        _check(lib.oracle_dense_bruteforce_ex(*self._common(), _ptr(out), _ptr(lse),
+                                              _ptr(self.local_bias), self.local_radius), "dense")
         return out, lse
 
 

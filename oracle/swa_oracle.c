@@ -31,6 +31,9 @@
  *               section "LongT5Config 参数全解": num_buckets 32, max_distance 128.
  *   [SWAN-3.3]  "SWAN-GPT：无需长文本训练" §3.3(1): decoder SWA-RoPE layers with
  *               a fixed 512-token causal window.
+ *   [LT5-LOCAL] LongT5 guide, "相对位置编码" section: the local attention adds a
+ *               relative-position bias bucketed on memory_position -
+ *               query_position, computed once over the local window.
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *   window bounds inclusive (2r+1 keys, non-causal); causal window t in [-r,0];
@@ -69,6 +72,8 @@ typedef struct {
     int causal;
     const int32_t *valid_len;
     double scale;
+    const float *local_bias;   /* [Hq, 2R+1] or NULL: bias of window keys by j - i */
+    int local_radius;          /* R */
 } oracle_problem;
 
 static int num_blocks(int n, int kb) { return kb > 0 ? (n + kb - 1) / kb : 0; }
@@ -134,6 +139,25 @@ static double side_bias(const oracle_problem *P, int h, int i, int s) {
     return (double)P->bias[(int64_t)h * cols + delta + nblk - 1];
 }
 
+/*
+ * Local relative-position bias of a window key [LT5-LOCAL]: added to s_ij when j
+ * is in the window W(i) of a non-global query, read from column (j - i) + R of
+ * the head's table.  Global query rows and global / side keys get none.
+ */
+static int in_window(const oracle_problem *P, int h, int i, int j) {
+    int64_t diff = (int64_t)i - j;
+    int64_t rd = (int64_t)P->window[h] * P->dilation[h];
+    int band = P->causal ? (diff >= 0 && diff <= rd) : (diff >= -rd && diff <= rd);
+    return band && (diff % P->dilation[h] == 0);
+}
+
+static double local_bias(const oracle_problem *P, int b, int h, int i, int j) {
+    if (!P->local_bias) return 0.0;
+    if (P->g > 0 && is_global(P, b, i)) return 0.0;
+    if (!in_window(P, h, i, j)) return 0.0;
+    return (double)P->local_bias[(int64_t)h * (2 * P->local_radius + 1) + (j - i) + P->local_radius];
+}
+
 static double dot(const float *a, const float *b, int D) {
     double acc = 0.0;
     for (int x = 0; x < D; ++x) acc += (double)a[x] * (double)b[x];
@@ -166,7 +190,7 @@ static void attend_row(const oracle_problem *P, int b, int h, int i,
     }
     double m = -INFINITY;
     for (int t = 0; t < nk; ++t) {
-        scores[t] = P->scale * dot(qi, kb + (int64_t)keys[t] * D, D);
+        scores[t] = P->scale * dot(qi, kb + (int64_t)keys[t] * D, D) + local_bias(P, b, h, i, keys[t]);
         if (scores[t] > m) m = scores[t];
     }
     for (int s = 0; s < S; ++s) {
@@ -203,6 +227,14 @@ static int check_problem(const oracle_problem *P) {
     if (P->S < 0 || (P->S > 0 && (!P->side_k || !P->side_v || P->side_block <= 0))) return ORACLE_EINVAL;
     for (int h = 0; h < P->Hq; ++h)
         if (P->window[h] < 0 || P->dilation[h] < 1) return ORACLE_EINVAL;
+    if (P->local_bias) {
+        /* the table must cover every offset j - i a window key can take */
+        for (int h = 0; h < P->Hq; ++h) {
+            int64_t reach = (int64_t)P->window[h] * P->dilation[h];
+            if (reach > P->n - 1) reach = P->n - 1;
+            if (P->local_radius < reach) return ORACLE_EINVAL;
+        }
+    }
     return ORACLE_OK;
 }
 
@@ -211,14 +243,16 @@ static int check_problem(const oracle_problem *P) {
  * means every row in that order) write o (fp64, D values), lse and
  * count = |K(i)| + (number of side keys attended) -- the attended pairs.
  */
-int oracle_forward(int B, int Hq, int Hkv, int n, int D, const float *q, const float *k,
-                   const float *v, const int32_t *global_idx, int g, const float *side_k,
-                   const float *side_v, int S, int side_block, const float *bias,
-                   const int32_t *window, const int32_t *dilation, int causal,
-                   const int32_t *valid_len, double scale, const int64_t *rows,
-                   int64_t nrows, double *out, double *lse, int64_t *count) {
+int oracle_forward_ex(int B, int Hq, int Hkv, int n, int D, const float *q, const float *k,
+                      const float *v, const int32_t *global_idx, int g, const float *side_k,
+                      const float *side_v, int S, int side_block, const float *bias,
+                      const int32_t *window, const int32_t *dilation, int causal,
+                      const int32_t *valid_len, double scale, const int64_t *rows,
+                      int64_t nrows, double *out, double *lse, int64_t *count,
+                      const float *local_bias_tab, int local_radius) {
     oracle_problem P = {B, Hq, Hkv, n, D, q, k, v, global_idx, g, side_k, side_v,
-                        S, side_block, bias, window, dilation, causal, valid_len, scale};
+                        S, side_block, bias, window, dilation, causal, valid_len, scale,
+                        local_bias_tab, local_radius};
     int rc = check_problem(&P);
     if (rc) return rc;
     int64_t total = rows ? nrows : (int64_t)B * Hq * n;
@@ -249,6 +283,17 @@ int oracle_forward(int B, int Hq, int Hkv, int n, int D, const float *q, const f
         free(scores);
     }
     return failed ? ORACLE_ENOMEM : ORACLE_OK;
+}
+
+int oracle_forward(int B, int Hq, int Hkv, int n, int D, const float *q, const float *k,
+                   const float *v, const int32_t *global_idx, int g, const float *side_k,
+                   const float *side_v, int S, int side_block, const float *bias,
+                   const int32_t *window, const int32_t *dilation, int causal,
+                   const int32_t *valid_len, double scale, const int64_t *rows,
+                   int64_t nrows, double *out, double *lse, int64_t *count) {
+    return oracle_forward_ex(B, Hq, Hkv, n, D, q, k, v, global_idx, g, side_k, side_v, S, side_block,
+                             bias, window, dilation, causal, valid_len, scale, rows, nrows, out, lse,
+                             count, NULL, 0);
 }
 
 /*
@@ -315,21 +360,29 @@ int oracle_key_list(int B, int Hq, int n, const int32_t *global_idx, int g,
  * appends every side column for valid rows, and runs a dense masked softmax
  * over all n + S columns.  Every row is written (flat order).
  */
-int oracle_dense_bruteforce(int B, int Hq, int Hkv, int n, int D, const float *q,
-                            const float *k, const float *v, const int32_t *global_idx, int g,
-                            const float *side_k, const float *side_v, int S, int side_block,
-                            const float *bias, const int32_t *window, const int32_t *dilation,
-                            int causal, const int32_t *valid_len, double scale, double *out,
-                            double *lse) {
+int oracle_dense_bruteforce_ex(int B, int Hq, int Hkv, int n, int D, const float *q,
+                               const float *k, const float *v, const int32_t *global_idx, int g,
+                               const float *side_k, const float *side_v, int S, int side_block,
+                               const float *bias, const int32_t *window, const int32_t *dilation,
+                               int causal, const int32_t *valid_len, double scale, double *out,
+                               double *lse, const float *local_bias_tab, int local_radius) {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || n < 0) return ORACLE_EINVAL;
+    if (local_bias_tab) {
+        for (int h = 0; h < Hq; ++h) {
+            int64_t reach = (int64_t)window[h] * dilation[h];
+            if (reach > n - 1) reach = n - 1;
+            if (local_radius < reach) return ORACLE_EINVAL;
+        }
+    }
     int G = Hq / Hkv;
     int nblk = side_block > 0 ? (n + side_block - 1) / side_block : 0;
     int cols = n + S;
     unsigned char *isg = (unsigned char *)calloc((size_t)n + 1, 1);
     unsigned char *allow = (unsigned char *)malloc((size_t)cols + 1);
+    unsigned char *inband = (unsigned char *)malloc((size_t)n + 1);
     double *s = (double *)malloc(sizeof(double) * ((size_t)cols + 1));
-    if (!isg || !allow || !s) {
-        free(isg); free(allow); free(s);
+    if (!isg || !allow || !s || !inband) {
+        free(isg); free(allow); free(s); free(inband);
         return ORACLE_ENOMEM;
     }
     for (int b = 0; b < B; ++b) {
@@ -348,6 +401,7 @@ int oracle_dense_bruteforce(int B, int Hq, int Hkv, int n, int D, const float *q
                     int band = causal ? (diff >= 0 && diff <= rd) : (llabs(diff) <= rd);
                     band = band && (diff % dilation[h] == 0);
                     int a = (band || isg[j] || isg[i]) && i < V && j < V;
+                    inband[j] = (unsigned char)(band && !isg[i]);
                     allow[j] = (unsigned char)a;
                     any |= a;
                 }
@@ -369,6 +423,8 @@ int oracle_dense_bruteforce(int B, int Hq, int Hkv, int n, int D, const float *q
                     double acc = 0.0;
                     for (int x = 0; x < D; ++x) acc += (double)qi[x] * (double)kk[x];
                     acc *= scale;
+                    if (c < n && local_bias_tab && inband[c])
+                        acc += (double)local_bias_tab[(int64_t)h * (2 * local_radius + 1) + (c - i) + local_radius];
                     if (c >= n && bias) {
                         int delta = (c - n) - i / side_block;
                         acc += (double)bias[(int64_t)h * (S + nblk - 1) + delta + nblk - 1];
@@ -395,7 +451,19 @@ int oracle_dense_bruteforce(int B, int Hq, int Hkv, int n, int D, const float *q
     free(isg);
     free(allow);
     free(s);
+    free(inband);
     return ORACLE_OK;
+}
+
+int oracle_dense_bruteforce(int B, int Hq, int Hkv, int n, int D, const float *q,
+                            const float *k, const float *v, const int32_t *global_idx, int g,
+                            const float *side_k, const float *side_v, int S, int side_block,
+                            const float *bias, const int32_t *window, const int32_t *dilation,
+                            int causal, const int32_t *valid_len, double scale, double *out,
+                            double *lse) {
+    return oracle_dense_bruteforce_ex(B, Hq, Hkv, n, D, q, k, v, global_idx, g, side_k, side_v, S,
+                                      side_block, bias, window, dilation, causal, valid_len, scale,
+                                      out, lse, NULL, 0);
 }
 
 /*

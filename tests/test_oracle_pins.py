@@ -317,3 +317,105 @@ def test_side_aggregate_block_means(oracle_mod):
     assert out.shape == (1, 1, 4, 2)
     assert out[0, 0, 0, 0] == 7.5
     assert out[0, 0, 3, 0] == np.mean(np.arange(48, 60))
+
+
+# --- local relative-position bias on window keys (LongT5 guide, 相对位置编码) ----------
+
+
+def _local_table(rng, Hq, R):
+    return _rand((Hq, 2 * R + 1), rng)
+
+
+def test_local_bias_matches_dense_bruteforce_grid(oracle_mod):
+    """The per-row path (bias looked up per key of K(i)) against the dense-mask brute
+    force (bias added on the band mask of non-global rows), globals, sides, dilation,
+    causal and padding included."""
+    rng = np.random.default_rng(41)
+    cases = 0
+    for n in (3, 8, 21, 40):
+        for r, d, causal, g, pad in itertools.product((0, 1, 3), (1, 2), (0, 1), (0, 2), (0, 3)):
+            if rng.random() > 0.5:
+                continue
+            S = int(rng.integers(0, 2)) * 3
+            p = _problem(oracle_mod, rng, 2, 4, 2, n, 8, r, d, causal, g, pad, S=S, kb=4, bias=bool(S))
+            R = min(r * d, n - 1) + int(rng.integers(0, 3))
+            lt = _local_table(rng, 4, R)
+            pb = oracle_mod.Problem(p.q, p.k, p.v, window=r, dilation=d, causal=causal,
+                                    global_idx=p.global_idx, side_k=p.side_k, side_v=p.side_v,
+                                    side_block=4, bias=p.bias, valid_len=p.valid_len, local_bias=lt)
+            o, lse, _ = pb.forward()
+            od, lsed = pb.dense_bruteforce()
+            assert np.max(np.abs(o - od)) <= 1e-12
+            _assert_close_lse(lse, lsed, 1e-12)
+            cases += 1
+    assert cases > 30
+
+
+def test_constant_local_bias_is_a_softmax_shift(oracle_mod):
+    """With no global or side keys every key is a window key, so a per-head constant
+    bias c shifts all scores: o is unchanged and lse moves by exactly c."""
+    rng = np.random.default_rng(43)
+    p = _problem(oracle_mod, rng, 2, 3, 3, 37, 16, 4, 2, 0, 0, 5)
+    c = np.array([0.5, -2.0, 3.25], np.float32)
+    lt = np.repeat(c[:, None], 2 * 8 + 1, axis=1)
+    pb = oracle_mod.Problem(p.q, p.k, p.v, window=4, dilation=2, valid_len=p.valid_len, local_bias=lt)
+    o0, l0, _ = p.forward()
+    o1, l1, _ = pb.forward()
+    assert np.max(np.abs(o0 - o1)) <= 1e-12
+    m = ~np.isneginf(l0)
+    assert np.max(np.abs((l1 - l0)[m] - np.broadcast_to(c[None, :, None], l0.shape)[m])) <= 1e-12
+
+
+def test_local_bias_offset_sign_closed_form(oracle_mod):
+    """q = 0 and bias = alpha * (j - i): the weight of window key j is
+    exp(alpha (j - i)) / sum over the window -- a closed form that fails if the
+    table is read at (i - j) or off by one."""
+    n, r, d, alpha = 30, 3, 2, 0.75   # alpha * integer is exact in fp32
+    R = r * d
+    q = np.zeros((1, 1, n, n), np.float32)
+    k = np.ones((1, 1, n, n), np.float32)
+    v = np.eye(n, dtype=np.float32)[None, None]
+    lt = (alpha * (np.arange(2 * R + 1) - R)).astype(np.float32)[None]
+    o, _, _ = oracle_mod.Problem(q, k, v, window=r, dilation=d, local_bias=lt).forward()
+    for i in range(n):
+        js = [i + d * t for t in range(-r, r + 1) if 0 <= i + d * t < n]
+        w = np.exp(alpha * (np.array(js) - i))
+        expect = np.zeros(n)
+        expect[js] = w / w.sum()
+        assert np.max(np.abs(o[0, 0, i] - expect)) <= 1e-14
+
+
+def test_local_bias_skips_global_rows_and_out_of_window_global_keys(oracle_mod):
+    """Table = -1e30 except offset 0: a non-global row keeps itself and the global
+    keys outside its window (a global key inside the window is a window key and is
+    suppressed too); a global row keeps plain full attention."""
+    rng = np.random.default_rng(47)
+    n, D, r = 40, 8, 3
+    q, k, v = _rand((1, 1, n, D), rng), _rand((1, 1, n, D), rng), _rand((1, 1, n, D), rng)
+    gi = np.array([[2, 5, 30]], np.int32)
+    lt = np.full((1, 2 * r + 1), -1e30, np.float32)
+    lt[0, r] = 0.0
+    o, lse, _ = oracle_mod.Problem(q, k, v, window=r, global_idx=gi, local_bias=lt).forward()
+    qd, kd, vd = (x[0, 0].astype(np.float64) for x in (q, k, v))
+    for i in range(n):
+        if i in gi[0]:
+            keys = list(range(n))
+        else:
+            keys = [i] + [j for j in gi[0] if abs(j - i) > r]
+        s = qd[i] @ kd[keys].T / np.sqrt(D)
+        m = s.max()
+        w = np.exp(s - m)
+        assert np.max(np.abs(o[0, 0, i] - (w @ vd[keys]) / w.sum())) <= 1e-12
+        assert abs(lse[0, 0, i] - (m + np.log(w.sum()))) <= 1e-12
+
+
+def test_local_bias_table_must_cover_the_window(oracle_mod):
+    rng = np.random.default_rng(49)
+    p = _problem(oracle_mod, rng, 1, 1, 1, 20, 4, 3, 2, 0, 0, 0)
+    short = oracle_mod.Problem(p.q, p.k, p.v, window=3, dilation=2, local_bias=_local_table(rng, 1, 5))
+    with pytest.raises(RuntimeError):
+        short.forward()
+    # a radius past n - 1 is never needed
+    big = oracle_mod.Problem(p.q[:, :, :4], p.k[:, :, :4], p.v[:, :, :4], window=50,
+                             local_bias=_local_table(rng, 1, 3))
+    big.forward()
