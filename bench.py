@@ -147,10 +147,11 @@ def replica_throughput(flop_per_rank: float, world: int, ms_max: float) -> float
 
 def prepare(w, device):
     """Device-resident inputs of one workload, built with the library's own kernels
-    (side keys: block means on the device; side bias: host bucket expansion)."""
+    (side keys: block means on the device; side and local bias: host bucket
+    expansion)."""
     import torch
 
-    from sliding_window_global_b200 import expand_side_bias, side_aggregate, workloads
+    from sliding_window_global_b200 import bucket_local_bias, expand_side_bias, side_aggregate, workloads
     inp = workloads.make_inputs(w)
     host = {k: v for k, v in inp.items()}
     dev = {}
@@ -163,8 +164,16 @@ def prepare(w, device):
             nblk = (w.seq_len + w.side_block - 1) // w.side_block
             host["bias"] = expand_side_bias(inp["bias_table"], w.num_side, nblk)
             dev["bias"] = host["bias"].to(device)
+    if inp.get("local_table") is not None:
+        host["local_bias"] = bucket_local_bias(inp["local_table"], local_radius(w))
+        dev["local_bias"] = host["local_bias"].to(device)
     torch.cuda.synchronize()
     return host, dev
+
+
+def local_radius(w) -> int:
+    """Radius of the local-bias table: the largest window offset, max min(r*d, n-1)."""
+    return max(min(r * d, w.seq_len - 1) for r, d in zip(w.window, w.dilation))
 
 
 def count_flops(w, host):
@@ -182,7 +191,7 @@ def time_device(w, plan, dev, steps, warmup, device):
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
     kw = dict(window=list(w.window), dilation=list(w.dilation), causal=w.causal,
               global_idx=dev["global_idx"], side_k=dev.get("side_k"), side_v=dev.get("side_v"),
-              bias=dev.get("bias"), valid_len=dev["valid_len"])
+              bias=dev.get("bias"), valid_len=dev["valid_len"], local_bias=dev.get("local_bias"))
     out = torch.empty((w.batch, w.q_heads, w.seq_len, w.head_dim), dtype=w.torch_dtype, device=device)
     lse = torch.empty((w.batch, w.q_heads, w.seq_len), dtype=torch.float32, device=device)
     for _ in range(warmup):
@@ -214,7 +223,8 @@ def time_e2e(w, plan, host, steps, warmup, device):
     import torch
 
     from sliding_window_global_b200 import side_aggregate
-    names = [k for k in ("q", "k", "v", "global_idx", "valid_len", "bias") if host.get(k) is not None]
+    names = [k for k in ("q", "k", "v", "global_idx", "valid_len", "bias", "local_bias")
+             if host.get(k) is not None]
     pinned = {k: host[k].contiguous().pin_memory() for k in names}
     dev = {k: torch.empty_like(pinned[k], device=device) for k in names}
     out_h = torch.empty((w.batch, w.q_heads, w.seq_len, w.head_dim), dtype=w.torch_dtype).pin_memory()
@@ -232,7 +242,8 @@ def time_e2e(w, plan, host, steps, warmup, device):
         out, lse = plan.forward(dev["q"], dev["k"], dev["v"], window=list(w.window),
                                 dilation=list(w.dilation), causal=w.causal,
                                 global_idx=dev.get("global_idx"), side_k=sk, side_v=sv,
-                                bias=dev.get("bias"), valid_len=dev.get("valid_len"))
+                                bias=dev.get("bias"), valid_len=dev.get("valid_len"),
+                                local_bias=dev.get("local_bias"))
         out_h.copy_(out, non_blocking=True)
         lse_h.copy_(lse, non_blocking=True)
 
@@ -260,11 +271,14 @@ def cpu_baseline(w, host, budget_s=12.0):
     if w.side_block:   # the oracle makes its own side keys from the same k/v
         inp["side_k"] = torch.from_numpy(oracle.side_aggregate(host["k"], w.side_block, host["valid_len"]))
         inp["side_v"] = torch.from_numpy(oracle.side_aggregate(host["v"], w.side_block, host["valid_len"]))
+    if host.get("local_table") is not None:
+        inp["local_bias"] = oracle.expand_local_bias(host["local_table"], local_radius(w))
     prob = oracle.Problem(inp["q"], inp["k"], inp["v"], window=np.array(w.window),
                           dilation=np.array(w.dilation), causal=w.causal,
                           global_idx=inp["global_idx"], side_k=inp.get("side_k"),
                           side_v=inp.get("side_v"), side_block=w.side_block or 16,
-                          bias=inp.get("bias"), valid_len=inp["valid_len"], scale=inp["scale"])
+                          bias=inp.get("bias"), valid_len=inp["valid_len"], scale=inp["scale"],
+                          local_bias=inp.get("local_bias"))
     rng = np.random.default_rng(0)
     total_rows = w.batch * w.q_heads * w.seq_len
     rows = np.sort(rng.choice(total_rows, min(total_rows, 2000), replace=False))
@@ -333,9 +347,10 @@ def run_ours(args):
         return res
 
     main = one(args.workload, True)
-    sec = None
-    if args.secondary and args.secondary != "none" and args.secondary != args.workload:
-        sec = one(args.secondary, False)
+    secs = []
+    for name in (args.secondary or "").split(","):
+        if name and name != "none" and name != args.workload:
+            secs.append(one(name, False))
     if rank == 0:
         w = main.pop("w")
         line = {
@@ -356,13 +371,16 @@ def run_ours(args):
         }
         if "cpu_baseline" in main:
             line["cpu_baseline"] = main["cpu_baseline"]
-        if sec is not None:
-            sw = sec.pop("w")
-            line["secondary"] = {"workload": sw.name, "value": sec["value"], "unit": "TFLOP/s",
-                                 "ms_per_step": sec["ms_per_step"],
-                                 "frac_of_peak": sec["value"] / world / peaks["bf16_tflops"],
-                                 "useful_gflop_per_step": sec["useful_gflop_per_step"],
-                                 "gpu_launches": sec["gpu_launches"], "clocks": sec["clocks"]}
+        if secs:
+            line["secondary"] = []
+            for sec in secs:
+                sw = sec.pop("w")
+                line["secondary"].append({
+                    "workload": sw.name, "value": sec["value"], "unit": "TFLOP/s",
+                    "ms_per_step": sec["ms_per_step"],
+                    "frac_of_peak": sec["value"] / world / peaks["bf16_tflops"],
+                    "useful_gflop_per_step": sec["useful_gflop_per_step"],
+                    "gpu_launches": sec["gpu_launches"], "clocks": sec["clocks"]})
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
@@ -414,7 +432,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="swan_swa")
-    ap.add_argument("--secondary", default="longt5_tglobal")
+    ap.add_argument("--secondary", default="longt5_tglobal,longt5_local",
+                    help="comma-separated workloads timed after the main one (device time only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

@@ -110,6 +110,50 @@ swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void
                        const int32_t* dilation, int causal, const int32_t* valid_len, void* out,
                        float* lse, void* stream);
 
+/* Arguments of swa_forward_ex: those of swa_forward, plus optional terms of the
+ * score that swa_forward does not take.  Zero-initialise the struct (fields may
+ * be appended in later versions; a zero field keeps its swa_forward meaning).
+ *
+ * local_bias: LongT5 local attention relative-position bias ("LongT5 长序列模型完全指南",
+ *   相对位置编码 section: a bias bucketed on memory_position - query_position,
+ *   computed once over the local window).  Device [Hq, 2*local_radius + 1] fp32,
+ *   4-byte aligned, or NULL.  For a query i that is not a global token and a key
+ *   j of its window W(i), local_bias[h][(j - i) + local_radius] is added to the
+ *   score (natural-log units, like bias).  Global query rows, global keys outside
+ *   W(i) and side keys get none; a global key inside W(i) is a window key.
+ *   local_radius must be >= min(window[h] * dilation[h], seq_len - 1) for every
+ *   head (else SWA_ERR_INVALID_ARG).  The bf16 kernels stage the bias rows of a
+ *   work unit in shared memory, which limits min(window[h], ceil(seq_len /
+ *   dilation[h])) to 766; larger windows with a local bias return
+ *   SWA_ERR_UNSUPPORTED.  Use swa_bucket_local_bias to expand a 32-bucket table. */
+typedef struct {
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* global_idx;
+  int num_global;
+  const void* side_k;
+  const void* side_v;
+  const float* bias;
+  const int32_t* window;       /* HOST */
+  const int32_t* dilation;     /* HOST */
+  int causal;
+  const int32_t* valid_len;
+  void* out;
+  float* lse;
+  const float* local_bias;     /* device [Hq, 2 * local_radius + 1] fp32, or NULL */
+  int local_radius;
+} swa_forward_args;
+
+/* swa_forward with the arguments in a struct (same statuses, same launches). */
+swa_status swa_forward_ex(swa_plan_t plan, const swa_forward_args* args, void* stream);
+
+/* Host helper: expand a per-head 32-bucket table [Hq][32] into the local-bias
+ * table [Hq][2R + 1] that swa_forward_ex reads, column c holding the T5
+ * bidirectional bucket of delta = c - R (memory position minus query position;
+ * the bucket function of swa_relative_bucket).  Host pointers. */
+swa_status swa_bucket_local_bias(int num_q_heads, int radius, const float* table, float* out);
+
 /* Synchronise `stream` and read (then clear) the plan's device error word:
  * SWA_ERR_TIMEOUT if a bounded wait expired in any kernel since the last check,
  * SWA_ERR_DEVICE_CHECK if a precondition check failed, SWA_ERR_CUDA if the

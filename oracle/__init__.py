@@ -215,6 +215,15 @@ def expand_side_bias(table, S: int, nblk: int):
     return out
 
 
+def expand_local_bias(table, radius: int):
+    """[Hq,32] bucket table -> [Hq, 2*radius + 1] fp32 local-bias table: column c
+    holds the T5 bucket of the token offset c - radius (memory minus query
+    position; LongT5 guide, 相对位置编码 section)."""
+    t = _f32(table)
+    cols = [relative_bucket(c - radius) for c in range(2 * radius + 1)]
+    return np.ascontiguousarray(t[:, cols], dtype=np.float32)
+
+
 def side_aggregate(x, block: int, valid_len=None):
     """Block means [B,H,n,D] -> [B,H,n//block,D] (fp64)."""
     a = _f32(x)

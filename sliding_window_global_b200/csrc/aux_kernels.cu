@@ -154,6 +154,9 @@ __global__ void simt_attn_kernel(AttnParams p, const T* __restrict__ q, const T*
       int j = is_global ? idx : i + d * (t_lo + idx);
       krow = kb + (size_t)j * D;
       vrow = vb + (size_t)j * D;
+      // local relative-position bias of window keys (offset j - i), non-global rows only
+      if (!is_global && p.local_bias)
+        bb = p.local_bias[(size_t)h * (2 * p.local_radius + 1) + p.local_radius + (j - i)];
     } else if (idx < nwin + ngl) {
       int j = gl[idx - nwin];
       int diff = i - j;

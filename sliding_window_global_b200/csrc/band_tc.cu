@@ -13,6 +13,9 @@
 //   side tiles   -- appended side keys with the additive bucketed bias of the
 //                   LongT5 Transient-Global attention ("LongT5 长序列模型完全指南",
 //                   Transient-Global and 源码级证据 sections).
+// Band tiles may carry a local relative-position bias indexed by key - query
+// offset (the LongT5 page, 相对位置编码: the local attention's bias is computed
+// once over the window); its row for the unit's head is staged in shared memory.
 // With dilation d a query at position c + d*u only meets keys c + d*u', so each
 // residue class is a plain band of radius r over rows c, c+d, ..., loaded through
 // strided TMA tensor maps.
@@ -30,7 +33,8 @@
 // warpgroups with setmaxnreg):
 //   warps 0-3   softmax of tile A, warps 4-7 softmax of tile B: thread t of the
 //               group owns query row t (TMEM lane t).  Per key tile: load S from
-//               TMEM, mask (boundary tiles only), scale, add bias (side tiles),
+//               TMEM, mask (boundary tiles only), scale, add bias (side tiles;
+//               band tiles with a local bias),
 //               running max m / sum l with a lazy O rescale (only when the max
 //               grows by more than 2^8), exponentiate -- part of the elements on
 //               the MUFU unit, part with a polynomial on the FMA pipe -- and write
@@ -58,7 +62,6 @@ constexpr uint32_t kSub = 128 * 128;          // one 128-row x 128-byte swizzle 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
-constexpr int kBiasCopy = 2048;               // floats per shifted copy of the side-bias segment
 
 #ifndef SWA_EMU_PER32
 #define SWA_EMU_PER32 8
@@ -356,6 +359,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const int lane = tid & 31;
   const int nunits = total_units<MODE>(p);
   const bool has_bias = p.bias && p.S > 0;
+  const bool has_local = MODE == 0 && p.local_bias != nullptr;
+  // shared bias area: 4 copies of the local-bias row (stride lstride floats), then
+  // 4 copies of the side-bias segment (stride side_stride)
+  const int lstride = has_local ? p.local_stride : 0;
+  const int side_stride = kBiasCopy - lstride;
+  float* sLocal = sBias;
+  float* sSide = sBias + 4 * lstride;
 
   if (tid == 0) {
     for (int x = 0; x < 2; ++x) {
@@ -555,8 +565,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       if (MODE == 0) pos = w.c + w.d * u;
       else if (row_valid) pos = p.global_idx[(size_t)w.b * p.g + w.u0[0] + row];
 
-      // side bias for this unit: four copies shifted by 0..3 floats so that every
-      // row can read 16-byte aligned vectors (both groups stage together)
+      // Bias rows of this unit, four copies shifted by 0..3 floats so that every
+      // row can read 16-byte aligned vectors (both groups stage together).
+      // Local bias: v[t + r_eff + kLocalPad] = bias of key offset d*t (class
+      // coordinates t), zero outside |t| <= r; band tiles read 128 consecutive
+      // entries starting anywhere in [-r_eff - 254, r_eff + 127] (r_eff = min(r, n_c)).
+      const int r_eff = min(w.r, p.cls[w.cls].n_c);
       int qblk_hi = 0;
       bool bias_staged = false;
       if (has_bias) {
@@ -571,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         qblk_hi = pos_hi / p.side_block;
         const int bias_len = p.S + (qblk_hi - pos_lo / p.side_block);
-        bias_staged = bias_len + 4 <= kBiasCopy;
+        bias_staged = bias_len + 4 <= side_stride;
         if (bias_staged) {
           named_barrier_sync(3, kSoftmaxThreads);     // both groups are done with the old segment
           const float* src = p.bias + (size_t)w.h * (p.S + p.nblk - 1) + (p.nblk - 1 - qblk_hi);
@@ -591,12 +605,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               if (idx < len) {
 #pragma unroll
                 for (int t = 0; t < 4; ++t)
-                  if (idx - t >= 0) sBias[t * kBiasCopy + idx - t] = v[q];
+                  if (idx - t >= 0) sSide[t * side_stride + idx - t] = v[q];
               }
             }
           }
-          named_barrier_sync(3, kSoftmaxThreads);
+          if (!has_local) named_barrier_sync(3, kSoftmaxThreads);
         }
+      }
+      if (has_local) {
+        if (!bias_staged) named_barrier_sync(3, kSoftmaxThreads);   // old rows are no longer read
+        const int R = p.local_radius;
+        const float* tab = p.local_bias + (size_t)w.h * (2 * R + 1) + R;
+        const int len = min((2 * r_eff + 2 * kLocalPad + 8) & ~3, lstride);
+        for (int idx = tid; idx < len; idx += kSoftmaxThreads) {
+          const int t = idx - r_eff - kLocalPad;
+          const long long off = (long long)w.d * t;
+          const bool in = t >= -w.r && t <= w.r && off >= -R && off <= R;
+          const float val = in ? __ldg(tab + off) * kLog2e : 0.f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            if (idx - c >= 0) sLocal[c * lstride + idx - c] = val;
+        }
+        named_barrier_sync(3, kSoftmaxThreads);
       }
       if (!w.active[x]) {
         if (MODE == 0) write_zero_row<D>(p, w, x, row);
@@ -648,6 +678,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         if (j < w.nband) {
           const int kv0 = w.band_lo + j * kTile;
           const int lo_t = klo - kv0, hi_t = khi - kv0;
+          if (has_local) {
+            // s * scale + bias, in log2 units (entries outside the window are masked below)
+            const int b0 = kv0 - u + r_eff + kLocalPad;
+            const float* cp = sLocal + (b0 & 3) * lstride + (b0 & ~3);
+#pragma unroll
+            for (int e = 0; e < kTile; e += 4) {
+              const float4 bb = *reinterpret_cast<const float4*>(cp + e);
+              ffma2(s[e], s[e + 1], s[e], s[e + 1], sl2, sl2, bb.x, bb.y);
+              ffma2(s[e + 2], s[e + 3], s[e + 2], s[e + 3], sl2, sl2, bb.z, bb.w);
+            }
+          }
           live = 0;
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch)
@@ -666,8 +707,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 #pragma unroll
             for (int e = 0; e < kTile; ++e) s[e] = (e < hi_t) ? s[e] : -INFINITY;
           }
-          tmax = row_max128(s) * sl2;
-          raw = true;
+          if (has_local) {
+            tmax = row_max128(s);
+          } else {
+            tmax = row_max128(s) * sl2;
+            raw = true;
+          }
         } else if (j < w.nband + w.ngc) {
           // global-column tile: stage its 128 positions in shared memory (one per
           // thread of the group), then mask the keys already inside the window
@@ -691,7 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           const int lim = row_valid ? p.S - s0 : 0;
           if (bias_row && bias_staged) {
             const int b0 = s0 + boff;
-            const float* cp = sBias + (b0 & 3) * kBiasCopy + (b0 & ~3);
+            const float* cp = sSide + (b0 & 3) * side_stride + (b0 & ~3);
 #pragma unroll
             for (int e = 0; e < kTile; e += 4) {
               const float4 bb = *reinterpret_cast<const float4*>(cp + e);
@@ -824,9 +869,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const bool has = row_valid && l > 0.f;
       const float inv = has ? 1.f / l : 0.f;
       const float lse_v = has ? (m + __log2f(l)) * kLn2 : -INFINITY;
-      if (MODE == 0 && !has_bias) {
-        // Coalesced store: 32-column chunks staged in shared memory (the side-bias
-        // area, unused without bias; two 8 KB buffers per group, 64-byte swizzle)
+      if (MODE == 0 && !has_bias && !has_local) {
+        // Coalesced store: 32-column chunks staged in shared memory (the bias area,
+        // unused without biases; two 8 KB buffers per group, 64-byte swizzle)
         // and written by TMA; rows beyond the class end are clipped by the map.
         uint8_t* stage = reinterpret_cast<uint8_t*>(sBias) + x * 2 * 8192;
         if (row == 0) tma_store_wait_read<0>();          // previous unit's stores have read

@@ -198,7 +198,38 @@ swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void
                        const void* side_v, const float* bias, const int32_t* window,
                        const int32_t* dilation, int causal, const int32_t* valid_len, void* out,
                        float* lse, void* stream) {
-  if (!plan) return SWA_ERR_INVALID_ARG;
+  swa_forward_args a;
+  memset(&a, 0, sizeof(a));
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.global_idx = global_idx;
+  a.num_global = num_global;
+  a.side_k = side_k;
+  a.side_v = side_v;
+  a.bias = bias;
+  a.window = window;
+  a.dilation = dilation;
+  a.causal = causal;
+  a.valid_len = valid_len;
+  a.out = out;
+  a.lse = lse;
+  return swa_forward_ex(plan, &a, stream);
+}
+
+swa_status swa_forward_ex(swa_plan_t plan, const swa_forward_args* args, void* stream) {
+  if (!plan || !args) return SWA_ERR_INVALID_ARG;
+  const void *q = args->q, *k = args->k, *v = args->v;
+  const int32_t* global_idx = args->global_idx;
+  const int num_global = args->num_global;
+  const void *side_k = args->side_k, *side_v = args->side_v;
+  const float* bias = args->bias;
+  const int32_t *window = args->window, *dilation = args->dilation;
+  const int causal = args->causal;
+  const int32_t* valid_len = args->valid_len;
+  void* out = args->out;
+  float* lse = args->lse;
+  const float* local_bias = args->local_bias;
   const swa_plan_desc& d = plan->desc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   plan->last_launches = 0;
@@ -213,7 +244,8 @@ swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void
     if (!aligned16(side_k) || !aligned16(side_v)) return SWA_ERR_INVALID_ARG;
   }
   if ((lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
-      (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+      (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) ||
+      (local_bias && (reinterpret_cast<uintptr_t>(local_bias) & 3u)))
     return SWA_ERR_INVALID_ARG;
   const int Hq = d.num_q_heads;
   for (int h = 0; h < Hq; ++h) {
@@ -222,6 +254,23 @@ swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void
     if ((long long)window[h] * (dilation ? dilation[h] : 1) > (1LL << 30)) return SWA_ERR_INVALID_ARG;
   }
   if (causal && num_global > 0) return SWA_ERR_UNSUPPORTED;
+  // local bias: the table covers every offset a window key can take; the band
+  // kernel stages [-r_eff - kLocalPad, r_eff + kLocalPad] of it per work unit,
+  // r_eff = min(r, ceil(n / d)) (offsets in class coordinates)
+  int local_stride = 0;
+  if (local_bias) {
+    if (args->local_radius < 0 || args->local_radius > (1 << 30)) return SWA_ERR_INVALID_ARG;
+    int r_eff_max = 0;
+    for (int h = 0; h < Hq; ++h) {
+      const long long dh = dilation ? dilation[h] : 1;
+      const long long reach = std::min((long long)window[h] * dh, (long long)d.seq_len - 1);
+      if (args->local_radius < reach) return SWA_ERR_INVALID_ARG;
+      const long long nc = (d.seq_len + dh - 1) / dh;
+      r_eff_max = (int)std::max<long long>(r_eff_max, std::min<long long>(window[h], nc));
+    }
+    local_stride = (int)align_up(2 * (size_t)r_eff_max + 2 * swa::kLocalPad + 4, 32);
+    if (d.dtype == SWA_BF16 && local_stride > swa::kBiasCopy) return SWA_ERR_UNSUPPORTED;
+  }
 
   // ---------------------------------------------------------- parameters
   AttnParams* pp = new (std::nothrow) AttnParams;
@@ -246,6 +295,9 @@ swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void
   p.valid_len = valid_len;
   p.global_idx = num_global > 0 ? global_idx : nullptr;
   p.bias = d.num_side > 0 ? bias : nullptr;
+  p.local_bias = local_bias;
+  p.local_radius = local_bias ? args->local_radius : 0;
+  p.local_stride = local_stride;
   p.out = out;
   p.lse = lse;
   p.err = plan->err;
@@ -277,9 +329,10 @@ swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void
   // Work units: two 128-row query tiles.  When query heads come in GQA pairs with
   // the same window and dilation (and no per-head side bias), a unit is the same
   // rows of two heads that share one KV head; otherwise it is two consecutive
-  // row tiles of one head.
+  // row tiles of one head.  (Per-head side or local bias rows are staged once per
+  // unit, so a unit keeps one head when either is present.)
   if (st == SWA_OK) {
-    bool pair = (p.G % 2 == 0) && !(d.num_side > 0 && bias);
+    bool pair = (p.G % 2 == 0) && !(d.num_side > 0 && bias) && !local_bias;
     for (int h = 0; pair && h < Hq; h += 2)
       pair = window[h] == window[h + 1] && p.class_base[h] == p.class_base[h + 1];
     p.pair_heads = pair ? 1 : 0;
@@ -414,6 +467,15 @@ int swa_relative_bucket(int delta) {
   for (int m = 1; m <= 7; ++m)
     if (a * a >= (64LL << m)) step = m;
   return bucket + 8 + step;
+}
+
+swa_status swa_bucket_local_bias(int num_q_heads, int radius, const float* table, float* out) {
+  if (num_q_heads < 1 || radius < 0 || radius > (1 << 28) || !table || !out) return SWA_ERR_INVALID_ARG;
+  const size_t cols = 2 * (size_t)radius + 1;
+  for (int h = 0; h < num_q_heads; ++h)
+    for (size_t c = 0; c < cols; ++c)
+      out[(size_t)h * cols + c] = table[h * 32 + swa_relative_bucket((int)c - radius)];
+  return SWA_OK;
 }
 
 swa_status swa_expand_side_bias(int num_q_heads, int num_side, int nblk, const float* table,

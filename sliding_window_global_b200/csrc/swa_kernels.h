@@ -13,6 +13,8 @@ constexpr int kTile = 128;           // query rows per tile and keys per KV tile
 constexpr int kMaxClasses = 16;      // distinct (dilation, residue) classes per forward
 constexpr int kMaxHeads = 128;       // query heads per plan
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
+constexpr int kBiasCopy = 2048;      // floats per staged bias copy (4 copies in shared memory)
+constexpr int kLocalPad = 256;       // zero entries staged on each side of a local-bias row
 
 // Bits of the device error word.
 constexpr int kDevErrTimeout = 1;    // a bounded wait expired
@@ -43,6 +45,9 @@ struct AttnParams {
   const int32_t* valid_len;          // [B] or nullptr (= n)
   const int32_t* global_idx;         // [B, g] or nullptr
   const float* bias;                 // [Hq, S + nblk - 1] or nullptr
+  const float* local_bias;           // [Hq, 2 * local_radius + 1] or nullptr (window keys)
+  int local_radius;
+  int local_stride;                  // floats per staged copy of a local-bias row (band kernel)
   void* out;                         // [B, Hq, n, D], input dtype
   float* lse;                        // [B, Hq, n] or nullptr
   float* part_o;                     // global-row partials [nsplit, B*Hq, gpad, D]

@@ -30,6 +30,7 @@ EXPORTS = (
     "swa_plan_create", "swa_forward", "swa_plan_check", "swa_plan_destroy",
     "swa_plan_workspace_bytes", "swa_plan_last_launches", "swa_status_string",
     "swa_side_aggregate", "swa_relative_bucket", "swa_expand_side_bias", "swa_forward_noalloc",
+    "swa_forward_ex", "swa_bucket_local_bias",
 )
 
 
@@ -45,6 +46,18 @@ class PlanDesc(ctypes.Structure):
         ("num_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("dtype", ctypes.c_int),
         ("max_global", ctypes.c_int), ("num_side", ctypes.c_int), ("side_block", ctypes.c_int),
         ("scale", ctypes.c_float), ("flags", ctypes.c_uint),
+    ]
+
+
+class ForwardArgs(ctypes.Structure):
+    """swa_forward_args of include/swa.h."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("global_idx", ctypes.c_void_p), ("num_global", ctypes.c_int),
+        ("side_k", ctypes.c_void_p), ("side_v", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+        ("window", ctypes.c_void_p), ("dilation", ctypes.c_void_p), ("causal", ctypes.c_int),
+        ("valid_len", ctypes.c_void_p), ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+        ("local_bias", ctypes.c_void_p), ("local_radius", ctypes.c_int),
     ]
 
 
@@ -85,6 +98,10 @@ def load_library():
         lib.swa_forward_noalloc.argtypes = [ctypes.POINTER(PlanDesc), P, P, P, P, I, P, P, P, P, P, I,
                                             P, P, P, P]
         lib.swa_forward_noalloc.restype = I
+        lib.swa_forward_ex.argtypes = [P, ctypes.POINTER(ForwardArgs), P]
+        lib.swa_forward_ex.restype = I
+        lib.swa_bucket_local_bias.argtypes = [I, I, P, P]
+        lib.swa_bucket_local_bias.restype = I
         _lib = lib
         return lib
 
@@ -166,7 +183,9 @@ class Plan:
                 side_k: Optional[torch.Tensor] = None, side_v: Optional[torch.Tensor] = None,
                 bias: Optional[torch.Tensor] = None, valid_len: Optional[torch.Tensor] = None,
                 out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                return_lse: bool = True, stream=None):
+                return_lse: bool = True, local_bias: Optional[torch.Tensor] = None, stream=None):
+        """``local_bias``: optional [Hq, 2R+1] fp32 device table of the LongT5 local
+        relative-position bias (window keys of non-global rows, column (j - i) + R)."""
         d = self.desc
         H = d.num_q_heads
         if out is None:
@@ -176,6 +195,23 @@ class Plan:
         w_arr, _ = _host_i32(window, H, "window")
         d_arr, _ = _host_i32(dilation, H, "dilation")
         g = 0 if global_idx is None else int(global_idx.shape[-1])
+        if local_bias is not None:
+            width = int(local_bias.shape[-1])
+            if local_bias.dim() != 2 or local_bias.shape[0] != H or width % 2 == 0:
+                raise ValueError("local_bias must be [Hq, 2R+1]")
+            a = ForwardArgs(
+                _dev_ptr(q, "q", self.dtype), _dev_ptr(k, "k", self.dtype), _dev_ptr(v, "v", self.dtype),
+                _dev_ptr(global_idx, "global_idx", torch.int32), g,
+                _dev_ptr(side_k, "side_k", self.dtype), _dev_ptr(side_v, "side_v", self.dtype),
+                _dev_ptr(bias, "bias", torch.float32), ctypes.cast(w_arr, ctypes.c_void_p),
+                None if d_arr is None else ctypes.cast(d_arr, ctypes.c_void_p), int(bool(causal)),
+                _dev_ptr(valid_len, "valid_len", torch.int32), _dev_ptr(out, "out", self.dtype),
+                _dev_ptr(lse, "lse", torch.float32), _dev_ptr(local_bias, "local_bias", torch.float32),
+                (width - 1) // 2)
+            st = self._lib.swa_forward_ex(self._h, ctypes.byref(a), _stream_handle(stream))
+            if st != 0:
+                raise SwaError(st, "swa_forward_ex")
+            return out, lse
         st = self._lib.swa_forward(
             self._h, _dev_ptr(q, "q", self.dtype), _dev_ptr(k, "k", self.dtype),
             _dev_ptr(v, "v", self.dtype), _dev_ptr(global_idx, "global_idx", torch.int32), g,
@@ -208,7 +244,8 @@ _plans = {}
 
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, window, dilation=None,
             causal: bool = False, global_idx=None, side_k=None, side_v=None, bias=None,
-            valid_len=None, side_block: int = 16, scale: float = 0.0, return_lse: bool = True):
+            valid_len=None, side_block: int = 16, scale: float = 0.0, return_lse: bool = True,
+            local_bias=None):
     """Banded sparse attention of q [B,Hq,n,D] over k/v [B,Hkv,n,D] (CUDA tensors).
 
     Returns ``(out, lse)``: out like q, lse fp32 [B,Hq,n] (natural log).  Plans are
@@ -225,7 +262,7 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, window, dilati
         _plans[key] = plan
     return plan.forward(q, k, v, window=window, dilation=dilation, causal=causal,
                         global_idx=global_idx, side_k=side_k, side_v=side_v, bias=bias,
-                        valid_len=valid_len, return_lse=return_lse)
+                        valid_len=valid_len, return_lse=return_lse, local_bias=local_bias)
 
 
 def side_aggregate(x: torch.Tensor, block: int, valid_len: Optional[torch.Tensor] = None,
@@ -256,4 +293,18 @@ def expand_side_bias(table: torch.Tensor, num_side: int, nblk: int) -> torch.Ten
                                   ctypes.c_void_p(out.data_ptr()))
     if st != 0:
         raise SwaError(st, "swa_expand_side_bias")
+    return out
+
+
+def bucket_local_bias(table: torch.Tensor, radius: int) -> torch.Tensor:
+    """[Hq,32] fp32 bucket table (host) -> [Hq, 2*radius + 1] local-bias table (host),
+    column c holding the bucket of the offset c - radius."""
+    lib = load_library()
+    t = table.detach().to("cpu", torch.float32).contiguous()
+    Hq = t.shape[0]
+    out = torch.empty((Hq, 2 * radius + 1), dtype=torch.float32)
+    st = lib.swa_bucket_local_bias(Hq, int(radius), ctypes.c_void_p(t.data_ptr()),
+                                   ctypes.c_void_p(out.data_ptr()))
+    if st != 0:
+        raise SwaError(st, "swa_bucket_local_bias")
     return out

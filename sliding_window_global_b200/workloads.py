@@ -14,11 +14,14 @@ cases:
   1024 side keys (block means of 16 tokens) with a 32-bucket side bias
 * ``swan_swa``         -- SWAN-GPT SWA-RoPE layer: 32 query / 8 KV heads, n=32768,
   D=128, causal window of 512 keys, q and k rotated by RoPE (base 10000)
+* ``longt5_local``     -- LongT5 Local attention: n=16384, 12 heads, r=127 with the
+  local relative-position bias (a 32-bucket table per head over the token offset)
 
 Inputs are N(0,1) from ``torch.Generator('cpu').manual_seed(seed)`` drawn in
-the order q, k, v, global positions, bias table, then rounded to the dtype.
-Side keys/values (block means) and the expanded side-bias table are NOT made
-here: each side (oracle and CUDA library) derives them with its own code.
+the order q, k, v, global positions, side-bias table, local-bias table, then
+rounded to the dtype.  Side keys/values (block means) and the expanded bias
+tables are NOT made here: each side (oracle and CUDA library) derives them with
+its own code.
 """
 from __future__ import annotations
 
@@ -46,6 +49,7 @@ class Workload:
     padding: int = 0                # trailing padded positions (valid_len = n - padding)
     side_block: int = 0             # k of the Transient-Global blocks (0: no side keys)
     side_bias: bool = False         # seeded 32-bucket side-bias table
+    local_bias: bool = False        # seeded 32-bucket local relative-position bias table
     rope: bool = False              # rotate q and k with RoPE (base 10000, all dims)
     seed: int = 0
 
@@ -90,6 +94,8 @@ WORKLOADS = {
                                _heads(1, 12), side_block=16, side_bias=True, seed=1004),
     "swan_swa": Workload("swan_swa", 1, 32, 8, 32768, 128, "bf16", _heads(511, 32), _heads(1, 32),
                          causal=True, rope=True, seed=1005),
+    "longt5_local": Workload("longt5_local", 1, 12, 12, 16384, 64, "bf16", _heads(127, 12),
+                             _heads(1, 12), local_bias=True, seed=1006),
 }
 
 # Reduced versions with the same structure (several tiles and a ragged tail) that the
@@ -109,6 +115,9 @@ SMALL = {
     "swan_swa": dataclasses.replace(WORKLOADS["swan_swa"], name="swan_swa_small", seq_len=1200,
                                     q_heads=8, kv_heads=2, window=_heads(300, 8),
                                     dilation=_heads(1, 8), seed=2005),
+    "longt5_local": dataclasses.replace(WORKLOADS["longt5_local"], name="longt5_local_small",
+                                        seq_len=1100, q_heads=3, kv_heads=3, window=_heads(127, 3),
+                                        dilation=_heads(1, 3), padding=45, seed=2006),
 }
 
 
@@ -150,6 +159,9 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> dict:
     bias_table = None
     if w.side_bias:
         bias_table = torch.randn((Hq, 32), generator=g, dtype=torch.float32)
+    local_table = None
+    if w.local_bias:
+        local_table = torch.randn((Hq, 32), generator=g, dtype=torch.float32)
     if w.rope:
         pos = torch.arange(n)
         q = _rope_(q, pos)
@@ -159,6 +171,7 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> dict:
         q=q.to(dt).contiguous(), k=k.to(dt).contiguous(), v=v.to(dt).contiguous(),
         global_idx=global_idx,
         bias_table=bias_table,
+        local_table=local_table,
         window=torch.tensor(w.window, dtype=torch.int32),
         dilation=torch.tensor(w.dilation, dtype=torch.int32),
         causal=w.causal,

@@ -31,7 +31,16 @@ def host_problem(w: workloads.Workload, inp: dict | None = None):
         if inp.get("bias_table") is not None:
             nblk = (w.seq_len + w.side_block - 1) // w.side_block
             inp["bias"] = torch.from_numpy(oracle.expand_side_bias(inp["bias_table"], w.num_side, nblk))
+    if inp.get("local_table") is not None:
+        R = local_radius(w)
+        inp["local_bias"] = torch.from_numpy(oracle.expand_local_bias(inp["local_table"], R))
     return inp
+
+
+def local_radius(w) -> int:
+    """Smallest table radius covering every window offset: max over heads of
+    min(r * d, n - 1)."""
+    return max(min(r * d, w.seq_len - 1) for r, d in zip(w.window, w.dilation))
 
 
 def oracle_problem(w, inp):
@@ -39,13 +48,14 @@ def oracle_problem(w, inp):
                           dilation=inp["dilation"].numpy(), causal=inp["causal"],
                           global_idx=inp["global_idx"], side_k=inp.get("side_k"),
                           side_v=inp.get("side_v"), side_block=w.side_block or 16,
-                          bias=inp.get("bias"), valid_len=inp["valid_len"], scale=inp["scale"])
+                          bias=inp.get("bias"), valid_len=inp["valid_len"], scale=inp["scale"],
+                          local_bias=inp.get("local_bias"))
 
 
 def to_dev(inp, device="cuda"):
     out = {}
     for k, v in inp.items():
-        if isinstance(v, torch.Tensor) and k not in ("window", "dilation", "bias_table"):
+        if isinstance(v, torch.Tensor) and k not in ("window", "dilation", "bias_table", "local_table"):
             out[k] = v.to(device).contiguous()
         else:
             out[k] = v
@@ -63,7 +73,7 @@ def run_gpu(w, dinp, plan=None, debug=False):
                             dilation=dinp["dilation"], causal=dinp["causal"],
                             global_idx=dinp["global_idx"], side_k=dinp.get("side_k"),
                             side_v=dinp.get("side_v"), bias=dinp.get("bias"),
-                            valid_len=dinp["valid_len"])
+                            valid_len=dinp["valid_len"], local_bias=dinp.get("local_bias"))
     torch.cuda.synchronize()
     return out, lse, plan
 

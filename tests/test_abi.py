@@ -94,3 +94,21 @@ def test_expand_side_bias_matches_oracle(lib):
         ours = binding.expand_side_bias(table, S, nblk).numpy()
         ref = oracle.expand_side_bias(table, S, nblk)
         assert np.array_equal(ours, ref)
+
+
+def test_bucket_local_bias_matches_oracle(lib):
+    gen = torch.Generator("cpu").manual_seed(6)
+    table = torch.randn((12, 32), generator=gen)
+    for R in (0, 1, 7, 127, 511, 2000):
+        ours = binding.bucket_local_bias(table, R).numpy()
+        ref = oracle.expand_local_bias(table, R)
+        assert ours.shape == (12, 2 * R + 1)
+        assert np.array_equal(ours, ref)
+    assert lib.swa_bucket_local_bias(0, 1, None, None) == 1
+    assert lib.swa_bucket_local_bias(1, -1, None, None) == 1
+
+
+def test_forward_ex_null_arguments(lib):
+    assert lib.swa_forward_ex(None, None, None) == 1
+    args = binding.ForwardArgs()
+    assert lib.swa_forward_ex(None, ctypes.byref(args), None) == 1

@@ -419,3 +419,17 @@ def test_local_bias_table_must_cover_the_window(oracle_mod):
     big = oracle_mod.Problem(p.q[:, :, :4], p.k[:, :, :4], p.v[:, :, :4], window=50,
                              local_bias=_local_table(rng, 1, 3))
     big.forward()
+
+
+def test_expand_local_bias_columns(oracle_mod):
+    table = np.arange(2 * 32, dtype=np.float32).reshape(2, 32)
+    R = 200
+    out = oracle_mod.expand_local_bias(table, R)
+    assert out.shape == (2, 2 * R + 1)
+    # column c holds delta = c - R (memory minus query position): 0 -> bucket 0,
+    # +1 -> 17 (the positive half starts at 16), -1 -> 1, |delta| >= 128 -> the last bucket
+    assert out[1, R] == 32 + 0
+    assert out[1, R + 1] == 32 + 17
+    assert out[1, R - 1] == 32 + 1
+    assert out[0, R + 7] == 16 + 7 and out[0, R + 8] == 16 + 8
+    assert out[0, 0] == 15 and out[0, 2 * R] == 31

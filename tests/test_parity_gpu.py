@@ -94,6 +94,19 @@ EDGE = [
                                           dilation=(1, 2, 1, 2), seq_len=300)),
     ("fp32_globals_pad", dataclasses.replace(workloads.SMALL["longformer_base"], dtype="fp32",
                                              seq_len=400, padding=33, num_global=7)),
+    # local relative-position bias on window keys (LongT5 local attention)
+    ("local_globals", _small("longformer_base", local_bias=True)),
+    ("local_tglobal_side_bias", _small("longt5_tglobal", local_bias=True, padding=30)),
+    ("local_dilated_globals", _small("dilated", local_bias=True)),
+    ("local_causal_gqa_d128", _small("swan_swa", local_bias=True)),
+    ("local_window_covers_seq", _small("longformer_base", seq_len=300, window=(5000,) * 4,
+                                       num_global=0, global_mode="none", padding=0,
+                                       local_bias=True)),
+    ("local_r766_d64", _small("longt5_local", seq_len=2000, window=(766,) * 3, padding=0)),
+    ("local_d128_noncausal", _small("swan_swa", causal=False, window=(200, 1, 0, 200, 37, 37, 5, 9),
+                                    local_bias=True)),
+    ("local_fp32_dilated", dataclasses.replace(workloads.SMALL["longt5_local"], dtype="fp32",
+                                               seq_len=500, window=(40,) * 3, dilation=(1, 2, 3))),
 ]
 
 
@@ -149,6 +162,31 @@ def test_support_exact(n, D, r, d, causal, g, pad):
                 row = o[b, h, i, :n]
                 assert np.all(row[~inside] == 0.0), (b, h, i)
                 assert np.all(row[inside] > 0.0), (b, h, i)
+
+
+def test_local_bias_window_beyond_staging_limit_is_unsupported():
+    """bf16 kernels stage the local-bias row of a unit: min(r, ceil(n/d)) <= 766."""
+    _need_gpu()
+    from sliding_window_global_b200 import SwaError
+    w = _small("longt5_local", seq_len=2000, window=(767,) * 3, padding=0)
+    dinp = helpers.to_dev(helpers.host_problem(w))
+    with pytest.raises(SwaError) as e:
+        helpers.run_gpu(w, dinp)
+    assert e.value.status == 2
+    # the same window with dilation 3 spans ceil(2000 / 3) = 667 class rows: supported
+    w = _small("longt5_local", seq_len=2000, window=(767,) * 3, dilation=(3,) * 3, padding=0)
+    _check_workload(w)
+
+
+def test_local_bias_table_too_small_is_invalid():
+    _need_gpu()
+    from sliding_window_global_b200 import SwaError
+    w = workloads.SMALL["longt5_local"]
+    dinp = helpers.to_dev(helpers.host_problem(w))
+    dinp["local_bias"] = dinp["local_bias"][:, 1:-1].contiguous()     # radius 126 < 127
+    with pytest.raises(SwaError) as e:
+        helpers.run_gpu(w, dinp)
+    assert e.value.status == 1
 
 
 def test_side_aggregate_matches_oracle():
