@@ -219,6 +219,33 @@ __device__ __forceinline__ bool uses(const Work& w, int x, int j) {
   return kv0 < w.hi[x] && kv0 + kTile > w.lo[x];
 }
 
+// The fields of one query tile as scalars: the softmax warps pick their tile at
+// run time, and indexing Work's two-element arrays with a run-time index would
+// put the whole struct in local memory.
+struct TileRows {
+  int u0, rows, nvalid, lo, hi, head;
+  bool active;
+};
+
+__device__ __forceinline__ TileRows tile_rows(const Work& w, int x) {
+  TileRows t;
+  t.u0 = x ? w.u0[1] : w.u0[0];
+  t.rows = x ? w.rows[1] : w.rows[0];
+  t.nvalid = x ? w.nvalid[1] : w.nvalid[0];
+  t.lo = x ? w.lo[1] : w.lo[0];
+  t.hi = x ? w.hi[1] : w.hi[0];
+  t.head = x ? w.hx[1] : w.hx[0];
+  t.active = x ? w.active[1] : w.active[0];
+  return t;
+}
+
+__device__ __forceinline__ bool uses(const Work& w, const TileRows& t, int j) {
+  if (!t.active || j < 0 || j >= w.total) return false;
+  if (j >= w.nband) return true;
+  const int kv0 = w.band_lo + j * kTile;
+  return kv0 < t.hi && kv0 + kTile > t.lo;
+}
+
 __device__ __forceinline__ void tile_source(const AttnParams& p, const Work& w, int j,
                                             const CUtensorMap*& mk, const CUtensorMap*& mv,
                                             int& y) {
@@ -302,15 +329,16 @@ __device__ __forceinline__ float row_max128(const float (&x)[kTile]) {
 }
 
 // ------------------------------------------------------------------ output rows
-__device__ __forceinline__ size_t out_row(const AttnParams& p, const Work& w, int x, int row) {
-  const int pos = w.c + w.d * (w.u0[x] + row);
-  return (size_t)(w.b * p.Hq + w.hx[x]) * p.n + pos;
+__device__ __forceinline__ size_t out_row(const AttnParams& p, const Work& w, const TileRows& t,
+                                          int row) {
+  const int pos = w.c + w.d * (t.u0 + row);
+  return (size_t)(w.b * p.Hq + t.head) * p.n + pos;
 }
 
 template <int D>
-__device__ void write_zero_row(const AttnParams& p, const Work& w, int x, int row) {
-  if (row >= w.rows[x] || row < w.nvalid[x]) return;
-  const size_t off = out_row(p, w, x, row);
+__device__ void write_zero_row(const AttnParams& p, const Work& w, const TileRows& t, int row) {
+  if (row >= t.rows || row < t.nvalid) return;
+  const size_t off = out_row(p, w, t, row);
   uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + off * D);
 #pragma unroll
   for (int i = 0; i < D / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
@@ -327,7 +355,9 @@ __device__ void write_neutral_partial(const AttnParams& p, const Work& w, int ro
   p.part_lse[prow] = -INFINITY;
 }
 
-template <int D, int MODE>
+// LOCAL: band tiles carry the local relative-position bias (MODE 0 only).  It is a
+// template parameter so that kernels without it keep their register schedule.
+template <int D, int MODE, bool LOCAL>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ AttnParams p) {
   using C = Cfg<D>;
   constexpr int NS = C::NS;
@@ -359,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const int lane = tid & 31;
   const int nunits = total_units<MODE>(p);
   const bool has_bias = p.bias && p.S > 0;
-  const bool has_local = MODE == 0 && p.local_bias != nullptr;
+  constexpr bool has_local = LOCAL && MODE == 0;
   // shared bias area: 4 copies of the local-bias row (stride lstride floats), then
   // 4 copies of the side-bias segment (stride side_stride)
   const int lstride = has_local ? p.local_stride : 0;
@@ -408,7 +438,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         if (!w.active[0]) continue;
         const CUtensorMap* mq = (MODE == 0) ? &p.mq[w.cls] : &p.mgq;
         const int kz = w.b * p.Hkv + w.hk;
-        for (int x = 0; x < 2 && ok; ++x) {
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (!ok) break;
           const int qz = w.b * p.Hq + w.hx[x];
           if (!w.active[x]) continue;
           if (qloads[x] > 0 &&
@@ -457,6 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         if (!w.active[0]) continue;
         const int T = w.total;
         int first[2] = {-1, -1}, last[2] = {-1, -1}, issued[2] = {-1, -1}, npv[2] = {0, 0};
+#pragma unroll
         for (int x = 0; x < 2; ++x)
           for (int j = 0; j < T; ++j)
             if (uses(w, x, j)) {
@@ -485,7 +518,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           issued[x] = j;
           return true;
         };
-        for (int x = 0; x < 2 && ok; ++x) {
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (!ok) break;
           if (!w.active[x]) continue;
           ok = mbar_wait_bounded(&q_full[x], qwaits[x] & 1, abort_v, kWaitLimitNs);
           ++qwaits[x];
@@ -494,17 +529,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         for (int j = 0; ok && j < T; ++j) {
           const int g = kv + j;
           const int st = g % NS;
-          for (int x = 0; x < 2 && ok; ++x)
-            if (uses(w, x, j) && issued[x] < j) ok = issue_qk(x, j);
+#pragma unroll
+          for (int x = 0; x < 2; ++x)
+            if (ok && uses(w, x, j) && issued[x] < j) ok = issue_qk(x, j);
           if (C::kSepP) {
             // the next S of each tile as soon as its softmax has read the current one
-            for (int x = 0; x < 2 && ok; ++x)
-              if (uses(w, x, j) && uses(w, x, j + 1) && issued[x] == j) ok = issue_qk(x, j + 1);
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+              if (ok && uses(w, x, j) && uses(w, x, j + 1) && issued[x] == j) ok = issue_qk(x, j + 1);
           }
           if (!ok) break;
           if (!mbar_wait_bounded(&v_full[st], (g / NS) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
           const uint32_t vt = v_base + st * C::kTileBytes;
-          for (int x = 0; x < 2 && ok; ++x) {
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            if (!ok) break;
             if (!uses(w, x, j)) continue;
             if (!C::kSepP) {
               // P over S: the first half of P (keys 0-63) is published early, so the
@@ -553,14 +592,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       Work w;
       decode_work<MODE>(p, uid, w);
       if (!w.valid) continue;
+      const TileRows tr = tile_rows(w, x);
       if (!w.active[0]) {
-        if (MODE == 0) write_zero_row<D>(p, w, x, row);
+        if (MODE == 0) write_zero_row<D>(p, w, tr, row);
         else if (x == 0) write_neutral_partial<D>(p, w, row);
         continue;
       }
       const int T = w.total;
-      const bool row_valid = row < w.nvalid[x];
-      const int u = w.u0[x] + row;
+      const bool row_valid = row < tr.nvalid;
+      const int u = tr.u0 + row;
       int pos = 0;
       if (MODE == 0) pos = w.c + w.d * u;
       else if (row_valid) pos = p.global_idx[(size_t)w.b * p.g + w.u0[0] + row];
@@ -628,8 +668,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         named_barrier_sync(3, kSoftmaxThreads);
       }
-      if (!w.active[x]) {
-        if (MODE == 0) write_zero_row<D>(p, w, x, row);
+      if (!tr.active) {
+        if (MODE == 0) write_zero_row<D>(p, w, tr, row);
         continue;
       }
 
@@ -652,7 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       float l = 0.f;
       int iu = 0;                              // tiles of this unit handled
       for (int j = 0; j < T; ++j) {
-        if (!uses(w, x, j)) continue;
+        if (!uses(w, tr, j)) continue;
         if (!mbar_wait_bounded(&s_full[x], it & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
         uint32_t xr[kTile];
@@ -899,20 +939,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           fence_proxy_async_smem();
           named_barrier_sync(1 + x, 128);
           if (row == 0) {
-            tma_store_3d(&p.mo[w.cls], buf, ch * 32, w.u0[x], w.b * p.Hq + w.hx[x]);
+            tma_store_3d(&p.mo[w.cls], buf, ch * 32, tr.u0, w.b * p.Hq + tr.head);
             tma_store_commit();
           }
         }
-        if (row < w.rows[x] && p.lse) p.lse[out_row(p, w, x, row)] = lse_v;
+        if (row < tr.rows && p.lse) p.lse[out_row(p, w, tr, row)] = lse_v;
       } else if (MODE == 0) {
-        const size_t off = out_row(p, w, x, row);
+        const size_t off = out_row(p, w, tr, row);
         uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + off * D);
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t rr[32];
           tmem_ld32(o_addr + ch * 32, rr);
           tmem_wait_ld_dep(rr);
-          if (row < w.rows[x]) {
+          if (row < tr.rows) {
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
               uint4 v;
@@ -924,7 +964,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             }
           }
         }
-        if (row < w.rows[x] && p.lse) p.lse[off] = lse_v;
+        if (row < tr.rows && p.lse) p.lse[off] = lse_v;
       } else {
         const size_t prow =
             ((size_t)w.split * p.B * p.Hq + (size_t)w.b * p.Hq + w.h) * p.gpad + w.u0[0] + row;
@@ -974,9 +1014,9 @@ size_t band_tc_smem_bytes(int D) {
   return D == 64 ? Cfg<64>::kSmemBytes : Cfg<128>::kSmemBytes;
 }
 
-template <int D, int MODE>
+template <int D, int MODE, bool LOCAL = false>
 static cudaError_t launch_one(const AttnParams& p, int units, int num_sms, cudaStream_t s) {
-  auto kern = attn_tc_kernel<D, MODE>;
+  auto kern = attn_tc_kernel<D, MODE, LOCAL>;
   const int smem = static_cast<int>(Cfg<D>::kSmemBytes);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -989,6 +1029,9 @@ static cudaError_t launch_one(const AttnParams& p, int units, int num_sms, cudaS
 // p.tiles[h] holds the number of two-tile units of head h, p.max_units their maximum.
 cudaError_t launch_band_tc(const AttnParams& p, int num_sms, cudaStream_t s) {
   const int units = p.max_units * p.B * p.Hq;
+  if (p.local_bias)
+    return p.D == 64 ? launch_one<64, 0, true>(p, units, num_sms, s)
+                     : launch_one<128, 0, true>(p, units, num_sms, s);
   return p.D == 64 ? launch_one<64, 0>(p, units, num_sms, s) : launch_one<128, 0>(p, units, num_sms, s);
 }
 
