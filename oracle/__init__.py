@@ -35,6 +35,24 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+class _Extras(ctypes.Structure):
+    """oracle_extras of swa_oracle.c."""
+    _fields_ = [("local_bias", ctypes.c_void_p), ("local_radius", ctypes.c_int),
+                ("rand_blocks", ctypes.c_void_p), ("num_rand", ctypes.c_int),
+                ("rand_block", ctypes.c_int)]
+
+
+def _extras(local_bias=None, local_radius=0, rand_blocks=None, rand_block=128):
+    ex = _Extras()
+    ex.local_bias = None if local_bias is None else local_bias.ctypes.data
+    ex.local_radius = int(local_radius)
+    if rand_blocks is not None and rand_blocks.shape[-1] > 0:
+        ex.rand_blocks = rand_blocks.ctypes.data
+        ex.num_rand = int(rand_blocks.shape[-1])
+        ex.rand_block = int(rand_block)
+    return ex
+
+
 def _load():
     global _lib
     with _lock:
@@ -48,14 +66,19 @@ def _load():
             lib.oracle_dense_bruteforce.argtypes = [I, I, I, I, I, P, P, P, P, I, P, P, I, I, P, P,
                                                     P, I, P, D, P, P]
             lib.oracle_dense_bruteforce.restype = I
-            lib.oracle_forward_ex.argtypes = lib.oracle_forward.argtypes + [P, I]
+            EX = ctypes.POINTER(_Extras)
+            lib.oracle_forward_ex.argtypes = lib.oracle_forward.argtypes + [EX]
             lib.oracle_forward_ex.restype = I
-            lib.oracle_dense_bruteforce_ex.argtypes = lib.oracle_dense_bruteforce.argtypes + [P, I]
+            lib.oracle_dense_bruteforce_ex.argtypes = lib.oracle_dense_bruteforce.argtypes + [EX]
             lib.oracle_dense_bruteforce_ex.restype = I
             lib.oracle_key_counts.argtypes = [I, I, I, P, I, I, P, P, I, P, P]
             lib.oracle_key_counts.restype = I
             lib.oracle_key_list.argtypes = [I, I, I, P, I, P, P, I, P, I, I, I, P]
             lib.oracle_key_list.restype = I
+            lib.oracle_key_counts_ex.argtypes = lib.oracle_key_counts.argtypes + [EX]
+            lib.oracle_key_counts_ex.restype = I
+            lib.oracle_key_list_ex.argtypes = lib.oracle_key_list.argtypes + [EX]
+            lib.oracle_key_list_ex.restype = I
             lib.oracle_relative_bucket.argtypes = [I]
             lib.oracle_relative_bucket.restype = I
             lib.oracle_expand_side_bias.argtypes = [I, I, I, P, P]
@@ -106,9 +129,11 @@ class Problem:
 
     def __init__(self, q, k, v, *, window, dilation=1, causal=False, global_idx=None,
                  side_k=None, side_v=None, side_block=16, bias=None, valid_len=None, scale=None,
-                 local_bias=None):
+                 local_bias=None, rand_blocks=None, rand_block=128):
         """``local_bias``: optional [Hq, 2R+1] table added to window keys of non-global
-        rows at column (j - i) + R (R inferred from the table width)."""
+        rows at column (j - i) + R (R inferred from the table width).
+        ``rand_blocks``: optional int [B, Hq, ceil(n / rand_block), r] random key
+        blocks of each query block (non-global rows attend their keys too)."""
         self.q, self.k, self.v = _f32(q), _f32(k), _f32(v)
         self.B, self.Hq, self.n, self.D = self.q.shape
         self.Hkv = self.k.shape[1]
@@ -132,6 +157,16 @@ class Problem:
             if self.local_bias.shape != (self.Hq, width) or width % 2 == 0:
                 raise ValueError("local_bias must be [Hq, 2R+1]")
             self.local_radius = (width - 1) // 2
+        self.rand_blocks = _i32(rand_blocks)
+        self.rand_block = int(rand_block)
+        if self.rand_blocks is not None:
+            nqb = (self.n + self.rand_block - 1) // self.rand_block
+            if self.rand_blocks.ndim != 4 or self.rand_blocks.shape[:3] != (self.B, self.Hq, nqb):
+                raise ValueError("rand_blocks must be [B, Hq, ceil(n / rand_block), r]")
+
+    def _ex(self):
+        self._exk = _extras(self.local_bias, self.local_radius, self.rand_blocks, self.rand_block)
+        return ctypes.byref(self._exk)
 
     def _common(self):
         return (self.B, self.Hq, self.Hkv, self.n, self.D, _ptr(self.q), _ptr(self.k), _ptr(self.v),
@@ -157,7 +192,7 @@ class Problem:
         lse = np.empty(total, dtype=np.float64)
         cnt = np.empty(total, dtype=np.int64)
         _check(lib.oracle_forward_ex(*self._common(), rp, total, _ptr(out), _ptr(lse), _ptr(cnt),
-                                     _ptr(self.local_bias), self.local_radius), "forward")
+                                     self._ex()), "forward")
         if rows is None:
             return (out.reshape(self.B, self.Hq, self.n, self.D), lse.reshape(self.B, self.Hq, self.n),
                     cnt.reshape(self.B, self.Hq, self.n))
@@ -167,36 +202,41 @@ class Problem:
         lib = _load()
         out = np.empty((self.B, self.Hq, self.n, self.D), dtype=np.float64)
         lse = np.empty((self.B, self.Hq, self.n), dtype=np.float64)
-        _check(lib.oracle_dense_bruteforce_ex(*self._common(), _ptr(out), _ptr(lse),
-                                              _ptr(self.local_bias), self.local_radius), "dense")
+        _check(lib.oracle_dense_bruteforce_ex(*self._common(), _ptr(out), _ptr(lse), self._ex()),
+               "dense")
         return out, lse
 
 
 def key_counts(B, Hq, n, *, window, dilation=1, causal=False, global_idx=None, S=0,
-               valid_len=None):
+               valid_len=None, rand_blocks=None, rand_block=128):
     """|K(i)| + S per row, [B,Hq,n] int64 (0 for padded rows)."""
     lib = _load()
     gi = _i32(global_idx)
     g = 0 if gi is None else int(gi.shape[-1])
     vl = _i32(valid_len)
+    rb = _i32(rand_blocks)
     cnt = np.empty((B, Hq, n), dtype=np.int64)
-    _check(lib.oracle_key_counts(B, Hq, n, _ptr(gi) if g else None, g, S,
-                                 _ptr(_per_head(window, Hq)), _ptr(_per_head(dilation, Hq)),
-                                 int(bool(causal)), _ptr(vl), _ptr(cnt)), "key_counts")
+    ex = _extras(rand_blocks=rb, rand_block=rand_block)
+    _check(lib.oracle_key_counts_ex(B, Hq, n, _ptr(gi) if g else None, g, S,
+                                    _ptr(_per_head(window, Hq)), _ptr(_per_head(dilation, Hq)),
+                                    int(bool(causal)), _ptr(vl), _ptr(cnt), ctypes.byref(ex)),
+           "key_counts")
     return cnt
 
 
 def key_list(B, Hq, n, b, h, i, *, window, dilation=1, causal=False, global_idx=None,
-             valid_len=None):
+             valid_len=None, rand_blocks=None, rand_block=128):
     """The explicit key set K(i) (ascending, no side keys) of one row."""
     lib = _load()
     gi = _i32(global_idx)
     g = 0 if gi is None else int(gi.shape[-1])
     vl = _i32(valid_len)
+    rb = _i32(rand_blocks)
     keys = np.empty(max(n, 1), dtype=np.int32)
     w, d = _per_head(window, Hq), _per_head(dilation, Hq)
-    nk = lib.oracle_key_list(B, Hq, n, _ptr(gi) if g else None, g, _ptr(w), _ptr(d),
-                             int(bool(causal)), _ptr(vl), b, h, i, _ptr(keys))
+    ex = _extras(rand_blocks=rb, rand_block=rand_block)
+    nk = lib.oracle_key_list_ex(B, Hq, n, _ptr(gi) if g else None, g, _ptr(w), _ptr(d),
+                                int(bool(causal)), _ptr(vl), b, h, i, _ptr(keys), ctypes.byref(ex))
     if nk < 0:
         raise MemoryError("oracle key_list")
     return keys[:nk].copy()

@@ -34,6 +34,10 @@
  *   [LT5-LOCAL] LongT5 guide, "相对位置编码" section: the local attention adds a
  *               relative-position bias bucketed on memory_position -
  *               query_position, computed once over the local window.
+ *   [BB-3.2.2]  "精读笔记：Big Bird" §3.2.2: every query also attends to r
+ *               randomly chosen keys.  Here the random keys come in blocks: the
+ *               rows of query block q = floor(i / bs) share rand_blocks[b][h][q][:],
+ *               each naming a block of bs consecutive keys (the draws are inputs).
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *   window bounds inclusive (2r+1 keys, non-causal); causal window t in [-r,0];
@@ -74,7 +78,30 @@ typedef struct {
     double scale;
     const float *local_bias;   /* [Hq, 2R+1] or NULL: bias of window keys by j - i */
     int local_radius;          /* R */
+    const int32_t *rand_blocks; /* [B, Hq, ceil(n / bs), num_rand] or NULL */
+    int num_rand;
+    int rand_block;            /* bs */
 } oracle_problem;
+
+/* Optional terms of the score and the key set, passed by pointer (NULL: none). */
+typedef struct {
+    const float *local_bias;
+    int local_radius;
+    const int32_t *rand_blocks;
+    int num_rand;
+    int rand_block;
+} oracle_extras;
+
+static void apply_extras(oracle_problem *P, const oracle_extras *ex) {
+    if (!ex) return;
+    P->local_bias = ex->local_bias;
+    P->local_radius = ex->local_radius;
+    if (ex->rand_blocks && ex->num_rand > 0 && ex->rand_block > 0) {
+        P->rand_blocks = ex->rand_blocks;
+        P->num_rand = ex->num_rand;
+        P->rand_block = ex->rand_block;
+    }
+}
 
 static int num_blocks(int n, int kb) { return kb > 0 ? (n + kb - 1) / kb : 0; }
 
@@ -87,13 +114,15 @@ static int is_global(const oracle_problem *P, int b, int i) {
 
 /*
  * The explicit key set K(i) of one query row, in increasing key order, without
- * duplicates [BB-3.2.1, BB-3.2.3, LF-2, SWAN-3.3]:
+ * duplicates [BB-3.2.1, BB-3.2.2, BB-3.2.3, LF-2, SWAN-3.3]:
  *   i >= V            -> empty (padded query row)
  *   i global          -> {0, .., V-1}
- *   otherwise         -> W(i) U G, W(i) = {i + d t : -r <= t <= r (t <= 0 if
- *                        causal), 0 <= i + d t < V}
- * The union is formed by merging the two ascending lists and dropping repeats.
- * Returns the number of keys written to keys[] (capacity n).
+ *   otherwise         -> W(i) U G U R(i), W(i) = {i + d t : -r <= t <= r (t <= 0
+ *                        if causal), 0 <= i + d t < V}, R(i) = the keys below V
+ *                        of the random blocks of i's query block
+ * W and G are merged as two ascending lists with repeats dropped; random blocks,
+ * when present, are added through a mark per key.  Returns the number of keys
+ * written to keys[] (capacity n).
  */
 static int key_set(const oracle_problem *P, int b, int h, int i, int32_t *keys,
                    int32_t *wbuf) {
@@ -122,6 +151,24 @@ static int key_set(const oracle_problem *P, int b, int h, int i, int32_t *keys,
             if (next >= V) continue; /* never attend a padded key */
         }
         if (m == 0 || keys[m - 1] != next) keys[m++] = next;
+    }
+    if (P->rand_blocks) {
+        unsigned char *mark = (unsigned char *)calloc((size_t)V + 1, 1);
+        if (!mark) return -1;
+        for (int t = 0; t < m; ++t) mark[keys[t]] = 1;
+        const int bs = P->rand_block;
+        const int nqb = (P->n + bs - 1) / bs;
+        const int32_t *rb = P->rand_blocks + (((int64_t)b * P->Hq + h) * nqb + i / bs) * P->num_rand;
+        for (int t = 0; t < P->num_rand; ++t) {
+            int64_t lo = (int64_t)rb[t] * bs, hi = lo + bs;
+            if (lo < 0) lo = 0;
+            if (hi > V) hi = V;
+            for (int64_t j = lo; j < hi; ++j) mark[j] = 1;
+        }
+        m = 0;
+        for (int j = 0; j < V; ++j)
+            if (mark[j]) keys[m++] = j;
+        free(mark);
     }
     return m;
 }
@@ -220,6 +267,11 @@ static void attend_row(const oracle_problem *P, int b, int h, int i,
 }
 
 static int check_problem(const oracle_problem *P) {
+    if (P->rand_blocks) {
+        const int nqb = (P->n + P->rand_block - 1) / P->rand_block;
+        for (int64_t t = 0; t < (int64_t)P->B * P->Hq * nqb * P->num_rand; ++t)
+            if (P->rand_blocks[t] < 0 || P->rand_blocks[t] >= nqb) return ORACLE_EINVAL;
+    }
     if (P->B <= 0 || P->Hq <= 0 || P->Hkv <= 0 || P->n < 0 || P->D <= 0) return ORACLE_EINVAL;
     if (P->Hq % P->Hkv) return ORACLE_EINVAL;
     if (!P->q || !P->k || !P->v || !P->window || !P->dilation) return ORACLE_EINVAL;
@@ -249,10 +301,11 @@ int oracle_forward_ex(int B, int Hq, int Hkv, int n, int D, const float *q, cons
                       const int32_t *window, const int32_t *dilation, int causal,
                       const int32_t *valid_len, double scale, const int64_t *rows,
                       int64_t nrows, double *out, double *lse, int64_t *count,
-                      const float *local_bias_tab, int local_radius) {
+                      const oracle_extras *ex) {
     oracle_problem P = {B, Hq, Hkv, n, D, q, k, v, global_idx, g, side_k, side_v,
                         S, side_block, bias, window, dilation, causal, valid_len, scale,
-                        local_bias_tab, local_radius};
+                        NULL, 0, NULL, 0, 0};
+    apply_extras(&P, ex);
     int rc = check_problem(&P);
     if (rc) return rc;
     int64_t total = rows ? nrows : (int64_t)B * Hq * n;
@@ -273,6 +326,11 @@ int oracle_forward_ex(int B, int Hq, int Hkv, int n, int D, const float *q, cons
                 int h = (int)((id / n) % Hq);
                 int b = (int)(id / ((int64_t)n * Hq));
                 int nk = key_set(&P, b, h, i, keys, wbuf);
+                if (nk < 0) {
+#pragma omp atomic write
+                    failed = 1;
+                    nk = 0;
+                }
                 int Vb = valid_len ? valid_len[b] : n;
                 attend_row(&P, b, h, i, keys, nk, scores, out + t * D, lse + t);
                 if (count) count[t] = (i < Vb) ? (int64_t)nk + S : 0;
@@ -293,20 +351,21 @@ int oracle_forward(int B, int Hq, int Hkv, int n, int D, const float *q, const f
                    int64_t nrows, double *out, double *lse, int64_t *count) {
     return oracle_forward_ex(B, Hq, Hkv, n, D, q, k, v, global_idx, g, side_k, side_v, S, side_block,
                              bias, window, dilation, causal, valid_len, scale, rows, nrows, out, lse,
-                             count, NULL, 0);
+                             count, NULL);
 }
 
 /*
  * oracle_key_counts: |K(i)| + S for every row (flat order), without touching
  * q/k/v -- the attended-pair count that defines the useful FLOPs 4*D*pairs.
  */
-int oracle_key_counts(int B, int Hq, int n, const int32_t *global_idx, int g, int S,
-                      const int32_t *window, const int32_t *dilation, int causal,
-                      const int32_t *valid_len, int64_t *count) {
+int oracle_key_counts_ex(int B, int Hq, int n, const int32_t *global_idx, int g, int S,
+                         const int32_t *window, const int32_t *dilation, int causal,
+                         const int32_t *valid_len, int64_t *count, const oracle_extras *ex) {
     oracle_problem P;
     memset(&P, 0, sizeof(P));
     P.B = B; P.Hq = Hq; P.Hkv = Hq; P.n = n; P.D = 1; P.global_idx = global_idx; P.g = g;
     P.S = S; P.window = window; P.dilation = dilation; P.causal = causal; P.valid_len = valid_len;
+    apply_extras(&P, ex);
     int failed = 0;
 #pragma omp parallel
     {
@@ -323,6 +382,11 @@ int oracle_key_counts(int B, int Hq, int n, const int32_t *global_idx, int g, in
                 int b = (int)(t / ((int64_t)n * Hq));
                 int Vb = valid_len ? valid_len[b] : n;
                 int nk = key_set(&P, b, h, i, keys, wbuf);
+                if (nk < 0) {
+#pragma omp atomic write
+                    failed = 1;
+                    nk = 0;
+                }
                 count[t] = (i < Vb) ? (int64_t)nk + S : 0;
             }
         }
@@ -332,22 +396,38 @@ int oracle_key_counts(int B, int Hq, int n, const int32_t *global_idx, int g, in
     return failed ? ORACLE_ENOMEM : ORACLE_OK;
 }
 
+int oracle_key_counts(int B, int Hq, int n, const int32_t *global_idx, int g, int S,
+                      const int32_t *window, const int32_t *dilation, int causal,
+                      const int32_t *valid_len, int64_t *count) {
+    return oracle_key_counts_ex(B, Hq, n, global_idx, g, S, window, dilation, causal, valid_len,
+                                count, NULL);
+}
+
 /*
  * oracle_key_list: the explicit key set K(i) of one row (no side keys), for
  * support checks.  Returns the count; keys[] must hold n entries.
  */
-int oracle_key_list(int B, int Hq, int n, const int32_t *global_idx, int g,
-                    const int32_t *window, const int32_t *dilation, int causal,
-                    const int32_t *valid_len, int b, int h, int i, int32_t *keys) {
+int oracle_key_list_ex(int B, int Hq, int n, const int32_t *global_idx, int g,
+                       const int32_t *window, const int32_t *dilation, int causal,
+                       const int32_t *valid_len, int b, int h, int i, int32_t *keys,
+                       const oracle_extras *ex) {
     oracle_problem P;
     memset(&P, 0, sizeof(P));
     P.B = B; P.Hq = Hq; P.Hkv = Hq; P.n = n; P.D = 1; P.global_idx = global_idx; P.g = g;
     P.window = window; P.dilation = dilation; P.causal = causal; P.valid_len = valid_len;
+    apply_extras(&P, ex);
     int32_t *wbuf = (int32_t *)malloc(sizeof(int32_t) * (size_t)(n + 1));
     if (!wbuf) return -1;
     int nk = key_set(&P, b, h, i, keys, wbuf);
     free(wbuf);
     return nk;
+}
+
+int oracle_key_list(int B, int Hq, int n, const int32_t *global_idx, int g,
+                    const int32_t *window, const int32_t *dilation, int causal,
+                    const int32_t *valid_len, int b, int h, int i, int32_t *keys) {
+    return oracle_key_list_ex(B, Hq, n, global_idx, g, window, dilation, causal, valid_len, b, h,
+                              i, keys, NULL);
 }
 
 /*
@@ -356,7 +436,8 @@ int oracle_key_list(int B, int Hq, int n, const int32_t *global_idx, int g,
  * matrix from the closed form
  *   non-causal: |i-j| <= r d  and  (i-j) mod d == 0
  *   causal:     0 <= i-j <= r d  and  (i-j) mod d == 0
- *   OR j global OR i global;   AND i < V AND j < V,
+ *   OR j global OR i global OR floor(j / bs) is a random block of floor(i / bs);
+ *   AND i < V AND j < V,
  * appends every side column for valid rows, and runs a dense masked softmax
  * over all n + S columns.  Every row is written (flat order).
  */
@@ -365,8 +446,13 @@ int oracle_dense_bruteforce_ex(int B, int Hq, int Hkv, int n, int D, const float
                                const float *side_k, const float *side_v, int S, int side_block,
                                const float *bias, const int32_t *window, const int32_t *dilation,
                                int causal, const int32_t *valid_len, double scale, double *out,
-                               double *lse, const float *local_bias_tab, int local_radius) {
+                               double *lse, const oracle_extras *ex) {
+    const float *local_bias_tab = ex ? ex->local_bias : NULL;
+    const int local_radius = ex ? ex->local_radius : 0;
+    const int32_t *rblk = (ex && ex->rand_blocks && ex->num_rand > 0) ? ex->rand_blocks : NULL;
+    const int nrand = rblk ? ex->num_rand : 0, bs = rblk ? ex->rand_block : 1;
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || n < 0) return ORACLE_EINVAL;
+    if (rblk && bs <= 0) return ORACLE_EINVAL;
     if (local_bias_tab) {
         for (int h = 0; h < Hq; ++h) {
             int64_t reach = (int64_t)window[h] * dilation[h];
@@ -400,7 +486,10 @@ int oracle_dense_bruteforce_ex(int B, int Hq, int Hkv, int n, int D, const float
                     int64_t diff = (int64_t)i - j;
                     int band = causal ? (diff >= 0 && diff <= rd) : (llabs(diff) <= rd);
                     band = band && (diff % dilation[h] == 0);
-                    int a = (band || isg[j] || isg[i]) && i < V && j < V;
+                    int rnd = 0;
+                    for (int t = 0; t < nrand; ++t)
+                        rnd |= (j / bs == rblk[(((int64_t)b * Hq + h) * ((n + bs - 1) / bs) + i / bs) * nrand + t]);
+                    int a = (band || isg[j] || isg[i] || rnd) && i < V && j < V;
                     inband[j] = (unsigned char)(band && !isg[i]);
                     allow[j] = (unsigned char)a;
                     any |= a;
@@ -463,7 +552,7 @@ int oracle_dense_bruteforce(int B, int Hq, int Hkv, int n, int D, const float *q
                             double *lse) {
     return oracle_dense_bruteforce_ex(B, Hq, Hkv, n, D, q, k, v, global_idx, g, side_k, side_v, S,
                                       side_block, bias, window, dilation, causal, valid_len, scale,
-                                      out, lse, NULL, 0);
+                                      out, lse, NULL);
 }
 
 /*

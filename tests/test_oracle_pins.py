@@ -433,3 +433,86 @@ def test_expand_local_bias_columns(oracle_mod):
     assert out[1, R - 1] == 32 + 1
     assert out[0, R + 7] == 16 + 7 and out[0, R + 8] == 16 + 8
     assert out[0, 0] == 15 and out[0, 2 * R] == 31
+
+
+# --- BigBird random key blocks (精读笔记：Big Bird §3.2.2) ------------------------------
+
+
+def _rand_blocks(rng, B, Hq, n, bs, r):
+    nqb = (n + bs - 1) // bs
+    return rng.integers(0, nqb, size=(B, Hq, nqb, r)).astype(np.int32)   # repeats allowed
+
+
+def test_random_blocks_match_dense_bruteforce_grid(oracle_mod):
+    """Per-row key sets with random blocks (repeats, overlaps with the window, globals
+    and padding included) against the dense mask that adds them by block membership."""
+    rng = np.random.default_rng(53)
+    cases = 0
+    for n in (5, 16, 29, 40):
+        for r, d, g, pad, nr, bs in itertools.product((0, 1, 3), (1, 2), (0, 2), (0, 3), (1, 3),
+                                                     (4, 7)):
+            if rng.random() > 0.3:
+                continue
+            S = int(rng.integers(0, 2)) * 2
+            p = _problem(oracle_mod, rng, 2, 2, 2, n, 8, r, d, 0, g, pad, S=S, kb=4, bias=bool(S))
+            rb = _rand_blocks(rng, 2, 2, n, bs, nr)
+            pr = oracle_mod.Problem(p.q, p.k, p.v, window=r, dilation=d, global_idx=p.global_idx,
+                                    side_k=p.side_k, side_v=p.side_v, side_block=4, bias=p.bias,
+                                    valid_len=p.valid_len, rand_blocks=rb, rand_block=bs)
+            o, lse, _ = pr.forward()
+            od, lsed = pr.dense_bruteforce()
+            assert np.max(np.abs(o - od)) <= 1e-12
+            _assert_close_lse(lse, lsed, 1e-12)
+            cases += 1
+    assert cases > 40
+
+
+def test_random_block_key_list_is_the_set_union(oracle_mod):
+    """K(i) = W(i) U G U (keys of the row's random blocks below V), as a set."""
+    rng = np.random.default_rng(59)
+    B, H, n, bs, nr, r = 2, 3, 50, 8, 3, 4
+    V = 45
+    gl = np.array([[3, 20], [0, 44]], np.int32)
+    rb = _rand_blocks(rng, B, H, n, bs, nr)
+    vl = np.array([V, V], np.int32)
+    for b in range(B):
+        for h in range(H):
+            for i in range(V):
+                got = oracle_mod.key_list(B, H, n, b, h, i, window=r, global_idx=gl, valid_len=vl,
+                                          rand_blocks=rb, rand_block=bs)
+                if i in gl[b]:
+                    want = set(range(V))
+                else:
+                    want = {j for j in range(i - r, i + r + 1) if 0 <= j < V} | set(gl[b].tolist())
+                    for blk in rb[b, h, i // bs]:
+                        want |= {j for j in range(blk * bs, blk * bs + bs) if j < V}
+                assert got.tolist() == sorted(want)
+
+
+def test_random_blocks_covering_everything_give_full_attention(oracle_mod):
+    """When the random blocks of every query block cover the whole sequence, every row
+    is a full-attention row (softmax over all valid keys, from torch)."""
+    rng = np.random.default_rng(61)
+    B, H, n, D, bs = 1, 2, 24, 8, 8
+    q, k, v = (_rand((B, H, n, D), rng) for _ in range(3))
+    rb = np.broadcast_to(np.arange(3, dtype=np.int32), (B, H, 3, 3)).copy()
+    o, lse, cnt = oracle_mod.Problem(q, k, v, window=1, rand_blocks=rb, rand_block=bs).forward()
+    s = torch.from_numpy(q).double() @ torch.from_numpy(k).double().transpose(-1, -2) / math.sqrt(D)
+    ref = torch.softmax(s, -1) @ torch.from_numpy(v).double()
+    assert np.max(np.abs(o - ref.numpy())) <= 1e-12
+    assert np.all(cnt == n)
+
+
+def test_random_blocks_zero_query_mean_over_key_set(oracle_mod):
+    """q = 0: o_i is the plain mean of V over |W U G U R| keys (a cardinality check)."""
+    rng = np.random.default_rng(67)
+    B, H, n, D, bs, r = 1, 1, 40, 4, 8, 2
+    q = np.zeros((B, H, n, D), np.float32)
+    k, v = _rand((B, H, n, D), rng), _rand((B, H, n, D), rng)
+    rb = _rand_blocks(rng, B, H, n, bs, 2)
+    p = oracle_mod.Problem(q, k, v, window=r, rand_blocks=rb, rand_block=bs)
+    o, _, cnt = p.forward()
+    for i in range(n):
+        keys = oracle_mod.key_list(B, H, n, 0, 0, i, window=r, rand_blocks=rb, rand_block=bs)
+        assert len(keys) == cnt[0, 0, i]
+        assert np.max(np.abs(o[0, 0, i] - v[0, 0, keys].astype(np.float64).mean(0))) <= 1e-12
