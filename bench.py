@@ -155,7 +155,7 @@ def prepare(w, device):
     inp = workloads.make_inputs(w)
     host = {k: v for k, v in inp.items()}
     dev = {}
-    for k in ("q", "k", "v", "global_idx", "valid_len"):
+    for k in ("q", "k", "v", "global_idx", "valid_len", "rand_blocks"):
         dev[k] = inp[k].to(device) if inp[k] is not None else None
     if w.side_block:
         dev["side_k"] = side_aggregate(dev["k"], w.side_block, dev["valid_len"])
@@ -180,8 +180,9 @@ def count_flops(w, host):
     from sliding_window_global_b200 import flops
     gl = host["global_idx"].numpy() if host["global_idx"] is not None else None
     vl = host["valid_len"].numpy() if host["valid_len"] is not None else None
+    rb = host["rand_blocks"].numpy() if host.get("rand_blocks") is not None else None
     pairs = flops.attended_pairs(w.seq_len, w.window, w.dilation, w.causal, gl, vl, w.batch,
-                                 w.num_side)
+                                 w.num_side, rb)
     return pairs, flops.useful_flops(pairs, w.head_dim)
 
 
@@ -191,7 +192,8 @@ def time_device(w, plan, dev, steps, warmup, device):
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
     kw = dict(window=list(w.window), dilation=list(w.dilation), causal=w.causal,
               global_idx=dev["global_idx"], side_k=dev.get("side_k"), side_v=dev.get("side_v"),
-              bias=dev.get("bias"), valid_len=dev["valid_len"], local_bias=dev.get("local_bias"))
+              bias=dev.get("bias"), valid_len=dev["valid_len"], local_bias=dev.get("local_bias"),
+              rand_blocks=dev.get("rand_blocks"))
     out = torch.empty((w.batch, w.q_heads, w.seq_len, w.head_dim), dtype=w.torch_dtype, device=device)
     lse = torch.empty((w.batch, w.q_heads, w.seq_len), dtype=torch.float32, device=device)
     for _ in range(warmup):
@@ -223,8 +225,8 @@ def time_e2e(w, plan, host, steps, warmup, device):
     import torch
 
     from sliding_window_global_b200 import side_aggregate
-    names = [k for k in ("q", "k", "v", "global_idx", "valid_len", "bias", "local_bias")
-             if host.get(k) is not None]
+    names = [k for k in ("q", "k", "v", "global_idx", "valid_len", "bias", "local_bias",
+                         "rand_blocks") if host.get(k) is not None]
     pinned = {k: host[k].contiguous().pin_memory() for k in names}
     dev = {k: torch.empty_like(pinned[k], device=device) for k in names}
     out_h = torch.empty((w.batch, w.q_heads, w.seq_len, w.head_dim), dtype=w.torch_dtype).pin_memory()
@@ -243,7 +245,7 @@ def time_e2e(w, plan, host, steps, warmup, device):
                                 dilation=list(w.dilation), causal=w.causal,
                                 global_idx=dev.get("global_idx"), side_k=sk, side_v=sv,
                                 bias=dev.get("bias"), valid_len=dev.get("valid_len"),
-                                local_bias=dev.get("local_bias"))
+                                local_bias=dev.get("local_bias"), rand_blocks=dev.get("rand_blocks"))
         out_h.copy_(out, non_blocking=True)
         lse_h.copy_(lse, non_blocking=True)
 
@@ -278,7 +280,8 @@ def cpu_baseline(w, host, budget_s=12.0):
                           global_idx=inp["global_idx"], side_k=inp.get("side_k"),
                           side_v=inp.get("side_v"), side_block=w.side_block or 16,
                           bias=inp.get("bias"), valid_len=inp["valid_len"], scale=inp["scale"],
-                          local_bias=inp.get("local_bias"))
+                          local_bias=inp.get("local_bias"), rand_blocks=inp.get("rand_blocks"),
+                          rand_block=128)
     rng = np.random.default_rng(0)
     total_rows = w.batch * w.q_heads * w.seq_len
     rows = np.sort(rng.choice(total_rows, min(total_rows, 2000), replace=False))
@@ -432,7 +435,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="swan_swa")
-    ap.add_argument("--secondary", default="longt5_tglobal,longt5_local",
+    ap.add_argument("--secondary", default="longt5_tglobal,longt5_local,bigbird_itc",
                     help="comma-separated workloads timed after the main one (device time only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -125,7 +125,19 @@ swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void
  *   head (else SWA_ERR_INVALID_ARG).  The bf16 kernels stage the bias rows of a
  *   work unit in shared memory, which limits min(window[h], ceil(seq_len /
  *   dilation[h])) to 766; larger windows with a local bias return
- *   SWA_ERR_UNSUPPORTED.  Use swa_bucket_local_bias to expand a 32-bucket table. */
+ *   SWA_ERR_UNSUPPORTED.  Use swa_bucket_local_bias to expand a 32-bucket table.
+ *
+ * rand_blocks, num_rand: BigBird random attention ("精读笔记：Big Bird" §3.2.2:
+ *   every query also attends to r randomly chosen keys), in blocks of 128 keys.
+ *   Device [B, Hq, ceil(seq_len / 128), num_rand] int32, 4-byte aligned: the
+ *   rows of query block q = floor(i / 128) of head h add the keys of blocks
+ *   rand_blocks[b][h][q][:] (keys 128*blk .. 128*blk + 127 below valid_len) to
+ *   their key set, as a set: keys already in the window or global, and repeated
+ *   blocks, count once.  Global query rows are unaffected (they attend every
+ *   key).  The caller draws the blocks.  0 <= num_rand <= 8; block indices must
+ *   lie in [0, ceil(seq_len / 128)) (not checked; an index outside attends
+ *   nothing).  Random blocks need dilation 1 on every head and causal == 0
+ *   (else SWA_ERR_UNSUPPORTED). */
 typedef struct {
   const void* q;
   const void* k;
@@ -143,6 +155,8 @@ typedef struct {
   float* lse;
   const float* local_bias;     /* device [Hq, 2 * local_radius + 1] fp32, or NULL */
   int local_radius;
+  const int32_t* rand_blocks;  /* device [B, Hq, ceil(n / 128), num_rand] int32, or NULL */
+  int num_rand;
 } swa_forward_args;
 
 /* swa_forward with the arguments in a struct (same statuses, same launches). */

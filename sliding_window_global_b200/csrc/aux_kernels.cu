@@ -133,7 +133,13 @@ __global__ void simt_attn_kernel(AttnParams p, const T* __restrict__ q, const T*
   int t_hi = p.causal ? 0 : min(r, (V - 1 - i) / d);
   const int nwin = is_global ? V : (t_hi - t_lo + 1);
   const int ngl = is_global ? 0 : p.g;
-  const int total = nwin + ngl + p.S;
+  // random key blocks of the row's query block (non-global rows)
+  const int nqb = (p.n + kTile - 1) / kTile;
+  const int32_t* rbp = (!is_global && p.rand_blocks)
+                           ? p.rand_blocks + (((size_t)b * p.Hq + h) * nqb + i / kTile) * p.num_rand
+                           : nullptr;
+  const int nrnd = rbp ? p.num_rand * kTile : 0;
+  const int total = nwin + ngl + p.S + nrnd;
   const T* kb = k + ((size_t)b * p.Hkv + hk) * p.n * D;
   const T* vb = v + ((size_t)b * p.Hkv + hk) * p.n * D;
   const T* skb = p.S ? side_k + ((size_t)b * p.Hkv + hk) * p.S * D : nullptr;
@@ -165,11 +171,28 @@ __global__ void simt_attn_kernel(AttnParams p, const T* __restrict__ q, const T*
         krow = kb + (size_t)j * D;
         vrow = vb + (size_t)j * D;
       }
-    } else if (idx < total) {
+    } else if (idx < nwin + ngl + p.S) {
       int sg = idx - nwin - ngl;
       krow = skb + (size_t)sg * D;
       vrow = svb + (size_t)sg * D;
       if (p.bias) bb = p.bias[(size_t)h * (p.S + p.nblk - 1) + sg - qblk + p.nblk - 1];
+    } else if (idx < total) {
+      // key e of random block t: counted unless it is padded, in the window, global,
+      // or in a block repeated earlier in the list
+      const int rr = idx - nwin - ngl - p.S;
+      const int t = rr / kTile;
+      const int blk = rbp[t];
+      const int j = blk * kTile + rr % kTile;
+      bool take = blk >= 0 && blk < nqb && j < V;
+      const int diff = i - j;
+      const bool inwin = (p.causal ? (diff >= 0 && diff <= r * d) : (abs(diff) <= r * d)) && (diff % d == 0);
+      take = take && !inwin;
+      for (int u = 0; take && u < p.g; ++u) take = gl[u] != j;
+      for (int t2 = 0; take && t2 < t; ++t2) take = rbp[t2] != blk;
+      if (take) {
+        krow = kb + (size_t)j * D;
+        vrow = vb + (size_t)j * D;
+      }
     }
     if (krow) {
       float dotv = 0.f;

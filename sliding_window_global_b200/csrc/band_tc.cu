@@ -12,7 +12,10 @@
 //                   minus those already inside its window (BigBird §3.2.3, ITC);
 //   side tiles   -- appended side keys with the additive bucketed bias of the
 //                   LongT5 Transient-Global attention ("LongT5 长序列模型完全指南",
-//                   Transient-Global and 源码级证据 sections).
+//                   Transient-Global and 源码级证据 sections);
+//   random tiles -- the random key blocks of each query tile (BigBird §3.2.2:
+//                   every query also attends to randomly chosen keys), minus keys
+//                   inside the row's window; only the tile they belong to uses them.
 // Band tiles may carry a local relative-position bias indexed by key - query
 // offset (the LongT5 page, 相对位置编码: the local attention's bias is computed
 // once over the window); its row for the unit's head is staged in shared memory.
@@ -106,6 +109,8 @@ struct Work {
   bool active[2];
   int band_lo;          // first key of band tile 0
   int nband, ngc, nside, total;
+  int rand0;            // first random tile: rand0 .. rand0+nrand-1 (tile A), then tile B's
+  int nrand[2];         // random tiles of tile A, B
   int key_end;          // MODE 1: keys at or beyond this are masked
   int lo[2], hi[2];     // band key range of each query tile (class coordinates)
 };
@@ -116,7 +121,7 @@ __device__ __forceinline__ int total_units(const AttnParams& p) {
                    : p.nsplit * (p.gpad / kTile) * p.B * p.Hq;
 }
 
-template <int MODE>
+template <int MODE, bool RAND>
 __device__ __forceinline__ void decode_work(const AttnParams& p, int unit_id, Work& w) {
   if (MODE == 0) {
     // unit ids run over (unit, batch, head or head pair), heads fastest
@@ -208,12 +213,22 @@ __device__ __forceinline__ void decode_work(const AttnParams& p, int unit_id, Wo
     w.hi[0] = w.key_end;
     w.lo[1] = w.hi[1] = 0;
   }
-  w.total = w.nband + w.ngc + w.nside;
+  w.rand0 = w.nband + w.ngc + w.nside;
+  w.nrand[0] = (RAND && MODE == 0 && w.active[0]) ? p.num_rand : 0;
+  w.nrand[1] = (RAND && MODE == 0 && w.active[1]) ? p.num_rand : 0;
+  w.total = w.rand0 + w.nrand[0] + w.nrand[1];
+}
+
+// Random key block t of query tile x (query block u0 / kTile; dilation 1 only).
+__device__ __forceinline__ int rand_block(const AttnParams& p, int b, int head, int u0, int t) {
+  const int nqb = (p.n + kTile - 1) / kTile;
+  return __ldg(p.rand_blocks + (((size_t)b * p.Hq + head) * nqb + u0 / kTile) * p.num_rand + t);
 }
 
 // Does query tile x use key tile j?
 __device__ __forceinline__ bool uses(const Work& w, int x, int j) {
   if (!w.active[x] || j < 0 || j >= w.total) return false;
+  if (j >= w.rand0) return (j < w.rand0 + w.nrand[0]) == (x == 0);   // a tile's own random blocks
   if (j >= w.nband) return true;                        // global and side tiles: every row
   const int kv0 = w.band_lo + j * kTile;
   return kv0 < w.hi[x] && kv0 + kTile > w.lo[x];
@@ -239,8 +254,9 @@ __device__ __forceinline__ TileRows tile_rows(const Work& w, int x) {
   return t;
 }
 
-__device__ __forceinline__ bool uses(const Work& w, const TileRows& t, int j) {
+__device__ __forceinline__ bool uses(const Work& w, const TileRows& t, int x, int j) {
   if (!t.active || j < 0 || j >= w.total) return false;
+  if (j >= w.rand0) return (j < w.rand0 + w.nrand[0]) == (x == 0);
   if (j >= w.nband) return true;
   const int kv0 = w.band_lo + j * kTile;
   return kv0 < t.hi && kv0 + kTile > t.lo;
@@ -257,10 +273,17 @@ __device__ __forceinline__ void tile_source(const AttnParams& p, const Work& w, 
     mk = &p.mgk;
     mv = &p.mgv;
     y = (j - w.nband) * kTile;
-  } else {
+  } else if (j < w.rand0) {
     mk = &p.msk;
     mv = &p.msv;
     y = (j - w.nband - w.ngc) * kTile;
+  } else {
+    // random key block (dilation 1: the class map is the plain key sequence)
+    const int x = (j < w.rand0 + w.nrand[0]) ? 0 : 1;
+    const int t = j - w.rand0 - (x ? w.nrand[0] : 0);
+    mk = &p.mk[w.cls];
+    mv = &p.mv[w.cls];
+    y = rand_block(p, w.b, x ? w.hx[1] : w.hx[0], x ? w.u0[1] : w.u0[0], t) * kTile;
   }
 }
 
@@ -355,9 +378,10 @@ __device__ void write_neutral_partial(const AttnParams& p, const Work& w, int ro
   p.part_lse[prow] = -INFINITY;
 }
 
-// LOCAL: band tiles carry the local relative-position bias (MODE 0 only).  It is a
-// template parameter so that kernels without it keep their register schedule.
-template <int D, int MODE, bool LOCAL>
+// LOCAL: band tiles carry the local relative-position bias; RAND: query tiles have
+// random key blocks (MODE 0 only).  They are template parameters so that kernels
+// without them keep their register schedule.
+template <int D, int MODE, bool LOCAL, bool RAND>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ AttnParams p) {
   using C = Cfg<D>;
   constexpr int NS = C::NS;
@@ -434,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       bool ok = true;
       for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
         Work w;
-        decode_work<MODE>(p, uid, w);
+        decode_work<MODE, RAND>(p, uid, w);
         if (!w.active[0]) continue;
         const CUtensorMap* mq = (MODE == 0) ? &p.mq[w.cls] : &p.mgq;
         const int kz = w.b * p.Hkv + w.hk;
@@ -485,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       bool ok = true;
       for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
         Work w;
-        decode_work<MODE>(p, uid, w);
+        decode_work<MODE, RAND>(p, uid, w);
         if (!w.active[0]) continue;
         const int T = w.total;
         int first[2] = {-1, -1}, last[2] = {-1, -1}, issued[2] = {-1, -1}, npv[2] = {0, 0};
@@ -590,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     bool ok = true;
     for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
       Work w;
-      decode_work<MODE>(p, uid, w);
+      decode_work<MODE, RAND>(p, uid, w);
       if (!w.valid) continue;
       const TileRows tr = tile_rows(w, x);
       if (!w.active[0]) {
@@ -674,6 +698,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
 
       const int rd = w.r * w.d;
+      // random key blocks of this query tile (MODE 0, dilation 1), kept in registers
+      constexpr bool has_rand = RAND && MODE == 0;
+      constexpr int kRandRegs = has_rand ? kMaxRand : 1;
+      int rbl[kRandRegs];
+#pragma unroll
+      for (int t = 0; t < kRandRegs; ++t)
+        rbl[t] = (has_rand && t < p.num_rand) ? rand_block(p, w.b, tr.head, tr.u0, t) : -1;
       int klo, khi;                            // band keys [klo, khi) of this row
       if (MODE == 0) {
         klo = u - w.r;
@@ -692,7 +723,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       float l = 0.f;
       int iu = 0;                              // tiles of this unit handled
       for (int j = 0; j < T; ++j) {
-        if (!uses(w, tr, j)) continue;
+        if (!uses(w, tr, x, j)) continue;
         if (!mbar_wait_bounded(&s_full[x], it & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
         uint32_t xr[kTile];
@@ -767,9 +798,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const int diff = pos - gp;
             bool inwin = p.causal ? (diff >= 0 && diff <= rd) : (abs(diff) <= rd);
             inwin = inwin && (diff % w.d == 0);
+            // a global key inside one of the tile's random blocks is counted there
+            if (has_rand) {
+#pragma unroll
+              for (int t = 0; t < kRandRegs; ++t) inwin = inwin || (rbl[t] >= 0 && (gp >> 7) == rbl[t]);
+            }
             const bool allowed = row_valid && gp >= 0 && !inwin;
             s[e] = allowed ? s[e] * sl2 : -INFINITY;
           }
+          tmax = row_max128(s);
+        } else if (has_rand && j >= w.rand0) {
+          // random key block: keys below the valid length and outside the row's
+          // window; a block repeated earlier in the list is masked whole
+          const int t = j - w.rand0 - (x ? w.nrand[0] : 0);
+          int kb = -1;
+#pragma unroll
+          for (int t2 = 0; t2 < kRandRegs; ++t2)
+            if (t2 == t) kb = rbl[t2];
+          bool dup = false;
+#pragma unroll
+          for (int t2 = 0; t2 < kRandRegs; ++t2) dup = dup || (t2 < t && rbl[t2] == kb);
+          const int kv0 = kb * kTile;
+          const int lo_t = klo - kv0, hi_t = khi - kv0, v_t = w.Vc - kv0;
+#pragma unroll
+          for (int e = 0; e < kTile; ++e) {
+            const bool allowed = row_valid && !dup && e < v_t && (e < lo_t || e >= hi_t);
+            s[e] = allowed ? s[e] * sl2 : -INFINITY;
+          }
+          live = 0;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch)
+            if (__any_sync(0xffffffffu, row_valid && !dup && 32 * ch < v_t)) live |= 1u << ch;
           tmax = row_max128(s);
         } else {
           const int s0 = (j - w.nband - w.ngc) * kTile;
@@ -1014,9 +1073,9 @@ size_t band_tc_smem_bytes(int D) {
   return D == 64 ? Cfg<64>::kSmemBytes : Cfg<128>::kSmemBytes;
 }
 
-template <int D, int MODE, bool LOCAL = false>
+template <int D, int MODE, bool LOCAL = false, bool RAND = false>
 static cudaError_t launch_one(const AttnParams& p, int units, int num_sms, cudaStream_t s) {
-  auto kern = attn_tc_kernel<D, MODE, LOCAL>;
+  auto kern = attn_tc_kernel<D, MODE, LOCAL, RAND>;
   const int smem = static_cast<int>(Cfg<D>::kSmemBytes);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -1029,6 +1088,13 @@ static cudaError_t launch_one(const AttnParams& p, int units, int num_sms, cudaS
 // p.tiles[h] holds the number of two-tile units of head h, p.max_units their maximum.
 cudaError_t launch_band_tc(const AttnParams& p, int num_sms, cudaStream_t s) {
   const int units = p.max_units * p.B * p.Hq;
+  if (p.num_rand > 0) {
+    if (p.local_bias)
+      return p.D == 64 ? launch_one<64, 0, true, true>(p, units, num_sms, s)
+                       : launch_one<128, 0, true, true>(p, units, num_sms, s);
+    return p.D == 64 ? launch_one<64, 0, false, true>(p, units, num_sms, s)
+                     : launch_one<128, 0, false, true>(p, units, num_sms, s);
+  }
   if (p.local_bias)
     return p.D == 64 ? launch_one<64, 0, true>(p, units, num_sms, s)
                      : launch_one<128, 0, true>(p, units, num_sms, s);

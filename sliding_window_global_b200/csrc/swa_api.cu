@@ -230,6 +230,7 @@ swa_status swa_forward_ex(swa_plan_t plan, const swa_forward_args* args, void* s
   void* out = args->out;
   float* lse = args->lse;
   const float* local_bias = args->local_bias;
+  const int32_t* rand_blocks = args->num_rand > 0 ? args->rand_blocks : nullptr;
   const swa_plan_desc& d = plan->desc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   plan->last_launches = 0;
@@ -245,8 +246,11 @@ swa_status swa_forward_ex(swa_plan_t plan, const swa_forward_args* args, void* s
   }
   if ((lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
       (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) ||
-      (local_bias && (reinterpret_cast<uintptr_t>(local_bias) & 3u)))
+      (local_bias && (reinterpret_cast<uintptr_t>(local_bias) & 3u)) ||
+      (rand_blocks && (reinterpret_cast<uintptr_t>(rand_blocks) & 3u)))
     return SWA_ERR_INVALID_ARG;
+  if (args->num_rand < 0 || args->num_rand > swa::kMaxRand) return SWA_ERR_INVALID_ARG;
+  if (args->num_rand > 0 && !rand_blocks) return SWA_ERR_INVALID_ARG;
   const int Hq = d.num_q_heads;
   for (int h = 0; h < Hq; ++h) {
     if (window[h] < 0) return SWA_ERR_INVALID_ARG;
@@ -254,6 +258,12 @@ swa_status swa_forward_ex(swa_plan_t plan, const swa_forward_args* args, void* s
     if ((long long)window[h] * (dilation ? dilation[h] : 1) > (1LL << 30)) return SWA_ERR_INVALID_ARG;
   }
   if (causal && num_global > 0) return SWA_ERR_UNSUPPORTED;
+  if (rand_blocks) {
+    // random key blocks are tiles of the plain key sequence: dilation 1, non-causal
+    if (causal) return SWA_ERR_UNSUPPORTED;
+    for (int h = 0; h < Hq; ++h)
+      if (dilation && dilation[h] != 1) return SWA_ERR_UNSUPPORTED;
+  }
   // local bias: the table covers every offset a window key can take; the band
   // kernel stages [-r_eff - kLocalPad, r_eff + kLocalPad] of it per work unit,
   // r_eff = min(r, ceil(n / d)) (offsets in class coordinates)
@@ -298,6 +308,8 @@ swa_status swa_forward_ex(swa_plan_t plan, const swa_forward_args* args, void* s
   p.local_bias = local_bias;
   p.local_radius = local_bias ? args->local_radius : 0;
   p.local_stride = local_stride;
+  p.rand_blocks = rand_blocks;
+  p.num_rand = rand_blocks ? args->num_rand : 0;
   p.out = out;
   p.lse = lse;
   p.err = plan->err;

@@ -15,6 +15,7 @@ constexpr int kMaxHeads = 128;       // query heads per plan
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
 constexpr int kBiasCopy = 2048;      // floats per staged bias copy (4 copies in shared memory)
 constexpr int kLocalPad = 256;       // zero entries staged on each side of a local-bias row
+constexpr int kMaxRand = 8;          // random key blocks per query block
 
 // Bits of the device error word.
 constexpr int kDevErrTimeout = 1;    // a bounded wait expired
@@ -48,6 +49,8 @@ struct AttnParams {
   const float* local_bias;           // [Hq, 2 * local_radius + 1] or nullptr (window keys)
   int local_radius;
   int local_stride;                  // floats per staged copy of a local-bias row (band kernel)
+  const int32_t* rand_blocks;        // [B, Hq, nqb, num_rand] random key blocks, or nullptr
+  int num_rand;                      // r (0: none); blocks are kTile keys, nqb = ceil(n / kTile)
   void* out;                         // [B, Hq, n, D], input dtype
   float* lse;                        // [B, Hq, n] or nullptr
   float* part_o;                     // global-row partials [nsplit, B*Hq, gpad, D]

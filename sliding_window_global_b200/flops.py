@@ -7,15 +7,30 @@ is the method's algorithmic work, not the dense n^2 work it avoids.
 Counted in closed form per row (vectorised over rows):
   window part |W(i)| = t_hi - t_lo + 1 with t_lo = max(-r, -floor(i/d)) and
   t_hi = 0 (causal) or min(r, floor((V-1-i)/d)); plus the global keys outside the
-  window; a global query row instead counts every valid key; plus S side keys.
+  window; plus the keys of the row's random key blocks that are neither global nor
+  in the window (counted once each); a global query row instead counts every valid
+  key; plus S side keys.
 """
 from __future__ import annotations
 
 import numpy as np
 
 
+def _random_extra(i, V, r, d, causal, gl, blocks, bs):
+    """Per row of one query block: keys of its random blocks outside W(i) and G."""
+    keys = np.unique(np.concatenate([np.arange(b * bs, b * bs + bs) for b in blocks]))
+    keys = keys[(keys >= 0) & (keys < V)]
+    keys = np.setdiff1d(keys, gl, assume_unique=False)
+    if keys.size == 0:
+        return np.zeros(i.size, np.int64)
+    diff = i[:, None] - keys[None, :]
+    inwin = diff % d == 0
+    inwin &= ((diff >= 0) & (diff <= r * d)) if causal else (np.abs(diff) <= r * d)
+    return (~inwin).sum(1).astype(np.int64)
+
+
 def attended_pairs(n: int, window, dilation, causal: bool, global_idx=None, valid_len=None,
-                   batch: int = 1, num_side: int = 0) -> int:
+                   batch: int = 1, num_side: int = 0, rand_blocks=None, rand_block: int = 128) -> int:
     window = np.asarray(window, dtype=np.int64).reshape(-1)
     dilation = np.asarray(dilation, dtype=np.int64).reshape(-1)
     if dilation.size == 1:
@@ -29,7 +44,7 @@ def attended_pairs(n: int, window, dilation, causal: bool, global_idx=None, vali
         gl = gl[gl < V]
         isg = np.zeros(V, bool)
         isg[gl] = True
-        for r, d in zip(window.tolist(), dilation.tolist()):
+        for h, (r, d) in enumerate(zip(window.tolist(), dilation.tolist())):
             t_lo = np.maximum(-r, -(i // d))
             t_hi = np.zeros_like(i) if causal else np.minimum(r, (V - 1 - i) // d)
             cnt = t_hi - t_lo + 1
@@ -41,6 +56,13 @@ def attended_pairs(n: int, window, dilation, causal: bool, global_idx=None, vali
                 else:
                     inwin &= np.abs(diff) <= r * d
                 cnt = cnt + (~inwin).sum(1)
+            if rand_blocks is not None and np.shape(rand_blocks)[-1] > 0:
+                rb = np.asarray(rand_blocks[b][h], dtype=np.int64)
+                for qb in range(rb.shape[0]):
+                    rows = i[qb * rand_block: (qb + 1) * rand_block]
+                    if rows.size:
+                        cnt[rows] += _random_extra(rows, V, r, d, causal, gl, rb[qb], rand_block)
+            if gl.size:
                 cnt = np.where(isg, V, cnt)
             total += int(cnt.sum()) + V * num_side
     return total

@@ -58,6 +58,7 @@ class ForwardArgs(ctypes.Structure):
         ("window", ctypes.c_void_p), ("dilation", ctypes.c_void_p), ("causal", ctypes.c_int),
         ("valid_len", ctypes.c_void_p), ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p),
         ("local_bias", ctypes.c_void_p), ("local_radius", ctypes.c_int),
+        ("rand_blocks", ctypes.c_void_p), ("num_rand", ctypes.c_int),
     ]
 
 
@@ -183,9 +184,12 @@ class Plan:
                 side_k: Optional[torch.Tensor] = None, side_v: Optional[torch.Tensor] = None,
                 bias: Optional[torch.Tensor] = None, valid_len: Optional[torch.Tensor] = None,
                 out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                return_lse: bool = True, local_bias: Optional[torch.Tensor] = None, stream=None):
+                return_lse: bool = True, local_bias: Optional[torch.Tensor] = None,
+                rand_blocks: Optional[torch.Tensor] = None, stream=None):
         """``local_bias``: optional [Hq, 2R+1] fp32 device table of the LongT5 local
-        relative-position bias (window keys of non-global rows, column (j - i) + R)."""
+        relative-position bias (window keys of non-global rows, column (j - i) + R).
+        ``rand_blocks``: optional int32 device tensor [B, Hq, ceil(n/128), r] of
+        BigBird random key blocks (128 keys each) per query block."""
         d = self.desc
         H = d.num_q_heads
         if out is None:
@@ -195,10 +199,17 @@ class Plan:
         w_arr, _ = _host_i32(window, H, "window")
         d_arr, _ = _host_i32(dilation, H, "dilation")
         g = 0 if global_idx is None else int(global_idx.shape[-1])
-        if local_bias is not None:
-            width = int(local_bias.shape[-1])
-            if local_bias.dim() != 2 or local_bias.shape[0] != H or width % 2 == 0:
+        if local_bias is not None or rand_blocks is not None:
+            width = 1 if local_bias is None else int(local_bias.shape[-1])
+            if local_bias is not None and (local_bias.dim() != 2 or local_bias.shape[0] != H
+                                           or width % 2 == 0):
                 raise ValueError("local_bias must be [Hq, 2R+1]")
+            nrand = 0
+            if rand_blocks is not None:
+                nqb = (d.seq_len + 127) // 128
+                if rand_blocks.dim() != 4 or tuple(rand_blocks.shape[:3]) != (d.batch, H, nqb):
+                    raise ValueError("rand_blocks must be [B, Hq, ceil(n/128), r]")
+                nrand = int(rand_blocks.shape[-1])
             a = ForwardArgs(
                 _dev_ptr(q, "q", self.dtype), _dev_ptr(k, "k", self.dtype), _dev_ptr(v, "v", self.dtype),
                 _dev_ptr(global_idx, "global_idx", torch.int32), g,
@@ -207,7 +218,7 @@ class Plan:
                 None if d_arr is None else ctypes.cast(d_arr, ctypes.c_void_p), int(bool(causal)),
                 _dev_ptr(valid_len, "valid_len", torch.int32), _dev_ptr(out, "out", self.dtype),
                 _dev_ptr(lse, "lse", torch.float32), _dev_ptr(local_bias, "local_bias", torch.float32),
-                (width - 1) // 2)
+                (width - 1) // 2, _dev_ptr(rand_blocks, "rand_blocks", torch.int32), nrand)
             st = self._lib.swa_forward_ex(self._h, ctypes.byref(a), _stream_handle(stream))
             if st != 0:
                 raise SwaError(st, "swa_forward_ex")
@@ -245,7 +256,7 @@ _plans = {}
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, window, dilation=None,
             causal: bool = False, global_idx=None, side_k=None, side_v=None, bias=None,
             valid_len=None, side_block: int = 16, scale: float = 0.0, return_lse: bool = True,
-            local_bias=None):
+            local_bias=None, rand_blocks=None):
     """Banded sparse attention of q [B,Hq,n,D] over k/v [B,Hkv,n,D] (CUDA tensors).
 
     Returns ``(out, lse)``: out like q, lse fp32 [B,Hq,n] (natural log).  Plans are
@@ -262,7 +273,8 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, window, dilati
         _plans[key] = plan
     return plan.forward(q, k, v, window=window, dilation=dilation, causal=causal,
                         global_idx=global_idx, side_k=side_k, side_v=side_v, bias=bias,
-                        valid_len=valid_len, return_lse=return_lse, local_bias=local_bias)
+                        valid_len=valid_len, return_lse=return_lse, local_bias=local_bias,
+                        rand_blocks=rand_blocks)
 
 
 def side_aggregate(x: torch.Tensor, block: int, valid_len: Optional[torch.Tensor] = None,

@@ -16,10 +16,15 @@ cases:
   D=128, causal window of 512 keys, q and k rotated by RoPE (base 10000)
 * ``longt5_local``     -- LongT5 Local attention: n=16384, 12 heads, r=127 with the
   local relative-position bias (a 32-bucket table per head over the token offset)
+* ``bigbird_itc``      -- BigBird-ITC pattern: n=4096, 12 heads, r=191 (three
+  128-key blocks), the first 128 tokens global, 3 random key blocks of 128 per
+  query block
 
 Inputs are N(0,1) from ``torch.Generator('cpu').manual_seed(seed)`` drawn in
-the order q, k, v, global positions, side-bias table, local-bias table, then
-rounded to the dtype.  Side keys/values (block means) and the expanded bias
+the order q, k, v, global positions, side-bias table, local-bias table, random
+key blocks, then rounded to the dtype.  Random blocks of query block q are drawn
+without replacement from the blocks other than q-1, q, q+1 and the global
+blocks, per (batch, head, query block).  Side keys/values (block means) and the expanded bias
 tables are NOT made here: each side (oracle and CUDA library) derives them with
 its own code.
 """
@@ -50,6 +55,7 @@ class Workload:
     side_block: int = 0             # k of the Transient-Global blocks (0: no side keys)
     side_bias: bool = False         # seeded 32-bucket side-bias table
     local_bias: bool = False        # seeded 32-bucket local relative-position bias table
+    num_rand: int = 0               # random key blocks of 128 per query block
     rope: bool = False              # rotate q and k with RoPE (base 10000, all dims)
     seed: int = 0
 
@@ -96,6 +102,9 @@ WORKLOADS = {
                          causal=True, rope=True, seed=1005),
     "longt5_local": Workload("longt5_local", 1, 12, 12, 16384, 64, "bf16", _heads(127, 12),
                              _heads(1, 12), local_bias=True, seed=1006),
+    "bigbird_itc": Workload("bigbird_itc", 1, 12, 12, 4096, 64, "bf16", _heads(191, 12),
+                            _heads(1, 12), num_global=128, global_mode="leading", num_rand=3,
+                            seed=1007),
 }
 
 # Reduced versions with the same structure (several tiles and a ragged tail) that the
@@ -118,6 +127,10 @@ SMALL = {
     "longt5_local": dataclasses.replace(WORKLOADS["longt5_local"], name="longt5_local_small",
                                         seq_len=1100, q_heads=3, kv_heads=3, window=_heads(127, 3),
                                         dilation=_heads(1, 3), padding=45, seed=2006),
+    "bigbird_itc": dataclasses.replace(WORKLOADS["bigbird_itc"], name="bigbird_itc_small",
+                                       seq_len=1300, q_heads=4, kv_heads=4, window=_heads(100, 4),
+                                       dilation=_heads(1, 4),
+                                       num_global=20, padding=37, seed=2007),
 }
 
 
@@ -162,6 +175,21 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> dict:
     local_table = None
     if w.local_bias:
         local_table = torch.randn((Hq, 32), generator=g, dtype=torch.float32)
+    rand_blocks = None
+    if w.num_rand:
+        nqb = (n + 127) // 128
+        gblocks = set()
+        if global_idx is not None:
+            gblocks = {int(x) // 128 for x in global_idx.reshape(-1).tolist()}
+        rand_blocks = torch.empty((B, Hq, nqb, w.num_rand), dtype=torch.int32)
+        for b in range(B):
+            for h in range(Hq):
+                for qb in range(nqb):
+                    cand = [x for x in range(nqb) if abs(x - qb) > 1 and x not in gblocks]
+                    if len(cand) < w.num_rand:
+                        cand = list(range(nqb))
+                    pick = torch.randperm(len(cand), generator=g)[: w.num_rand]
+                    rand_blocks[b, h, qb] = torch.tensor([cand[int(t)] for t in pick], dtype=torch.int32)
     if w.rope:
         pos = torch.arange(n)
         q = _rope_(q, pos)
@@ -172,6 +200,7 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> dict:
         global_idx=global_idx,
         bias_table=bias_table,
         local_table=local_table,
+        rand_blocks=rand_blocks,
         window=torch.tensor(w.window, dtype=torch.int32),
         dilation=torch.tensor(w.dilation, dtype=torch.int32),
         causal=w.causal,

@@ -49,7 +49,8 @@ def oracle_problem(w, inp):
                           global_idx=inp["global_idx"], side_k=inp.get("side_k"),
                           side_v=inp.get("side_v"), side_block=w.side_block or 16,
                           bias=inp.get("bias"), valid_len=inp["valid_len"], scale=inp["scale"],
-                          local_bias=inp.get("local_bias"))
+                          local_bias=inp.get("local_bias"), rand_blocks=inp.get("rand_blocks"),
+                          rand_block=128)
 
 
 def to_dev(inp, device="cuda"):
@@ -73,7 +74,8 @@ def run_gpu(w, dinp, plan=None, debug=False):
                             dilation=dinp["dilation"], causal=dinp["causal"],
                             global_idx=dinp["global_idx"], side_k=dinp.get("side_k"),
                             side_v=dinp.get("side_v"), bias=dinp.get("bias"),
-                            valid_len=dinp["valid_len"], local_bias=dinp.get("local_bias"))
+                            valid_len=dinp["valid_len"], local_bias=dinp.get("local_bias"),
+                            rand_blocks=dinp.get("rand_blocks"))
     torch.cuda.synchronize()
     return out, lse, plan
 

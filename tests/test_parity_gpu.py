@@ -164,6 +164,55 @@ def test_support_exact(n, D, r, d, causal, g, pad):
                 assert np.all(row[inside] > 0.0), (b, h, i)
 
 
+RANDOM = [
+    # BigBird random key blocks on top of windows, globals, padding, GQA and D = 128
+    ("rand_globals_pad", _small("bigbird_itc")),
+    ("rand_no_globals", _small("bigbird_itc", num_global=0, global_mode="none", padding=0)),
+    ("rand_gqa_pairs_d128", _small("swan_swa", causal=False, window=(150,) * 8, num_rand=2)),
+    ("rand_local_bias", _small("bigbird_itc", local_bias=True, num_rand=4)),
+    ("rand_window_covers_seq", _small("bigbird_itc", window=(3000,) * 4, num_global=0,
+                                      global_mode="none")),
+    ("rand_tiny_seq", _small("bigbird_itc", seq_len=100, num_global=3, padding=7)),
+    ("rand_fp32", dataclasses.replace(workloads.SMALL["bigbird_itc"], dtype="fp32", seq_len=500,
+                                      num_global=5)),
+]
+
+
+@pytest.mark.parametrize("name,w", RANDOM, ids=[e[0] for e in RANDOM])
+def test_random_blocks(name, w):
+    _need_gpu()
+    _check_workload(w)
+
+
+def test_random_blocks_with_repeats_and_overlaps():
+    """Hand-written draws: a block repeated in the list, the query block itself, its
+    neighbours (overlapping the window), a block holding global keys and the block
+    holding the padded tail -- each key must still count once."""
+    _need_gpu()
+    w = _small("bigbird_itc", seq_len=1000, num_rand=5, padding=60)
+    inp = workloads.make_inputs(w)
+    nqb = (w.seq_len + 127) // 128
+    rb = torch.empty((1, w.q_heads, nqb, 5), dtype=torch.int32)
+    for h in range(w.q_heads):
+        for qb in range(nqb):
+            rb[0, h, qb] = torch.tensor([qb, (qb + 3) % nqb, max(qb - 1, 0), 0, nqb - 1])
+            if h % 2:
+                rb[0, h, qb, 1] = rb[0, h, qb, 0]          # a repeated block
+    inp["rand_blocks"] = rb
+    _check_workload(w, inp)
+
+
+def test_random_blocks_unsupported_with_dilation_or_causal():
+    _need_gpu()
+    from sliding_window_global_b200 import SwaError
+    for w in (_small("bigbird_itc", dilation=(1, 2, 1, 1)),
+              _small("bigbird_itc", causal=True, num_global=0, global_mode="none")):
+        dinp = helpers.to_dev(helpers.host_problem(w))
+        with pytest.raises(SwaError) as e:
+            helpers.run_gpu(w, dinp)
+        assert e.value.status == 2
+
+
 def test_local_bias_window_beyond_staging_limit_is_unsupported():
     """bf16 kernels stage the local-bias row of a unit: min(r, ceil(n/d)) <= 766."""
     _need_gpu()
