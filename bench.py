@@ -149,31 +149,13 @@ def prepare(w, device):
     """Device-resident inputs of one workload, built with the library's own kernels
     (side keys: block means on the device; side and local bias: host bucket
     expansion)."""
-    import torch
-
-    from sliding_window_global_b200 import bucket_local_bias, expand_side_bias, side_aggregate, workloads
-    inp = workloads.make_inputs(w)
-    host = {k: v for k, v in inp.items()}
-    dev = {}
-    for k in ("q", "k", "v", "global_idx", "valid_len", "rand_blocks"):
-        dev[k] = inp[k].to(device) if inp[k] is not None else None
-    if w.side_block:
-        dev["side_k"] = side_aggregate(dev["k"], w.side_block, dev["valid_len"])
-        dev["side_v"] = side_aggregate(dev["v"], w.side_block, dev["valid_len"])
-        if inp["bias_table"] is not None:
-            nblk = (w.seq_len + w.side_block - 1) // w.side_block
-            host["bias"] = expand_side_bias(inp["bias_table"], w.num_side, nblk)
-            dev["bias"] = host["bias"].to(device)
-    if inp.get("local_table") is not None:
-        host["local_bias"] = bucket_local_bias(inp["local_table"], local_radius(w))
-        dev["local_bias"] = host["local_bias"].to(device)
-    torch.cuda.synchronize()
-    return host, dev
+    from sliding_window_global_b200.profile_case import device_inputs
+    return device_inputs(w, device)
 
 
 def local_radius(w) -> int:
-    """Radius of the local-bias table: the largest window offset, max min(r*d, n-1)."""
-    return max(min(r * d, w.seq_len - 1) for r, d in zip(w.window, w.dilation))
+    from sliding_window_global_b200.profile_case import local_radius as radius
+    return radius(w)
 
 
 def count_flops(w, host):
@@ -190,10 +172,8 @@ def time_device(w, plan, dev, steps, warmup, device):
     """Per-step CUDA-event time of one forward, L2 flushed before each step."""
     import torch
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
-    kw = dict(window=list(w.window), dilation=list(w.dilation), causal=w.causal,
-              global_idx=dev["global_idx"], side_k=dev.get("side_k"), side_v=dev.get("side_v"),
-              bias=dev.get("bias"), valid_len=dev["valid_len"], local_bias=dev.get("local_bias"),
-              rand_blocks=dev.get("rand_blocks"))
+    from sliding_window_global_b200.profile_case import forward_kwargs
+    kw = forward_kwargs(w, dev)
     out = torch.empty((w.batch, w.q_heads, w.seq_len, w.head_dim), dtype=w.torch_dtype, device=device)
     lse = torch.empty((w.batch, w.q_heads, w.seq_len), dtype=torch.float32, device=device)
     for _ in range(warmup):

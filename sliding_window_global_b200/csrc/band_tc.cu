@@ -109,8 +109,8 @@ struct Work {
   bool active[2];
   int band_lo;          // first key of band tile 0
   int nband, ngc, nside, total;
-  int rand0;            // first random tile: rand0 .. rand0+nrand-1 (tile A), then tile B's
-  int nrand[2];         // random tiles of tile A, B
+  int rand0;            // first random tile; with both tiles active they alternate A, B, A, ...
+  int nrand[2];         // random tiles of tile A, B (equal when both are active)
   int key_end;          // MODE 1: keys at or beyond this are masked
   int lo[2], hi[2];     // band key range of each query tile (class coordinates)
 };
@@ -219,6 +219,18 @@ __device__ __forceinline__ void decode_work(const AttnParams& p, int unit_id, Wo
   w.total = w.rand0 + w.nrand[0] + w.nrand[1];
 }
 
+// Owner (query tile) and index t of random tile j >= w.rand0.  Alternating the two
+// tiles' random blocks lets one tile's softmax overlap the other tile's MMAs.
+__device__ __forceinline__ int rand_owner(const Work& w, int j, int& t) {
+  const int k = j - w.rand0;
+  if (w.nrand[1] > 0 && w.nrand[0] > 0) {
+    t = k >> 1;
+    return k & 1;
+  }
+  t = k;
+  return w.nrand[0] > 0 ? 0 : 1;
+}
+
 // Random key block t of query tile x (query block u0 / kTile; dilation 1 only).
 __device__ __forceinline__ int rand_block(const AttnParams& p, int b, int head, int u0, int t) {
   const int nqb = (p.n + kTile - 1) / kTile;
@@ -228,7 +240,10 @@ __device__ __forceinline__ int rand_block(const AttnParams& p, int b, int head, 
 // Does query tile x use key tile j?
 __device__ __forceinline__ bool uses(const Work& w, int x, int j) {
   if (!w.active[x] || j < 0 || j >= w.total) return false;
-  if (j >= w.rand0) return (j < w.rand0 + w.nrand[0]) == (x == 0);   // a tile's own random blocks
+  if (j >= w.rand0) {                                   // a tile's own random blocks
+    int t;
+    return rand_owner(w, j, t) == x;
+  }
   if (j >= w.nband) return true;                        // global and side tiles: every row
   const int kv0 = w.band_lo + j * kTile;
   return kv0 < w.hi[x] && kv0 + kTile > w.lo[x];
@@ -256,7 +271,10 @@ __device__ __forceinline__ TileRows tile_rows(const Work& w, int x) {
 
 __device__ __forceinline__ bool uses(const Work& w, const TileRows& t, int x, int j) {
   if (!t.active || j < 0 || j >= w.total) return false;
-  if (j >= w.rand0) return (j < w.rand0 + w.nrand[0]) == (x == 0);
+  if (j >= w.rand0) {
+    int t;
+    return rand_owner(w, j, t) == x;
+  }
   if (j >= w.nband) return true;
   const int kv0 = w.band_lo + j * kTile;
   return kv0 < t.hi && kv0 + kTile > t.lo;
@@ -279,8 +297,8 @@ __device__ __forceinline__ void tile_source(const AttnParams& p, const Work& w, 
     y = (j - w.nband - w.ngc) * kTile;
   } else {
     // random key block (dilation 1: the class map is the plain key sequence)
-    const int x = (j < w.rand0 + w.nrand[0]) ? 0 : 1;
-    const int t = j - w.rand0 - (x ? w.nrand[0] : 0);
+    int t;
+    const int x = rand_owner(w, j, t);
     mk = &p.mk[w.cls];
     mv = &p.mv[w.cls];
     y = rand_block(p, w.b, x ? w.hx[1] : w.hx[0], x ? w.u0[1] : w.u0[0], t) * kTile;
@@ -558,9 +576,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (ok && uses(w, x, j) && issued[x] < j) ok = issue_qk(x, j);
           if (C::kSepP) {
             // the next S of each tile as soon as its softmax has read the current one
+            // (its next key tile may be j + 2 when random tiles alternate; a tile up
+            // to j + NS - 1 is loadable: its ring slot was freed by tile <= j - 1)
 #pragma unroll
-            for (int x = 0; x < 2; ++x)
-              if (ok && uses(w, x, j) && uses(w, x, j + 1) && issued[x] == j) ok = issue_qk(x, j + 1);
+            for (int x = 0; x < 2; ++x) {
+              if (!ok || !uses(w, x, j) || issued[x] != j) continue;
+              int jn = j + 1;
+              while (jn < T && jn < j + NS && !uses(w, x, jn)) ++jn;
+              if (jn < T && jn < j + NS) ok = issue_qk(x, jn);
+            }
           }
           if (!ok) break;
           if (!mbar_wait_bounded(&v_full[st], (g / NS) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
@@ -705,6 +729,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 #pragma unroll
       for (int t = 0; t < kRandRegs; ++t)
         rbl[t] = (has_rand && t < p.num_rand) ? rand_block(p, w.b, tr.head, tr.u0, t) : -1;
+      // this thread's position of the unit's first global-column tile, loaded early
+      const int gpos0 = (w.ngc > 0 && row < p.g) ? __ldg(p.global_idx + (size_t)w.b * p.g + row) : -1;
       int klo, khi;                            // band keys [klo, khi) of this row
       if (MODE == 0) {
         klo = u - w.r;
@@ -786,31 +812,40 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
         } else if (j < w.nband + w.ngc) {
           // global-column tile: stage its 128 positions in shared memory (one per
-          // thread of the group), then mask the keys already inside the window
+          // thread of the group), each with the per-key facts every row shares:
+          // -1 for no key (or a key a random block of this tile already counts),
+          // bit 30 set for a key of another residue class (never inside a window of
+          // this tile's rows, whose positions are all c mod d).  Rows then mask the
+          // keys already inside their window.
           const int e0 = (j - w.nband) * kTile;
+          int code = (j == w.nband) ? gpos0
+                     : ((e0 + row < p.g) ? __ldg(p.global_idx + (size_t)w.b * p.g + e0 + row) : -1);
+          if (code >= 0) {
+            bool in_rand = false;
+            if (has_rand) {
+#pragma unroll
+              for (int t = 0; t < kRandRegs; ++t) in_rand = in_rand || (rbl[t] >= 0 && (code >> 7) == rbl[t]);
+            }
+            if (in_rand) code = -1;
+            else if (w.d > 1 && code % w.d != w.c) code |= 1 << 30;
+          }
           named_barrier_sync(1 + x, 128);      // the previous tile's readers are done
-          sGpos[x * kTile + row] =
-              (e0 + row < p.g) ? __ldg(p.global_idx + (size_t)w.b * p.g + e0 + row) : -1;
+          sGpos[x * kTile + row] = code;
           named_barrier_sync(1 + x, 128);
 #pragma unroll
           for (int e = 0; e < kTile; ++e) {
-            const int gp = sGpos[x * kTile + e];
-            const int diff = pos - gp;
-            bool inwin = p.causal ? (diff >= 0 && diff <= rd) : (abs(diff) <= rd);
-            inwin = inwin && (diff % w.d == 0);
-            // a global key inside one of the tile's random blocks is counted there
-            if (has_rand) {
-#pragma unroll
-              for (int t = 0; t < kRandRegs; ++t) inwin = inwin || (rbl[t] >= 0 && (gp >> 7) == rbl[t]);
-            }
-            const bool allowed = row_valid && gp >= 0 && !inwin;
+            const int cv = sGpos[x * kTile + e];
+            const int diff = pos - (cv & ~(1 << 30));
+            const bool inwin = !(cv & (1 << 30)) && (p.causal ? (diff >= 0 && diff <= rd) : (abs(diff) <= rd));
+            const bool allowed = row_valid && cv >= 0 && !inwin;
             s[e] = allowed ? s[e] * sl2 : -INFINITY;
           }
           tmax = row_max128(s);
         } else if (has_rand && j >= w.rand0) {
           // random key block: keys below the valid length and outside the row's
           // window; a block repeated earlier in the list is masked whole
-          const int t = j - w.rand0 - (x ? w.nrand[0] : 0);
+          int t;
+          rand_owner(w, j, t);
           int kb = -1;
 #pragma unroll
           for (int t2 = 0; t2 < kRandRegs; ++t2)
