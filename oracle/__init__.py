@@ -85,6 +85,8 @@ def _load():
             lib.oracle_expand_side_bias.restype = I
             lib.oracle_side_aggregate.argtypes = [I, I, I, I, I, P, P, P]
             lib.oracle_side_aggregate.restype = I
+            lib.oracle_backward.argtypes = [I, I, I, I, I, P, P, P, P, P, I, P, P, I, P, D, EX, P, P, P]
+            lib.oracle_backward.restype = I
             lib.oracle_num_threads.argtypes = []
             lib.oracle_num_threads.restype = I
             _lib = lib
@@ -197,6 +199,22 @@ class Problem:
             return (out.reshape(self.B, self.Hq, self.n, self.D), lse.reshape(self.B, self.Hq, self.n),
                     cnt.reshape(self.B, self.Hq, self.n))
         return out, lse, cnt
+
+    def backward(self, dout):
+        """fp64 (dq, dk, dv) for the upstream gradient ``dout`` (like q); no side keys."""
+        if self.S:
+            raise ValueError("the oracle backward covers problems without side keys")
+        lib = _load()
+        do = _f32(dout)
+        dq = np.empty((self.B, self.Hq, self.n, self.D), dtype=np.float64)
+        dk = np.empty((self.B, self.Hkv, self.n, self.D), dtype=np.float64)
+        dv = np.empty((self.B, self.Hkv, self.n, self.D), dtype=np.float64)
+        _check(lib.oracle_backward(self.B, self.Hq, self.Hkv, self.n, self.D, _ptr(self.q),
+                                   _ptr(self.k), _ptr(self.v), _ptr(do), _ptr(self.global_idx),
+                                   self.g, _ptr(self.window), _ptr(self.dilation), self.causal,
+                                   _ptr(self.valid_len), self.scale, self._ex(), _ptr(dq), _ptr(dk),
+                                   _ptr(dv)), "backward")
+        return dq, dk, dv
 
     def dense_bruteforce(self):
         lib = _load()

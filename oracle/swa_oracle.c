@@ -624,6 +624,98 @@ int oracle_side_aggregate(int B, int H, int n, int D, int kb, const float *x,
     return ORACLE_OK;
 }
 
+/*
+ * oracle_backward: gradients of the attention (no side keys) with respect to q,
+ * k and v for an upstream gradient dout = dL/do, by the chain rule through the
+ * softmax of each row [definition of softmax attention; the key sets are those
+ * of oracle_forward]:
+ *   p_j  = exp(s_j - lse),  s_j = scale <q_i, k_j> (+ local bias)
+ *   dp_j = <dout_i, v_j>,   Delta_i = sum_j p_j dp_j,   ds_j = p_j (dp_j - Delta_i)
+ *   dq_i = scale sum_j ds_j k_j,  dk_j += scale ds_j q_i,  dv_j += p_j dout_i
+ * Padded rows contribute nothing.  dq [B,Hq,n,D], dk/dv [B,Hkv,n,D] (fp64) are
+ * overwritten.  Work is split over (batch, KV head) pairs, so the accumulations
+ * into dk/dv never race.
+ */
+int oracle_backward(int B, int Hq, int Hkv, int n, int D, const float *q, const float *k,
+                    const float *v, const float *dout, const int32_t *global_idx, int g,
+                    const int32_t *window, const int32_t *dilation, int causal,
+                    const int32_t *valid_len, double scale, const oracle_extras *ex,
+                    double *dq, double *dk, double *dv) {
+    oracle_problem P = {B, Hq, Hkv, n, D, q, k, v, global_idx, g, NULL, NULL,
+                        0, 0, NULL, window, dilation, causal, valid_len, scale,
+                        NULL, 0, NULL, 0, 0};
+    apply_extras(&P, ex);
+    int rc = check_problem(&P);
+    if (rc) return rc;
+    if (!dout || !dq || !dk || !dv) return ORACLE_EINVAL;
+    const int G = Hq / Hkv;
+    memset(dq, 0, sizeof(double) * (size_t)B * Hq * n * D);
+    memset(dk, 0, sizeof(double) * (size_t)B * Hkv * n * D);
+    memset(dv, 0, sizeof(double) * (size_t)B * Hkv * n * D);
+    int failed = 0;
+#pragma omp parallel
+    {
+        int32_t *keys = (int32_t *)malloc(sizeof(int32_t) * (size_t)(n + 1));
+        int32_t *wbuf = (int32_t *)malloc(sizeof(int32_t) * (size_t)(n + 1));
+        double *sc = (double *)malloc(sizeof(double) * (size_t)(n + 1));
+        double *dp = (double *)malloc(sizeof(double) * (size_t)(n + 1));
+        if (!keys || !wbuf || !sc || !dp) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int bk = 0; bk < B * Hkv; ++bk) {
+                const int b = bk / Hkv, hk = bk % Hkv;
+                const int V = valid_len ? valid_len[b] : n;
+                const float *kb = k + ((int64_t)b * Hkv + hk) * n * D;
+                const float *vb = v + ((int64_t)b * Hkv + hk) * n * D;
+                double *dkb = dk + ((int64_t)b * Hkv + hk) * n * D;
+                double *dvb = dv + ((int64_t)b * Hkv + hk) * n * D;
+                for (int h = hk * G; h < (hk + 1) * G; ++h) {
+                    for (int i = 0; i < V && i < n; ++i) {
+                        int nk = key_set(&P, b, h, i, keys, wbuf);
+                        if (nk <= 0) continue;
+                        const int64_t row = ((int64_t)b * Hq + h) * n + i;
+                        const float *qi = q + row * D;
+                        const float *doi = dout + row * D;
+                        double m = -INFINITY;
+                        for (int t = 0; t < nk; ++t) {
+                            sc[t] = scale * dot(qi, kb + (int64_t)keys[t] * D, D) + local_bias(&P, b, h, i, keys[t]);
+                            if (sc[t] > m) m = sc[t];
+                        }
+                        double l = 0.0;
+                        for (int t = 0; t < nk; ++t) l += exp(sc[t] - m);
+                        const double lse = m + log(l);
+                        double delta = 0.0;
+                        for (int t = 0; t < nk; ++t) {
+                            sc[t] = exp(sc[t] - lse);                        /* p */
+                            dp[t] = dot(doi, vb + (int64_t)keys[t] * D, D);
+                            delta += sc[t] * dp[t];
+                        }
+                        double *dqi = dq + row * D;
+                        for (int t = 0; t < nk; ++t) {
+                            const double ds = sc[t] * (dp[t] - delta);
+                            const float *kj = kb + (int64_t)keys[t] * D;
+                            double *dkj = dkb + (int64_t)keys[t] * D;
+                            double *dvj = dvb + (int64_t)keys[t] * D;
+                            for (int x = 0; x < D; ++x) {
+                                dqi[x] += scale * ds * (double)kj[x];
+                                dkj[x] += scale * ds * (double)qi[x];
+                                dvj[x] += sc[t] * (double)doi[x];
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        free(keys);
+        free(wbuf);
+        free(sc);
+        free(dp);
+    }
+    return failed ? ORACLE_ENOMEM : ORACLE_OK;
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -516,3 +516,84 @@ def test_random_blocks_zero_query_mean_over_key_set(oracle_mod):
         keys = oracle_mod.key_list(B, H, n, 0, 0, i, window=r, rand_blocks=rb, rand_block=bs)
         assert len(keys) == cnt[0, 0, i]
         assert np.max(np.abs(o[0, 0, i] - v[0, 0, keys].astype(np.float64).mean(0))) <= 1e-12
+
+
+# --- backward (gradients of softmax attention through the same key sets) ----------------
+
+
+def _dense_mask(n, r, d, causal, gl, V):
+    """The closed-form allowed matrix (band by dilation, causal, global rows/cols, padding)."""
+    i = np.arange(n)[:, None]
+    j = np.arange(n)[None, :]
+    diff = i - j
+    band = (diff % d == 0) & (((diff >= 0) & (diff <= r * d)) if causal else (np.abs(diff) <= r * d))
+    isg = np.zeros(n, bool)
+    if gl is not None:
+        isg[gl] = True
+    allow = band | isg[None, :] | isg[:, None]
+    return allow & (i < V) & (j < V)
+
+
+def test_backward_matches_torch_autograd_on_dense_masked_attention(oracle_mod):
+    rng = np.random.default_rng(71)
+    cases = 0
+    for n, r, d, causal, g, pad, G in [(13, 2, 1, 0, 0, 0, 1), (20, 3, 2, 0, 2, 3, 2), (17, 4, 1, 1, 0, 2, 2),
+                                       (24, 1, 3, 1, 0, 0, 1), (9, 20, 1, 0, 1, 0, 3), (30, 2, 2, 0, 3, 5, 1)]:
+        B, Hkv, D = 2, 2, 8
+        Hq = Hkv * G
+        p = _problem(oracle_mod, rng, B, Hq, Hkv, n, D, r, d, causal, g, pad)
+        dout = _rand((B, Hq, n, D), rng)
+        dq, dk, dv = p.backward(dout)
+        V = n - pad
+        q = torch.from_numpy(p.q).double().requires_grad_()
+        k = torch.from_numpy(p.k).double().requires_grad_()
+        v = torch.from_numpy(p.v).double().requires_grad_()
+        kk = k.repeat_interleave(G, dim=1)
+        vv = v.repeat_interleave(G, dim=1)
+        s = q @ kk.transpose(-1, -2) * p.scale
+        outs = []
+        for b in range(B):
+            gl = p.global_idx[b] if p.global_idx is not None else None
+            allow = torch.from_numpy(_dense_mask(n, r, d, causal, gl, V))
+            sb = s[b].masked_fill(~allow, float("-inf"))
+            w = torch.softmax(sb, -1).nan_to_num(0.0)          # padded rows: no keys, o = 0
+            outs.append(w @ vv[b])
+        o = torch.stack(outs)
+        (o * torch.from_numpy(dout).double()).sum().backward()
+        assert np.max(np.abs(dq - q.grad.numpy())) <= 1e-12
+        assert np.max(np.abs(dk - k.grad.numpy())) <= 1e-12
+        assert np.max(np.abs(dv - v.grad.numpy())) <= 1e-12
+        cases += 1
+    assert cases == 6
+
+
+def test_backward_finite_differences(oracle_mod):
+    """Central differences of L = sum(dout * o) through the oracle's forward, with the
+    local bias and random blocks in play (the terms torch does not see above)."""
+    rng = np.random.default_rng(73)
+    B, H, n, D, r, bs = 1, 2, 20, 4, 2, 4
+    q, k, v = (_rand((B, H, n, D), rng) for _ in range(3))
+    dout = _rand((B, H, n, D), rng)
+    gl = np.array([[5, 17]], np.int32)
+    lt = _local_table(rng, H, r)
+    rb = _rand_blocks(rng, B, H, n, bs, 2)
+    kw = dict(window=r, global_idx=gl, local_bias=lt, rand_blocks=rb, rand_block=bs)
+    dq, dk, dv = oracle_mod.Problem(q, k, v, **kw).backward(dout)
+
+    def loss(qq, kk, vv):
+        o, _, _ = oracle_mod.Problem(qq, kk, vv, **kw).forward()
+        return float((o * dout.astype(np.float64)).sum())
+
+    h = 2.0 ** -10
+    for name, arr, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for _ in range(6):
+            idx = tuple(int(rng.integers(0, s)) for s in arr.shape)
+            plus, minus = arr.copy(), arr.copy()
+            plus[idx] += np.float32(h)
+            minus[idx] -= np.float32(h)
+            step = float(plus[idx]) - float(minus[idx])
+            args = {"q": (q, k, v), "k": (q, k, v), "v": (q, k, v)}[name]
+            a_p = [plus if x is arr else x for x in args]
+            a_m = [minus if x is arr else x for x in args]
+            fd = (loss(*a_p) - loss(*a_m)) / step
+            assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, abs(grad[idx])), (name, idx, fd, grad[idx])
