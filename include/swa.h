@@ -168,6 +168,40 @@ swa_status swa_forward_ex(swa_plan_t plan, const swa_forward_args* args, void* s
  * the bucket function of swa_relative_bucket).  Host pointers. */
 swa_status swa_bucket_local_bias(int num_q_heads, int radius, const float* table, float* out);
 
+/* ---------------------------------------------------------------------------
+ * Backward pass: gradients of the forward's output with respect to q, k and v,
+ * through the chain rule of each row's softmax (p = exp(s - lse), dp = dout . v,
+ * ds = p (dp - rowsum(dout * out)), dq = scale ds k, dk = scale ds^T q,
+ * dv = p^T dout) over the same key sets: the dilated / causal sliding window
+ * ("精读笔记：Big Bird" §3.2.1, the Longformer page §二, SWAN-GPT §3.3(1)) with GQA
+ * and padding.  Global tokens, side keys, local bias and random blocks are not
+ * covered: a plan with side keys returns SWA_ERR_UNSUPPORTED, and the arguments
+ * have no fields for the others.  bf16 plans only (else SWA_ERR_UNSUPPORTED);
+ * the query heads of one KV head must share window and dilation (else
+ * SWA_ERR_UNSUPPORTED).  Gradients are written in fp32; dk and dv hold the sums
+ * over the query heads of each KV head.  Every element of dq, dk, dv is written
+ * (padded rows get 0).  The plan's workspace holds rowsum(dout * out).
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  const void* q;               /* device [B, Hq, n, D] bf16, 16-byte aligned */
+  const void* k;               /* device [B, Hkv, n, D] bf16 */
+  const void* v;               /* device [B, Hkv, n, D] bf16 */
+  const void* out;             /* device [B, Hq, n, D] bf16: the forward's output */
+  const float* lse;            /* device [B, Hq, n] fp32: the forward's lse */
+  const void* dout;            /* device [B, Hq, n, D] bf16: upstream gradient */
+  const int32_t* window;       /* HOST [Hq] */
+  const int32_t* dilation;     /* HOST [Hq] or NULL (all 1) */
+  int causal;
+  const int32_t* valid_len;    /* device [B] or NULL */
+  float* dq;                   /* device [B, Hq, n, D] fp32 */
+  float* dk;                   /* device [B, Hkv, n, D] fp32 */
+  float* dv;                   /* device [B, Hkv, n, D] fp32 */
+} swa_backward_args;
+
+/* Three launches on `stream`: rowsum(dout * out), the query-stationary dq pass,
+ * the key-stationary dk/dv pass.  Statuses as swa_forward. */
+swa_status swa_backward(swa_plan_t plan, const swa_backward_args* args, void* stream);
+
 /* Synchronise `stream` and read (then clear) the plan's device error word:
  * SWA_ERR_TIMEOUT if a bounded wait expired in any kernel since the last check,
  * SWA_ERR_DEVICE_CHECK if a precondition check failed, SWA_ERR_CUDA if the

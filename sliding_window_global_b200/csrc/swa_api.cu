@@ -40,6 +40,7 @@ struct swa_plan_s {
   void* gv;
   float* part_o;
   float* part_lse;
+  float* delta;        // backward: rowsum(dout * out) [B, Hq, n]
   int last_launches;
   int num_sms;         // persistent grid size
 };
@@ -141,6 +142,11 @@ swa_status swa_plan_create(swa_plan_t* out_plan, const swa_plan_desc* d) {
     o_po = off; off = align_up(off + (size_t)p->nsplit_max * B * Hq * p->gpad * D * 4, 256);
     o_pl = off; off = align_up(off + (size_t)p->nsplit_max * B * Hq * p->gpad * 4, 256);
   }
+  size_t o_delta = 0;
+  if (d->dtype == SWA_BF16) {
+    o_delta = off;
+    off = align_up(off + B * Hq * (size_t)d->seq_len * 4, 256);
+  }
   p->ws_bytes = off;
   if (cudaMalloc(&p->ws, p->ws_bytes) != cudaSuccess) {
     cudaGetLastError();
@@ -153,6 +159,7 @@ swa_status swa_plan_create(swa_plan_t* out_plan, const swa_plan_desc* d) {
     return SWA_ERR_CUDA;
   }
   p->err = reinterpret_cast<int*>(p->ws);
+  if (o_delta) p->delta = reinterpret_cast<float*>(p->ws + o_delta);
   if (o_gq) {
     p->gq = p->ws + o_gq;
     p->gk = p->ws + o_gk;
@@ -450,6 +457,123 @@ swa_status swa_forward_ex(swa_plan_t plan, const swa_forward_args* args, void* s
         ++launches;
       }
     }
+  }
+  delete pp;
+  plan->last_launches = launches;
+  if (ce != cudaSuccess) return SWA_ERR_CUDA;
+  if (d.flags & SWA_DEBUG_CHECKS) return swa_plan_check(plan, stream);
+  return SWA_OK;
+}
+
+swa_status swa_backward(swa_plan_t plan, const swa_backward_args* a, void* stream) {
+  if (!plan || !a) return SWA_ERR_INVALID_ARG;
+  const swa_plan_desc& d = plan->desc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  plan->last_launches = 0;
+  if (!a->q || !a->k || !a->v || !a->out || !a->lse || !a->dout || !a->window || !a->dq || !a->dk ||
+      !a->dv)
+    return SWA_ERR_INVALID_ARG;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out) ||
+      !aligned16(a->dout) || !aligned16(a->dq) || !aligned16(a->dk) || !aligned16(a->dv) ||
+      (reinterpret_cast<uintptr_t>(a->lse) & 3u))
+    return SWA_ERR_INVALID_ARG;
+  if (a->causal != 0 && a->causal != 1) return SWA_ERR_INVALID_ARG;
+  const int Hq = d.num_q_heads, n = d.seq_len, D = d.head_dim;
+  for (int h = 0; h < Hq; ++h) {
+    if (a->window[h] < 0) return SWA_ERR_INVALID_ARG;
+    if (a->dilation && a->dilation[h] < 1) return SWA_ERR_INVALID_ARG;
+    if ((long long)a->window[h] * (a->dilation ? a->dilation[h] : 1) > (1LL << 30)) return SWA_ERR_INVALID_ARG;
+  }
+  if (d.dtype != SWA_BF16 || d.num_side > 0 || !plan->delta) return SWA_ERR_UNSUPPORTED;
+  const int G = Hq / d.num_kv_heads;
+  for (int h = 0; h < Hq; ++h) {
+    const int h0 = (h / G) * G;
+    if (a->window[h] != a->window[h0] || (a->dilation && a->dilation[h] != a->dilation[h0]))
+      return SWA_ERR_UNSUPPORTED;
+  }
+
+  swa::BwdParams* pp = new (std::nothrow) swa::BwdParams;
+  if (!pp) return SWA_ERR_OOM;
+  swa::BwdParams& p = *pp;
+  memset(&p, 0, sizeof(p));
+  p.B = d.batch;
+  p.Hq = Hq;
+  p.Hkv = d.num_kv_heads;
+  p.n = n;
+  p.D = D;
+  p.G = G;
+  p.causal = a->causal;
+  p.scale = d.scale > 0.f ? d.scale : 1.0f / sqrtf((float)D);
+  p.scale_log2 = p.scale * 1.4426950408889634f;
+  p.valid_len = a->valid_len;
+  p.out = a->out;
+  p.dout = a->dout;
+  p.lse = a->lse;
+  p.delta = plan->delta;
+  p.dq = a->dq;
+  p.dk = a->dk;
+  p.dv = a->dv;
+  p.err = plan->err;
+  // residue classes (as in the forward) and tiles per head
+  int nclass = 0;
+  swa_status st = SWA_OK;
+  for (int h = 0; h < Hq && st == SWA_OK; ++h) {
+    const int dh = a->dilation ? a->dilation[h] : 1;
+    p.window[h] = a->window[h];
+    int base = -1;
+    for (int c = 0; c < nclass; ++c)
+      if (p.cls[c].d == dh && p.cls[c].c == 0) base = c;
+    if (base < 0) {
+      const int need = std::min(dh, n);
+      if (nclass + need > kMaxClasses) { st = SWA_ERR_UNSUPPORTED; break; }
+      base = nclass;
+      for (int c = 0; c < need; ++c) {
+        p.cls[nclass].d = dh;
+        p.cls[nclass].c = c;
+        p.cls[nclass].n_c = (n - c + dh - 1) / dh;
+        p.cls[nclass].nres = need;
+        ++nclass;
+      }
+    }
+    p.class_base[h] = base;
+    int tiles = 0;
+    for (int c = 0; c < std::min(dh, n); ++c) tiles += (p.cls[base + c].n_c + kTile - 1) / kTile;
+    p.qtiles[h] = tiles;
+    p.ktiles[h / G] = tiles;
+    p.max_qtiles = std::max(p.max_qtiles, tiles);
+    p.max_ktiles = std::max(p.max_ktiles, tiles);
+  }
+  if (st != SWA_OK) {
+    delete pp;
+    return st;
+  }
+  const size_t row = (size_t)D * 2;
+  bool ok = true;
+  for (int c = 0; c < nclass && ok; ++c) {
+    const int dd = p.cls[c].d, cc = p.cls[c].c, nc = p.cls[c].n_c;
+    ok = ok && make_map(&p.mq[c], static_cast<const char*>(a->q) + cc * row, D, nc, (uint64_t)p.B * Hq,
+                        dd * row, (uint64_t)n * row);
+    ok = ok && make_map(&p.mdo[c], static_cast<const char*>(a->dout) + cc * row, D, nc,
+                        (uint64_t)p.B * Hq, dd * row, (uint64_t)n * row);
+    ok = ok && make_map(&p.mk[c], static_cast<const char*>(a->k) + cc * row, D, nc,
+                        (uint64_t)p.B * p.Hkv, dd * row, (uint64_t)n * row);
+    ok = ok && make_map(&p.mv[c], static_cast<const char*>(a->v) + cc * row, D, nc,
+                        (uint64_t)p.B * p.Hkv, dd * row, (uint64_t)n * row);
+  }
+  if (!ok) {
+    delete pp;
+    return SWA_ERR_CUDA;
+  }
+  int launches = 0;
+  cudaError_t ce = swa::launch_bwd_delta(p, s);
+  ++launches;
+  if (ce == cudaSuccess) {
+    ce = swa::launch_bwd_dq(p, s);
+    ++launches;
+  }
+  if (ce == cudaSuccess) {
+    ce = swa::launch_bwd_dkv(p, s);
+    ++launches;
   }
   delete pp;
   plan->last_launches = launches;

@@ -30,7 +30,7 @@ EXPORTS = (
     "swa_plan_create", "swa_forward", "swa_plan_check", "swa_plan_destroy",
     "swa_plan_workspace_bytes", "swa_plan_last_launches", "swa_status_string",
     "swa_side_aggregate", "swa_relative_bucket", "swa_expand_side_bias", "swa_forward_noalloc",
-    "swa_forward_ex", "swa_bucket_local_bias",
+    "swa_forward_ex", "swa_bucket_local_bias", "swa_backward",
 )
 
 
@@ -59,6 +59,17 @@ class ForwardArgs(ctypes.Structure):
         ("valid_len", ctypes.c_void_p), ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p),
         ("local_bias", ctypes.c_void_p), ("local_radius", ctypes.c_int),
         ("rand_blocks", ctypes.c_void_p), ("num_rand", ctypes.c_int),
+    ]
+
+
+class BackwardArgs(ctypes.Structure):
+    """swa_backward_args of include/swa.h."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("dout", ctypes.c_void_p),
+        ("window", ctypes.c_void_p), ("dilation", ctypes.c_void_p), ("causal", ctypes.c_int),
+        ("valid_len", ctypes.c_void_p), ("dq", ctypes.c_void_p), ("dk", ctypes.c_void_p),
+        ("dv", ctypes.c_void_p),
     ]
 
 
@@ -103,6 +114,8 @@ def load_library():
         lib.swa_forward_ex.restype = I
         lib.swa_bucket_local_bias.argtypes = [I, I, P, P]
         lib.swa_bucket_local_bias.restype = I
+        lib.swa_backward.argtypes = [P, ctypes.POINTER(BackwardArgs), P]
+        lib.swa_backward.restype = I
         _lib = lib
         return lib
 
@@ -233,6 +246,37 @@ class Plan:
         if st != 0:
             raise SwaError(st, "swa_forward")
         return out, lse
+
+    def backward(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                 lse: torch.Tensor, dout: torch.Tensor, *, window, dilation=None,
+                 causal: bool = False, valid_len: Optional[torch.Tensor] = None,
+                 dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
+                 dv: Optional[torch.Tensor] = None, stream=None):
+        """Gradients (dq, dk, dv), fp32, of the band attention for the upstream gradient
+        ``dout``; ``out`` and ``lse`` are the forward's results."""
+        d = self.desc
+        H, Hkv = d.num_q_heads, d.num_kv_heads
+        shape_q = (d.batch, H, d.seq_len, d.head_dim)
+        shape_k = (d.batch, Hkv, d.seq_len, d.head_dim)
+        if dq is None:
+            dq = torch.empty(shape_q, dtype=torch.float32, device=q.device)
+        if dk is None:
+            dk = torch.empty(shape_k, dtype=torch.float32, device=q.device)
+        if dv is None:
+            dv = torch.empty(shape_k, dtype=torch.float32, device=q.device)
+        w_arr, _ = _host_i32(window, H, "window")
+        d_arr, _ = _host_i32(dilation, H, "dilation")
+        a = BackwardArgs(
+            _dev_ptr(q, "q", self.dtype), _dev_ptr(k, "k", self.dtype), _dev_ptr(v, "v", self.dtype),
+            _dev_ptr(out, "out", self.dtype), _dev_ptr(lse, "lse", torch.float32),
+            _dev_ptr(dout, "dout", self.dtype), ctypes.cast(w_arr, ctypes.c_void_p),
+            None if d_arr is None else ctypes.cast(d_arr, ctypes.c_void_p), int(bool(causal)),
+            _dev_ptr(valid_len, "valid_len", torch.int32), _dev_ptr(dq, "dq", torch.float32),
+            _dev_ptr(dk, "dk", torch.float32), _dev_ptr(dv, "dv", torch.float32))
+        st = self._lib.swa_backward(self._h, ctypes.byref(a), _stream_handle(stream))
+        if st != 0:
+            raise SwaError(st, "swa_backward")
+        return dq, dk, dv
 
     def check(self, stream=None) -> int:
         """Synchronise and return the status of the device error word (0 = OK)."""

@@ -112,3 +112,9 @@ def test_forward_ex_null_arguments(lib):
     assert lib.swa_forward_ex(None, None, None) == 1
     args = binding.ForwardArgs()
     assert lib.swa_forward_ex(None, ctypes.byref(args), None) == 1
+
+
+def test_backward_null_arguments(lib):
+    assert lib.swa_backward(None, None, None) == 1
+    args = binding.BackwardArgs()
+    assert lib.swa_backward(None, ctypes.byref(args), None) == 1
