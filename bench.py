@@ -198,6 +198,39 @@ def time_device(w, plan, dev, steps, warmup, device):
     return sum(ms) / steps, launches
 
 
+def time_backward(w, plan, dev, steps, warmup, device):
+    """Per-step CUDA-event time of one backward (dq, dk, dv) from the forward's out and
+    lse and a seeded upstream gradient, L2 flushed before each step."""
+    import torch
+    from sliding_window_global_b200.profile_case import forward_kwargs
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    out, lse = plan.forward(dev["q"], dev["k"], dev["v"], **forward_kwargs(w, dev))
+    g = torch.Generator(device=device).manual_seed(11)
+    dout = torch.randn(out.shape, generator=g, device=device).to(out.dtype)
+    kw = dict(window=list(w.window), dilation=list(w.dilation), causal=w.causal,
+              valid_len=dev["valid_len"])
+    grads = plan.backward(dev["q"], dev["k"], dev["v"], out, lse, dout, **kw)
+    for _ in range(warmup):
+        flush.fill_(1.0)
+        plan.backward(dev["q"], dev["k"], dev["v"], out, lse, dout, dq=grads[0], dk=grads[1],
+                      dv=grads[2], **kw)
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    launches = 0
+    for s in range(steps):
+        flush.fill_(float(s))
+        starts[s].record()
+        plan.backward(dev["q"], dev["k"], dev["v"], out, lse, dout, dq=grads[0], dk=grads[1],
+                      dv=grads[2], **kw)
+        ends[s].record()
+        launches += plan.last_launches
+    torch.cuda.synchronize()
+    if plan.check() != 0:
+        raise RuntimeError("device error word set during the backward")
+    return sum(starts[s].elapsed_time(ends[s]) for s in range(steps)) / steps, launches
+
+
 def time_e2e(w, plan, host, steps, warmup, device):
     """Same metric through the public API with pinned host buffers: every step copies
     the inputs host->device, builds side keys on the device, runs the forward and
@@ -324,6 +357,17 @@ def run_ours(args):
                                "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peak)}
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
                 res["cpu_baseline"] = cpu_baseline(w, host)
+            if not args.no_backward and not w.num_global and not w.num_side and not w.local_bias \
+                    and not w.num_rand:
+                bms, blaunch = time_backward(w, plan, dev, args.steps, args.warmup, device)
+                bms = _max_over_ranks(dist, bms, device)
+                # useful backward work: five products per attended pair (S, dP, dV, dK, dQ)
+                bflop = 2.5 * flop
+                res["backward"] = {"workload": name, "value": replica_throughput(bflop, world, bms),
+                                   "unit": "TFLOP/s", "ms_per_step": bms,
+                                   "useful_gflop_per_step": bflop / 1e9, "gpu_launches": blaunch,
+                                   "frac_of_peak": bflop / (bms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                                   "kernels": "bwd_delta + bwd_dq_kernel<D> + bwd_dkv_kernel<D>"}
         plan.close()
         del dev
         torch.cuda.empty_cache()
@@ -352,6 +396,8 @@ def run_ours(args):
             "roofline": main["roofline"], "e2e": main["e2e"], "gpu_launches": main["gpu_launches"],
             "clocks": main["clocks"],
         }
+        if "backward" in main:
+            line["backward"] = main["backward"]
         if "cpu_baseline" in main:
             line["cpu_baseline"] = main["cpu_baseline"]
         if secs:
@@ -418,6 +464,7 @@ def main():
     ap.add_argument("--secondary", default="longt5_tglobal,longt5_local,bigbird_itc",
                     help="comma-separated workloads timed after the main one (device time only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass timing")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
