@@ -2,6 +2,7 @@
 profilers (ncu) and quick timing.  No parity checks; use the tests for those.
 
     python -m sliding_window_global_b200.profile_case WORKLOAD [--seq-len N] [--batch B] [--reps R]
+        [--backward]
 
 The inputs, kernels and launch configuration are those of the bench's timed step
 (``device_inputs`` builds the bench's inputs too).
@@ -58,6 +59,8 @@ def main(argv=None):
     ap.add_argument("--seq-len", type=int, default=None)
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--reps", type=int, default=4)
+    ap.add_argument("--backward", action="store_true",
+                    help="after the forwards, run the backward pass --reps times")
     a = ap.parse_args(argv)
     w = workloads.WORKLOADS[a.workload]
     if a.seq_len:
@@ -70,6 +73,13 @@ def main(argv=None):
                 max_global=w.num_global, num_side=w.num_side, side_block=w.side_block or 16)
     for _ in range(a.reps):
         out, _ = plan.forward(dev["q"], dev["k"], dev["v"], **forward_kwargs(w, dev))
+    if a.backward:
+        out, lse = plan.forward(dev["q"], dev["k"], dev["v"], **forward_kwargs(w, dev))
+        dout = torch.randn(out.shape, device=out.device, generator=torch.Generator("cuda").manual_seed(1))
+        dout = dout.to(out.dtype)
+        for _ in range(a.reps):
+            plan.backward(dev["q"], dev["k"], dev["v"], out, lse, dout, window=list(w.window),
+                          dilation=list(w.dilation), causal=w.causal, valid_len=dev["valid_len"])
     torch.cuda.synchronize()
     status = plan.check()
     print(f"{w.name} B={w.batch} n={w.seq_len}: status {status}, launches/forward "
