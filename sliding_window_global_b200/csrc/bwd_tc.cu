@@ -13,18 +13,22 @@
 //   bwd_dq_kernel<D>     query-stationary: one CTA per 128-row query tile walks
 //                        its band's key tiles: S = Q K^T and dP = dO V^T into
 //                        TMEM, dS written back as bf16 over S, dQ += dS K;
-//   bwd_dkv_kernel<D>    key-stationary: one CTA per 128-key tile walks the query
-//                        tiles (of every query head of its GQA group) that reach
-//                        it: S^T = K Q^T and dP^T = V dO^T, P^T and dS^T written
-//                        back as bf16, dV += P^T dO and dK += dS^T Q.
+//   bwd_dkv_kernel<D>    key-stationary: one CTA per 128-key tile walks the 64-row
+//                        query tiles (of every query head of its GQA group) that
+//                        reach it, two compute warpgroups taking alternate tiles:
+//                        S^T = K Q^T and dP^T = V dO^T into the group's TMEM
+//                        columns, P^T and dS^T as bf16 into shared memory, then
+//                        dV += P^T dO and dK += dS^T Q.
 // Neither needs atomics: every output row belongs to one CTA.  S and dP are
 // computed by both passes (seven tile products instead of five), the price of
 // keeping dQ out of the key-stationary pass's TMEM, which D = 128 fills.
 //
-// Warp roles (192 threads): warps 0-3 compute (thread t owns TMEM lane t),
-// warp 4 issues the TMA loads, warp 5 allocates TMEM and issues the MMAs.
+// Warp roles of the dQ pass (192 threads): warps 0-3 compute (thread t owns TMEM
+// lane t), warp 4 issues the TMA loads, warp 5 allocates TMEM and issues the MMAs;
+// the dK/dV pass (320 threads) has two compute warpgroups, then the same two.
 #include "ptx.cuh"
 #include "swa_kernels.h"
+#include "bwd_kernels.h"
 
 namespace swa {
 namespace {
@@ -45,9 +49,8 @@ struct BCfg {
   static constexpr uint32_t kBarOff = kStageOff + 4 * kStage * 4;
   static constexpr uint32_t kSmemBytes = kBarOff + 16 * 8 + 1024;
   static constexpr uint32_t kTmemCols = 512;
-  // TMEM columns: S (or S^T) 0-127 with P / dS written over 0-63; dP (or dP^T)
-  // 128-255 (dS^T over 128-191 in the key-stationary pass); accumulators after.
-  static constexpr uint32_t kS = 0, kDP = 128, kAcc0 = 256, kAcc1 = 256 + D;
+  // TMEM columns (dQ pass): S 0-127 with dS written over 0-63, dP 128-255, dQ after.
+  static constexpr uint32_t kS = 0, kDP = 128, kAcc0 = 256;
 };
 
 // TMA load of one 128 x D bf16 tile (two 64-column boxes when D = 128).
@@ -322,20 +325,46 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
 }
 
 // ------------------------------------------------------------------ dK, dV
+// Key-stationary pass with 64-row query tiles and two compute warpgroups that take
+// alternate query tiles, each with its own S^T / dP^T columns in TMEM (M = 128 keys,
+// N = 64 queries), so one group's exponentials overlap the other group's products.
+// P^T and dS^T go to shared memory (128 keys x 64 queries, K-major with the
+// 128-byte swizzle) and feed dV += P^T dO and dK += dS^T Q as shared-memory operands.
+constexpr int kQT = 64;                        // query rows per tile of this pass
+constexpr int kDkvThreads = 320;               // warps 0-3, 4-7 compute; 8 TMA; 9 MMA / TMEM
+
 template <int D>
-__global__ void __launch_bounds__(kBThreads, 1) bwd_dkv_kernel(const __grid_constant__ BwdParams p) {
-  using C = BCfg<D>;
+struct KCfg {
+  static constexpr uint32_t kKVBytes = 128u * D * 2u;      // a 128 x D tile
+  static constexpr uint32_t kQBytes = kQT * D * 2u;        // a 64 x D tile
+  static constexpr uint32_t kQSub = kQT * 128u;            // 64-row x 128-byte sub-tile
+  static constexpr uint32_t kK = 0, kV = kKVBytes;
+  static constexpr uint32_t kRing = 2 * kKVBytes;          // stage s: Q at kRing + 2 s Q, dO after
+  static constexpr uint32_t kPds = kRing + 4 * kQBytes;    // group g: P^T at kPds + 2 g P, dS^T after
+  static constexpr uint32_t kPBytes = 128u * kQT * 2u;     // 16 KB
+  static constexpr uint32_t kStg = kPds + 4 * kPBytes;     // [group][buffer][lse2 64 | delta 64] floats
+  static constexpr uint32_t kBarOff = kStg + 2 * 2 * 128 * 4;
+  static constexpr uint32_t kSmemBytes = kBarOff + 16 * 8 + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  // TMEM: group g S^T at 128 g, dP^T at 128 g + 64; dV at 256, dK at 256 + D
+  static constexpr uint32_t kAccV = 256, kAccK = 256 + D;
+};
+static_assert(KCfg<128>::kSmemBytes <= 227 * 1024, "shared memory of the dK/dV pass");
+
+template <int D>
+__global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_constant__ BwdParams p) {
+  using C = KCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-  float* sStage = reinterpret_cast<float*>(smem + C::kStageOff);   // [2][lse2, delta][128]
   uint64_t* a_full = bars;          // K and V loaded
-  uint64_t* r_full = bars + 1;      // [2] Q, dO of a stage loaded
-  uint64_t* r_empty = bars + 3;     // [2]
-  uint64_t* s_full = bars + 5;      // S^T and dP^T in TMEM
-  uint64_t* p_full = bars + 6;      // P^T and dS^T written (128 arrivals)
-  uint64_t* acc_full = bars + 7;    // dK, dV complete
+  uint64_t* r_full = bars + 1;      // [2] Q, dO of a ring stage loaded
+  uint64_t* r_empty = bars + 3;     // [2] that stage's products are done
+  uint64_t* s_full = bars + 5;      // [2] S^T, dP^T of group g in TMEM
+  uint64_t* p_full = bars + 7;      // [2] group g wrote P^T, dS^T (and read its TMEM), 128 arrivals
+  uint64_t* pds_free = bars + 9;    // [2] group g's P^T / dS^T buffers read by the products
+  uint64_t* acc_full = bars + 11;   // dK, dV complete
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -343,26 +372,26 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dkv_kernel(const __grid_cons
   BUnit u;
   decode_bunit(p, blockIdx.x, true, u);
   if (!u.valid) return;
-  // query rows (class coordinates) whose window reaches the valid keys of this tile
   const int lastk = u.u0 + u.nvalid - 1;
   const int qlo = p.causal ? u.u0 : max(0, u.u0 - u.r);
   const int qhi = u.nvalid > 0 ? min(u.Vc, lastk + u.r + 1) : qlo;
-  const int NQ = qhi > qlo ? (qhi - qlo + kTile - 1) / kTile : 0;
-  const int T = NQ * p.G;                     // query tiles of every head of the group
+  const int NQ = qhi > qlo ? (qhi - qlo + kQT - 1) / kQT : 0;
+  const int T = NQ * p.G;                     // 64-row query tiles of every head of the group
 
   if (tid == 0) {
     mbar_init(a_full, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&r_full[s], 1);
       mbar_init(&r_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&pds_free[s], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
     mbar_init(acc_full, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(&tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
@@ -373,64 +402,91 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dkv_kernel(const __grid_cons
   volatile int* abort_v = &abort_flag;
   const int kz = u.b * p.Hkv + u.hk;
 
-  if (warp == 4) {
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0 && T > 0) {
-      mbar_arrive_expect_tx(a_full, 2 * C::kTileBytes);
-      load_tile<D>(smem + C::kStat0, &p.mk[u.cls], a_full, u.u0, kz);
-      load_tile<D>(smem + C::kStat1, &p.mv[u.cls], a_full, u.u0, kz);
+      mbar_arrive_expect_tx(a_full, 2 * C::kKVBytes);
+      load_tile<D>(smem + C::kK, &p.mk[u.cls], a_full, u.u0, kz);
+      load_tile<D>(smem + C::kV, &p.mv[u.cls], a_full, u.u0, kz);
       for (int j = 0; j < T; ++j) {
         const int st = j & 1;
         if (j >= 2 && !mbar_wait_bounded(&r_empty[st], ((j >> 1) - 1) & 1, abort_v, kWaitLimitNs)) break;
         const int qz = u.b * p.Hq + u.h + j / NQ;
-        const int y = qlo + (j % NQ) * kTile;
-        uint8_t* dst = smem + C::kRing + st * 2 * C::kTileBytes;
-        mbar_arrive_expect_tx(&r_full[st], 2 * C::kTileBytes);
-        load_tile<D>(dst, &p.mq[u.cls], &r_full[st], y, qz);
-        load_tile<D>(dst + C::kTileBytes, &p.mdo[u.cls], &r_full[st], y, qz);
+        const int y = qlo + (j % NQ) * kQT;
+        uint8_t* dst = smem + C::kRing + st * 2 * C::kQBytes;
+        mbar_arrive_expect_tx(&r_full[st], 2 * C::kQBytes);
+        tma_load_3d(dst, &p.mq64[u.cls], &r_full[st], 0, y, qz);
+        if (D == 128) tma_load_3d(dst + C::kQSub, &p.mq64[u.cls], &r_full[st], 64, y, qz);
+        tma_load_3d(dst + C::kQBytes, &p.mdo64[u.cls], &r_full[st], 0, y, qz);
+        if (D == 128) tma_load_3d(dst + C::kQBytes + C::kQSub, &p.mdo64[u.cls], &r_full[st], 64, y, qz);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && T > 0) {
-      const uint32_t ka = smem_u32(smem + C::kStat0), va = smem_u32(smem + C::kStat1);
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kQT, false);    // S^T, dP^T: 128 x 64
+      constexpr uint32_t idesc_a = idesc_bf16_f32(128, D, true);       // dV, dK: 128 x D, B MN-major
+      const uint32_t ka = smem_u32(smem + C::kK), va = smem_u32(smem + C::kV);
+      // S^T = K Q^T and dP^T = V dO^T of tile j into group (j & 1)'s columns
+      auto issue_s = [&](int j) -> bool {
+        const int st = j & 1, g = j & 1;
+        if (!mbar_wait_bounded(&r_full[st], (j >> 1) & 1, abort_v, kWaitLimitNs)) return false;
+        tc_fence_after();
+        const uint32_t qb = smem_u32(smem + C::kRing + st * 2 * C::kQBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t offa = (kk >> 2) * kBSub + (kk & 3) * 32;
+          const uint32_t offb = (kk >> 2) * C::kQSub + (kk & 3) * 32;
+          umma_ss(tmem + 128 * g, sdesc_sw128(ka + offa, 16, 1024), sdesc_sw128(qb + offb, 16, 1024),
+                  idesc_s, kk > 0 ? 1u : 0u);
+          umma_ss(tmem + 128 * g + 64, sdesc_sw128(va + offa, 16, 1024),
+                  sdesc_sw128(qb + C::kQBytes + offb, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[g]);
+        return true;
+      };
       bool ok = mbar_wait_bounded(a_full, 0, abort_v, kWaitLimitNs);
-      for (int j = 0; ok && j <= T; ++j) {
-        if (j > 0) {
-          // dV += P^T dO and dK += dS^T Q for tile j-1, then its stage may be refilled
-          if (!mbar_wait_bounded(p_full, (j - 1) & 1, abort_v, kWaitLimitNs)) break;
-          tc_fence_after();
-          const int sp = (j - 1) & 1;
-          const uint32_t qb = smem_u32(smem + C::kRing + sp * 2 * C::kTileBytes);
-          mma_px<D>(tmem + C::kAcc0, tmem + C::kS, qb + C::kTileBytes, j > 1);   // dV
-          mma_px<D>(tmem + C::kAcc1, tmem + C::kDP, qb, j > 1);                  // dK
-          umma_commit(&r_empty[sp]);
-          if (j == T) umma_commit(acc_full);
+      if (ok) ok = issue_s(0);
+      if (ok && T > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < T; ++j) {
+        const int g = j & 1, st = j & 1;
+        if (!mbar_wait_bounded(&p_full[g], (j >> 1) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+        fence_proxy_async_smem();
+        tc_fence_after();
+        const uint32_t pt = smem_u32(smem + C::kPds + g * 2 * C::kPBytes);
+        const uint32_t qb = smem_u32(smem + C::kRing + st * 2 * C::kQBytes);
+        // dV += P^T dO, dK += dS^T Q (A: 128 x 64 K-major from shared memory; B: 64 x D MN-major)
+#pragma unroll
+        for (int kk = 0; kk < kQT / 16; ++kk) {
+          umma_ss(tmem + C::kAccV, sdesc_sw128(pt + kk * 32, 16, 1024),
+                  sdesc_sw128(qb + C::kQBytes + kk * 2048, C::kQSub, 1024), idesc_a, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_ss(tmem + C::kAccK, sdesc_sw128(pt + C::kPBytes + kk * 32, 16, 1024),
+                  sdesc_sw128(qb + kk * 2048, C::kQSub, 1024), idesc_a, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        if (j < T) {
-          const int st = j & 1;
-          if (!mbar_wait_bounded(&r_full[st], (j >> 1) & 1, abort_v, kWaitLimitNs)) break;
-          tc_fence_after();
-          const uint32_t qb = smem_u32(smem + C::kRing + st * 2 * C::kTileBytes);
-          mma_abt<D>(tmem + C::kS, ka, qb);                          // S^T = K Q^T
-          mma_abt<D>(tmem + C::kDP, va, qb + C::kTileBytes);         // dP^T = V dO^T
-          umma_commit(s_full);
-        }
+        umma_commit(&pds_free[g]);
+        umma_commit(&r_empty[st]);
+        if (j + 2 < T) ok = issue_s(j + 2);     // the group has read its S^T, dP^T of tile j
       }
+      if (ok) umma_commit(acc_full);
     }
   } else {
-    // ------------------------------------------------------------ compute
-    const int row = tid;                       // key row, TMEM lane
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    // ------------------------------------------------------------ compute warpgroups
+    const int g = warp >> 2;                  // takes query tiles j with j & 1 == g
+    const int row = tid & 127;                // key row, TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const bool key_valid = row < u.nvalid;
     const int uk = u.u0 + row;
     const float sl2 = p.scale_log2;
+    uint8_t* pts = smem + C::kPds + g * 2 * C::kPBytes;   // P^T rows, then dS^T rows
     bool ok = true;
-    for (int j = 0; j < T; ++j) {
-      // stage lse2 and Delta of the tile's 128 query rows (a padded or missing row
-      // gets lse2 = +inf, so its p is 0)
+    int nt = 0;                               // tiles handled by this group
+    for (int j = g; j < T; j += 2, ++nt) {
+      // lse2 and Delta of the tile's 64 query rows (a padded or missing row gets
+      // lse2 = +inf, so its p is 0)
       const int head = u.h + j / NQ;
-      const int q0 = qlo + (j % NQ) * kTile;
-      float* stg = sStage + (j & 1) * 256;
-      {
+      const int q0 = qlo + (j % NQ) * kQT;
+      float* stg = reinterpret_cast<float*>(smem + C::kStg) + (g * 2 + (nt & 1)) * 128;
+      if (row < kQT) {
         const int uq = q0 + row;
         float l2 = INFINITY, dl = 0.f;
         if (uq < u.Vc) {
@@ -439,74 +495,82 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dkv_kernel(const __grid_cons
           dl = p.delta[pr];
         }
         stg[row] = l2;
-        stg[128 + row] = dl;
+        stg[kQT + row] = dl;
       }
-      named_barrier_sync(1, 128);
-      if (!mbar_wait_bounded(s_full, j & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+      named_barrier_sync(1 + g, 128);
+      if (!mbar_wait_bounded(&s_full[g], nt & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
       tc_fence_after();
+      // the products of tile j - 2 have read this group's P^T / dS^T buffers
+      if (nt > 0 && !mbar_wait_bounded(&pds_free[g], (nt - 1) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
       const int d0 = q0 - uk;                  // query - key offset of column 0
+      uint8_t* prow = pts + row * 128;
+      uint8_t* drow = pts + C::kPBytes + row * 128;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int half = 0; half < 2; ++half) {   // 32 query columns at a time
         uint32_t sr[32], dr[32];
-        tmem_ld32(lane_base + C::kS + ch * 32, sr);
-        tmem_ld32(lane_base + C::kDP + ch * 32, dr);
+        tmem_ld32(lane_base + 128 * g + 32 * half, sr);
+        tmem_ld32(lane_base + 128 * g + 64 + 32 * half, dr);
         tmem_wait_ld_dep(sr);
         tmem_wait_ld_dep(dr);
-        uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int q = 0; q < 32; q += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(stg + ch * 32 + q);
-          const float4 dl4 = *reinterpret_cast<const float4*>(stg + 128 + ch * 32 + q);
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-          const float dv[4] = {dl4.x, dl4.y, dl4.z, dl4.w};
-          float pr[4], ds[4];
+        for (int c4 = 0; c4 < 4; ++c4) {       // 16-byte chunks of 8 queries
+          const int c = half * 4 + c4;
+          const float4 la = *reinterpret_cast<const float4*>(stg + c * 8);
+          const float4 lb = *reinterpret_cast<const float4*>(stg + c * 8 + 4);
+          const float4 da = *reinterpret_cast<const float4*>(stg + kQT + c * 8);
+          const float4 db = *reinterpret_cast<const float4*>(stg + kQT + c * 8 + 4);
+          const float lv[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
+          const float dv[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+          float pr[8], ds[8];
 #pragma unroll
-          for (int e4 = 0; e4 < 4; ++e4) {
-            const int off = d0 + ch * 32 + q + e4;   // query - key
+          for (int e = 0; e < 8; ++e) {
+            const int off = d0 + c * 8 + e;
             const bool inband = p.causal ? (off >= 0 && off <= u.r) : (off >= -u.r && off <= u.r);
             const bool allowed = key_valid && inband;
-            pr[e4] = allowed ? ex2_approx(__uint_as_float(sr[q + e4]) * sl2 - lv[e4]) : 0.f;
-            ds[e4] = pr[e4] * (__uint_as_float(dr[q + e4]) - dv[e4]);
+            pr[e] = allowed ? ex2_approx(__uint_as_float(sr[c4 * 8 + e]) * sl2 - lv[e]) : 0.f;
+            ds[e] = pr[e] * (__uint_as_float(dr[c4 * 8 + e]) - dv[e]);
           }
-          pk[q / 2] = pack_bf16x2(pr[0], pr[1]);
-          pk[q / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
-          dk[q / 2] = pack_bf16x2(ds[0], ds[1]);
-          dk[q / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+          uint4 pv, dsv;
+          pv.x = pack_bf16x2(pr[0], pr[1]);
+          pv.y = pack_bf16x2(pr[2], pr[3]);
+          pv.z = pack_bf16x2(pr[4], pr[5]);
+          pv.w = pack_bf16x2(pr[6], pr[7]);
+          dsv.x = pack_bf16x2(ds[0], ds[1]);
+          dsv.y = pack_bf16x2(ds[2], ds[3]);
+          dsv.z = pack_bf16x2(ds[4], ds[5]);
+          dsv.w = pack_bf16x2(ds[6], ds[7]);
+          const int sw = (c ^ (row & 7)) << 4; // 128-byte swizzle within the 8-row atom
+          *reinterpret_cast<uint4*>(prow + sw) = pv;
+          *reinterpret_cast<uint4*>(drow + sw) = dsv;
         }
-        tmem_st16(lane_base + C::kS + ch * 16, pk);     // P^T over S^T
-        tmem_st16(lane_base + C::kDP + ch * 16, dk);    // dS^T over dP^T
       }
-      tmem_wait_st();
+      fence_proxy_async_smem();                // generic writes -> tensor-core reads
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[g]);
     }
-    // epilogue: dK = scale * (dS^T Q), dV = P^T dO, fp32; padded keys get zeros.
-    // The TMEM loads are warp-wide, so every thread issues them; only rows of the
-    // tile store.
+    // epilogue: group 0 writes dV, group 1 writes dK = scale * (dS^T Q), fp32; padded
+    // keys get zeros.  The TMEM loads are warp-wide, so every thread issues them.
     if (ok && T > 0) ok = mbar_wait_bounded(acc_full, 0, abort_v, kWaitLimitNs);
     if (ok) {
       tc_fence_after();
-      const size_t prow = row < u.rows ? pos_row(p, u, u.hk, p.Hkv, uk) : 0;
+      const size_t prw = row < u.rows ? pos_row(p, u, u.hk, p.Hkv, uk) : 0;
+      float* dst = (g ? p.dk : p.dv) + prw * D;
+      const float mul = g ? p.scale : 1.f;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        float* dst = (which ? p.dk : p.dv) + prow * D;
-        const float mul = which ? p.scale : 1.f;
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t rr[32];
+        if (T > 0) {
+          tmem_ld32(lane_base + (g ? C::kAccK : C::kAccV) + ch * 32, rr);
+          tmem_wait_ld_dep(rr);
+        }
+        if (row < u.rows) {
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t rr[32];
-          if (T > 0) {
-            tmem_ld32(lane_base + (which ? C::kAcc1 : C::kAcc0) + ch * 32, rr);
-            tmem_wait_ld_dep(rr);
-          }
-          if (row < u.rows) {
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-              float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-              if (T > 0 && key_valid)
-                v4 = make_float4(__uint_as_float(rr[q4 * 4]) * mul, __uint_as_float(rr[q4 * 4 + 1]) * mul,
-                                 __uint_as_float(rr[q4 * 4 + 2]) * mul, __uint_as_float(rr[q4 * 4 + 3]) * mul);
-              reinterpret_cast<float4*>(dst)[ch * 8 + q4] = v4;
-            }
+          for (int q4 = 0; q4 < 8; ++q4) {
+            float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (T > 0 && key_valid)
+              v4 = make_float4(__uint_as_float(rr[q4 * 4]) * mul, __uint_as_float(rr[q4 * 4 + 1]) * mul,
+                               __uint_as_float(rr[q4 * 4 + 2]) * mul, __uint_as_float(rr[q4 * 4 + 3]) * mul);
+            reinterpret_cast<float4*>(dst)[ch * 8 + q4] = v4;
           }
         }
       }
@@ -524,7 +588,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dkv_kernel(const __grid_cons
     }
     __syncthreads();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
@@ -532,11 +596,11 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dkv_kernel(const __grid_cons
 }
 
 template <typename K>
-cudaError_t launch_bwd(K kern, uint32_t smem, int grid, const BwdParams& p, cudaStream_t s) {
+cudaError_t launch_kern(K kern, uint32_t smem, int grid, int threads, const BwdParams& p, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, kBThreads, smem, s>>>(p);
+  kern<<<grid, threads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -551,14 +615,14 @@ cudaError_t launch_bwd_delta(const BwdParams& p, cudaStream_t s) {
 
 cudaError_t launch_bwd_dq(const BwdParams& p, cudaStream_t s) {
   const int grid = p.max_qtiles * p.B * p.Hq;
-  return p.D == 64 ? launch_bwd(bwd_dq_kernel<64>, BCfg<64>::kSmemBytes, grid, p, s)
-                   : launch_bwd(bwd_dq_kernel<128>, BCfg<128>::kSmemBytes, grid, p, s);
+  return p.D == 64 ? launch_kern(bwd_dq_kernel<64>, BCfg<64>::kSmemBytes, grid, kBThreads, p, s)
+                   : launch_kern(bwd_dq_kernel<128>, BCfg<128>::kSmemBytes, grid, kBThreads, p, s);
 }
 
 cudaError_t launch_bwd_dkv(const BwdParams& p, cudaStream_t s) {
   const int grid = p.max_ktiles * p.B * p.Hkv;
-  return p.D == 64 ? launch_bwd(bwd_dkv_kernel<64>, BCfg<64>::kSmemBytes, grid, p, s)
-                   : launch_bwd(bwd_dkv_kernel<128>, BCfg<128>::kSmemBytes, grid, p, s);
+  return p.D == 64 ? launch_kern(bwd_dkv_kernel<64>, KCfg<64>::kSmemBytes, grid, kDkvThreads, p, s)
+                   : launch_kern(bwd_dkv_kernel<128>, KCfg<128>::kSmemBytes, grid, kDkvThreads, p, s);
 }
 
 }  // namespace swa

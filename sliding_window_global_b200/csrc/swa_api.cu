@@ -21,6 +21,7 @@
 
 #include "../../include/swa.h"
 #include "swa_kernels.h"
+#include "bwd_kernels.h"
 
 using swa::AttnParams;
 using swa::kMaxClasses;
@@ -74,12 +75,13 @@ EncodeTiledFn encode_fn() {
 // of 64 columns with the 128-byte swizzle (the tcgen05 operand layout); output
 // stores use a box of 32 columns with the 64-byte swizzle (the staging layout).
 bool make_map(CUtensorMap* m, const void* base, int D, uint64_t rows, uint64_t planes,
-              uint64_t row_stride_bytes, uint64_t plane_stride_bytes, bool store_box = false) {
+              uint64_t row_stride_bytes, uint64_t plane_stride_bytes, bool store_box = false,
+              int box_rows = kTile) {
   EncodeTiledFn fn = encode_fn();
   if (!fn || rows == 0 || planes == 0) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, rows, planes};
   cuuint64_t strides[2] = {row_stride_bytes, plane_stride_bytes};
-  cuuint32_t box[3] = {store_box ? 32u : 64u, (cuuint32_t)kTile, 1};
+  cuuint32_t box[3] = {store_box ? 32u : 64u, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -559,6 +561,11 @@ swa_status swa_backward(swa_plan_t plan, const swa_backward_args* a, void* strea
                         (uint64_t)p.B * p.Hkv, dd * row, (uint64_t)n * row);
     ok = ok && make_map(&p.mv[c], static_cast<const char*>(a->v) + cc * row, D, nc,
                         (uint64_t)p.B * p.Hkv, dd * row, (uint64_t)n * row);
+    // 64-row query / dout boxes for the key-stationary pass
+    ok = ok && make_map(&p.mq64[c], static_cast<const char*>(a->q) + cc * row, D, nc, (uint64_t)p.B * Hq,
+                        dd * row, (uint64_t)n * row, false, 64);
+    ok = ok && make_map(&p.mdo64[c], static_cast<const char*>(a->dout) + cc * row, D, nc,
+                        (uint64_t)p.B * Hq, dd * row, (uint64_t)n * row, false, 64);
   }
   if (!ok) {
     delete pp;
