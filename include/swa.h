@@ -217,6 +217,15 @@ size_t swa_plan_workspace_bytes(swa_plan_t plan);
 /* Number of kernel launches the most recent swa_forward enqueued. */
 int swa_plan_last_launches(swa_plan_t plan);
 
+/* Self-test of the failure path (an addition of this library: the pages describe
+ * nothing like it).  Enqueues one small kernel that waits, with the bounded wait
+ * every kernel of the library uses, on a barrier that nothing signals; after
+ * limit_ns (0 < limit_ns <= 5e9, else SWA_ERR_INVALID_ARG) the wait gives up and
+ * sets the timeout bit of the plan's error word, as an expired wait in the
+ * attention kernels does, and the kernel returns.  The next swa_plan_check
+ * reports SWA_ERR_TIMEOUT (and clears the word); the context stays usable. */
+swa_status swa_selftest_wait_timeout(swa_plan_t plan, uint64_t limit_ns, void* stream);
+
 /* Static, human-readable name of a status. */
 const char* swa_status_string(swa_status s);
 

@@ -11,6 +11,7 @@
 //   * a device-side check of the global-index precondition.
 #include <cuda_bf16.h>
 
+#include "ptx.cuh"
 #include "swa_kernels.h"
 
 namespace swa {
@@ -269,7 +270,31 @@ __global__ void check_globals_kernel(const int32_t* __restrict__ gidx, int g, in
   if (bad) atomicOr(err, kDevErrCheck);
 }
 
+// ------------------------------------------------------------------ failure-path self test
+// One thread waits on an mbarrier that nothing arrives at, with the bounded wait the
+// attention kernels use; when the limit expires it reports a timeout in the error
+// word, as those kernels do, and returns.
+__global__ void wait_probe_kernel(int* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    volatile int* a = &abort_flag;
+    if (!mbar_wait_bounded(&bar, 0, a, limit_ns)) atomicOr(err, kDevErrTimeout);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_wait_probe(int* err, uint64_t limit_ns, cudaStream_t s) {
+  wait_probe_kernel<<<1, 32, 0, s>>>(err, limit_ns);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_gather_globals(const AttnParams& p, const void* q, const void* k, const void* v,
                                   void* gq, void* gk, void* gv, int elem_bytes, cudaStream_t s) {

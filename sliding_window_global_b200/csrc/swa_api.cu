@@ -589,6 +589,12 @@ swa_status swa_backward(swa_plan_t plan, const swa_backward_args* a, void* strea
   return SWA_OK;
 }
 
+swa_status swa_selftest_wait_timeout(swa_plan_t plan, uint64_t limit_ns, void* stream) {
+  if (!plan || limit_ns == 0 || limit_ns > 5000000000ull) return SWA_ERR_INVALID_ARG;
+  plan->last_launches = 1;
+  return cuda_status(swa::launch_wait_probe(plan->err, limit_ns, static_cast<cudaStream_t>(stream)));
+}
+
 swa_status swa_side_aggregate(const void* x, void* out, int batch, int heads, int seq_len,
                               int head_dim, int block, const int32_t* valid_len, swa_dtype dtype,
                               void* stream) {

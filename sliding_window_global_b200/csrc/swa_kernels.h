@@ -75,6 +75,7 @@ cudaError_t launch_merge_global_rows(const AttnParams& p, int bf16_out, cudaStre
 cudaError_t launch_simt(const AttnParams& p, const void* q, const void* k, const void* v,
                         const void* side_k, const void* side_v, int bf16, cudaStream_t s);
 cudaError_t launch_check_globals(const AttnParams& p, cudaStream_t s);
+cudaError_t launch_wait_probe(int* err, uint64_t limit_ns, cudaStream_t s);
 cudaError_t launch_side_aggregate(const void* x, void* out, int B, int H, int n, int D, int kb,
                                   const int32_t* valid_len, int bf16, cudaStream_t s);
 size_t band_tc_smem_bytes(int D);

@@ -30,7 +30,7 @@ EXPORTS = (
     "swa_plan_create", "swa_forward", "swa_plan_check", "swa_plan_destroy",
     "swa_plan_workspace_bytes", "swa_plan_last_launches", "swa_status_string",
     "swa_side_aggregate", "swa_relative_bucket", "swa_expand_side_bias", "swa_forward_noalloc",
-    "swa_forward_ex", "swa_bucket_local_bias", "swa_backward",
+    "swa_forward_ex", "swa_bucket_local_bias", "swa_backward", "swa_selftest_wait_timeout",
 )
 
 
@@ -116,6 +116,8 @@ def load_library():
         lib.swa_bucket_local_bias.restype = I
         lib.swa_backward.argtypes = [P, ctypes.POINTER(BackwardArgs), P]
         lib.swa_backward.restype = I
+        lib.swa_selftest_wait_timeout.argtypes = [P, ctypes.c_uint64, P]
+        lib.swa_selftest_wait_timeout.restype = I
         _lib = lib
         return lib
 
@@ -277,6 +279,13 @@ class Plan:
         if st != 0:
             raise SwaError(st, "swa_backward")
         return dq, dk, dv
+
+    def selftest_wait_timeout(self, limit_ns: int, stream=None) -> None:
+        """Enqueue the failure-path self test: a bounded wait that expires after
+        ``limit_ns`` and sets the timeout bit that ``check()`` then reports."""
+        st = self._lib.swa_selftest_wait_timeout(self._h, int(limit_ns), _stream_handle(stream))
+        if st != 0:
+            raise SwaError(st, "swa_selftest_wait_timeout")
 
     def check(self, stream=None) -> int:
         """Synchronise and return the status of the device error word (0 = OK)."""

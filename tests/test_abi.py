@@ -118,3 +118,7 @@ def test_backward_null_arguments(lib):
     assert lib.swa_backward(None, None, None) == 1
     args = binding.BackwardArgs()
     assert lib.swa_backward(None, ctypes.byref(args), None) == 1
+
+
+def test_selftest_rejects_bad_limits(lib):
+    assert lib.swa_selftest_wait_timeout(None, 1000, None) == 1

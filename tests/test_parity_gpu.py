@@ -279,3 +279,22 @@ def test_repeat_calls_deterministic_and_launch_count():
     o2, l2, _ = helpers.run_gpu(w, dinp, plan=plan)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
     assert plan.last_launches == 6   # gather x3, band, global rows, merge
+
+
+def test_bounded_wait_expires_into_a_status_and_the_context_survives():
+    """Failure path: a wait on a barrier nothing signals gives up after its limit,
+    the error word reports SWA_ERR_TIMEOUT once, and the next forward is unaffected."""
+    _need_gpu()
+    import time
+    w = workloads.SMALL["longformer_base"]
+    dinp = helpers.to_dev(helpers.host_problem(w))
+    out0, lse0, plan = helpers.run_gpu(w, dinp)
+    assert plan.check() == 0
+    t0 = time.perf_counter()
+    plan.selftest_wait_timeout(50_000_000)          # 50 ms
+    assert plan.check() == 5                        # SWA_ERR_TIMEOUT
+    assert time.perf_counter() - t0 >= 0.04
+    assert plan.check() == 0                        # the word was cleared
+    out1, lse1, _ = helpers.run_gpu(w, dinp, plan=plan)
+    assert plan.check() == 0
+    assert torch.equal(out0, out1) and torch.equal(lse0, lse1)
