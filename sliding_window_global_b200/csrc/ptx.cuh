@@ -92,7 +92,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 3-D tiled load (no multicast) into this CTA's shared memory; completion is
+// 3-D tiled load into this CTA's own shared memory; completion is
 // signalled as transaction bytes on `bar`.  x (innermost) must be a multiple of
 // 8 elements for 16-bit types (callers pass 0 or 64).
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
