@@ -43,12 +43,17 @@
 //               the MUFU unit, part with a polynomial on the FMA pipe -- and write
 //               P (bf16) back into the TMEM columns of S.  Epilogue: O / l.
 //   warp 8      TMA producer: Q tiles, then K/V tiles into an NS-stage ring.
-//   warp 9      TMEM allocator and MMA issuer (warps 10-11 idle).  Per key tile j, for A then B:
-//               O += P(j) V(j) (P read from TMEM), immediately followed by
-//               S = Q K(j+1)^T into the same TMEM columns, so the tensor core
-//               works on one query tile while the other one's softmax runs.
-//               MMAs from one thread execute in order, so a new S never
-//               overwrites a P that an earlier MMA still reads.
+//   warp 9      TMEM allocator and MMA issuer.  P over S (D = 128): it issues
+//               both tiles' MMAs; per key tile j, for A then B, O += P(j) V(j)
+//               (P read from TMEM) immediately followed by S = Q K(j+1)^T into
+//               the same TMEM columns, so the tensor core works on one query
+//               tile while the other one's softmax runs.  MMAs from one thread
+//               execute in order, so a new S never overwrites a P that an
+//               earlier MMA still reads.  Separate P (D = 64): warp 9 issues
+//               tile A's MMAs and warp 10 tile B's, each the next S of its tile
+//               as soon as the softmax has read the current one; the two
+//               issuers share only the K/V ring (read-only) and release each
+//               slot together.  Other warps of the group idle.
 #include "ptx.cuh"
 #include "swa_kernels.h"
 
@@ -237,18 +242,6 @@ __device__ __forceinline__ int rand_block(const AttnParams& p, int b, int head, 
   return __ldg(p.rand_blocks + (((size_t)b * p.Hq + head) * nqb + u0 / kTile) * p.num_rand + t);
 }
 
-// Does query tile x use key tile j?
-__device__ __forceinline__ bool uses(const Work& w, int x, int j) {
-  if (!w.active[x] || j < 0 || j >= w.total) return false;
-  if (j >= w.rand0) {                                   // a tile's own random blocks
-    int t;
-    return rand_owner(w, j, t) == x;
-  }
-  if (j >= w.nband) return true;                        // global and side tiles: every row
-  const int kv0 = w.band_lo + j * kTile;
-  return kv0 < w.hi[x] && kv0 + kTile > w.lo[x];
-}
-
 // The fields of one query tile as scalars: the softmax warps pick their tile at
 // run time, and indexing Work's two-element arrays with a run-time index would
 // put the whole struct in local memory.
@@ -269,13 +262,14 @@ __device__ __forceinline__ TileRows tile_rows(const Work& w, int x) {
   return t;
 }
 
+// Does query tile x (fields t) use key tile j?
 __device__ __forceinline__ bool uses(const Work& w, const TileRows& t, int x, int j) {
   if (!t.active || j < 0 || j >= w.total) return false;
-  if (j >= w.rand0) {
+  if (j >= w.rand0) {                                   // a tile's own random blocks
     int t;
     return rand_owner(w, j, t) == x;
   }
-  if (j >= w.nband) return true;
+  if (j >= w.nband) return true;                        // global and side tiles: every row
   const int kv0 = w.band_lo + j * kTile;
   return kv0 < t.hi && kv0 + kTile > t.lo;
 }
@@ -403,6 +397,8 @@ template <int D, int MODE, bool LOCAL, bool RAND>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ AttnParams p) {
   using C = Cfg<D>;
   constexpr int NS = C::NS;
+  constexpr int kIssuers = C::kSepP ? 2 : 1;              // MMA-issuing warps
+  constexpr int kTilesPerIssuer = 2 / kIssuers;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -453,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     for (int s = 0; s < NS; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], kIssuers);    // released by every MMA issuer
     }
     abort_flag = 0;
     fence_barrier_init();
@@ -511,18 +507,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
       }
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 9 || (kIssuers == 2 && warp == 10)) {
+    // ------------------------------------------------------------ MMA issuers
+    // P over S (D = 128): warp 9 issues both tiles' MMAs in one fixed order, which
+    // keeps the two softmax groups half a period apart.  Separate P (D = 64): warp
+    // 9 issues tile A's MMAs and warp 10 tile B's, so neither tile's products wait
+    // behind the other tile's barriers.
     setmaxnreg_dec<kRegsControl>();
     if (lane == 0) {
+      const int x0 = (kIssuers == 2) ? warp - 9 : 0;   // first tile of this issuer
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
       const uint32_t q_base = smem_u32(sQ);
       const uint32_t k_base = smem_u32(sK);
       const uint32_t v_base = smem_u32(sV);
-      int qwaits[2] = {0, 0};
-      int pwaits[2] = {0, 0};
-      int nqk[2] = {0, 0};                          // QKs issued per tile buffer (kernel-wide)
+      int qwaits[kTilesPerIssuer] = {}, pwaits[kTilesPerIssuer] = {};
+      int nqk[kTilesPerIssuer] = {};                    // QKs issued per tile buffer (kernel-wide)
       int kv = 0;
       bool ok = true;
       for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
@@ -530,22 +530,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         decode_work<MODE, RAND>(p, uid, w);
         if (!w.active[0]) continue;
         const int T = w.total;
-        int first[2] = {-1, -1}, last[2] = {-1, -1}, issued[2] = {-1, -1}, npv[2] = {0, 0};
+        // the tiles' fields as scalars (x0 is a run-time value with two issuers)
+        TileRows tr[kTilesPerIssuer];
+        int first[kTilesPerIssuer], last[kTilesPerIssuer], issued[kTilesPerIssuer], npv[kTilesPerIssuer];
 #pragma unroll
-        for (int x = 0; x < 2; ++x)
+        for (int i = 0; i < kTilesPerIssuer; ++i) {
+          tr[i] = tile_rows(w, x0 + i);
+          first[i] = last[i] = issued[i] = -1;
+          npv[i] = 0;
           for (int j = 0; j < T; ++j)
-            if (uses(w, x, j)) {
-              if (first[x] < 0) first[x] = j;
-              last[x] = j;
+            if (uses(w, tr[i], x0 + i, j)) {
+              if (first[i] < 0) first[i] = j;
+              last[i] = j;
             }
-        auto issue_qk = [&](int x, int j) -> bool {
+        }
+        auto issue_qk = [&](int i, int j) -> bool {
+          const int x = x0 + i;
           const int g = kv + j;
           if (!mbar_wait_bounded(&k_full[g % NS], (g / NS) & 1, abort_v, kWaitLimitNs)) return false;
           // separate-P layout: S_x is rewritten only after the softmax read the last one
-          if (C::kSepP && nqk[x] > 0 &&
-              !mbar_wait_bounded(&s_free[x], (nqk[x] - 1) & 1, abort_v, kWaitLimitNs))
+          if (C::kSepP && nqk[i] > 0 &&
+              !mbar_wait_bounded(&s_free[x], (nqk[i] - 1) & 1, abort_v, kWaitLimitNs))
             return false;
-          ++nqk[x];
+          ++nqk[i];
           tc_fence_after();
           const uint32_t qt = q_base + x * C::kTileBytes;
           const uint32_t kt = k_base + (g % NS) * C::kTileBytes;
@@ -556,64 +563,76 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     sdesc_sw128(kt + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
           }
           umma_commit(&s_full[x]);
-          if (j == last[x]) umma_commit(&q_empty[x]);   // Q_x may be refilled once this QK is done
-          issued[x] = j;
+          if (j == last[i]) umma_commit(&q_empty[x]);   // Q_x may be refilled once this QK is done
+          issued[i] = j;
           return true;
         };
 #pragma unroll
-        for (int x = 0; x < 2; ++x) {
+        for (int i = 0; i < kTilesPerIssuer; ++i) {
           if (!ok) break;
-          if (!w.active[x]) continue;
-          ok = mbar_wait_bounded(&q_full[x], qwaits[x] & 1, abort_v, kWaitLimitNs);
-          ++qwaits[x];
-          if (ok) ok = issue_qk(x, first[x]);
+          if (!tr[i].active) continue;
+          ok = mbar_wait_bounded(&q_full[x0 + i], qwaits[i] & 1, abort_v, kWaitLimitNs);
+          ++qwaits[i];
+          if (ok) ok = issue_qk(i, first[i]);
         }
         for (int j = 0; ok && j < T; ++j) {
           const int g = kv + j;
           const int st = g % NS;
+          bool any = false;                           // this issuer reads the slot of tile j
 #pragma unroll
-          for (int x = 0; x < 2; ++x)
-            if (ok && uses(w, x, j) && issued[x] < j) ok = issue_qk(x, j);
+          for (int i = 0; i < kTilesPerIssuer; ++i) {
+            const bool u = uses(w, tr[i], x0 + i, j);
+            any = any || u;
+            if (ok && u && issued[i] < j) ok = issue_qk(i, j);
+          }
           if (C::kSepP) {
             // the next S of each tile as soon as its softmax has read the current one
             // (its next key tile may be j + 2 when random tiles alternate; a tile up
             // to j + NS - 1 is loadable: its ring slot was freed by tile <= j - 1)
 #pragma unroll
-            for (int x = 0; x < 2; ++x) {
-              if (!ok || !uses(w, x, j) || issued[x] != j) continue;
+            for (int i = 0; i < kTilesPerIssuer; ++i) {
+              if (!ok || !uses(w, tr[i], x0 + i, j) || issued[i] != j) continue;
               int jn = j + 1;
-              while (jn < T && jn < j + NS && !uses(w, x, jn)) ++jn;
-              if (jn < T && jn < j + NS) ok = issue_qk(x, jn);
+              while (jn < T && jn < j + NS && !uses(w, tr[i], x0 + i, jn)) ++jn;
+              if (jn < T && jn < j + NS) ok = issue_qk(i, jn);
             }
           }
           if (!ok) break;
+          // With two issuers both wait for V of every tile of the unit, used or not,
+          // before they release its ring slot: the slot's next load needs both
+          // releases, so neither issuer can arrive twice on one phase of kv_empty.
           if (!mbar_wait_bounded(&v_full[st], (g / NS) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+          if (!any) {
+            mbar_arrive(&kv_empty[st]);               // no MMA of this issuer reads the slot
+            continue;
+          }
           const uint32_t vt = v_base + st * C::kTileBytes;
 #pragma unroll
-          for (int x = 0; x < 2; ++x) {
+          for (int i = 0; i < kTilesPerIssuer; ++i) {
+            const int x = x0 + i;
             if (!ok) break;
-            if (!uses(w, x, j)) continue;
+            if (!uses(w, tr[i], x, j)) continue;
             if (!C::kSepP) {
               // P over S: the first half of P (keys 0-63) is published early, so the
               // PV over it overlaps the exponentials of the second half
-              if (!mbar_wait_bounded(&p_half[x], pwaits[x] & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+              if (!mbar_wait_bounded(&p_half[x], pwaits[i] & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
               tc_fence_after();
 #pragma unroll
               for (int kk = 0; kk < kTile / 32; ++kk)
                 umma_ts(tmem + C::o_col(x), tmem + C::p_col(x) + kk * 8,
-                        sdesc_sw128(vt + kk * 2048, kSub, 1024), idesc_pv, (npv[x] > 0 || kk > 0) ? 1u : 0u);
+                        sdesc_sw128(vt + kk * 2048, kSub, 1024), idesc_pv, (npv[i] > 0 || kk > 0) ? 1u : 0u);
             }
-            if (!mbar_wait_bounded(&p_full[x], pwaits[x] & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
-            ++pwaits[x];
+            if (!mbar_wait_bounded(&p_full[x], pwaits[i] & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+            ++pwaits[i];
             tc_fence_after();
 #pragma unroll
             for (int kk = C::kSepP ? 0 : kTile / 32; kk < kTile / 16; ++kk)
               umma_ts(tmem + C::o_col(x), tmem + C::p_col(x) + kk * 8,
-                      sdesc_sw128(vt + kk * 2048, kSub, 1024), idesc_pv, (npv[x] > 0 || kk > 0) ? 1u : 0u);
-            ++npv[x];
+                      sdesc_sw128(vt + kk * 2048, kSub, 1024), idesc_pv, (npv[i] > 0 || kk > 0) ? 1u : 0u);
+            ++npv[i];
             if (C::kSepP) umma_commit(&pv_done[x]);
-            if (j == last[x]) umma_commit(&o_full[x]);
-            else if (!C::kSepP && uses(w, x, j + 1)) ok = issue_qk(x, j + 1);
+            if (j == last[i]) umma_commit(&o_full[x]);
+            else if (!C::kSepP && uses(w, tr[i], x, j + 1)) ok = issue_qk(i, j + 1);
           }
           umma_commit(&kv_empty[st]);
         }
