@@ -116,6 +116,34 @@ def test_edge_cases(name, w):
     _check_workload(w)
 
 
+# Key rows scaled up so that later key tiles score far above the running max of the
+# earlier ones: x30 makes some rows jump by more than 2^64 (log2 units) within a
+# unit, x3 by a few powers of two, x0.01 shrinks a block.  The separate-P kernels
+# (D = 64) take a tile's exponentials against the running max and find the tile max
+# alongside them, redoing a tile that jumps past the guard; D = 128 takes the max
+# first.  Both must still match the oracle.
+JUMPS = [
+    ("d64_window", _small("longt5_local", local_bias=False, window=(300,) * 3, padding=0)),
+    ("d64_local_bias", _small("longt5_local", window=(300,) * 3)),
+    ("d64_side_keys", _small("longt5_tglobal")),
+    ("d64_globals_padding", _small("longformer_base")),
+    ("d128_causal_gqa", _small("swan_swa")),
+]
+
+
+@pytest.mark.parametrize("name,w", JUMPS, ids=[e[0] for e in JUMPS])
+def test_scores_jumping_between_key_tiles(name, w):
+    _need_gpu()
+    inp = workloads.make_inputs(w)
+    k = inp["k"].float()
+    n = k.shape[2]
+    for lo, hi, f in ((n * 3 // 8, n * 3 // 8 + 120, 30.0), (n * 5 // 8, n * 5 // 8 + 100, 3.0),
+                      (n * 7 // 8, n * 7 // 8 + 60, 0.01)):
+        k[:, :, lo:hi] *= f
+    inp["k"] = k.to(w.torch_dtype)
+    _check_workload(w, inp)
+
+
 SUPPORT = [
     # (n, D, r, dilation, causal, g, padding)
     (128, 128, 5, 1, False, 0, 0),
