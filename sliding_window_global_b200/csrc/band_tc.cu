@@ -71,12 +71,26 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 
-#ifndef SWA_EMU_PER32
-#define SWA_EMU_PER32 8
+#ifndef SWA_EMU_PER32_D128
+#define SWA_EMU_PER32_D128 0
 #endif
-// Of every 32 exponentials, this many are evaluated by the FMA-pipe polynomial
-// instead of MUFU.EX2, balancing the two pipes.
-constexpr int kEmuPer32 = SWA_EMU_PER32;
+#ifndef SWA_EMU_PER32_D64
+#define SWA_EMU_PER32_D64 8
+#endif
+// Of every 32 exponentials, this many (a multiple of 4) are evaluated by the
+// FMA-pipe polynomial instead of MUFU.EX2; measured best per head size.
+template <int D>
+__host__ __device__ constexpr int emu_per32() {
+  return D == 128 ? SWA_EMU_PER32_D128 : SWA_EMU_PER32_D64;
+}
+
+// Where the tile max is taken: once after the tile-kind branches (D = 128), or
+// inside each branch (D = 64).  Both compute the same value; the code placement
+// was measured faster for each head size.
+template <int D>
+__host__ __device__ constexpr bool max_after_branches() {
+  return D == 128;
+}
 
 template <int D>
 struct Cfg {
@@ -397,6 +411,7 @@ template <int D, int MODE, bool LOCAL, bool RAND>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ AttnParams p) {
   using C = Cfg<D>;
   constexpr int NS = C::NS;
+  constexpr bool kMaxAfter = max_after_branches<D>();
   constexpr int kIssuers = C::kSepP ? 2 : 1;              // MMA-issuing warps
   constexpr int kTilesPerIssuer = 2 / kIssuers;
   extern __shared__ uint8_t smem_raw[];
@@ -824,9 +839,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             for (int e = 0; e < kTile; ++e) s[e] = (e < hi_t) ? s[e] : -INFINITY;
           }
           if (has_local) {
-            tmax = row_max128(s);
+            if (!kMaxAfter) tmax = row_max128(s);
           } else {
-            tmax = row_max128(s) * sl2;
+            if (!kMaxAfter) tmax = row_max128(s) * sl2;
             raw = true;
           }
         } else if (j < w.nband + w.ngc) {
@@ -859,7 +874,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const bool allowed = row_valid && cv >= 0 && !inwin;
             s[e] = allowed ? s[e] * sl2 : -INFINITY;
           }
-          tmax = row_max128(s);
+          if (!kMaxAfter) tmax = row_max128(s);
         } else if (has_rand && j >= w.rand0) {
           // random key block: keys below the valid length and outside the row's
           // window; a block repeated earlier in the list is masked whole
@@ -883,7 +898,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch)
             if (__any_sync(0xffffffffu, row_valid && !dup && 32 * ch < v_t)) live |= 1u << ch;
-          tmax = row_max128(s);
+          if (!kMaxAfter) tmax = row_max128(s);
         } else {
           const int s0 = (j - w.nband - w.ngc) * kTile;
           const int lim = row_valid ? p.S - s0 : 0;
@@ -917,11 +932,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             for (int ch = 0; ch < 4; ++ch)
               if (__any_sync(0xffffffffu, 32 * ch < lim)) live |= 1u << ch;
           }
-          tmax = row_max128(s);
+          if (!kMaxAfter) tmax = row_max128(s);
         }
 
         // Online softmax with a lazy rescale: the reference max m only moves when
         // the tile max exceeds it by more than 2^8 (l and O always share m).
+        if (kMaxAfter) tmax = row_max128(s) * (raw ? sl2 : 1.f);
         const float m_new = fmaxf(m, tmax);
         const bool need = (m == -INFINITY) ? (m_new > -INFINITY) : (m_new > m + kRescaleThreshold);
         const bool rescale = __any_sync(0xffffffffu, need);
@@ -969,7 +985,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               float a0, a1, a2, a3;
               ffma2(a0, a1, s[e], s[e + 1], mul, mul, neg_m, neg_m);
               ffma2(a2, a3, s[e + 2], s[e + 3], mul, mul, neg_m, neg_m);
-              if (q < kEmuPer32) {
+              if (q < emu_per32<D>()) {
                 exp2_poly2(a0, a1, a0, a1);
                 exp2_poly2(a2, a3, a2, a3);
               } else {
