@@ -115,6 +115,16 @@ struct Cfg {
   }
 };
 
+// The register split must fit the budget the CTA is launched with (a larger sum
+// would leave setmaxnreg.inc waiting), and the shared memory one CTA per SM.
+static_assert(kSoftmaxThreads * kRegsSoftmax + (kThreads - kSoftmaxThreads) * kRegsControl <= kThreads * 168,
+              "setmaxnreg split exceeds the launch register budget");
+static_assert(Cfg<64>::kSmemBytes + 2 * kTile * 4 + 16 <= 227 * 1024, "shared memory, D = 64");
+static_assert(Cfg<128>::kSmemBytes + 2 * kTile * 4 + 16 <= 227 * 1024, "shared memory, D = 128");
+static_assert(emu_per32<64>() % 4 == 0 && emu_per32<64>() <= 32 && emu_per32<128>() % 4 == 0 &&
+                  emu_per32<128>() <= 32,
+              "polynomial exponentials come in groups of four");
+
 // ------------------------------------------------------------------ work description
 struct Work {
   bool valid;           // the unit id names real work
