@@ -1,0 +1,319 @@
+"""Model check of the band kernel's barrier protocol (host only, no GPU).
+
+The persistent band kernel runs one TMA producer, one or two MMA issuers and two
+softmax groups that hand work to each other through mbarriers (csrc/band_tc.cu).
+This test replays that protocol as a discrete-event simulation with a random
+scheduler over random unit shapes, for both TMEM layouts:
+
+* P over S (D = 128): one issuer for both query tiles, P published in two halves,
+  the next S issued after the PV that reads P;
+* separate P (D = 64): one issuer per query tile, the next S issued as soon as the
+  softmax has read the current one (up to NS - 1 key tiles ahead), and every
+  issuer releasing every K/V ring slot of the unit (kv_empty counts two arrivals).
+
+MMAs complete asynchronously and in issue order per issuer; a commit arrives on its
+barrier once the MMAs issued before it have completed.  Checked on every run:
+
+* no deadlock: every agent finishes;
+* no parity-ambiguous wait: a barrier is never two phases ahead of a waiter (the
+  hardware's parity test would then block for good);
+* no K/V slot is refilled while an MMA that reads its previous contents is pending;
+* every query tile's softmax sees exactly its own key tiles, in order.
+
+Optionally both softmax groups also meet at every unit start, as they do when a side
+or local bias is staged in shared memory.
+"""
+import random
+
+import pytest
+
+
+class Barrier:
+    def __init__(self, name, count):
+        self.name, self.count, self.arrivals, self.done = name, count, 0, 0
+
+    def arrive(self):
+        self.arrivals += 1
+        assert self.arrivals <= self.count
+        if self.arrivals == self.count:
+            self.arrivals = 0
+            self.done += 1
+
+
+class ProtocolError(AssertionError):
+    pass
+
+
+def wait(bar, k):
+    """Generator step: wait for the completion of phase k (parity wait)."""
+    while True:
+        if bar.done - k >= 2:
+            raise ProtocolError(f"{bar.name}: {bar.done} phases done, waiter on phase {k}")
+        if bar.done > k:
+            return
+        yield
+
+
+def random_units(rng, n_units):
+    """Tile lists of random units, shaped as the kernel builds them: band tiles from
+    the first key of tile A's window, so A uses tiles 0..a_hi and B, whose rows start
+    128 class rows later, tiles b_lo..nband-1 with b_lo 0 (paired heads or a window
+    reaching back a whole tile) or 1; the band is the union of the two windows; then
+    global and side tiles (both tiles), then the random tiles, alternating A, B."""
+    units = []
+    for _ in range(n_units):
+        kind = rng.random()
+        nband = rng.randint(1, 5)
+        b_active = rng.random() > 0.15
+        if b_active:
+            b_lo = rng.randint(0, min(1, nband - 1))
+            a_hi = rng.randint(max(0, b_lo - 1), nband - 1)
+        else:
+            b_lo, a_hi = nband, nband - 1
+        use_a = [j <= a_hi for j in range(nband)]
+        use_b = [b_active and j >= b_lo for j in range(nband)]
+        extra = rng.randint(0, 3) if kind < 0.5 else 0        # global / side tiles: both tiles
+        use_a += [True] * extra
+        use_b += [b_active] * extra
+        nr = rng.randint(0, 3) if kind > 0.7 else 0           # random tiles, alternating
+        for t in range(nr):
+            for x in range(2 if b_active else 1):
+                use_a.append(x == 0)
+                use_b.append(x == 1)
+        units.append((use_a, use_b, b_active))
+    return units
+
+
+def simulate(seed, sep_p, staged=False, n_units=12):
+    rng = random.Random(seed)
+    NS = 4 if sep_p else 2
+    issuers = 2 if sep_p else 1
+    units = random_units(rng, n_units)
+    B = {}
+
+    def bar(name, count=1):
+        B[name] = Barrier(name, count)
+        return B[name]
+
+    q_full = [bar(f"q_full{x}") for x in range(2)]
+    q_empty = [bar(f"q_empty{x}") for x in range(2)]
+    k_full = [bar(f"k_full{s}") for s in range(NS)]
+    v_full = [bar(f"v_full{s}") for s in range(NS)]
+    kv_empty = [bar(f"kv_empty{s}", issuers) for s in range(NS)]
+    s_full = [bar(f"s_full{x}") for x in range(2)]
+    s_free = [bar(f"s_free{x}", 128) for x in range(2)]
+    p_half = [bar(f"p_half{x}", 128) for x in range(2)]
+    p_full = [bar(f"p_full{x}", 128) for x in range(2)]
+    pv_done = [bar(f"pv_done{x}") for x in range(2)]
+    o_full = [bar(f"o_full{x}") for x in range(2)]
+
+    # per issuer: FIFO of ('mma', slot, use) and ('commit', barrier) entries
+    pipes = [[] for _ in range(issuers)]
+    pending_reads = {}                       # (slot, use) -> MMAs not yet complete
+    loads = [0] * NS                         # loads into each slot so far
+    seen = [[], []]                          # key tiles each softmax group processed
+
+    def mma(i, slot):
+        key = (slot, loads[slot] - 1)
+        pending_reads[key] = pending_reads.get(key, 0) + 1
+        pipes[i].append(("mma", key))
+
+    def commit(i, b):
+        pipes[i].append(("commit", b))
+
+    def producer():
+        qloads = [0, 0]
+        kv = 0
+        for use_a, use_b, b_act in units:
+            for x, act in ((0, True), (1, b_act)):
+                if not act:
+                    continue
+                if qloads[x] > 0:
+                    yield from wait(q_empty[x], qloads[x] - 1)
+                q_full[x].arrive()
+                qloads[x] += 1
+            for j in range(len(use_a)):
+                st = kv % NS
+                if kv >= NS:
+                    yield from wait(kv_empty[st], kv // NS - 1)
+                if pending_reads.get((st, loads[st] - 1), 0):
+                    raise ProtocolError(f"slot {st} refilled while an MMA still reads it")
+                loads[st] += 1
+                yield
+                k_full[st].arrive()
+                yield
+                v_full[st].arrive()
+                kv += 1
+
+    def issuer(i):
+        xs = [i] if issuers == 2 else [0, 1]
+        qwaits = {x: 0 for x in xs}
+        pwaits = {x: 0 for x in xs}
+        nqk = {x: 0 for x in xs}
+        kv = 0
+        for use_a, use_b, b_act in units:
+            use = {0: use_a, 1: use_b}
+            T = len(use_a)
+            act = {x: (x == 0 or b_act) for x in xs}
+            first = {x: next((j for j in range(T) if use[x][j]), -1) for x in xs}
+            last = {x: max((j for j in range(T) if use[x][j]), default=-1) for x in xs}
+            issued = {x: -1 for x in xs}
+            npv = {x: 0 for x in xs}
+
+            def issue_qk(x, j):
+                g = kv + j
+                yield from wait(k_full[g % NS], g // NS)
+                if sep_p and nqk[x] > 0:
+                    yield from wait(s_free[x], nqk[x] - 1)
+                nqk[x] += 1
+                mma(i, g % NS)
+                commit(i, s_full[x])
+                if j == last[x]:
+                    commit(i, q_empty[x])
+                issued[x] = j
+
+            for x in xs:
+                if act[x] and first[x] >= 0:
+                    yield from wait(q_full[x], qwaits[x])
+                    qwaits[x] += 1
+                    yield from issue_qk(x, first[x])
+            for j in range(T):
+                g = kv + j
+                st = g % NS
+                anyuse = False
+                for x in xs:
+                    u = act[x] and use[x][j]
+                    anyuse = anyuse or u
+                    if u and issued[x] < j:
+                        yield from issue_qk(x, j)
+                if sep_p:
+                    for x in xs:
+                        if not (act[x] and use[x][j]) or issued[x] != j:
+                            continue
+                        jn = j + 1
+                        while jn < T and jn < j + NS and not use[x][jn]:
+                            jn += 1
+                        if jn < T and jn < j + NS:
+                            yield from issue_qk(x, jn)
+                yield from wait(v_full[st], g // NS)
+                if not anyuse:
+                    kv_empty[st].arrive()
+                    continue
+                for x in xs:
+                    if not (act[x] and use[x][j]):
+                        continue
+                    if not sep_p:
+                        yield from wait(p_half[x], pwaits[x])
+                        mma(i, st)
+                    yield from wait(p_full[x], pwaits[x])
+                    pwaits[x] += 1
+                    mma(i, st)
+                    npv[x] += 1
+                    if sep_p:
+                        commit(i, pv_done[x])
+                    if j == last[x]:
+                        commit(i, o_full[x])
+                    elif not sep_p and j + 1 < T and use[x][j + 1]:
+                        yield from issue_qk(x, j + 1)
+                commit(i, kv_empty[st])
+            kv += T
+
+    met = {}                                 # unit -> softmax groups at the staging barrier
+
+    def softmax(x):
+        it = pw = oc = 0
+        for u, (use_a, use_b, b_act) in enumerate(units):
+            if staged:
+                # a side or local bias is staged per unit by both groups together
+                # (a named barrier over both groups, also when tile B is inactive)
+                met[u] = met.get(u, 0) + 1
+                while met[u] < 2:
+                    yield
+            if x == 1 and not b_act:
+                continue
+            use = use_a if x == 0 else use_b
+            for j in range(len(use)):
+                if not use[j]:
+                    continue
+                yield from wait(s_full[x], it)
+                seen[x].append(j)
+                if sep_p:
+                    for _ in range(128):
+                        s_free[x].arrive()
+                yield
+                if sep_p and pw > 0:
+                    yield from wait(pv_done[x], pw - 1)
+                if not sep_p:
+                    for _ in range(128):
+                        p_half[x].arrive()
+                    yield
+                for _ in range(128):
+                    p_full[x].arrive()
+                pw += 1
+                it += 1
+            yield from wait(o_full[x], oc)
+            oc += 1
+
+    agents = [producer()] + [issuer(i) for i in range(issuers)] + [softmax(0), softmax(1)]
+    alive = list(range(len(agents)))
+
+    def step_pipe(i):
+        kind, val = pipes[i].pop(0)
+        if kind == "mma":
+            pending_reads[val] -= 1
+        else:
+            val.arrive()
+
+    stalls = 0
+    while alive or any(pipes):
+        choices = [("agent", a) for a in alive] + [("pipe", i) for i in range(issuers) if pipes[i]]
+        kind, who = rng.choice(choices)
+        if kind == "pipe":
+            step_pipe(who)
+            stalls = 0
+            continue
+        try:
+            next(agents[who])
+            stalls += 1
+        except StopIteration:
+            alive.remove(who)
+            stalls = 0
+        if stalls > 20000:
+            raise ProtocolError("deadlock: no agent can make progress")
+
+    for x in range(2):
+        expect = []
+        for use_a, use_b, b_act in units:
+            if x == 1 and not b_act:
+                continue
+            expect += [j for j, u in enumerate(use_a if x == 0 else use_b) if u]
+        assert seen[x] == expect
+
+
+@pytest.mark.parametrize("staged", [False, True], ids=["", "bias_staged"])
+@pytest.mark.parametrize("sep_p", [False, True], ids=["p_over_s_one_issuer", "separate_p_two_issuers"])
+def test_barrier_protocol_random_schedules(sep_p, staged):
+    for seed in range(300):
+        simulate(seed, sep_p, staged)
+
+
+def test_model_detects_a_broken_release_count():
+    """The model is not vacuous: with kv_empty counting one arrival while two
+    issuers release every slot, a slot gets refilled under a pending reader or a
+    barrier runs two phases ahead of a waiter on some schedule."""
+    orig = Barrier.__init__
+
+    def one_arrival(self, name, count):
+        orig(self, name, 1 if name.startswith("kv_empty") else count)
+
+    Barrier.__init__ = one_arrival
+    try:
+        caught = 0
+        for seed in range(300):
+            try:
+                simulate(seed, True)
+            except AssertionError:
+                caught += 1
+        assert caught > 0
+    finally:
+        Barrier.__init__ = orig
