@@ -21,7 +21,8 @@ barrier once the MMAs issued before it have completed.  Checked on every run:
 * every query tile's softmax sees exactly its own key tiles, in order.
 
 Optionally both softmax groups also meet at every unit start, as they do when a side
-or local bias is staged in shared memory.
+or local bias is staged in shared memory.  A second model covers the key-stationary
+dK/dV pass of the backward (csrc/bwd_tc.cu).  Each model has a planted-mistake test.
 """
 import random
 
@@ -317,3 +318,123 @@ def test_model_detects_a_broken_release_count():
         assert caught > 0
     finally:
         Barrier.__init__ = orig
+
+
+def simulate_dkv(seed, T, early_next=False):
+    """The key-stationary dK/dV pass (csrc/bwd_tc.cu): one key tile per CTA, its T
+    query tiles through a two-stage ring, compute groups taking alternate tiles, Pᵀ
+    and dSᵀ in one shared-memory buffer per group, the next Sᵀ/dPᵀ of a group issued
+    once its products have read the current ones."""
+    rng = random.Random(seed)
+    a_full = Barrier("a_full", 1)
+    r_full = [Barrier(f"r_full{s}", 1) for s in range(2)]
+    r_empty = [Barrier(f"r_empty{s}", 1) for s in range(2)]
+    s_full = [Barrier(f"s_full{g}", 1) for g in range(2)]
+    p_full = [Barrier(f"p_full{g}", 128) for g in range(2)]
+    pds_free = [Barrier(f"pds_free{g}", 1) for g in range(2)]
+    acc_full = Barrier("acc_full", 1)
+    pipe = []
+    pending = {}
+    loads = [0, 0]
+    pbuf_uses = [0, 0]
+    consumed = [0, 0]                       # tiles whose S^T/dP^T each group has read
+
+    def mma(key):
+        pending[key] = pending.get(key, 0) + 1
+        pipe.append(("mma", key))
+
+    def producer():
+        a_full.arrive()
+        for j in range(T):
+            st = j & 1
+            if j >= 2:
+                yield from wait(r_empty[st], (j >> 1) - 1)
+            if pending.get(("ring", st, loads[st] - 1), 0):
+                raise ProtocolError(f"ring slot {st} refilled under a pending reader")
+            loads[st] += 1
+            yield
+            r_full[st].arrive()
+
+    def issuer():
+        def issue_s(j):
+            st, g = j & 1, j & 1
+            yield from wait(r_full[st], j >> 1)
+            if consumed[g] < (j >> 1):
+                raise ProtocolError(f"S^T of tile {j} written before group {g} read tile {j - 2}")
+            mma(("ring", st, loads[st] - 1))
+            pipe.append(("commit", s_full[g]))
+
+        yield from wait(a_full, 0)
+        yield from issue_s(0)
+        if T > 1:
+            yield from issue_s(1)
+        for j in range(T):
+            g = st = j & 1
+            if early_next and j + 2 < T:         # planted mistake: before the group read S(j)
+                yield from issue_s(j + 2)
+            yield from wait(p_full[g], j >> 1)
+            mma(("ring", st, loads[st] - 1))
+            mma(("pbuf", g, pbuf_uses[g] - 1))
+            pipe.append(("commit", pds_free[g]))
+            pipe.append(("commit", r_empty[st]))
+            if j + 2 < T and not early_next:
+                yield from issue_s(j + 2)
+        pipe.append(("commit", acc_full))
+
+    def compute(g):
+        nt = 0
+        for j in range(g, T, 2):
+            yield from wait(s_full[g], nt)
+            consumed[g] += 1
+            if nt > 0:
+                yield from wait(pds_free[g], nt - 1)
+            if pending.get(("pbuf", g, pbuf_uses[g] - 1), 0):
+                raise ProtocolError(f"P/dS buffer {g} rewritten under a pending reader")
+            pbuf_uses[g] += 1
+            yield
+            for _ in range(128):
+                p_full[g].arrive()
+            nt += 1
+        if T > 0:
+            yield from wait(acc_full, 0)
+
+    agents = [producer(), issuer(), compute(0), compute(1)]
+    alive = list(range(len(agents)))
+    stalls = 0
+    while alive or pipe:
+        choices = [("agent", a) for a in alive] + ([("pipe", 0)] if pipe else [])
+        kind, who = rng.choice(choices)
+        if kind == "pipe":
+            k, val = pipe.pop(0)
+            if k == "mma":
+                pending[val] -= 1
+            else:
+                val.arrive()
+            stalls = 0
+            continue
+        try:
+            next(agents[who])
+            stalls += 1
+        except StopIteration:
+            alive.remove(who)
+            stalls = 0
+        if stalls > 20000:
+            raise ProtocolError("deadlock: no agent can make progress")
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 4, 7, 12])
+def test_dkv_pass_protocol_random_schedules(T):
+    for seed in range(200):
+        simulate_dkv(seed, T)
+
+
+def test_dkv_model_detects_an_early_next_product():
+    """Issuing a group's next S^T before its softmax has read the current one is
+    caught (as an overwrite, a parity-ambiguous wait or a deadlock)."""
+    caught = 0
+    for seed in range(100):
+        try:
+            simulate_dkv(seed, 6, early_next=True)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
