@@ -363,7 +363,8 @@ def test_constant_local_bias_is_a_softmax_shift(oracle_mod):
     o1, l1, _ = pb.forward()
     assert np.max(np.abs(o0 - o1)) <= 1e-12
     m = ~np.isneginf(l0)
-    assert np.max(np.abs((l1 - l0)[m] - np.broadcast_to(c[None, :, None], l0.shape)[m])) <= 1e-12
+    assert np.array_equal(np.isneginf(l1), ~m)          # padded rows stay empty
+    assert np.max(np.abs(l1[m] - l0[m] - np.broadcast_to(c[None, :, None], l0.shape)[m])) <= 1e-12
 
 
 def test_local_bias_offset_sign_closed_form(oracle_mod):
