@@ -108,7 +108,7 @@ def simulate(seed, sep_p, staged=False, n_units=12):
     pv_done = [bar(f"pv_done{x}") for x in range(2)]
     o_full = [bar(f"o_full{x}") for x in range(2)]
 
-    # per issuer: FIFO of ('mma', slot, use) and ('commit', barrier) entries
+    # per issuer: FIFO of ('mma', (slot, use)) and ('commit', barrier) entries
     pipes = [[] for _ in range(issuers)]
     pending_reads = {}                       # (slot, use) -> MMAs not yet complete
     loads = [0] * NS                         # loads into each slot so far
@@ -159,7 +159,6 @@ def simulate(seed, sep_p, staged=False, n_units=12):
             first = {x: next((j for j in range(T) if use[x][j]), -1) for x in xs}
             last = {x: max((j for j in range(T) if use[x][j]), default=-1) for x in xs}
             issued = {x: -1 for x in xs}
-            npv = {x: 0 for x in xs}
 
             def issue_qk(x, j):
                 g = kv + j
@@ -209,7 +208,6 @@ def simulate(seed, sep_p, staged=False, n_units=12):
                     yield from wait(p_full[x], pwaits[x])
                     pwaits[x] += 1
                     mma(i, st)
-                    npv[x] += 1
                     if sep_p:
                         commit(i, pv_done[x])
                     if j == last[x]:
