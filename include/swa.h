@@ -101,9 +101,15 @@ swa_status swa_plan_create(swa_plan_t* out_plan, const swa_plan_desc* desc);
  * aligned, window < 0, dilation < 1, num_global out of range; SWA_ERR_UNSUPPORTED
  * for causal together with num_global > 0, or more than 16 distinct
  * (dilation, residue) classes; SWA_ERR_CUDA when a launch fails.  In
- * SWA_DEBUG_CHECKS mode it also synchronises and returns SWA_ERR_DEVICE_CHECK
- * (bad global_idx) or SWA_ERR_TIMEOUT.  Global-index preconditions are NOT
- * checked outside debug mode. */
+ * SWA_DEBUG_CHECKS mode a device kernel first checks global_idx (and the random
+ * blocks of swa_forward_ex); the call synchronises and reads the result back
+ * before it enqueues anything that indexes with them, returning
+ * SWA_ERR_DEVICE_CHECK with only that check launched; after the forward it
+ * synchronises again and returns SWA_ERR_TIMEOUT if a bounded wait expired.
+ * Outside debug mode the index preconditions are not checked; a position outside
+ * [0, seq_len) still never makes a kernel read or write out of bounds (its
+ * gathered row is zero and its global row is not written), but the results are
+ * then undefined. */
 swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void* v,
                        const int32_t* global_idx, int num_global, const void* side_k,
                        const void* side_v, const float* bias, const int32_t* window,
@@ -135,9 +141,9 @@ swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void
  *   their key set, as a set: keys already in the window or global, and repeated
  *   blocks, count once.  Global query rows are unaffected (they attend every
  *   key).  The caller draws the blocks.  0 <= num_rand <= 8; block indices must
- *   lie in [0, ceil(seq_len / 128)) (not checked; an index outside attends
- *   nothing).  Random blocks need dilation 1 on every head and causal == 0
- *   (else SWA_ERR_UNSUPPORTED). */
+ *   lie in [0, ceil(seq_len / 128)) (checked in SWA_DEBUG_CHECKS mode; outside
+ *   it an index outside attends nothing).  Random blocks need dilation 1 on every
+ *   head and causal == 0 (else SWA_ERR_UNSUPPORTED). */
 typedef struct {
   const void* q;
   const void* k;
@@ -274,7 +280,12 @@ swa_status swa_expand_side_bias(int num_q_heads, int num_side, int nblk, const f
  * array: each clears the error word and rewrites the rest before reading it, but
  * calls that overlap on the GPU (unordered streams or threads) race on it.
  * Arguments, layouts and the other statuses are those of swa_plan_create plus
- * swa_forward (desc: the plan descriptor; stream: a cudaStream_t).
+ * swa_forward (desc: the plan descriptor; stream: a cudaStream_t); validation
+ * and launches are shared with swa_forward.  With no plan there is no
+ * swa_plan_check: outside SWA_DEBUG_CHECKS mode this entry point never
+ * synchronises and cannot report an expired bounded wait (the next call clears
+ * the error word); set SWA_DEBUG_CHECKS in desc->flags to have each call
+ * synchronise and return SWA_ERR_TIMEOUT or SWA_ERR_DEVICE_CHECK.
  * ------------------------------------------------------------------------- */
 #define SWA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 

@@ -46,8 +46,10 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ src, uint4* __restr
     int b = (int)(bh / H);
     uint4 v = make_uint4(0, 0, 0, 0);
     if (e < g) {
-      int pos = gidx[(size_t)b * g + e];
-      v = src[(bh * n + pos) * row_vecs + x];
+      // a position outside the sequence (a broken precondition) gathers zeros
+      // instead of reading out of bounds
+      const int pos = gidx[(size_t)b * g + e];
+      if (pos >= 0 && pos < n) v = src[(bh * n + pos) * row_vecs + x];
     }
     dst[t] = v;
   }
@@ -85,6 +87,7 @@ __global__ void merge_global_rows_kernel(AttnParams p) {
     }
   }
   const int pos = p.global_idx[(size_t)b * p.g + e];
+  if (pos < 0 || pos >= p.n) return;      // broken precondition: never write out of bounds
   const size_t off = (size_t)bh * p.n + pos;
   T* o = static_cast<T*>(p.out) + off * D;
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
@@ -168,7 +171,7 @@ __global__ void simt_attn_kernel(AttnParams p, const T* __restrict__ q, const T*
       int j = gl[idx - nwin];
       int diff = i - j;
       bool inwin = (p.causal ? (diff >= 0 && diff <= r * d) : (abs(diff) <= r * d)) && (diff % d == 0);
-      if (!inwin && j < V) {
+      if (!inwin && j >= 0 && j < V) {
         krow = kb + (size_t)j * D;
         vrow = vb + (size_t)j * D;
       }
@@ -258,15 +261,25 @@ __global__ void side_aggregate_kernel(const T* __restrict__ x, T* __restrict__ o
 }
 
 // ------------------------------------------------------------------ precondition check
-// global_idx rows must be strictly increasing and inside [0, valid_len).
-__global__ void check_globals_kernel(const int32_t* __restrict__ gidx, int g, int B, int n,
-                                     const int32_t* __restrict__ valid_len, int* err) {
-  int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= B * g) return;
-  int b = t / g, e = t % g;
-  int V = valid_len ? min(valid_len[b], n) : n;
-  int pos = gidx[t];
-  bool bad = pos < 0 || pos >= V || (e > 0 && gidx[t - 1] >= pos);
+// global_idx rows must be strictly increasing and inside [0, valid_len); random
+// key blocks must lie inside [0, nqb).  Threads [0, B*g) check global_idx, the
+// next nrand_total threads the random blocks.
+__global__ void check_inputs_kernel(const int32_t* __restrict__ gidx, int g, int B, int n,
+                                    const int32_t* __restrict__ valid_len,
+                                    const int32_t* __restrict__ rand_blocks, long long nrand_total,
+                                    int nqb, int* err) {
+  const long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const long long ng = (long long)B * g;
+  bool bad = false;
+  if (t < ng) {
+    const int b = (int)(t / g), e = (int)(t % g);
+    const int V = valid_len ? min(valid_len[b], n) : n;
+    const int pos = gidx[t];
+    bad = pos < 0 || pos >= V || (e > 0 && gidx[t - 1] >= pos);
+  } else if (t - ng < nrand_total) {
+    const int blk = rand_blocks[t - ng];
+    bad = blk < 0 || blk >= nqb;
+  }
   if (bad) atomicOr(err, kDevErrCheck);
 }
 
@@ -350,10 +363,13 @@ cudaError_t launch_simt(const AttnParams& p, const void* q, const void* k, const
   return cudaGetLastError();
 }
 
-cudaError_t launch_check_globals(const AttnParams& p, cudaStream_t s) {
-  const int t = p.B * p.g;
+cudaError_t launch_check_inputs(const AttnParams& p, cudaStream_t s) {
+  const int nqb = (p.n + kTile - 1) / kTile;
+  const long long nrand = p.rand_blocks ? (long long)p.B * p.Hq * nqb * p.num_rand : 0;
+  const long long t = (long long)p.B * p.g + nrand;
   if (t == 0) return cudaSuccess;
-  check_globals_kernel<<<(t + 255) / 256, 256, 0, s>>>(p.global_idx, p.g, p.B, p.n, p.valid_len, p.err);
+  check_inputs_kernel<<<(unsigned)((t + 255) / 256), 256, 0, s>>>(p.global_idx, p.g, p.B, p.n, p.valid_len,
+                                                                   p.rand_blocks, nrand, nqb, p.err);
   return cudaGetLastError();
 }
 

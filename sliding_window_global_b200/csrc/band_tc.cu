@@ -695,7 +695,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int u = tr.u0 + row;
       int pos = 0;
       if (MODE == 0) pos = w.c + w.d * u;
-      else if (row_valid) pos = p.global_idx[(size_t)w.b * p.g + w.u0[0] + row];
+      else if (row_valid)   // clamped: a broken precondition must not index the bias out of bounds
+        pos = min(max(p.global_idx[(size_t)w.b * p.g + w.u0[0] + row], 0), p.n - 1);
 
       // Bias rows of this unit, four copies shifted by 0..3 floats so that every
       // row can read 16-byte aligned vectors (both groups stage together).
@@ -703,7 +704,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       // coordinates t), zero outside |t| <= r; band tiles read 128 consecutive
       // entries starting anywhere in [-r_eff - 254, r_eff + 127] (r_eff = min(r, n_c)).
       const int r_eff = min(w.r, p.cls[w.cls].n_c);
-      int qblk_hi = 0;
+      int qblk_hi = 0, qblk_lo = 0;
       bool bias_staged = false;
       if (has_bias) {
         int pos_lo, pos_hi;
@@ -712,11 +713,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           pos_lo = w.c + w.d * w.u0[0];
           pos_hi = w.c + w.d * last_row;
         } else {
-          pos_lo = p.global_idx[(size_t)w.b * p.g + w.u0[0]];
-          pos_hi = p.global_idx[(size_t)w.b * p.g + w.u0[0] + w.nvalid[0] - 1];
+          pos_lo = min(max(p.global_idx[(size_t)w.b * p.g + w.u0[0]], 0), p.n - 1);
+          pos_hi = min(max(p.global_idx[(size_t)w.b * p.g + w.u0[0] + w.nvalid[0] - 1], 0), p.n - 1);
+          pos_hi = max(pos_hi, pos_lo);
         }
         qblk_hi = pos_hi / p.side_block;
-        const int bias_len = p.S + (qblk_hi - pos_lo / p.side_block);
+        qblk_lo = pos_lo / p.side_block;
+        const int bias_len = p.S + (qblk_hi - qblk_lo);
         bias_staged = bias_len + 4 <= side_stride;
         if (bias_staged) {
           named_barrier_sync(3, kSoftmaxThreads);     // both groups are done with the old segment
@@ -785,7 +788,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
       if (!row_valid) khi = klo;               // padded row: attends nothing
       const int qblk = (p.S > 0) ? pos / p.side_block : 0;
-      const int boff = qblk_hi - qblk;
+      // offset of this row's bias segment inside the staged one; it lies in range
+      // whenever global_idx is sorted (clamped so that unsorted input stays in bounds)
+      const int boff = min(max(qblk_hi - qblk, 0), qblk_hi - qblk_lo);
       const float* bias_row =
           has_bias ? p.bias + (size_t)w.h * (p.S + p.nblk - 1) + (p.nblk - 1 - qblk) : nullptr;
 
@@ -894,7 +899,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 #pragma unroll
           for (int t2 = 0; t2 < kRandRegs; ++t2)
             if (t2 == t) kb = rbl[t2];
-          bool dup = false;
+          // an index outside the key blocks attends nothing (masked like a repeat)
+          bool dup = kb < 0 || kb * kTile >= p.n;
 #pragma unroll
           for (int t2 = 0; t2 < kRandRegs; ++t2) dup = dup || (t2 < t && rbl[t2] == kb);
           const int kv0 = kb * kTile;

@@ -74,7 +74,9 @@ cudaError_t launch_gather_globals(const AttnParams& p, const void* q, const void
 cudaError_t launch_merge_global_rows(const AttnParams& p, int bf16_out, cudaStream_t s);
 cudaError_t launch_simt(const AttnParams& p, const void* q, const void* k, const void* v,
                         const void* side_k, const void* side_v, int bf16, cudaStream_t s);
-cudaError_t launch_check_globals(const AttnParams& p, cudaStream_t s);
+// Debug check of the index inputs: global_idx rows strictly increasing inside
+// [0, valid_len), random key blocks inside [0, ceil(n / 128)); sets kDevErrCheck.
+cudaError_t launch_check_inputs(const AttnParams& p, cudaStream_t s);
 cudaError_t launch_wait_probe(int* err, uint64_t limit_ns, cudaStream_t s);
 cudaError_t launch_side_aggregate(const void* x, void* out, int B, int H, int n, int D, int kb,
                                   const int32_t* valid_len, int bf16, cudaStream_t s);

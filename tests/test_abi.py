@@ -60,6 +60,28 @@ def test_plan_create_rejects_bad_descriptors(lib, bad):
     assert not h.value
 
 
+_BAD_DESCRIPTORS = [
+    (dict(batch=0), 1), (dict(seq_len=0), 1), (dict(num_q_heads=3), 1), (dict(num_kv_heads=0), 1),
+    (dict(dtype=7), 1), (dict(max_global=-1), 1), (dict(max_global=300), 1),
+    (dict(num_side=4, side_block=0), 1), (dict(scale=-1.0), 1), (dict(flags=8), 1),
+    (dict(head_dim=0), 1), (dict(head_dim=96), 2), (dict(num_q_heads=256, num_kv_heads=1), 2),
+    (dict(batch=2**31 - 1), 2),
+]
+
+
+@pytest.mark.parametrize("bad,status", _BAD_DESCRIPTORS)
+def test_both_forward_entry_points_validate_descriptors_alike(lib, bad, status):
+    """swa_plan_create and swa_forward_noalloc share one descriptor validator: the same
+    bad descriptor gives the same status from both, before any device work."""
+    h = ctypes.c_void_p()
+    d = _desc(**bad)
+    assert lib.swa_plan_create(ctypes.byref(h), ctypes.byref(d)) == status
+    win = (ctypes.c_int32 * max(1, d.num_q_heads))()
+    st = lib.swa_forward_noalloc(ctypes.byref(d), None, None, None, None, 0, None, None, None, win,
+                                 None, 0, None, None, None, None)
+    assert st == status
+
+
 def test_plan_create_unsupported_head_dim(lib):
     h = ctypes.c_void_p()
     d = _desc(head_dim=96)

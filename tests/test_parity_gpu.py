@@ -280,23 +280,55 @@ def test_side_aggregate_matches_oracle():
 
 
 def test_debug_mode_flags_bad_global_index():
-    """A global index out of [0, valid_len) is a precondition failure that debug mode
-    reports as a status (the kernels never read it: the check runs first)."""
+    """A global index list that is not strictly increasing inside [0, valid_len) is a
+    precondition failure.  Debug mode checks it on the device and reads the result
+    back before any kernel that indexes with global_idx is enqueued: the status is
+    SWA_ERR_DEVICE_CHECK, only the check kernel ran, and out is untouched."""
     _need_gpu()
     from sliding_window_global_b200 import Plan, SwaError
     w = workloads.SMALL["longformer_base"]
     inp = helpers.to_dev(helpers.host_problem(w))
+    n, V = w.seq_len, w.valid_len
     plan = Plan(w.batch, w.seq_len, w.q_heads, w.kv_heads, w.head_dim, torch.bfloat16,
                 max_global=4, debug=True)
-    bad = torch.tensor([[3, 2, 5, 9]], dtype=torch.int32, device="cuda")  # not increasing
-    with pytest.raises(SwaError) as e:
-        plan.forward(inp["q"], inp["k"], inp["v"], window=inp["window"], global_idx=bad,
-                     valid_len=inp["valid_len"])
-    assert e.value.status == 6
+    out = torch.full((w.batch, w.q_heads, n, w.head_dim), 7.0, dtype=torch.bfloat16, device="cuda")
+    for bad in ([3, 2, 5, 9],            # not increasing
+                [2, 3, 5, n + 40],       # beyond the sequence
+                [2, 3, 5, V],            # a padded position
+                [-1, 3, 5, 9]):          # negative
+        idx = torch.tensor([bad], dtype=torch.int32, device="cuda")
+        with pytest.raises(SwaError) as e:
+            plan.forward(inp["q"], inp["k"], inp["v"], window=inp["window"], global_idx=idx,
+                         valid_len=inp["valid_len"], out=out)
+        assert e.value.status == 6, bad
+        assert plan.last_launches == 1, bad          # the check kernel alone
+        assert plan.check() == 0                     # the word was read and cleared
+        torch.cuda.synchronize()
+        assert bool((out == 7.0).all()), bad
     good = torch.tensor([[2, 3, 5, 9]], dtype=torch.int32, device="cuda")
     plan.forward(inp["q"], inp["k"], inp["v"], window=inp["window"], global_idx=good,
                  valid_len=inp["valid_len"])
     assert plan.check() == 0
+
+
+def test_debug_mode_flags_bad_random_block():
+    """Random key blocks outside [0, ceil(n/128)) fail the debug check the same way."""
+    _need_gpu()
+    from sliding_window_global_b200 import Plan, SwaError
+    w = workloads.SMALL["bigbird_itc"]
+    dinp = helpers.to_dev(helpers.host_problem(w))
+    plan = Plan(w.batch, w.seq_len, w.q_heads, w.kv_heads, w.head_dim, torch.bfloat16,
+                max_global=w.num_global, debug=True)
+    kw = dict(window=dinp["window"], global_idx=dinp["global_idx"], valid_len=dinp["valid_len"])
+    plan.forward(dinp["q"], dinp["k"], dinp["v"], rand_blocks=dinp["rand_blocks"], **kw)
+    assert plan.check() == 0
+    nqb = (w.seq_len + 127) // 128
+    for val in (nqb, -1):
+        rb = dinp["rand_blocks"].clone()
+        rb[0, 1, 2, 0] = val
+        with pytest.raises(SwaError) as e:
+            plan.forward(dinp["q"], dinp["k"], dinp["v"], rand_blocks=rb, **kw)
+        assert e.value.status == 6 and plan.last_launches == 1
 
 
 def test_repeat_calls_deterministic_and_launch_count():

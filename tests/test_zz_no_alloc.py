@@ -72,6 +72,16 @@ CASES = [
     ("dilated_globals", workloads.SMALL["dilated"], 3002),
     ("gqa_causal", workloads.SMALL["swan_swa"], 3003),
     ("fp32", workloads.SMALL["longformer_tiny"], 3004),
+    # global tokens together with side keys and their bias: one more split (the side
+    # keys') in the scratch layout
+    ("globals_side_bias", dataclasses.replace(workloads.SMALL["longt5_tglobal"], name="tglobal_globals",
+                                              num_global=12, global_mode="leading"), 3005),
+    # 1000 global slots at D=128: the full set of global-row splits would exceed the
+    # scratch array, so the entry point uses fewer splits than the plan-based path
+    ("globals_near_limit", dataclasses.replace(workloads.SMALL["longformer_base"], name="many_globals",
+                                               q_heads=2, kv_heads=2, head_dim=128, seq_len=2048,
+                                               num_global=1000, window=(64, 64), dilation=(1, 1),
+                                               padding=0), 3006),
 ]
 
 
