@@ -87,6 +87,9 @@ def _load():
             lib.oracle_side_aggregate.restype = I
             lib.oracle_backward.argtypes = [I, I, I, I, I, P, P, P, P, P, I, P, P, I, P, D, EX, P, P, P]
             lib.oracle_backward.restype = I
+            lib.oracle_backward_ex.argtypes = [I, I, I, I, I, P, P, P, P, P, I, P, P, I, I, P, P, P, I,
+                                               P, D, EX, P, P, P, P, P]
+            lib.oracle_backward_ex.restype = I
             lib.oracle_num_threads.argtypes = []
             lib.oracle_num_threads.restype = I
             _lib = lib
@@ -201,19 +204,26 @@ class Problem:
         return out, lse, cnt
 
     def backward(self, dout):
-        """fp64 (dq, dk, dv) for the upstream gradient ``dout`` (like q); no side keys."""
-        if self.S:
-            raise ValueError("the oracle backward covers problems without side keys")
+        """fp64 gradients for the upstream gradient ``dout`` (like q): (dq, dk, dv), plus
+        (dside_k, dside_v) when the problem has side keys (a 5-tuple then)."""
         lib = _load()
         do = _f32(dout)
         dq = np.empty((self.B, self.Hq, self.n, self.D), dtype=np.float64)
         dk = np.empty((self.B, self.Hkv, self.n, self.D), dtype=np.float64)
         dv = np.empty((self.B, self.Hkv, self.n, self.D), dtype=np.float64)
-        _check(lib.oracle_backward(self.B, self.Hq, self.Hkv, self.n, self.D, _ptr(self.q),
-                                   _ptr(self.k), _ptr(self.v), _ptr(do), _ptr(self.global_idx),
-                                   self.g, _ptr(self.window), _ptr(self.dilation), self.causal,
-                                   _ptr(self.valid_len), self.scale, self._ex(), _ptr(dq), _ptr(dk),
-                                   _ptr(dv)), "backward")
+        dsk = dsv = None
+        if self.S:
+            dsk = np.empty((self.B, self.Hkv, self.S, self.D), dtype=np.float64)
+            dsv = np.empty((self.B, self.Hkv, self.S, self.D), dtype=np.float64)
+        _check(lib.oracle_backward_ex(self.B, self.Hq, self.Hkv, self.n, self.D, _ptr(self.q),
+                                      _ptr(self.k), _ptr(self.v), _ptr(do), _ptr(self.global_idx),
+                                      self.g, _ptr(self.side_k), _ptr(self.side_v), self.S,
+                                      self.side_block, _ptr(self.bias), _ptr(self.window),
+                                      _ptr(self.dilation), self.causal, _ptr(self.valid_len),
+                                      self.scale, self._ex(), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dsk),
+                                      _ptr(dsv)), "backward")
+        if self.S:
+            return dq, dk, dv, dsk, dsv
         return dq, dk, dv
 
     def dense_bruteforce(self):

@@ -625,40 +625,50 @@ int oracle_side_aggregate(int B, int H, int n, int D, int kb, const float *x,
 }
 
 /*
- * oracle_backward: gradients of the attention (no side keys) with respect to q,
- * k and v for an upstream gradient dout = dL/do, by the chain rule through the
- * softmax of each row [definition of softmax attention; the key sets are those
- * of oracle_forward]:
- *   p_j  = exp(s_j - lse),  s_j = scale <q_i, k_j> (+ local bias)
+ * oracle_backward_ex: gradients of the attention with respect to q, k, v and the
+ * side keys / values, for an upstream gradient dout = dL/do, by the chain rule
+ * through the softmax of each row [definition of softmax attention; the key sets
+ * are those of oracle_forward, side keys appended to every valid row]:
+ *   p_j  = exp(s_j - lse),  s_j = scale <q_i, k_j> (+ local bias / side bias)
  *   dp_j = <dout_i, v_j>,   Delta_i = sum_j p_j dp_j,   ds_j = p_j (dp_j - Delta_i)
  *   dq_i = scale sum_j ds_j k_j,  dk_j += scale ds_j q_i,  dv_j += p_j dout_i
- * Padded rows contribute nothing.  dq [B,Hq,n,D], dk/dv [B,Hkv,n,D] (fp64) are
- * overwritten.  Work is split over (batch, KV head) pairs, so the accumulations
- * into dk/dv never race.
+ * with j running over K(i) and the side keys (whose rows of dk / dv are dside_k /
+ * dside_v).  The biases are inputs, not differentiated.  Padded rows contribute
+ * nothing.  dq [B,Hq,n,D], dk/dv [B,Hkv,n,D], dside_k/dside_v [B,Hkv,S,D] (fp64,
+ * may be NULL when S = 0) are overwritten.  Work is split over (batch, KV head)
+ * pairs, so the accumulations into dk/dv and dside_k/dside_v never race.
  */
-int oracle_backward(int B, int Hq, int Hkv, int n, int D, const float *q, const float *k,
-                    const float *v, const float *dout, const int32_t *global_idx, int g,
-                    const int32_t *window, const int32_t *dilation, int causal,
-                    const int32_t *valid_len, double scale, const oracle_extras *ex,
-                    double *dq, double *dk, double *dv) {
-    oracle_problem P = {B, Hq, Hkv, n, D, q, k, v, global_idx, g, NULL, NULL,
-                        0, 0, NULL, window, dilation, causal, valid_len, scale,
+int oracle_backward_ex(int B, int Hq, int Hkv, int n, int D, const float *q, const float *k,
+                       const float *v, const float *dout, const int32_t *global_idx, int g,
+                       const float *side_k, const float *side_v, int S, int side_block,
+                       const float *bias, const int32_t *window, const int32_t *dilation,
+                       int causal, const int32_t *valid_len, double scale,
+                       const oracle_extras *ex, double *dq, double *dk, double *dv,
+                       double *dside_k, double *dside_v) {
+    oracle_problem P = {B, Hq, Hkv, n, D, q, k, v, global_idx, g, side_k, side_v,
+                        S, side_block, bias, window, dilation, causal, valid_len, scale,
                         NULL, 0, NULL, 0, 0};
     apply_extras(&P, ex);
     int rc = check_problem(&P);
     if (rc) return rc;
     if (!dout || !dq || !dk || !dv) return ORACLE_EINVAL;
+    if (S > 0 && (!dside_k || !dside_v)) return ORACLE_EINVAL;
     const int G = Hq / Hkv;
     memset(dq, 0, sizeof(double) * (size_t)B * Hq * n * D);
     memset(dk, 0, sizeof(double) * (size_t)B * Hkv * n * D);
     memset(dv, 0, sizeof(double) * (size_t)B * Hkv * n * D);
+    if (S > 0) {
+        memset(dside_k, 0, sizeof(double) * (size_t)B * Hkv * S * D);
+        memset(dside_v, 0, sizeof(double) * (size_t)B * Hkv * S * D);
+    }
     int failed = 0;
 #pragma omp parallel
     {
+        const size_t cap = (size_t)n + 1 + (size_t)(S > 0 ? S : 0);
         int32_t *keys = (int32_t *)malloc(sizeof(int32_t) * (size_t)(n + 1));
         int32_t *wbuf = (int32_t *)malloc(sizeof(int32_t) * (size_t)(n + 1));
-        double *sc = (double *)malloc(sizeof(double) * (size_t)(n + 1));
-        double *dp = (double *)malloc(sizeof(double) * (size_t)(n + 1));
+        double *sc = (double *)malloc(sizeof(double) * cap);
+        double *dp = (double *)malloc(sizeof(double) * cap);
         if (!keys || !wbuf || !sc || !dp) {
 #pragma omp atomic write
             failed = 1;
@@ -669,35 +679,55 @@ int oracle_backward(int B, int Hq, int Hkv, int n, int D, const float *q, const 
                 const int V = valid_len ? valid_len[b] : n;
                 const float *kb = k + ((int64_t)b * Hkv + hk) * n * D;
                 const float *vb = v + ((int64_t)b * Hkv + hk) * n * D;
+                const float *skb = S > 0 ? side_k + ((int64_t)b * Hkv + hk) * S * D : NULL;
+                const float *svb = S > 0 ? side_v + ((int64_t)b * Hkv + hk) * S * D : NULL;
                 double *dkb = dk + ((int64_t)b * Hkv + hk) * n * D;
                 double *dvb = dv + ((int64_t)b * Hkv + hk) * n * D;
+                double *dskb = S > 0 ? dside_k + ((int64_t)b * Hkv + hk) * S * D : NULL;
+                double *dsvb = S > 0 ? dside_v + ((int64_t)b * Hkv + hk) * S * D : NULL;
                 for (int h = hk * G; h < (hk + 1) * G; ++h) {
                     for (int i = 0; i < V && i < n; ++i) {
                         int nk = key_set(&P, b, h, i, keys, wbuf);
-                        if (nk <= 0) continue;
+                        if (nk < 0) continue;
+                        const int total = nk + S;
+                        if (total <= 0) continue;
                         const int64_t row = ((int64_t)b * Hq + h) * n + i;
                         const float *qi = q + row * D;
                         const float *doi = dout + row * D;
                         double m = -INFINITY;
-                        for (int t = 0; t < nk; ++t) {
-                            sc[t] = scale * dot(qi, kb + (int64_t)keys[t] * D, D) + local_bias(&P, b, h, i, keys[t]);
+                        for (int t = 0; t < total; ++t) {
+                            if (t < nk)
+                                sc[t] = scale * dot(qi, kb + (int64_t)keys[t] * D, D) +
+                                        local_bias(&P, b, h, i, keys[t]);
+                            else
+                                sc[t] = scale * dot(qi, skb + (int64_t)(t - nk) * D, D) +
+                                        side_bias(&P, h, i, t - nk);
                             if (sc[t] > m) m = sc[t];
                         }
                         double l = 0.0;
-                        for (int t = 0; t < nk; ++t) l += exp(sc[t] - m);
+                        for (int t = 0; t < total; ++t) l += exp(sc[t] - m);
                         const double lse = m + log(l);
                         double delta = 0.0;
-                        for (int t = 0; t < nk; ++t) {
+                        for (int t = 0; t < total; ++t) {
+                            const float *vj = t < nk ? vb + (int64_t)keys[t] * D : svb + (int64_t)(t - nk) * D;
                             sc[t] = exp(sc[t] - lse);                        /* p */
-                            dp[t] = dot(doi, vb + (int64_t)keys[t] * D, D);
+                            dp[t] = dot(doi, vj, D);
                             delta += sc[t] * dp[t];
                         }
                         double *dqi = dq + row * D;
-                        for (int t = 0; t < nk; ++t) {
+                        for (int t = 0; t < total; ++t) {
                             const double ds = sc[t] * (dp[t] - delta);
-                            const float *kj = kb + (int64_t)keys[t] * D;
-                            double *dkj = dkb + (int64_t)keys[t] * D;
-                            double *dvj = dvb + (int64_t)keys[t] * D;
+                            const float *kj;
+                            double *dkj, *dvj;
+                            if (t < nk) {
+                                kj = kb + (int64_t)keys[t] * D;
+                                dkj = dkb + (int64_t)keys[t] * D;
+                                dvj = dvb + (int64_t)keys[t] * D;
+                            } else {
+                                kj = skb + (int64_t)(t - nk) * D;
+                                dkj = dskb + (int64_t)(t - nk) * D;
+                                dvj = dsvb + (int64_t)(t - nk) * D;
+                            }
                             for (int x = 0; x < D; ++x) {
                                 dqi[x] += scale * ds * (double)kj[x];
                                 dkj[x] += scale * ds * (double)qi[x];
@@ -714,6 +744,17 @@ int oracle_backward(int B, int Hq, int Hkv, int n, int D, const float *q, const 
         free(dp);
     }
     return failed ? ORACLE_ENOMEM : ORACLE_OK;
+}
+
+/* oracle_backward_ex without side keys. */
+int oracle_backward(int B, int Hq, int Hkv, int n, int D, const float *q, const float *k,
+                    const float *v, const float *dout, const int32_t *global_idx, int g,
+                    const int32_t *window, const int32_t *dilation, int causal,
+                    const int32_t *valid_len, double scale, const oracle_extras *ex,
+                    double *dq, double *dk, double *dv) {
+    return oracle_backward_ex(B, Hq, Hkv, n, D, q, k, v, dout, global_idx, g, NULL, NULL, 0, 0,
+                              NULL, window, dilation, causal, valid_len, scale, ex, dq, dk, dv,
+                              NULL, NULL);
 }
 
 int oracle_num_threads(void) {

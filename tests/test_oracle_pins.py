@@ -386,6 +386,36 @@ def test_local_bias_offset_sign_closed_form(oracle_mod):
         assert np.max(np.abs(o[0, 0, i] - expect)) <= 1e-14
 
 
+def test_side_bias_direction_closed_form(oracle_mod):
+    """q = 0, window radius 0, one-hot V over the sequence and the side rows, and a
+    side-bias table that is a known function f of delta = memory block - query block
+    (LongT5 guide, 相对位置编码: the side keys' bias is bucketed on the block
+    distance, memory minus query).  Row i then has weight 1 on itself and
+    exp(f(sigma - floor(i / k))) on side key sigma, normalised -- a closed form that
+    fails if the table is read at the query-minus-memory distance or off by one."""
+    n, k, S = 40, 4, 6
+    nblk = -(-n // k)
+    f = lambda dlt: 0.25 * dlt + 0.03125 * dlt * dlt          # asymmetric, exact in fp32
+    D = n + S
+    q = np.zeros((1, 1, n, D), np.float32)
+    kk = np.ones((1, 1, n, D), np.float32)
+    v = np.eye(n, D, dtype=np.float32)[None, None]
+    side_k = np.ones((1, 1, S, D), np.float32)
+    side_v = np.eye(S, D, k=n, dtype=np.float32)[None, None]
+    # the table layout of the interface: column c holds delta = c - (nblk - 1)
+    bias = np.array([[f(c - (nblk - 1)) for c in range(S + nblk - 1)]], np.float32)
+    o, lse, _ = oracle_mod.Problem(q, kk, v, window=0, side_k=side_k, side_v=side_v, side_block=k,
+                                   bias=bias).forward()
+    for i in range(n):
+        w_side = np.exp([f(sig - i // k) for sig in range(S)])
+        z = 1.0 + w_side.sum()
+        expect = np.zeros(D)
+        expect[i] = 1.0 / z
+        expect[n:] = w_side / z
+        assert np.max(np.abs(o[0, 0, i] - expect)) <= 1e-14
+        assert abs(lse[0, 0, i] - np.log(z)) <= 1e-13
+
+
 def test_local_bias_skips_global_rows_and_out_of_window_global_keys(oracle_mod):
     """Table = -1e30 except offset 0: a non-global row keeps itself and the global
     keys outside its window (a global key inside the window is a window key and is
@@ -598,3 +628,72 @@ def test_backward_finite_differences(oracle_mod):
             a_m = [minus if x is arr else x for x in args]
             fd = (loss(*a_p) - loss(*a_m)) / step
             assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, abs(grad[idx])), (name, idx, fd, grad[idx])
+
+
+def test_backward_with_side_keys_matches_torch_autograd(oracle_mod):
+    """Side keys (and their additive bias) appended to every valid row: the oracle's
+    gradients for q, k, v, side_k and side_v equal torch autograd through a dense
+    masked attention over [K; side_k] and [V; side_v] (globals, padding, GQA, causal
+    and dilation in play)."""
+    rng = np.random.default_rng(79)
+    for n, r, d, causal, g, pad, G, S, kb in [(16, 2, 1, 0, 0, 0, 1, 4, 4), (21, 3, 2, 0, 2, 3, 2, 5, 4),
+                                              (18, 4, 1, 1, 0, 2, 2, 3, 6), (12, 1, 1, 0, 1, 0, 1, 6, 2)]:
+        B, Hkv, D = 2, 2, 8
+        Hq = Hkv * G
+        p = _problem(oracle_mod, rng, B, Hq, Hkv, n, D, r, d, causal, g, pad, S=S, kb=kb, bias=True)
+        dout = _rand((B, Hq, n, D), rng)
+        dq, dk, dv, dsk, dsv = p.backward(dout)
+        V = n - pad
+        nblk = -(-n // kb)
+        q = torch.from_numpy(p.q).double().requires_grad_()
+        k = torch.from_numpy(p.k).double().requires_grad_()
+        v = torch.from_numpy(p.v).double().requires_grad_()
+        sk = torch.from_numpy(p.side_k).double().requires_grad_()
+        sv = torch.from_numpy(p.side_v).double().requires_grad_()
+        kk = torch.cat([k, sk], 2).repeat_interleave(G, dim=1)
+        vv = torch.cat([v, sv], 2).repeat_interleave(G, dim=1)
+        s = q @ kk.transpose(-1, -2) * p.scale
+        # side-key bias: row i, side key sigma -> table column sigma - floor(i / kb) + nblk - 1
+        col = (torch.arange(S)[None, :] - (torch.arange(n) // kb)[:, None]) + nblk - 1
+        sb_bias = torch.from_numpy(p.bias).double()[:, col]               # [Hq, n, S]
+        bias_full = torch.cat([torch.zeros(Hq, n, n, dtype=torch.float64), sb_bias], -1)
+        outs = []
+        for b in range(B):
+            gl = p.global_idx[b] if p.global_idx is not None else None
+            allow = np.concatenate([_dense_mask(n, r, d, causal, gl, V),
+                                    np.repeat((np.arange(n) < V)[:, None], S, 1)], 1)
+            sc = (s[b] + bias_full).masked_fill(~torch.from_numpy(allow), float("-inf"))
+            w = torch.softmax(sc, -1).nan_to_num(0.0)
+            outs.append(w @ vv[b])
+        o = torch.stack(outs)
+        (o * torch.from_numpy(dout).double()).sum().backward()
+        for mine, ref in ((dq, q), (dk, k), (dv, v), (dsk, sk), (dsv, sv)):
+            assert np.max(np.abs(mine - ref.grad.numpy())) <= 1e-12
+
+
+def test_backward_with_side_keys_finite_differences(oracle_mod):
+    """Central differences of L = sum(dout * o) through the oracle's forward, for every
+    input the side-key backward differentiates (side keys, bias and globals in play)."""
+    rng = np.random.default_rng(83)
+    p = _problem(oracle_mod, rng, 1, 2, 1, 18, 4, 2, 1, 0, 2, 2, S=4, kb=4, bias=True)
+    dout = _rand((1, 2, 18, 4), rng)
+    grads = p.backward(dout)
+    inputs = [p.q, p.k, p.v, p.side_k, p.side_v]
+    kw = dict(window=p.window, dilation=p.dilation, global_idx=p.global_idx, side_block=p.side_block,
+              bias=p.bias, valid_len=p.valid_len)
+
+    def loss(arrs):
+        o, _, _ = oracle_mod.Problem(arrs[0], arrs[1], arrs[2], side_k=arrs[3], side_v=arrs[4],
+                                     **kw).forward()
+        return float((o * dout.astype(np.float64)).sum())
+
+    h = 2.0 ** -10
+    for a_i, (arr, grad) in enumerate(zip(inputs, grads)):
+        for _ in range(5):
+            idx = tuple(int(rng.integers(0, s)) for s in arr.shape)
+            plus, minus = [x.copy() for x in inputs], [x.copy() for x in inputs]
+            plus[a_i][idx] += np.float32(h)
+            minus[a_i][idx] -= np.float32(h)
+            step = float(plus[a_i][idx]) - float(minus[a_i][idx])
+            fd = (loss(plus) - loss(minus)) / step
+            assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, abs(grad[idx])), (a_i, idx, fd, grad[idx])
