@@ -118,6 +118,29 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def launch_decision(gpus: int, env) -> str:
+    """How to run for --gpus N: "run" (this process is the whole job, or one rank of
+    a torchrun job of N ranks), "relaunch" (N > 1 without torchrun: start N ranks
+    with torchrun), or "error" (torchrun started a different number of ranks)."""
+    if "WORLD_SIZE" in env:
+        return "run" if int(env["WORLD_SIZE"]) == gpus else "error"
+    return "relaunch" if gpus > 1 else "run"
+
+
+def torchrun_command(gpus: int, argv, port: int, timeout_s: int):
+    """One rank per GPU on this node, rendezvous on 127.0.0.1, bounded by timeout."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+    return ["timeout", "-k", "60", str(timeout_s), *cmd]
+
+
+def _free_port() -> int:
+    import socket
+    with socket.socket() as sck:
+        sck.bind(("127.0.0.1", 0))
+        return sck.getsockname()[1]
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     if ws > 1:
@@ -233,45 +256,74 @@ def time_backward(w, plan, dev, steps, warmup, device):
 
 def time_e2e(w, plan, host, steps, warmup, device):
     """Same metric through the public API with pinned host buffers: every step copies
-    the inputs host->device, builds side keys on the device, runs the forward and
-    reads the output and lse back."""
+    its inputs host->device, runs the forward (which builds the side keys from k and
+    v on the device) and reads the output and lse back.  Steps are pipelined over two buffer sets on
+    three streams (copy-in, compute, copy-out), so the host->device copy of one step
+    overlaps the forward and the device->host copy of the previous one; the time is
+    taken with CUDA events from the first copy-in to the last copy-out."""
     import torch
 
-    from sliding_window_global_b200 import side_aggregate
     names = [k for k in ("q", "k", "v", "global_idx", "valid_len", "bias", "local_bias",
                          "rand_blocks") if host.get(k) is not None]
     pinned = {k: host[k].contiguous().pin_memory() for k in names}
-    dev = {k: torch.empty_like(pinned[k], device=device) for k in names}
-    out_h = torch.empty((w.batch, w.q_heads, w.seq_len, w.head_dim), dtype=w.torch_dtype).pin_memory()
-    lse_h = torch.empty((w.batch, w.q_heads, w.seq_len), dtype=torch.float32).pin_memory()
     h2d = sum(pinned[k].numel() * pinned[k].element_size() for k in names)
-    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * 4
+    oshape = (w.batch, w.q_heads, w.seq_len, w.head_dim)
+    lshape = (w.batch, w.q_heads, w.seq_len)
+    nbuf = 2
+    dev = [{k: torch.empty_like(pinned[k], device=device) for k in names} for _ in range(nbuf)]
+    outs = [(torch.empty(oshape, dtype=w.torch_dtype, device=device),
+             torch.empty(lshape, dtype=torch.float32, device=device)) for _ in range(nbuf)]
+    host_out = [(torch.empty(oshape, dtype=w.torch_dtype).pin_memory(),
+                 torch.empty(lshape, dtype=torch.float32).pin_memory()) for _ in range(nbuf)]
+    d2h = host_out[0][0].numel() * host_out[0][0].element_size() + host_out[0][1].numel() * 4
+    s_in, s_comp, s_out = (torch.cuda.Stream(device) for _ in range(3))
+    ev_in = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_comp = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_out = [torch.cuda.Event() for _ in range(nbuf)]
+    used = [False] * nbuf
 
-    def step():
-        for k in names:
-            dev[k].copy_(pinned[k], non_blocking=True)
-        sk = sv = None
-        if w.side_block:
-            sk = side_aggregate(dev["k"], w.side_block, dev.get("valid_len"))
-            sv = side_aggregate(dev["v"], w.side_block, dev.get("valid_len"))
-        out, lse = plan.forward(dev["q"], dev["k"], dev["v"], window=list(w.window),
-                                dilation=list(w.dilation), causal=w.causal,
-                                global_idx=dev.get("global_idx"), side_k=sk, side_v=sv,
-                                bias=dev.get("bias"), valid_len=dev.get("valid_len"),
-                                local_bias=dev.get("local_bias"), rand_blocks=dev.get("rand_blocks"))
-        out_h.copy_(out, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
+    def step(i):
+        b = i % nbuf
+        d, (o, lse), (ho, hl) = dev[b], outs[b], host_out[b]
+        with torch.cuda.stream(s_in):
+            if used[b]:
+                s_in.wait_event(ev_comp[b])           # the forward that read these inputs is done
+            for k in names:
+                d[k].copy_(pinned[k], non_blocking=True)
+            ev_in[b].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(ev_in[b])
+            if used[b]:
+                s_comp.wait_event(ev_out[b])          # out of this slot has been read back
+            # Transient-Global side keys: block means of k and v, built inside the forward
+            plan.forward(d["q"], d["k"], d["v"], window=list(w.window), dilation=list(w.dilation),
+                         causal=w.causal, global_idx=d.get("global_idx"),
+                         bias=d.get("bias"), valid_len=d.get("valid_len"), out=o, lse=lse,
+                         local_bias=d.get("local_bias"), rand_blocks=d.get("rand_blocks"),
+                         side_from_kv=bool(w.side_block), stream=s_comp)
+            ev_comp[b].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[b])
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+            ev_out[b].record(s_out)
+        used[b] = True
 
-    for _ in range(max(1, warmup)):
-        step()
+    for i in range(max(1, warmup)):
+        step(i)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(steps):
-        step()
-    t1.record()
+    t0.record(s_in)
+    s_comp.wait_event(t0)
+    s_out.wait_event(t0)
+    for i in range(steps):
+        step(i)
+    s_in.wait_stream(s_out)
+    t1.record(s_in)
     torch.cuda.synchronize()
+    if plan.check() != 0:
+        raise RuntimeError("device error word set during the end-to-end run")
     return t0.elapsed_time(t1) / steps, h2d, d2h
 
 
@@ -433,7 +485,7 @@ def run_reference(args):
         import oracle
         nblk = (w.seq_len + w.side_block - 1) // w.side_block
         host["bias"] = torch.from_numpy(oracle.expand_side_bias(host["bias_table"], w.num_side, nblk))
-    per_step = max(1.0, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    per_step = args.ref_budget or max(1.0, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
     vals = []
     base = None
     for s in range(args.warmup + args.steps):
@@ -442,7 +494,8 @@ def run_reference(args):
             vals.append(r["value"])
             base = r
     v = float(np.mean(vals))
-    line = {"metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+    line = {"metric": METRIC, "value": v, "unit": "TFLOP/s",
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
@@ -461,11 +514,22 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="swan_swa")
-    ap.add_argument("--secondary", default="longt5_tglobal,longt5_local,bigbird_itc",
+    ap.add_argument("--secondary", default="longt5_tglobal,longformer_base,dilated,longt5_local,bigbird_itc",
                     help="comma-separated workloads timed after the main one (device time only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass timing")
+    ap.add_argument("--ref-budget", type=float, default=None,
+                    help="reference arm: seconds of oracle work per step (default: fit a few minutes)")
     args = ap.parse_args()
+    how = launch_decision(args.gpus, os.environ)
+    if how == "error":
+        print(f"bench.py: --gpus {args.gpus} but torchrun started WORLD_SIZE="
+              f"{os.environ.get('WORLD_SIZE')} ranks", file=sys.stderr)
+        sys.exit(2)
+    if how == "relaunch":
+        # N GPUs were asked for without torchrun: start one rank per GPU ourselves
+        cmd = torchrun_command(args.gpus, sys.argv[1:], _free_port(), 1800)
+        sys.exit(subprocess.call(cmd))
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":

@@ -143,7 +143,21 @@ swa_status swa_forward(swa_plan_t plan, const void* q, const void* k, const void
  *   key).  The caller draws the blocks.  0 <= num_rand <= 8; block indices must
  *   lie in [0, ceil(seq_len / 128)) (checked in SWA_DEBUG_CHECKS mode; outside
  *   it an index outside attends nothing).  Random blocks need dilation 1 on every
- *   head and causal == 0 (else SWA_ERR_UNSUPPORTED). */
+ *   head and causal == 0 (else SWA_ERR_UNSUPPORTED).
+ *
+ * side_from_kv: 1 to have the forward build the Transient-Global side keys and
+ *   values itself from k and v ("LongT5 长序列模型完全指南", Transient-Global: the
+ *   tokens of each side_block-token block are summed and normalised into one
+ *   global token; 源码级证据: padding tokens belong to no block, a trailing
+ *   partial block joins the previous one) -- the block means that
+ *   swa_side_aggregate computes, bit for bit, into the plan's workspace.  In a
+ *   bf16 plan the band kernel builds them in a prologue (each CTA its share,
+ *   launched cooperatively so that every CTA is resident; a CTA loads side tiles
+ *   once all CTAs have counted themselves done, a wait bounded like the others),
+ *   so the forward stays one launch; an fp32 plan runs one block-mean launch for
+ *   k and v first.  side_k and side_v must then be NULL, and the plan's num_side
+ *   must equal seq_len / side_block (else SWA_ERR_INVALID_ARG).  0 (the
+ *   default): side_k / side_v are inputs. */
 typedef struct {
   const void* q;
   const void* k;
@@ -163,6 +177,7 @@ typedef struct {
   int local_radius;
   const int32_t* rand_blocks;  /* device [B, Hq, ceil(n / 128), num_rand] int32, or NULL */
   int num_rand;
+  int side_from_kv;            /* 1: build side keys / values from k and v (block means) */
 } swa_forward_args;
 
 /* swa_forward with the arguments in a struct (same statuses, same launches). */
@@ -180,13 +195,18 @@ swa_status swa_bucket_local_bias(int num_q_heads, int radius, const float* table
  * ds = p (dp - rowsum(dout * out)), dq = scale ds k, dk = scale ds^T q,
  * dv = p^T dout) over the same key sets: the dilated / causal sliding window
  * ("精读笔记：Big Bird" §3.2.1, the Longformer page §二, SWAN-GPT §3.3(1)) with GQA
- * and padding.  Global tokens, side keys, local bias and random blocks are not
- * covered: a plan with side keys returns SWA_ERR_UNSUPPORTED, and the arguments
- * have no fields for the others.  bf16 plans only (else SWA_ERR_UNSUPPORTED);
- * the query heads of one KV head must share window and dilation (else
+ * and padding, plus, when their fields are set, the other terms of the forward:
+ * global rows and columns (BigBird §3.2.3), the Transient-Global side keys and
+ * their bias (LongT5 guide, Transient-Global; gradients of the side keys and
+ * values in dside_k / dside_v), the local relative-position bias (LongT5 guide,
+ * 相对位置编码) and random blocks (BigBird §3.2.2).  The biases are inputs: no
+ * gradient is formed for them.  The terms must be those the forward ran with
+ * (its out and lse are read).  bf16 plans only (else SWA_ERR_UNSUPPORTED); the
+ * query heads of one KV head must share window and dilation (else
  * SWA_ERR_UNSUPPORTED).  Gradients are written in fp32; dk and dv hold the sums
- * over the query heads of each KV head.  Every element of dq, dk, dv is written
- * (padded rows get 0).  The plan's workspace holds rowsum(dout * out).
+ * over the query heads of each KV head.  Every element of dq, dk, dv (and
+ * dside_k, dside_v) is written (padded rows get 0).  The plan's workspace holds
+ * rowsum(dout * out) and, with global tokens, the gathered global rows.
  * ------------------------------------------------------------------------- */
 typedef struct {
   const void* q;               /* device [B, Hq, n, D] bf16, 16-byte aligned */
@@ -202,6 +222,19 @@ typedef struct {
   float* dq;                   /* device [B, Hq, n, D] fp32 */
   float* dk;                   /* device [B, Hkv, n, D] fp32 */
   float* dv;                   /* device [B, Hkv, n, D] fp32 */
+  /* Optional terms, as in swa_forward_ex (zero-initialise the struct; zero fields
+   * keep the band-only meaning): */
+  const int32_t* global_idx;   /* device [B, num_global] int32 or NULL */
+  int num_global;              /* <= the plan's max_global */
+  const void* side_k;          /* device [B, Hkv, S, D] bf16, required when the plan has side keys */
+  const void* side_v;
+  const float* bias;           /* device [Hq, S + nblk - 1] fp32 side bias, or NULL */
+  const float* local_bias;     /* device [Hq, 2 * local_radius + 1] fp32, or NULL */
+  int local_radius;
+  const int32_t* rand_blocks;  /* device [B, Hq, ceil(n / 128), num_rand] int32, or NULL */
+  int num_rand;
+  float* dside_k;              /* device [B, Hkv, S, D] fp32, required when the plan has side keys */
+  float* dside_v;
 } swa_backward_args;
 
 /* Three launches on `stream`: rowsum(dout * out), the query-stationary dq pass,
@@ -231,6 +264,17 @@ int swa_plan_last_launches(swa_plan_t plan);
  * attention kernels does, and the kernel returns.  The next swa_plan_check
  * reports SWA_ERR_TIMEOUT (and clears the word); the context stays usable. */
 swa_status swa_selftest_wait_timeout(swa_plan_t plan, uint64_t limit_ns, void* stream);
+
+/* Self-test of the exponential the band kernel evaluates on the FMA pipe (an
+ * addition of this library: the pages describe nothing like it).  For part of
+ * the softmax exponentials the tensor-core kernel computes 2^x with a degree-3
+ * polynomial instead of the MUFU unit; this entry point runs exactly that
+ * device function on y[i] = 2^x[i], i < n (device pointers, fp32, enqueued on
+ * `stream`), so that tests can hold it to its stated bound: relative error at
+ * most 1.02e-4 for x in [-125.5, 128], a value in [0, 2^-125] below -125.5, and
+ * exactly +0 for x <= -127 (and -inf).  SWA_ERR_INVALID_ARG for n < 0 or null
+ * pointers with n > 0. */
+swa_status swa_selftest_exp2_poly(const float* x, float* y, int n, void* stream);
 
 /* Static, human-readable name of a status. */
 const char* swa_status_string(swa_status s);

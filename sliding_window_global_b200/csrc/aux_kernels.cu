@@ -12,6 +12,8 @@
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "side_mean.cuh"
+#include "softmax_math.cuh"
 #include "swa_kernels.h"
 
 namespace swa {
@@ -260,6 +262,32 @@ __global__ void side_aggregate_kernel(const T* __restrict__ x, T* __restrict__ o
   }
 }
 
+// Both side keys and side values in one launch (for the fp32 path of a forward
+// handed raw K/V): the block means of side_aggregate_kernel, bit for bit, VEC
+// consecutive columns per thread with 16-byte loads.  Threads [0, total) produce
+// side keys, [total, 2 total) side values.
+template <typename T>
+__global__ void side_aggregate_kv_kernel(const T* __restrict__ k, const T* __restrict__ v,
+                                         T* __restrict__ sk, T* __restrict__ sv, int B, int H, int n,
+                                         int D, int kb, const int32_t* __restrict__ valid_len) {
+  constexpr int VEC = 16 / sizeof(T);
+  const int S = n / kb;
+  const int groups = D / VEC;
+  const size_t total = (size_t)B * H * S * groups;
+  for (size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x; t < 2 * total;
+       t += (size_t)gridDim.x * blockDim.x) {
+    const bool is_v = t >= total;
+    const size_t u = is_v ? t - total : t;
+    const int cg = (int)(u % groups);
+    const size_t r = u / groups;
+    const int s = (int)(r % S);
+    const size_t bh = r / S;
+    const int b = (int)(bh / H);
+    const int V = valid_len ? min(valid_len[b], n) : n;
+    side_mean_vec<T>(is_v ? v : k, is_v ? sv : sk, bh, s, cg, n, D, kb, V);
+  }
+}
+
 // ------------------------------------------------------------------ precondition check
 // global_idx rows must be strictly increasing and inside [0, valid_len); random
 // key blocks must lie inside [0, nqb).  Threads [0, B*g) check global_idx, the
@@ -302,7 +330,26 @@ __global__ void wait_probe_kernel(int* err, unsigned long long limit_ns) {
   }
 }
 
+// ------------------------------------------------------------------ exp2 self test
+// y = the band kernel's FMA-pipe 2^x (exp2_poly2), two elements per thread.
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const long long i = 2 * (blockIdx.x * (long long)blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const bool two = i + 1 < n;
+  float y0, y1;
+  exp2_poly2(y0, y1, x[i], two ? x[i + 1] : 0.f);
+  y[i] = y0;
+  if (two) y[i + 1] = y1;
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const long long pairs = (n + 1LL) / 2;
+  exp2_poly_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0, s>>>(x, y, n);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_wait_probe(int* err, uint64_t limit_ns, cudaStream_t s) {
   wait_probe_kernel<<<1, 32, 0, s>>>(err, limit_ns);
@@ -322,6 +369,18 @@ cudaError_t launch_gather_globals(const AttnParams& p, const void* q, const void
                                                     p.global_idx, p.Hkv, p.n, p.g, p.gpad, row_vecs, p.B);
   gather_rows_kernel<<<blocks(tk), threads, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(gv),
                                                     p.global_idx, p.Hkv, p.n, p.g, p.gpad, row_vecs, p.B);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* gidx, int B, int H, int n, int g,
+                               int gpad, int D, int elem_bytes, cudaStream_t s) {
+  const int row_vecs = D * elem_bytes / 16;
+  const size_t total = (size_t)B * H * gpad * row_vecs;
+  if (total == 0) return cudaSuccess;
+  const int threads = 256;
+  const int blocks = (int)min((total + threads - 1) / threads, (size_t)4096);
+  gather_rows_kernel<<<blocks, threads, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), gidx,
+                                                H, n, g, gpad, row_vecs, B);
   return cudaGetLastError();
 }
 
@@ -370,6 +429,24 @@ cudaError_t launch_check_inputs(const AttnParams& p, cudaStream_t s) {
   if (t == 0) return cudaSuccess;
   check_inputs_kernel<<<(unsigned)((t + 255) / 256), 256, 0, s>>>(p.global_idx, p.g, p.B, p.n, p.valid_len,
                                                                    p.rand_blocks, nrand, nqb, p.err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_side_aggregate_kv(const void* k, const void* v, void* sk, void* sv, int B, int H,
+                                     int n, int D, int kb, const int32_t* valid_len, int bf16,
+                                     cudaStream_t s) {
+  const int vec = bf16 ? 8 : 4;
+  const size_t total = 2 * (size_t)B * H * (n / kb) * (D / vec);
+  const int threads = 256;
+  const int blocks = (int)min((total + threads - 1) / threads, (size_t)8192);
+  if (bf16) {
+    using T = __nv_bfloat16;
+    side_aggregate_kv_kernel<T><<<blocks, threads, 0, s>>>((const T*)k, (const T*)v, (T*)sk, (T*)sv, B, H,
+                                                              n, D, kb, valid_len);
+  } else {
+    side_aggregate_kv_kernel<float><<<blocks, threads, 0, s>>>((const float*)k, (const float*)v, (float*)sk,
+                                                                  (float*)sv, B, H, n, D, kb, valid_len);
+  }
   return cudaGetLastError();
 }
 

@@ -54,18 +54,37 @@
 //               as soon as the softmax has read the current one; the two
 //               issuers share only the K/V ring (read-only) and release each
 //               slot together.  Other warps of the group idle.
+#include <algorithm>
+
 #include "ptx.cuh"
+#include "side_mean.cuh"
+#include "softmax_math.cuh"
 #include "swa_kernels.h"
 
 namespace swa {
 namespace {
 
+#ifndef SWA_EPI_WG
+#define SWA_EPI_WG 0
+#endif
+// A fourth warpgroup drains O from TMEM and stores it, so that the softmax
+// warpgroups go on to the next unit at once.
+constexpr bool kEpiWG = SWA_EPI_WG != 0;
 constexpr int kSoftmaxThreads = 256;
-constexpr int kThreads = 384;                 // 3 warpgroups: softmax A, softmax B, control
-// Registers per thread after reallocation: 256 * 200 + 128 * 104 = 384 * 168, the
-// budget the CTA is launched with (168 per thread for 384 threads).
-constexpr int kRegsSoftmax = 200;
-constexpr int kRegsControl = 104;
+constexpr int kThreads = kEpiWG ? 512 : 384;  // softmax A, softmax B, control (, epilogue)
+constexpr int kLaunchRegs = kEpiWG ? 128 : 168;   // 65536 / threads, rounded down to 8
+// Registers per thread after reallocation; the sum must fit the launch budget
+// (kThreads * kLaunchRegs).
+#ifndef SWA_REGS_SOFTMAX
+#define SWA_REGS_SOFTMAX (kEpiWG ? 192 : 200)
+#endif
+#ifndef SWA_REGS_CONTROL
+#define SWA_REGS_CONTROL (kEpiWG ? 72 : 104)
+#endif
+constexpr int kRegsSoftmax = SWA_REGS_SOFTMAX;
+constexpr int kRegsControl = SWA_REGS_CONTROL;
+constexpr int kRegsEpi = kEpiWG ? (kThreads * kLaunchRegs - kSoftmaxThreads * kRegsSoftmax - 128 * kRegsControl) / 128
+                                : 0;
 constexpr uint32_t kSub = 128 * 128;          // one 128-row x 128-byte swizzle sub-tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -84,6 +103,12 @@ __host__ __device__ constexpr int emu_per32() {
   return D == 128 ? SWA_EMU_PER32_D128 : SWA_EMU_PER32_D64;
 }
 
+#ifndef SWA_EX2_PACKED
+#define SWA_EX2_PACKED 0
+#endif
+// MUFU exponentials on bf16 pairs (ex2.approx.ftz.bf16x2) instead of fp32 singles.
+constexpr bool kEx2Packed = SWA_EX2_PACKED != 0;
+
 // Where the tile max is taken: once after the tile-kind branches (D = 128), or
 // inside each branch (D = 64).  Both compute the same value; the code placement
 // was measured faster for each head size.
@@ -101,7 +126,7 @@ struct Cfg {
   static constexpr uint32_t kVOff = kKOff + NS * kTileBytes;
   static constexpr uint32_t kBiasOff = kVOff + NS * kTileBytes;  // 4 shifted copies
   static constexpr uint32_t kBarOff = kBiasOff + 4 * kBiasCopy * 4;
-  static constexpr int kNumBars = 2 + 2 + 3 * NS + 2 + 2 + 2 + 2 + 2 + 2;
+  static constexpr int kNumBars = 2 + 2 + 3 * NS + 2 + 2 + 2 + 2 + 2 + 2 + 2 + 2;
   static constexpr uint32_t kSmemBytes = kBarOff + kNumBars * 8 + 1024;
   // TMEM columns.  D = 128: S_A | S_B | O_A | O_B, P written over S.  D = 64 has
   // room for separate P buffers (S_A | S_B | P_A | P_B | O_A | O_B), so the next
@@ -117,8 +142,11 @@ struct Cfg {
 
 // The register split must fit the budget the CTA is launched with (a larger sum
 // would leave setmaxnreg.inc waiting), and the shared memory one CTA per SM.
-static_assert(kSoftmaxThreads * kRegsSoftmax + (kThreads - kSoftmaxThreads) * kRegsControl <= kThreads * 168,
+static_assert(kSoftmaxThreads * kRegsSoftmax + 128 * kRegsControl + (kEpiWG ? 128 * kRegsEpi : 0) <=
+                  kThreads * kLaunchRegs,
               "setmaxnreg split exceeds the launch register budget");
+static_assert(!kEpiWG || (kRegsEpi >= 24 && kRegsEpi % 8 == 0), "epilogue register share");
+static_assert(kRegsSoftmax % 8 == 0 && kRegsControl % 8 == 0, "setmaxnreg takes multiples of 8");
 static_assert(Cfg<64>::kSmemBytes + 2 * kTile * 4 + 16 <= 227 * 1024, "shared memory, D = 64");
 static_assert(Cfg<128>::kSmemBytes + 2 * kTile * 4 + 16 <= 227 * 1024, "shared memory, D = 128");
 static_assert(emu_per32<64>() % 4 == 0 && emu_per32<64>() <= 32 && emu_per32<128>() % 4 == 0 &&
@@ -144,49 +172,104 @@ struct Work {
   int lo[2], hi[2];     // band key range of each query tile (class coordinates)
 };
 
+// Work schedule.  MODE 0: the band units in the linear order (batch, head or head
+// pair, residue class, row unit); each CTA walks one contiguous range of it, so
+// consecutive units of a CTA are usually the next row tiles of the same head (pair):
+// they reuse most of their K/V tiles through L2 and need no fresh decode, only the
+// row offset moves.  MODE 1: global-row units, strided over the CTAs.
+struct Sched {
+  long long id, end;    // current unit, end of this CTA's range (MODE 0); uid, count (MODE 1)
+  int b, hp, c, u;      // batch, head (pair), class offset within the head, unit within the class
+  int uc;               // units of class c
+  int V;                // valid length of batch b
+};
+
+__device__ __forceinline__ int class_units(const AttnParams& p, int cls) {
+  const int tc = (p.cls[cls].n_c + kTile - 1) / kTile;
+  return p.pair_heads ? tc : (tc + 1) / 2;
+}
+
+__device__ __forceinline__ int batch_valid(const AttnParams& p, int b) {
+  return min(p.valid_len ? __ldg(p.valid_len + b) : p.n, p.n);
+}
+
 template <int MODE>
-__device__ __forceinline__ int total_units(const AttnParams& p) {
-  return MODE == 0 ? p.max_units * p.B * (p.pair_heads ? p.Hq / 2 : p.Hq)
-                   : p.nsplit * (p.gpad / kTile) * p.B * p.Hq;
+__device__ __forceinline__ void sched_begin(const AttnParams& p, Sched& s) {
+  if (MODE == 0) {
+    const long long T = p.units_total, G = gridDim.x;
+    s.id = T * blockIdx.x / G;
+    s.end = T * (blockIdx.x + 1) / G;
+    if (s.id >= s.end) return;
+    const int per_b = p.unit_prefix[p.num_hp];
+    s.b = (int)(s.id / per_b);
+    int rem = (int)(s.id - (long long)s.b * per_b);
+    s.hp = 0;
+    while (s.hp + 1 < p.num_hp && p.unit_prefix[s.hp + 1] <= rem) ++s.hp;
+    rem -= p.unit_prefix[s.hp];
+    const int base = p.class_base[p.pair_heads ? 2 * s.hp : s.hp];
+    s.c = 0;
+    s.uc = class_units(p, base);
+    while (rem >= s.uc && s.c + 1 < p.cls[base].nres) {
+      rem -= s.uc;
+      ++s.c;
+      s.uc = class_units(p, base + s.c);
+    }
+    s.u = rem;
+    s.V = batch_valid(p, s.b);
+  } else {
+    s.id = blockIdx.x;
+    s.end = (long long)p.nsplit * (p.gpad / kTile) * p.B * p.Hq;
+  }
+}
+
+template <int MODE>
+__device__ __forceinline__ void sched_next(const AttnParams& p, Sched& s) {
+  if (MODE == 0) {
+    ++s.id;
+    if (s.id >= s.end) return;
+    if (++s.u < s.uc) return;
+    s.u = 0;
+    const int base = p.class_base[p.pair_heads ? 2 * s.hp : s.hp];
+    if (s.c + 1 < p.cls[base].nres) {
+      ++s.c;
+    } else {
+      s.c = 0;
+      if (++s.hp == p.num_hp) {
+        s.hp = 0;
+        ++s.b;
+        s.V = batch_valid(p, s.b);
+      }
+    }
+    const int nb = p.class_base[p.pair_heads ? 2 * s.hp : s.hp];
+    s.uc = class_units(p, nb + s.c);
+  } else {
+    s.id += gridDim.x;
+  }
 }
 
 template <int MODE, bool RAND>
-__device__ __forceinline__ void decode_work(const AttnParams& p, int unit_id, Work& w) {
+__device__ __forceinline__ void decode_work(const AttnParams& p, const Sched& sc, Work& w) {
   if (MODE == 0) {
-    // unit ids run over (unit, batch, head or head pair), heads fastest
-    const int hunits = p.pair_heads ? p.Hq / 2 : p.Hq;
-    const int BH = p.B * hunits;
-    const int bh = unit_id % BH;
-    int unit = unit_id / BH;
-    w.b = bh / hunits;
-    w.h = p.pair_heads ? 2 * (bh % hunits) : bh % hunits;
+    w.valid = true;
+    w.b = sc.b;
+    w.h = p.pair_heads ? 2 * sc.hp : sc.hp;
     w.hx[0] = w.h;
     w.hx[1] = p.pair_heads ? w.h + 1 : w.h;
-    w.valid = unit < p.tiles[w.h];
     w.hk = w.h / p.G;
     w.r = p.window[w.h];
     const int base = p.class_base[w.h];
     w.d = p.cls[base].d;
-    const int nres = p.cls[base].nres;
-    const int per_unit = p.pair_heads ? 1 : 2;           // row tiles per unit and class
-    int c = 0;
-    for (; c < nres - 1; ++c) {
-      const int tc = (p.cls[base + c].n_c + kTile - 1) / kTile;
-      const int uc = (tc + per_unit - 1) / per_unit;
-      if (unit < uc) break;
-      unit -= uc;
-    }
-    w.c = c;
-    w.cls = base + c;
+    w.c = sc.c;
+    w.cls = base + sc.c;
     const int nc = p.cls[w.cls].n_c;
-    int V = p.valid_len ? p.valid_len[w.b] : p.n;
-    V = min(V, p.n);
-    w.Vc = V > c ? (V - c + w.d - 1) / w.d : 0;
+    const int V = sc.V;
+    w.Vc = V > w.c ? (V - w.c + w.d - 1) / w.d : 0;
     w.split = 0;
     w.key_end = 0;
+    const int unit = sc.u;
     for (int x = 0; x < 2; ++x) {
       w.u0[x] = p.pair_heads ? unit * kTile : unit * 2 * kTile + x * kTile;
-      w.rows[x] = w.valid ? max(0, min(kTile, nc - w.u0[x])) : 0;
+      w.rows[x] = max(0, min(kTile, nc - w.u0[x]));
       w.nvalid[x] = max(0, min(w.rows[x], w.Vc - w.u0[x]));
       w.active[x] = w.nvalid[x] > 0;
       w.lo[x] = max(0, w.u0[x] - w.r);
@@ -199,6 +282,7 @@ __device__ __forceinline__ void decode_work(const AttnParams& p, int unit_id, Wo
     w.ngc = (w.active[0] && p.g > 0) ? (p.g + kTile - 1) / kTile : 0;
     w.nside = (w.active[0] && p.S > 0) ? (p.S + kTile - 1) / kTile : 0;
   } else {
+    const int unit_id = (int)sc.id;
     w.valid = true;
     w.split = unit_id % p.nsplit;
     const int rest = unit_id / p.nsplit;
@@ -330,50 +414,6 @@ __device__ __forceinline__ void tma_tile(void* dst, const CUtensorMap* map, uint
   if (D == 128) tma_load_3d(static_cast<uint8_t*>(dst) + kSub, map, bar, 64, y, z);
 }
 
-// ------------------------------------------------------------------ packed fp32 helpers
-__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
-                                      float c0, float c1) {
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
-}
-__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
-// 2^a for a pair of arguments <= 2^7 on the FMA pipe: round to the nearest
-// integer i (adding 1.5*2^23 leaves i in the low mantissa bits), f = a - i in
-// [-1/2, 1/2], 2^f by a degree-3 polynomial (coefficients fitted for this
-// kernel by iterated weighted least squares on Chebyshev nodes, c0 = 1 exactly;
-// relative error 1.0e-4), then i is added to the exponent field.  Arguments
-// below -127 (masked scores are -inf) are clamped to -127, which yields +0.
-__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float a0, float a1) {
-  constexpr float kRound = 12582912.0f;         // 1.5 * 2^23
-  constexpr float c1 = 0.6932829022407532f, c2 = 0.2422109693288803f, c3 = 0.05500892549753189f;
-  a0 = fmaxf(a0, -127.f);
-  a1 = fmaxf(a1, -127.f);
-  float r0, r1, i0, i1, f0, f1, q0, q1;
-  fadd2(r0, r1, a0, a1, kRound, kRound);
-  fadd2(i0, i1, r0, r1, -kRound, -kRound);
-  fadd2(f0, f1, a0, a1, -i0, -i1);
-  ffma2(q0, q1, f0, f1, c3, c3, c2, c2);
-  ffma2(q0, q1, q0, q1, f0, f1, c1, c1);
-  ffma2(q0, q1, q0, q1, f0, f1, 1.f, 1.f);
-  y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(r0) << 23));
-  y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(r1) << 23));
-}
-
 // Row max of 128 values: 8 independent chains of 3-input maxima, then a tree.
 __device__ __forceinline__ float row_max128(const float (&x)[kTile]) {
   float m[8];
@@ -414,6 +454,121 @@ __device__ void write_neutral_partial(const AttnParams& p, const Work& w, int ro
   p.part_lse[prow] = -INFINITY;
 }
 
+// Fused Transient-Global prologue: this CTA's share of the side keys and values
+// (16-byte column groups of the side rows of k, then of v), all threads.
+template <int D>
+__device__ __forceinline__ void side_prologue(const AttnParams& p, int tid, int nthreads) {
+  constexpr int VEC = 8;                                   // bf16
+  constexpr int groups = D / VEC;
+  const long long rows = (long long)p.B * p.Hkv * p.S;     // per tensor
+  const long long items = 2 * rows * groups;
+  const long long lo = items * blockIdx.x / gridDim.x, hi = items * (blockIdx.x + 1) / gridDim.x;
+  for (long long t = lo + tid; t < hi; t += nthreads) {
+    const bool is_v = t >= rows * groups;
+    const long long u = is_v ? t - rows * groups : t;
+    const int cg = (int)(u % groups);
+    const long long r = u / groups;
+    const int s = (int)(r % p.S);
+    const long long bh = r / p.S;
+    const int b = (int)(bh / p.Hkv);
+    const int V = min(p.valid_len ? __ldg(p.valid_len + b) : p.n, p.n);
+    side_mean_vec<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(is_v ? p.agg_v : p.agg_k),
+                                 static_cast<__nv_bfloat16*>(is_v ? p.agg_sv : p.agg_sk), (size_t)bh, s, cg,
+                                 p.n, D, p.side_block, V);
+  }
+}
+
+// Epilogue of one query tile: O_x (TMEM) times 1/l -> out (bf16; MODE 0) or the
+// fp32 partials of a global-row split (MODE 1).  Thread `row` owns TMEM lane row.
+// staged: 32-column chunks go through shared memory (two 8 KB buffers at `stage`,
+// 64-byte swizzle) and are written by TMA, the `bar` named barrier (128 threads)
+// ordering the buffer reuse; else each thread stores its row.  o_free: if set, it
+// is arrived at once the last chunk has left TMEM.
+template <int D, int MODE>
+__device__ __forceinline__ void store_o(const AttnParams& p, const Work& w, const TileRows& tr, int row,
+                                        uint32_t o_addr, float inv, bool staged, uint8_t* stage, int bar,
+                                        uint64_t* o_free) {
+  constexpr int NCH = D / 32;
+  if (MODE == 0 && staged) {
+    if (row == 0) tma_store_wait_read<0>();          // previous stores have read the buffers
+    named_barrier_sync(bar, 128);
+#pragma unroll
+    for (int ch = 0; ch < NCH; ++ch) {
+      uint8_t* buf = stage + (ch & 1) * 8192;
+      if (ch >= 2) {
+        if (row == 0) tma_store_wait_read<1>();      // the store of chunk ch-2 has read buf
+        named_barrier_sync(bar, 128);
+      }
+      uint32_t rr[32];
+      tmem_ld32(o_addr + ch * 32, rr);
+      tmem_wait_ld_dep(rr);
+      if (o_free && ch == NCH - 1) {
+        tc_fence_before();
+        mbar_arrive(o_free);
+      }
+      uint8_t* rbase = buf + row * 64;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint4 v;
+        v.x = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 0]) * inv, __uint_as_float(rr[q4 * 8 + 1]) * inv);
+        v.y = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 2]) * inv, __uint_as_float(rr[q4 * 8 + 3]) * inv);
+        v.z = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 4]) * inv, __uint_as_float(rr[q4 * 8 + 5]) * inv);
+        v.w = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 6]) * inv, __uint_as_float(rr[q4 * 8 + 7]) * inv);
+        *reinterpret_cast<uint4*>(rbase + ((q4 ^ ((row >> 1) & 3)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      named_barrier_sync(bar, 128);
+      if (row == 0) {
+        tma_store_3d(&p.mo[w.cls], buf, ch * 32, tr.u0, w.b * p.Hq + tr.head);
+        tma_store_commit();
+      }
+    }
+  } else if (MODE == 0) {
+    const size_t off = out_row(p, w, tr, row);
+    uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + off * D);
+#pragma unroll
+    for (int ch = 0; ch < NCH; ++ch) {
+      uint32_t rr[32];
+      tmem_ld32(o_addr + ch * 32, rr);
+      tmem_wait_ld_dep(rr);
+      if (o_free && ch == NCH - 1) {
+        tc_fence_before();
+        mbar_arrive(o_free);
+      }
+      if (row < tr.rows) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 0]) * inv, __uint_as_float(rr[q4 * 8 + 1]) * inv);
+          v.y = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 2]) * inv, __uint_as_float(rr[q4 * 8 + 3]) * inv);
+          v.z = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 4]) * inv, __uint_as_float(rr[q4 * 8 + 5]) * inv);
+          v.w = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 6]) * inv, __uint_as_float(rr[q4 * 8 + 7]) * inv);
+          orow[ch * 4 + q4] = v;
+        }
+      }
+    }
+  } else {
+    const size_t prow = ((size_t)w.split * p.B * p.Hq + (size_t)w.b * p.Hq + w.h) * p.gpad + w.u0[0] + row;
+    float4* po = reinterpret_cast<float4*>(p.part_o + prow * D);
+#pragma unroll
+    for (int ch = 0; ch < NCH; ++ch) {
+      uint32_t rr[32];
+      tmem_ld32(o_addr + ch * 32, rr);
+      tmem_wait_ld_dep(rr);
+      if (o_free && ch == NCH - 1) {
+        tc_fence_before();
+        mbar_arrive(o_free);
+      }
+      if (row < w.rows[0]) {
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4)
+          po[ch * 8 + q4] = make_float4(__uint_as_float(rr[q4 * 4 + 0]) * inv, __uint_as_float(rr[q4 * 4 + 1]) * inv,
+                                        __uint_as_float(rr[q4 * 4 + 2]) * inv, __uint_as_float(rr[q4 * 4 + 3]) * inv);
+      }
+    }
+  }
+}
+
 // LOCAL: band tiles carry the local relative-position bias; RAND: query tiles have
 // random key blocks (MODE 0 only).  They are template parameters so that kernels
 // without them keep their register schedule.
@@ -443,14 +598,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   uint64_t* s_free = o_full + 2;          // [2] S read into registers (separate-P layout)
   uint64_t* pv_done = s_free + 2;         // [2] a PV finished: P buffer free, O updated
   uint64_t* p_half = pv_done + 2;         // [2] P of keys 0-63 written (P-over-S layout)
+  uint64_t* epi_in = p_half + 2;          // [2] softmax finished a unit: 1/l of each row staged
+  uint64_t* o_free = epi_in + 2;          // [2] the epilogue has read O_x out of TMEM
   __shared__ uint32_t tmem_slot;
+  __shared__ float sInv[2][2][kTile];     // [unit parity][tile][row] 1/l for the epilogue warpgroup
   __shared__ int abort_flag;
   __shared__ int sGpos[2 * kTile];        // positions of the current global tile, per group
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int nunits = total_units<MODE>(p);
   const bool has_bias = p.bias && p.S > 0;
   constexpr bool has_local = LOCAL && MODE == 0;
   // shared bias area: 4 copies of the local-bias row (stride lstride floats), then
@@ -470,6 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_init(&s_free[x], kTile);
       mbar_init(&pv_done[x], 1);
       mbar_init(&p_half[x], kTile);
+      mbar_init(&epi_in[x], kTile);
+      mbar_init(&o_free[x], kTile);
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(&k_full[s], 1);
@@ -488,6 +647,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
   volatile int* abort_v = &abort_flag;
+  if (MODE == 0 && p.agg_count) {
+    side_prologue<D>(p, tid, kThreads);
+    fence_proxy_async_global();                // side rows written here are read by TMA
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) atomicAdd(p.agg_count, 1u);  // after the whole CTA's stores
+  }
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     setmaxnreg_dec<kRegsControl>();
@@ -495,9 +661,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       int qloads[2] = {0, 0};
       int kv = 0;                                   // K/V tiles loaded so far (ring position)
       bool ok = true;
-      for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
+      bool side_ready = false;                      // fused prologue: all CTAs counted
+      Sched sc;
+      sched_begin<MODE>(p, sc);
+      for (; ok && sc.id < sc.end; sched_next<MODE>(p, sc)) {
         Work w;
-        decode_work<MODE, RAND>(p, uid, w);
+        decode_work<MODE, RAND>(p, sc, w);
         if (!w.active[0]) continue;
         const CUtensorMap* mq = (MODE == 0) ? &p.mq[w.cls] : &p.mgq;
         const int kz = w.b * p.Hkv + w.hk;
@@ -521,6 +690,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           if (kv >= NS && !mbar_wait_bounded(&kv_empty[st], (use - 1) & 1, abort_v, kWaitLimitNs)) {
             ok = false;
             break;
+          }
+          if (MODE == 0 && p.agg_count && !side_ready && j >= w.nband + w.ngc && j < w.rand0) {
+            // first side tile of this CTA: every CTA must have built its share
+            if (!wait_count_bounded(p.agg_count, gridDim.x, abort_v, kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            side_ready = true;
           }
           const CUtensorMap *mk, *mv;
           int y;
@@ -547,12 +724,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const uint32_t k_base = smem_u32(sK);
       const uint32_t v_base = smem_u32(sV);
       int qwaits[kTilesPerIssuer] = {}, pwaits[kTilesPerIssuer] = {};
+      int ounits[kTilesPerIssuer] = {};                 // units whose O_x was handed to the epilogue
       int nqk[kTilesPerIssuer] = {};                    // QKs issued per tile buffer (kernel-wide)
       int kv = 0;
       bool ok = true;
-      for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
+      Sched sc;
+      sched_begin<MODE>(p, sc);
+      for (; ok && sc.id < sc.end; sched_next<MODE>(p, sc)) {
         Work w;
-        decode_work<MODE, RAND>(p, uid, w);
+        decode_work<MODE, RAND>(p, sc, w);
         if (!w.active[0]) continue;
         const int T = w.total;
         // the tiles' fields as scalars (x0 is a run-time value with two issuers)
@@ -637,6 +817,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const int x = x0 + i;
             if (!ok) break;
             if (!uses(w, tr[i], x, j)) continue;
+            // the first PV of a unit overwrites O_x: the epilogue warpgroup must have
+            // read the previous unit's O_x out of TMEM
+            if (kEpiWG && npv[i] == 0 && ounits[i] > 0 &&
+                !mbar_wait_bounded(&o_free[x], (ounits[i] - 1) & 1, abort_v, kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
             if (!C::kSepP) {
               // P over S: the first half of P (keys 0-63) is published early, so the
               // PV over it overlaps the exponentials of the second half
@@ -656,7 +843,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                       sdesc_sw128(vt + kk * 2048, kSub, 1024), idesc_pv, (npv[i] > 0 || kk > 0) ? 1u : 0u);
             ++npv[i];
             if (C::kSepP) umma_commit(&pv_done[x]);
-            if (j == last[i]) umma_commit(&o_full[x]);
+            if (j == last[i]) {
+              umma_commit(&o_full[x]);
+              ++ounits[i];
+            }
             else if (!C::kSepP && uses(w, tr[i], x, j + 1)) ok = issue_qk(i, j + 1);
           }
           umma_commit(&kv_empty[st]);
@@ -664,9 +854,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         kv += T;
       }
     }
-  } else if (warp >= 10) {
+  } else if (warp >= 10 && warp < 12) {
     setmaxnreg_dec<kRegsControl>();
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax warpgroups
     setmaxnreg_inc<kRegsSoftmax>();
     const int x = warp >> 2;                   // 0: tile A, 1: tile B
@@ -680,9 +870,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     int it = 0;                                // S/P tiles handled so far (barrier phase)
     int oc = 0;                                // units finished (o_full phase)
     bool ok = true;
-    for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
+    Sched sc;
+    sched_begin<MODE>(p, sc);
+    for (; ok && sc.id < sc.end; sched_next<MODE>(p, sc)) {
       Work w;
-      decode_work<MODE, RAND>(p, uid, w);
+      decode_work<MODE, RAND>(p, sc, w);
       if (!w.valid) continue;
       const TileRows tr = tile_rows(w, x);
       if (!w.active[0]) {
@@ -1004,6 +1196,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               if (q < emu_per32<D>()) {
                 exp2_poly2(a0, a1, a0, a1);
                 exp2_poly2(a2, a3, a2, a3);
+              } else if (kEx2Packed) {
+                // the exponent rounded to bf16, two exponentials per MUFU operation; P
+                // comes out packed, and l sums exactly the P the PV product reads
+                const uint32_t p01 = ex2_bf16x2(pack_bf16x2(a0, a1));
+                const uint32_t p23 = ex2_bf16x2(pack_bf16x2(a2, a3));
+                pk[q / 2] = p01;
+                pk[q / 2 + 1] = p23;
+                acc0 = add_bf16_lo(p01, acc0);
+                acc1 = add_bf16_hi(p01, acc1);
+                acc2 = add_bf16_lo(p23, acc2);
+                acc3 = add_bf16_hi(p23, acc3);
+                continue;
               } else {
                 a0 = ex2_approx(a0);
                 a1 = ex2_approx(a1);
@@ -1046,93 +1250,68 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       if (!ok) break;
 
       // ---------------------------------------------------------- epilogue
-      // O_x is read out of TMEM before this group's next p_full arrival, which is
-      // what the MMA warp waits for before it overwrites O_x.
-      if (!mbar_wait_bounded(&o_full[x], oc & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
-      ++oc;
-      tc_fence_after();
       const bool has = row_valid && l > 0.f;
       const float inv = has ? 1.f / l : 0.f;
       const float lse_v = has ? (m + __log2f(l)) * kLn2 : -INFINITY;
-      if (MODE == 0 && !has_bias && !has_local) {
-        // Coalesced store: 32-column chunks staged in shared memory (the bias area,
-        // unused without biases; two 8 KB buffers per group, 64-byte swizzle)
-        // and written by TMA; rows beyond the class end are clipped by the map.
-        uint8_t* stage = reinterpret_cast<uint8_t*>(sBias) + x * 2 * 8192;
-        if (row == 0) tma_store_wait_read<0>();          // previous unit's stores have read
-        named_barrier_sync(1 + x, 128);
-#pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint8_t* buf = stage + (ch & 1) * 8192;
-          if (ch >= 2) {
-            if (row == 0) tma_store_wait_read<1>();      // the store of chunk ch-2 has read buf
-            named_barrier_sync(1 + x, 128);
-          }
-          uint32_t rr[32];
-          tmem_ld32(o_addr + ch * 32, rr);
-          tmem_wait_ld_dep(rr);
-          uint8_t* rbase = buf + row * 64;
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 0]) * inv, __uint_as_float(rr[q4 * 8 + 1]) * inv);
-            v.y = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 2]) * inv, __uint_as_float(rr[q4 * 8 + 3]) * inv);
-            v.z = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 4]) * inv, __uint_as_float(rr[q4 * 8 + 5]) * inv);
-            v.w = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 6]) * inv, __uint_as_float(rr[q4 * 8 + 7]) * inv);
-            *reinterpret_cast<uint4*>(rbase + ((q4 ^ ((row >> 1) & 3)) << 4)) = v;
-          }
-          fence_proxy_async_smem();
-          named_barrier_sync(1 + x, 128);
-          if (row == 0) {
-            tma_store_3d(&p.mo[w.cls], buf, ch * 32, tr.u0, w.b * p.Hq + tr.head);
-            tma_store_commit();
-          }
-        }
+      if (MODE == 0) {
         if (row < tr.rows && p.lse) p.lse[out_row(p, w, tr, row)] = lse_v;
-      } else if (MODE == 0) {
-        const size_t off = out_row(p, w, tr, row);
-        uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + off * D);
-#pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t rr[32];
-          tmem_ld32(o_addr + ch * 32, rr);
-          tmem_wait_ld_dep(rr);
-          if (row < tr.rows) {
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 0]) * inv, __uint_as_float(rr[q4 * 8 + 1]) * inv);
-              v.y = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 2]) * inv, __uint_as_float(rr[q4 * 8 + 3]) * inv);
-              v.z = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 4]) * inv, __uint_as_float(rr[q4 * 8 + 5]) * inv);
-              v.w = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 6]) * inv, __uint_as_float(rr[q4 * 8 + 7]) * inv);
-              orow[ch * 4 + q4] = v;
-            }
-          }
-        }
-        if (row < tr.rows && p.lse) p.lse[off] = lse_v;
-      } else {
-        const size_t prow =
-            ((size_t)w.split * p.B * p.Hq + (size_t)w.b * p.Hq + w.h) * p.gpad + w.u0[0] + row;
-        float4* po = reinterpret_cast<float4*>(p.part_o + prow * D);
-#pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t rr[32];
-          tmem_ld32(o_addr + ch * 32, rr);
-          tmem_wait_ld_dep(rr);
-          if (row < w.rows[0]) {
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4)
-              po[ch * 8 + q4] = make_float4(__uint_as_float(rr[q4 * 4 + 0]) * inv, __uint_as_float(rr[q4 * 4 + 1]) * inv,
-                                            __uint_as_float(rr[q4 * 4 + 2]) * inv, __uint_as_float(rr[q4 * 4 + 3]) * inv);
-          }
-        }
-        if (row < w.rows[0]) p.part_lse[prow] = lse_v;
+      } else if (row < w.rows[0]) {
+        p.part_lse[((size_t)w.split * p.B * p.Hq + (size_t)w.b * p.Hq + w.h) * p.gpad + w.u0[0] + row] = lse_v;
       }
-      tc_fence_before();
+      if (kEpiWG) {
+        // hand the unit to the epilogue warpgroup: 1/l per row, then go on
+        sInv[oc & 1][x][row] = inv;
+        ++oc;
+        mbar_arrive(&epi_in[x]);
+      } else {
+        // O_x is read out of TMEM before this group's next p_full arrival, which is
+        // what the MMA warp waits for before it overwrites O_x.
+        if (!mbar_wait_bounded(&o_full[x], oc & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+        ++oc;
+        tc_fence_after();
+        store_o<D, MODE>(p, w, tr, row, o_addr, inv, !has_bias && !has_local,
+                         reinterpret_cast<uint8_t*>(sBias) + x * 2 * 8192, 1 + x, nullptr);
+        tc_fence_before();
+      }
     }
   }
 
-  if (warp < 8 && (tid & 127) == 0) tma_store_wait_read<0>();   // staged stores have read smem
+  if (kEpiWG && warp >= 12) {
+    // ------------------------------------------------------------ epilogue warpgroup
+    // Per unit and query tile: wait for the softmax's 1/l and for the last PV, read
+    // O_x out of TMEM (then release it to the MMA warp), scale and store it.
+    setmaxnreg_dec<kRegsEpi>();
+    const int row = tid & 127;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const bool has_local_e = LOCAL && MODE == 0;
+    int ocx[2] = {0, 0};
+    bool ok = true;
+    Sched sc;
+    sched_begin<MODE>(p, sc);
+    for (; ok && sc.id < sc.end; sched_next<MODE>(p, sc)) {
+      Work w;
+      decode_work<MODE, RAND>(p, sc, w);
+      if (!w.valid || !w.active[0]) continue;
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        if (!ok) break;
+        if (!(x ? w.active[1] : w.active[0])) continue;
+        const int par = ocx[x] & 1;
+        if (!mbar_wait_bounded(&epi_in[x], par, abort_v, kWaitLimitNs) ||
+            !mbar_wait_bounded(&o_full[x], par, abort_v, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        ++ocx[x];
+        tc_fence_after();
+        const TileRows tr = tile_rows(w, x);
+        store_o<D, MODE>(p, w, tr, row, lane_base + C::o_col(x), sInv[par][x][row], !has_bias && !has_local_e,
+                         reinterpret_cast<uint8_t*>(sBias) + x * 2 * 8192, 4, &o_free[x]);
+      }
+    }
+  }
+
+  if ((kEpiWG ? warp >= 12 : warp < 8) && (tid & 127) == 0) tma_store_wait_read<0>();   // staged stores have read smem
   tc_fence_before();
   __syncthreads();
   if (abort_flag) {
@@ -1167,13 +1346,28 @@ static cudaError_t launch_one(const AttnParams& p, int units, int num_sms, cudaS
   if (e != cudaSuccess) return e;
   const int grid = units < num_sms ? units : num_sms;
   if (grid <= 0) return cudaSuccess;
+  if (MODE == 0 && p.agg_count) {
+    // the fused side-key prologue waits for every CTA: a cooperative launch makes
+    // them all resident at once (one CTA per SM, grid <= SM count)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
+  }
   kern<<<grid, kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
 // p.tiles[h] holds the number of two-tile units of head h, p.max_units their maximum.
 cudaError_t launch_band_tc(const AttnParams& p, int num_sms, cudaStream_t s) {
-  const int units = p.max_units * p.B * p.Hq;
+  const int units = (int)std::min<long long>(p.units_total, 1LL << 30);
   if (p.num_rand > 0) {
     if (p.local_bias)
       return p.D == 64 ? launch_one<64, 0, true, true>(p, units, num_sms, s)

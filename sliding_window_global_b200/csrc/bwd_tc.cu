@@ -139,8 +139,43 @@ __global__ void bwd_delta_kernel(const __grid_constant__ BwdParams p) {
   if (lane == 0) p.delta[warp] = acc;
 }
 
+// ------------------------------------------------------------------ shared facts
+// Position sets of the forward, written out per (query position, key position):
+// the window W(i) of a head (radius r, dilation d, causal or not).
+__device__ __forceinline__ bool in_window(int qpos, int kpos, int rd, int d, int causal) {
+  const int diff = qpos - kpos;
+  const bool span = causal ? (diff >= 0 && diff <= rd) : (diff >= -rd && diff <= rd);
+  return span && (d == 1 || diff % d == 0);
+}
+
+// Is position `pos` one of batch b's global tokens?  (binary search: sorted list)
+__device__ __forceinline__ bool is_global_pos(const BwdParams& p, int b, int pos) {
+  if (p.g == 0) return false;
+  const int32_t* gl = p.global_idx + (size_t)b * p.g;
+  int lo = 0, hi = p.g;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    const int v = __ldg(gl + mid);
+    if (v == pos) return true;
+    if (v < pos) lo = mid + 1;
+    else hi = mid;
+  }
+  return false;
+}
+
+__device__ __forceinline__ int batch_valid_len(const BwdParams& p, int b) {
+  return min(p.valid_len ? __ldg(p.valid_len + b) : p.n, p.n);
+}
+
 // ------------------------------------------------------------------ dQ
-template <int D>
+// Query-stationary: a 128-row query tile (Q and dO resident) walks a list of key
+// tiles through a two-stage ring.  X: after the band's tiles come the global-column
+// tiles (gathered K/V of the global tokens), the side tiles and the random tiles of
+// the row block, with the masks and biases of the forward; global query rows take
+// only their window and side keys here.  GROWS: the stationary tile is 128 gathered
+// global query rows, the key tiles are every tile of the sequence, and the mask keeps
+// the keys outside each row's window; the result is added to dq.
+template <int D, bool X, bool GROWS>
 __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_constant__ BwdParams p) {
   using C = BCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -155,16 +190,46 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
   uint64_t* acc_full = bars + 7;    // dQ complete
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  __shared__ int sGpos[kTile];      // key positions of the current global-column tile
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   BUnit u;
-  decode_bunit(p, blockIdx.x, false, u);
-  if (!u.valid) return;
-  // band key range of the tile: [klo_t, khi_t) in class coordinates
-  const int last = u.u0 + u.nvalid - 1;
-  const int klo_t = max(0, u.u0 - u.r);
-  const int khi_t = u.nvalid > 0 ? (p.causal ? min(u.Vc, last + 1) : min(u.Vc, last + u.r + 1)) : klo_t;
-  const int T = khi_t > klo_t ? (khi_t - klo_t + kTile - 1) / kTile : 0;
+  int klo_t = 0, T = 0, nband = 0, ngc = 0, nside = 0, nrand = 0;
+  if (!GROWS) {
+    decode_bunit(p, blockIdx.x, false, u);
+    if (!u.valid) return;
+    // band key range of the tile: [klo_t, khi_t) in class coordinates
+    const int last = u.u0 + u.nvalid - 1;
+    klo_t = max(0, u.u0 - u.r);
+    const int khi_t = u.nvalid > 0 ? (p.causal ? min(u.Vc, last + 1) : min(u.Vc, last + u.r + 1)) : klo_t;
+    nband = khi_t > klo_t ? (khi_t - klo_t + kTile - 1) / kTile : 0;
+    if (X && u.nvalid > 0) {
+      ngc = p.g > 0 ? (p.g + kTile - 1) / kTile : 0;
+      nside = p.S > 0 ? (p.S + kTile - 1) / kTile : 0;
+      nrand = p.rand_blocks ? p.num_rand : 0;
+    }
+    T = nband + ngc + nside + nrand;
+  } else {
+    // global rows: unit = (batch, query head, tile of 128 global slots)
+    const int gtiles = p.gpad / kTile;
+    const int bh = blockIdx.x / gtiles, gt = blockIdx.x % gtiles;
+    u.valid = true;
+    u.b = bh / p.Hq;
+    u.h = bh % p.Hq;
+    u.hk = u.h / p.G;
+    u.cls = p.dense_class;
+    u.c = 0;
+    u.d = p.cls[p.class_base[u.h]].d;             // the head's own dilation, for its window
+    u.r = p.window[u.h];
+    u.nc = p.n;
+    u.Vc = batch_valid_len(p, u.b);
+    u.u0 = gt * kTile;
+    u.rows = min(kTile, p.gpad - u.u0);
+    u.nvalid = max(0, min(u.rows, p.g - u.u0));
+    if (u.nvalid == 0) return;
+    T = (u.Vc + kTile - 1) / kTile;
+    nband = T;
+  }
 
   if (tid == 0) {
     mbar_init(a_full, 1);
@@ -189,19 +254,33 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
   volatile int* abort_v = &abort_flag;
   const int qz = u.b * p.Hq + u.h;
   const int kz = u.b * p.Hkv + u.hk;
+  const int qb = u.u0 / kTile;                     // query block of the tile (random blocks: d = 1)
+  const int nqb = (p.n + kTile - 1) / kTile;
 
   if (warp == 4) {
     if (lane == 0 && T > 0) {
       mbar_arrive_expect_tx(a_full, 2 * C::kTileBytes);
-      load_tile<D>(smem + C::kStat0, &p.mq[u.cls], a_full, u.u0, qz);
-      load_tile<D>(smem + C::kStat1, &p.mdo[u.cls], a_full, u.u0, qz);
+      load_tile<D>(smem + C::kStat0, GROWS ? &p.mgq : &p.mq[u.cls], a_full, u.u0, qz);
+      load_tile<D>(smem + C::kStat1, GROWS ? &p.mgdo : &p.mdo[u.cls], a_full, u.u0, qz);
       for (int j = 0; j < T; ++j) {
         const int st = j & 1;
         if (j >= 2 && !mbar_wait_bounded(&r_empty[st], ((j >> 1) - 1) & 1, abort_v, kWaitLimitNs)) break;
+        const CUtensorMap *mk = &p.mk[u.cls], *mv = &p.mv[u.cls];
+        int y = GROWS ? j * kTile : klo_t + j * kTile;
+        if (X && j >= nband) {
+          if (j < nband + ngc) {
+            mk = &p.mgk; mv = &p.mgv; y = (j - nband) * kTile;
+          } else if (j < nband + ngc + nside) {
+            mk = &p.msk; mv = &p.msv; y = (j - nband - ngc) * kTile;
+          } else {
+            const int t = j - nband - ngc - nside;
+            y = __ldg(p.rand_blocks + (((size_t)u.b * p.Hq + u.h) * nqb + qb) * p.num_rand + t) * kTile;
+          }
+        }
         uint8_t* dst = smem + C::kRing + st * 2 * C::kTileBytes;
         mbar_arrive_expect_tx(&r_full[st], 2 * C::kTileBytes);
-        load_tile<D>(dst, &p.mk[u.cls], &r_full[st], klo_t + j * kTile, kz);
-        load_tile<D>(dst + C::kTileBytes, &p.mv[u.cls], &r_full[st], klo_t + j * kTile, kz);
+        load_tile<D>(dst, mk, &r_full[st], y, kz);
+        load_tile<D>(dst + C::kTileBytes, mv, &r_full[st], y, kz);
       }
     }
   } else if (warp == 5) {
@@ -235,23 +314,72 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     const bool row_valid = row < u.nvalid;
     const int uq = u.u0 + row;
+    const int rd = u.r * u.d;
+    // the row's position; band rows: class coordinates -> position; global rows: gathered
+    int qpos = u.c + u.d * uq;
+    if (GROWS) qpos = row_valid ? __ldg(p.global_idx + (size_t)u.b * p.g + uq) : 0;
     const int klo = uq - u.r;
     const int khi = row_valid ? min(p.causal ? uq : uq + u.r, u.Vc - 1) + 1 : klo;
     size_t prow = 0;
     float lse2 = 0.f, delta = 0.f;
-    if (row < u.rows) {
-      prow = pos_row(p, u, u.h, p.Hq, uq);
+    if (row < u.rows && (!GROWS || row_valid)) {
+      prow = GROWS ? ((size_t)u.b * p.Hq + u.h) * p.n + qpos : pos_row(p, u, u.h, p.Hq, uq);
       if (row_valid) {
         lse2 = p.lse[prow] * kBLog2e;
         delta = p.delta[prow];
       }
     }
+    // terms beyond the band (X): the row's facts
+    bool row_global = false;
+    const float* lrow = nullptr;               // local-bias table of the head at offset 0
+    const float* srow = nullptr;               // side-bias row of the row's query block
+    int rbl[kMaxRand];
+#pragma unroll
+    for (int t = 0; t < kMaxRand; ++t) rbl[t] = -1;
+    if (X) {
+      row_global = row_valid && is_global_pos(p, u.b, qpos);
+      if (p.local_bias && !row_global)
+        lrow = p.local_bias + (size_t)u.h * (2 * p.local_radius + 1) + p.local_radius;
+      if (p.bias && p.S > 0)
+        srow = p.bias + (size_t)u.h * (p.S + p.nblk - 1) + (p.nblk - 1 - qpos / p.side_block);
+#pragma unroll
+      for (int t = 0; t < kMaxRand; ++t)
+        if (t < nrand) rbl[t] = __ldg(p.rand_blocks + (((size_t)u.b * p.Hq + u.h) * nqb + qb) * p.num_rand + t);
+    }
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int j = 0; j < T; ++j) {
+      // tile kind: 0 band (or every key, GROWS), 1 global columns, 2 side, 3 random
+      int kind = 0, base = 0, t_rand = 0;
+      if (X && j >= nband) {
+        if (j < nband + ngc) { kind = 1; base = (j - nband) * kTile; }
+        else if (j < nband + ngc + nside) { kind = 2; base = (j - nband - ngc) * kTile; }
+        else { kind = 3; t_rand = j - nband - ngc - nside; }
+      }
+      if (X && kind == 1) {
+        // stage the tile's global key positions: -1 for empty slots and for keys a
+        // random block of this row block already counts (the forward's rule)
+        int cv = base + row < p.g ? __ldg(p.global_idx + (size_t)u.b * p.g + base + row) : -1;
+#pragma unroll
+        for (int t = 0; t < kMaxRand; ++t)
+          if (cv >= 0 && rbl[t] >= 0 && (cv >> 7) == rbl[t]) cv = -1;
+        named_barrier_sync(1, 128);            // readers of the previous tile are done
+        sGpos[row] = cv;
+        named_barrier_sync(1, 128);
+      }
+      int kb = 0;
+      bool dup = false;
+      if (X && kind == 3) {
+#pragma unroll
+        for (int t = 0; t < kMaxRand; ++t)
+          if (t == t_rand) kb = rbl[t];
+#pragma unroll
+        for (int t = 0; t < kMaxRand; ++t) dup = dup || (t < t_rand && rbl[t] == kb);
+        dup = dup || kb < 0 || kb >= nqb;
+      }
       if (!mbar_wait_bounded(s_full, j & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
       tc_fence_after();
-      const int kv0 = klo_t + j * kTile;
+      const int kv0 = GROWS ? j * kTile : (kind == 3 ? kb * kTile : klo_t + j * kTile);
       const int lo_t = klo - kv0, hi_t = khi - kv0;
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
@@ -267,8 +395,27 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
             const int e = ch * 32 + q + h2;
-            const bool allowed = e >= lo_t && e < hi_t;
-            const float pr = allowed ? ex2_approx(__uint_as_float(sr[q + h2]) * sl2 - lse2) : 0.f;
+            bool allowed;
+            float b2 = 0.f;                    // bias in log2 units
+            if (GROWS) {
+              const int key = kv0 + e;
+              allowed = row_valid && key < u.Vc && !in_window(qpos, key, rd, u.d, p.causal);
+            } else if (!X || kind == 0) {
+              allowed = e >= lo_t && e < hi_t;
+              if (X && lrow && allowed) b2 = __ldg(lrow + u.d * (kv0 + e - uq)) * kBLog2e;
+            } else if (kind == 1) {
+              const int cv = sGpos[e];
+              allowed = row_valid && !row_global && cv >= 0 && !in_window(qpos, cv, rd, u.d, p.causal);
+            } else if (kind == 2) {
+              const int sg = base + e;
+              allowed = row_valid && sg < p.S;
+              if (srow && allowed) b2 = __ldg(srow + sg) * kBLog2e;
+            } else {
+              const int key = kv0 + e;
+              allowed = row_valid && !row_global && !dup && key < u.Vc &&
+                        !in_window(qpos, key, rd, 1, p.causal);
+            }
+            const float pr = allowed ? ex2_approx(__uint_as_float(sr[q + h2]) * sl2 + b2 - lse2) : 0.f;
             ds[h2] = pr * (__uint_as_float(dr[q + h2]) - delta);
           }
           pk[q / 2] = pack_bf16x2(ds[0], ds[1]);
@@ -280,7 +427,8 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
       tc_fence_before();
       mbar_arrive(ds_full);
     }
-    // epilogue: dQ = scale * (dS K), fp32; padded rows get zeros
+    // epilogue: dQ = scale * (dS K), fp32; padded rows get zeros.  Global rows (GROWS)
+    // add their part to what the band pass wrote.
     if (ok && T > 0) ok = mbar_wait_bounded(acc_full, 0, abort_v, kWaitLimitNs);
     if (ok) {
       tc_fence_after();
@@ -292,14 +440,19 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
           tmem_ld32(lane_base + C::kAcc0 + ch * 32, rr);
           tmem_wait_ld_dep(rr);
         }
-        if (row < u.rows) {
+        if (GROWS ? row_valid : row < u.rows) {
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
             float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
             if (T > 0 && row_valid)
               v4 = make_float4(__uint_as_float(rr[q4 * 4]) * p.scale, __uint_as_float(rr[q4 * 4 + 1]) * p.scale,
                                __uint_as_float(rr[q4 * 4 + 2]) * p.scale, __uint_as_float(rr[q4 * 4 + 3]) * p.scale);
-            reinterpret_cast<float4*>(dst)[ch * 8 + q4] = v4;
+            float4* d4 = reinterpret_cast<float4*>(dst) + ch * 8 + q4;
+            if (GROWS) {
+              const float4 o = *d4;
+              v4 = make_float4(o.x + v4.x, o.y + v4.y, o.z + v4.z, o.w + v4.w);
+            }
+            *d4 = v4;
           }
         }
       }
@@ -331,6 +484,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
 // P^T and dS^T go to shared memory (128 keys x 64 queries, K-major with the
 // 128-byte swizzle) and feed dV += P^T dO and dK += dS^T Q as shared-memory operands.
 constexpr int kQT = 64;                        // query rows per tile of this pass
+constexpr int kMaxRandList = 2048;             // (query head in group, query block) pairs per key block
 constexpr int kDkvThreads = 320;               // warps 0-3, 4-7 compute; 8 TMA; 9 MMA / TMEM
 
 template <int D>
@@ -342,8 +496,10 @@ struct KCfg {
   static constexpr uint32_t kRing = 2 * kKVBytes;          // stage s: Q at kRing + 2 s Q, dO after
   static constexpr uint32_t kPds = kRing + 4 * kQBytes;    // group g: P^T at kPds + 2 g P, dS^T after
   static constexpr uint32_t kPBytes = 128u * kQT * 2u;     // 16 KB
-  static constexpr uint32_t kStg = kPds + 4 * kPBytes;     // [group][buffer][lse2 64 | delta 64] floats
-  static constexpr uint32_t kBarOff = kStg + 2 * 2 * 128 * 4;
+  // [group][buffer][lse2 64 | delta 64 | position 64 | row fact 64] (floats, ints)
+  static constexpr uint32_t kStg = kPds + 4 * kPBytes;
+  static constexpr uint32_t kList = kStg + 2 * 2 * 256 * 4;  // random job: query blocks drawing the key block
+  static constexpr uint32_t kBarOff = kList + kMaxRandList * 4;
   static constexpr uint32_t kSmemBytes = kBarOff + 16 * 8 + 1024;
   static constexpr uint32_t kTmemCols = 512;
   // TMEM: group g S^T at 128 g, dP^T at 128 g + 64; dV at 256, dK at 256 + D
@@ -351,9 +507,28 @@ struct KCfg {
 };
 static_assert(KCfg<128>::kSmemBytes <= 227 * 1024, "shared memory of the dK/dV pass");
 
-template <int D>
+// Jobs of the key-stationary pass.
+enum DkvJob {
+  kJobBand = 0,        // band key tile of a class, its band query tiles (overwrites dk, dv)
+  kJobBandX = 1,       // the same with the local bias, and the global query rows outside the
+                       // key's window appended (gathered rows)
+  kJobGlobalKeys = 2,  // gathered global keys: every query row of the sequence whose window,
+                       // and whose row block's random blocks, miss the key (adds to dk, dv)
+  kJobSide = 3,        // a side tile: every valid query row, with the side bias (dside_k, dside_v)
+  kJobRandom = 4,      // a random key block: the rows of the query blocks that drew it (adds)
+};
+
+// Query tiles of one key-stationary unit.  A tile is 64 query rows of one query
+// head of the unit's GQA group; `src` 0 reads the class view (band), 1 the gathered
+// global rows, 2 the whole sequence (dense class).
+struct QTile {
+  int head, y, src;
+};
+
+template <int D, int JOB>
 __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_constant__ BwdParams p) {
   using C = KCfg<D>;
+  constexpr bool kBandJob = JOB == kJobBand || JOB == kJobBandX;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -367,16 +542,107 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
   uint64_t* acc_full = bars + 11;   // dK, dV complete
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  __shared__ int sCount;
+  int* sList = reinterpret_cast<int*>(smem + C::kList);   // random job: head-in-group * nqb + query block
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nqb = (p.n + kTile - 1) / kTile;
 
   BUnit u;
-  decode_bunit(p, blockIdx.x, true, u);
-  if (!u.valid) return;
-  const int lastk = u.u0 + u.nvalid - 1;
-  const int qlo = p.causal ? u.u0 : max(0, u.u0 - u.r);
-  const int qhi = u.nvalid > 0 ? min(u.Vc, lastk + u.r + 1) : qlo;
-  const int NQ = qhi > qlo ? (qhi - qlo + kQT - 1) / kQT : 0;
-  const int T = NQ * p.G;                     // 64-row query tiles of every head of the group
+  int qlo = 0, NQ = 0, NG = 0, ND = 0, T = 0;
+  int kpos0 = 0;                    // position of key row 0 (band: class coordinates handled below)
+  if (kBandJob) {
+    decode_bunit(p, blockIdx.x, true, u);
+    if (!u.valid) return;
+    const int lastk = u.u0 + u.nvalid - 1;
+    qlo = p.causal ? u.u0 : max(0, u.u0 - u.r);
+    const int qhi = u.nvalid > 0 ? min(u.Vc, lastk + u.r + 1) : qlo;
+    NQ = qhi > qlo ? (qhi - qlo + kQT - 1) / kQT : 0;
+    NG = (JOB == kJobBandX && p.g > 0 && u.nvalid > 0) ? (p.g + kQT - 1) / kQT : 0;
+    T = (NQ + NG) * p.G;            // 64-row query tiles of every head of the group
+  } else {
+    // unit = (batch, KV head, key tile of the job's key set)
+    int per = 0;
+    if (JOB == kJobGlobalKeys) per = p.gpad / kTile;
+    if (JOB == kJobSide) per = (p.S + kTile - 1) / kTile;
+    if (JOB == kJobRandom) per = nqb;
+    const int bk = blockIdx.x / per, kt = blockIdx.x % per;
+    u.valid = true;
+    u.b = bk / p.Hkv;
+    u.hk = bk % p.Hkv;
+    u.h = u.hk * p.G;
+    u.cls = p.dense_class;
+    u.c = 0;
+    u.d = p.cls[p.class_base[u.h]].d;
+    u.r = p.window[u.h];
+    u.nc = p.n;
+    u.Vc = batch_valid_len(p, u.b);
+    u.u0 = kt * kTile;
+    if (JOB == kJobGlobalKeys) {
+      u.rows = min(kTile, p.gpad - u.u0);
+      u.nvalid = max(0, min(u.rows, p.g - u.u0));
+    } else if (JOB == kJobSide) {
+      u.rows = min(kTile, p.S - u.u0);
+      u.nvalid = u.rows;            // every side key; with no valid row T = 0 writes zeros
+    } else {
+      u.rows = min(kTile, p.n - u.u0);
+      u.nvalid = max(0, min(u.rows, u.Vc - u.u0));
+    }
+    if (u.nvalid == 0) return;      // no key of this tile exists: nothing to add
+    kpos0 = u.u0;
+    ND = (u.Vc + kQT - 1) / kQT;
+    if (JOB == kJobRandom) {
+      // the (head, query block) pairs of the group whose random list names this key
+      // block, each counted at its first occurrence; built in a fixed order
+      const int pairs = p.G * nqb;
+      int* flags = reinterpret_cast<int*>(smem + C::kPds);     // free until the first tile
+      if (pairs > kMaxRandList) {
+        if (tid == 0) atomicOr(p.err, kDevErrCheck);   // more pairs than the list holds: reported
+        return;
+      }
+      for (int i = tid; i < pairs; i += blockDim.x) {
+        const int32_t* rl = p.rand_blocks + (((size_t)u.b * p.Hq + u.h + i / nqb) * nqb + i % nqb) * p.num_rand;
+        int f = 0;
+        for (int t = 0; t < p.num_rand; ++t) f |= (__ldg(rl + t) == kt);   // a repeat counts once
+        flags[i] = f;
+      }
+      __syncthreads();
+      if (warp == 0) {                                  // ordered compaction, 32 pairs a step
+        int cnt = 0;
+        for (int base = 0; base < pairs; base += 32) {
+          const int i = base + lane;
+          const bool f = i < pairs && flags[i];
+          const unsigned m = __ballot_sync(0xffffffffu, f);
+          if (f) sList[cnt + __popc(m & ((1u << lane) - 1u))] = i;
+          cnt += __popc(m);
+        }
+        if (lane == 0) sCount = cnt;
+      }
+      __syncthreads();
+      T = 2 * sCount;               // two 64-row halves per query block
+    } else {
+      T = ND * p.G;
+    }
+  }
+  auto qtile = [&](int j) -> QTile {
+    QTile t;
+    if (kBandJob) {
+      const int per = NQ + NG;
+      t.head = u.h + j / per;
+      const int jj = j % per;
+      if (jj < NQ) { t.y = qlo + jj * kQT; t.src = 0; }
+      else { t.y = (jj - NQ) * kQT; t.src = 1; }
+    } else if (JOB == kJobRandom) {
+      const int e = sList[j >> 1];
+      t.head = u.h + e / nqb;
+      t.y = (e % nqb) * kTile + (j & 1) * kQT;
+      t.src = 2;
+    } else {
+      t.head = u.h + j / ND;
+      t.y = (j % ND) * kQT;
+      t.src = 2;
+    }
+    return t;
+  };
 
   if (tid == 0) {
     mbar_init(a_full, 1);
@@ -405,20 +671,24 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && T > 0) {
+      const CUtensorMap* km = JOB == kJobGlobalKeys ? &p.mgk : JOB == kJobSide ? &p.msk : &p.mk[u.cls];
+      const CUtensorMap* vm = JOB == kJobGlobalKeys ? &p.mgv : JOB == kJobSide ? &p.msv : &p.mv[u.cls];
       mbar_arrive_expect_tx(a_full, 2 * C::kKVBytes);
-      load_tile<D>(smem + C::kK, &p.mk[u.cls], a_full, u.u0, kz);
-      load_tile<D>(smem + C::kV, &p.mv[u.cls], a_full, u.u0, kz);
+      load_tile<D>(smem + C::kK, km, a_full, u.u0, kz);
+      load_tile<D>(smem + C::kV, vm, a_full, u.u0, kz);
       for (int j = 0; j < T; ++j) {
         const int st = j & 1;
         if (j >= 2 && !mbar_wait_bounded(&r_empty[st], ((j >> 1) - 1) & 1, abort_v, kWaitLimitNs)) break;
-        const int qz = u.b * p.Hq + u.h + j / NQ;
-        const int y = qlo + (j % NQ) * kQT;
+        const QTile qt = qtile(j);
+        const int qz = u.b * p.Hq + qt.head;
+        const CUtensorMap* qm = qt.src == 0 ? &p.mq64[u.cls] : qt.src == 1 ? &p.mgq64 : &p.mq64[p.dense_class];
+        const CUtensorMap* dm = qt.src == 0 ? &p.mdo64[u.cls] : qt.src == 1 ? &p.mgdo64 : &p.mdo64[p.dense_class];
         uint8_t* dst = smem + C::kRing + st * 2 * C::kQBytes;
         mbar_arrive_expect_tx(&r_full[st], 2 * C::kQBytes);
-        tma_load_3d(dst, &p.mq64[u.cls], &r_full[st], 0, y, qz);
-        if (D == 128) tma_load_3d(dst + C::kQSub, &p.mq64[u.cls], &r_full[st], 64, y, qz);
-        tma_load_3d(dst + C::kQBytes, &p.mdo64[u.cls], &r_full[st], 0, y, qz);
-        if (D == 128) tma_load_3d(dst + C::kQBytes + C::kQSub, &p.mdo64[u.cls], &r_full[st], 64, y, qz);
+        tma_load_3d(dst, qm, &r_full[st], 0, qt.y, qz);
+        if (D == 128) tma_load_3d(dst + C::kQSub, qm, &r_full[st], 64, qt.y, qz);
+        tma_load_3d(dst + C::kQBytes, dm, &r_full[st], 0, qt.y, qz);
+        if (D == 128) tma_load_3d(dst + C::kQBytes + C::kQSub, dm, &r_full[st], 64, qt.y, qz);
       }
     }
   } else if (warp == 9) {
@@ -476,33 +746,74 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const bool key_valid = row < u.nvalid;
     const int uk = u.u0 + row;
+    const int rd = u.r * u.d;
+    // the key's position (band jobs: class coordinates c + d * uk)
+    int kpos = kBandJob ? u.c + u.d * uk : kpos0 + row;
+    if (JOB == kJobGlobalKeys) kpos = key_valid ? __ldg(p.global_idx + (size_t)u.b * p.g + uk) : 0;
     const float sl2 = p.scale_log2;
     uint8_t* pts = smem + C::kPds + g * 2 * C::kPBytes;   // P^T rows, then dS^T rows
     bool ok = true;
     int nt = 0;                               // tiles handled by this group
     for (int j = g; j < T; j += 2, ++nt) {
-      // lse2 and Delta of the tile's 64 query rows (a padded or missing row gets
-      // lse2 = +inf, so its p is 0)
-      const int head = u.h + j / NQ;
-      const int q0 = qlo + (j % NQ) * kQT;
-      float* stg = reinterpret_cast<float*>(smem + C::kStg) + (g * 2 + (nt & 1)) * 128;
+      // per query row of the tile: lse2 (+inf excludes the row: padded, missing, or
+      // outside the job's rows), Delta, and the row's position or block facts
+      const QTile qt = qtile(j);
+      float* stg = reinterpret_cast<float*>(smem + C::kStg) + (g * 2 + (nt & 1)) * 256;
+      int* stgi = reinterpret_cast<int*>(stg + 2 * kQT);   // [64] positions, [64] extra
       if (row < kQT) {
-        const int uq = q0 + row;
+        const int uq = qt.y + row;
         float l2 = INFINITY, dl = 0.f;
-        if (uq < u.Vc) {
-          const size_t pr = pos_row(p, u, head, p.Hq, uq);
+        int qp = 0, ex = 0;
+        bool take = false;
+        if (qt.src == 0) {
+          take = uq < u.Vc;
+          qp = u.c + u.d * uq;
+          // the local bias applies to the window keys of non-global rows
+          if (JOB == kJobBandX) ex = (p.local_bias && take && !is_global_pos(p, u.b, qp)) ? 1 : 0;
+        } else if (qt.src == 1) {
+          take = uq < p.g;
+          qp = take ? __ldg(p.global_idx + (size_t)u.b * p.g + uq) : 0;
+        } else {
+          take = uq < u.Vc;
+          qp = uq;
+          if (JOB == kJobGlobalKeys || JOB == kJobRandom) take = take && !is_global_pos(p, u.b, qp);
+          if (JOB == kJobSide) ex = qp / p.side_block;                 // query block of the side bias
+        }
+        if (take) {
+          const size_t pr = ((size_t)u.b * p.Hq + qt.head) * p.n + qp;
           l2 = p.lse[pr] * kBLog2e;
           dl = p.delta[pr];
         }
         stg[row] = l2;
         stg[kQT + row] = dl;
+        stgi[row] = qp;
+        stgi[kQT + row] = ex;
       }
+      // global-key job: the random blocks of the tile's query block (one block per tile)
+      int trb[kMaxRand];
+#pragma unroll
+      for (int t = 0; t < kMaxRand; ++t) trb[t] = -1;
+      if (JOB == kJobGlobalKeys && p.rand_blocks) {
+        const int qbk = qt.y / kTile;
+#pragma unroll
+        for (int t = 0; t < kMaxRand; ++t)
+          if (t < p.num_rand) trb[t] = __ldg(p.rand_blocks + (((size_t)u.b * p.Hq + qt.head) * nqb + qbk) * p.num_rand + t);
+      }
+      bool key_in_rand = false;
+#pragma unroll
+      for (int t = 0; t < kMaxRand; ++t) key_in_rand = key_in_rand || (trb[t] >= 0 && (kpos >> 7) == trb[t]);
+      const float* lrow = (JOB == kJobBandX && p.local_bias)
+                              ? p.local_bias + (size_t)qt.head * (2 * p.local_radius + 1) + p.local_radius
+                              : nullptr;
+      const float* sbias = (JOB == kJobSide && p.bias)
+                               ? p.bias + (size_t)qt.head * (p.S + p.nblk - 1) + (p.nblk - 1) + uk
+                               : nullptr;
       named_barrier_sync(1 + g, 128);
       if (!mbar_wait_bounded(&s_full[g], nt & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
       tc_fence_after();
       // the products of tile j - 2 have read this group's P^T / dS^T buffers
       if (nt > 0 && !mbar_wait_bounded(&pds_free[g], (nt - 1) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
-      const int d0 = q0 - uk;                  // query - key offset of column 0
+      const int d0 = qt.y - uk;                // query - key offset of column 0 (band, class coordinates)
       uint8_t* prow = pts + row * 128;
       uint8_t* drow = pts + C::kPBytes + row * 128;
 #pragma unroll
@@ -524,10 +835,26 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
           float pr[8], ds[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const int off = d0 + c * 8 + e;
-            const bool inband = p.causal ? (off >= 0 && off <= u.r) : (off >= -u.r && off <= u.r);
-            const bool allowed = key_valid && inband;
-            pr[e] = allowed ? ex2_approx(__uint_as_float(sr[c4 * 8 + e]) * sl2 - lv[e]) : 0.f;
+            bool allowed;
+            float b2 = 0.f;
+            if (JOB == kJobBand || (JOB == kJobBandX && qt.src == 0)) {
+              const int off = d0 + c * 8 + e;
+              const bool inband = p.causal ? (off >= 0 && off <= u.r) : (off >= -u.r && off <= u.r);
+              allowed = key_valid && inband;
+              if (JOB == kJobBandX && lrow && allowed && stgi[kQT + c * 8 + e])
+                b2 = __ldg(lrow - u.d * off) * kBLog2e;
+            } else if (JOB == kJobBandX) {
+              // a global query row: keys outside its window (inside it the band tile counts)
+              allowed = key_valid && !in_window(stgi[c * 8 + e], kpos, rd, u.d, p.causal);
+            } else if (JOB == kJobGlobalKeys) {
+              allowed = key_valid && !key_in_rand && !in_window(stgi[c * 8 + e], kpos, rd, u.d, p.causal);
+            } else if (JOB == kJobSide) {
+              allowed = key_valid;
+              if (sbias) b2 = __ldg(sbias - stgi[kQT + c * 8 + e]) * kBLog2e;
+            } else {
+              allowed = key_valid && !in_window(stgi[c * 8 + e], kpos, rd, 1, p.causal);
+            }
+            pr[e] = allowed ? ex2_approx(__uint_as_float(sr[c4 * 8 + e]) * sl2 + b2 - lv[e]) : 0.f;
             ds[e] = pr[e] * (__uint_as_float(dr[c4 * 8 + e]) - dv[e]);
           }
           uint4 pv, dsv;
@@ -548,13 +875,27 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
       tc_fence_before();
       mbar_arrive(&p_full[g]);
     }
-    // epilogue: group 0 writes dV, group 1 writes dK = scale * (dS^T Q), fp32; padded
-    // keys get zeros.  The TMEM loads are warp-wide, so every thread issues them.
+    // epilogue: group 0 writes dV, group 1 writes dK = scale * (dS^T Q), fp32.  Band and
+    // side jobs overwrite (padded keys get zeros); the global-key and random jobs add
+    // to the rows the band pass wrote.  The TMEM loads are warp-wide, so every thread
+    // issues them.
     if (ok && T > 0) ok = mbar_wait_bounded(acc_full, 0, abort_v, kWaitLimitNs);
     if (ok) {
       tc_fence_after();
-      const size_t prw = row < u.rows ? pos_row(p, u, u.hk, p.Hkv, uk) : 0;
-      float* dst = (g ? p.dk : p.dv) + prw * D;
+      constexpr bool kAdd = JOB == kJobGlobalKeys || JOB == kJobRandom;
+      size_t prw = 0;
+      float* base = g ? p.dk : p.dv;
+      bool write = row < u.rows;
+      if (JOB == kJobSide) {
+        base = g ? p.dsk : p.dsv;
+        prw = ((size_t)u.b * p.Hkv + u.hk) * p.S + uk;
+      } else if (kAdd) {
+        write = key_valid;
+        prw = ((size_t)u.b * p.Hkv + u.hk) * p.n + kpos;
+      } else if (write) {
+        prw = pos_row(p, u, u.hk, p.Hkv, uk);
+      }
+      float* dst = base + prw * D;
       const float mul = g ? p.scale : 1.f;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
@@ -563,14 +904,19 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
           tmem_ld32(lane_base + (g ? C::kAccK : C::kAccV) + ch * 32, rr);
           tmem_wait_ld_dep(rr);
         }
-        if (row < u.rows) {
+        if (write) {
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
             float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
             if (T > 0 && key_valid)
               v4 = make_float4(__uint_as_float(rr[q4 * 4]) * mul, __uint_as_float(rr[q4 * 4 + 1]) * mul,
                                __uint_as_float(rr[q4 * 4 + 2]) * mul, __uint_as_float(rr[q4 * 4 + 3]) * mul);
-            reinterpret_cast<float4*>(dst)[ch * 8 + q4] = v4;
+            float4* d4 = reinterpret_cast<float4*>(dst) + ch * 8 + q4;
+            if (kAdd) {
+              const float4 o = *d4;
+              v4 = make_float4(o.x + v4.x, o.y + v4.y, o.z + v4.z, o.w + v4.w);
+            }
+            *d4 = v4;
           }
         }
       }
@@ -615,14 +961,44 @@ cudaError_t launch_bwd_delta(const BwdParams& p, cudaStream_t s) {
 
 cudaError_t launch_bwd_dq(const BwdParams& p, cudaStream_t s) {
   const int grid = p.max_qtiles * p.B * p.Hq;
-  return p.D == 64 ? launch_kern(bwd_dq_kernel<64>, BCfg<64>::kSmemBytes, grid, kBThreads, p, s)
-                   : launch_kern(bwd_dq_kernel<128>, BCfg<128>::kSmemBytes, grid, kBThreads, p, s);
+  if (p.extras)
+    return p.D == 64 ? launch_kern(bwd_dq_kernel<64, true, false>, BCfg<64>::kSmemBytes, grid, kBThreads, p, s)
+                     : launch_kern(bwd_dq_kernel<128, true, false>, BCfg<128>::kSmemBytes, grid, kBThreads, p, s);
+  return p.D == 64 ? launch_kern(bwd_dq_kernel<64, false, false>, BCfg<64>::kSmemBytes, grid, kBThreads, p, s)
+                   : launch_kern(bwd_dq_kernel<128, false, false>, BCfg<128>::kSmemBytes, grid, kBThreads, p, s);
+}
+
+cudaError_t launch_bwd_dq_global_rows(const BwdParams& p, cudaStream_t s) {
+  if (p.g == 0) return cudaSuccess;
+  const int grid = p.B * p.Hq * (p.gpad / kTile);
+  return p.D == 64 ? launch_kern(bwd_dq_kernel<64, false, true>, BCfg<64>::kSmemBytes, grid, kBThreads, p, s)
+                   : launch_kern(bwd_dq_kernel<128, false, true>, BCfg<128>::kSmemBytes, grid, kBThreads, p, s);
+}
+
+template <int JOB>
+static cudaError_t launch_dkv_job(const BwdParams& p, int grid, cudaStream_t s) {
+  return p.D == 64 ? launch_kern(bwd_dkv_kernel<64, JOB>, KCfg<64>::kSmemBytes, grid, kDkvThreads, p, s)
+                   : launch_kern(bwd_dkv_kernel<128, JOB>, KCfg<128>::kSmemBytes, grid, kDkvThreads, p, s);
 }
 
 cudaError_t launch_bwd_dkv(const BwdParams& p, cudaStream_t s) {
   const int grid = p.max_ktiles * p.B * p.Hkv;
-  return p.D == 64 ? launch_kern(bwd_dkv_kernel<64>, KCfg<64>::kSmemBytes, grid, kDkvThreads, p, s)
-                   : launch_kern(bwd_dkv_kernel<128>, KCfg<128>::kSmemBytes, grid, kDkvThreads, p, s);
+  return p.extras ? launch_dkv_job<kJobBandX>(p, grid, s) : launch_dkv_job<kJobBand>(p, grid, s);
+}
+
+cudaError_t launch_bwd_dkv_global_keys(const BwdParams& p, cudaStream_t s) {
+  if (p.g == 0) return cudaSuccess;
+  return launch_dkv_job<kJobGlobalKeys>(p, p.B * p.Hkv * (p.gpad / kTile), s);
+}
+
+cudaError_t launch_bwd_dkv_side(const BwdParams& p, cudaStream_t s) {
+  if (p.S == 0) return cudaSuccess;
+  return launch_dkv_job<kJobSide>(p, p.B * p.Hkv * ((p.S + kTile - 1) / kTile), s);
+}
+
+cudaError_t launch_bwd_dkv_random(const BwdParams& p, cudaStream_t s) {
+  if (!p.rand_blocks || p.num_rand == 0) return cudaSuccess;
+  return launch_dkv_job<kJobRandom>(p, p.B * p.Hkv * ((p.n + kTile - 1) / kTile), s);
 }
 
 }  // namespace swa

@@ -87,6 +87,39 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// Acquire load of a global counter (gpu scope).
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Order this thread's generic-proxy global accesses with its async-proxy (TMA)
+// accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Wait until *count >= target (written by other CTAs of the same cooperative
+// launch), bounded like mbar_wait_bounded; then order the async proxy after it.
+__device__ __forceinline__ bool wait_count_bounded(const unsigned* count, unsigned target,
+                                                   volatile int* abort_flag, uint64_t limit_ns) {
+  uint64_t t0 = 0;
+  while (ld_acquire_gpu(count) < target) {
+    if (*abort_flag) return false;
+    const uint64_t now = global_timer_ns();
+    if (t0 == 0) {
+      t0 = now;
+    } else if (now - t0 > limit_ns) {
+      *abort_flag = 1;
+      return false;
+    }
+    __nanosleep(256);
+  }
+  fence_proxy_async_global();
+  return true;
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

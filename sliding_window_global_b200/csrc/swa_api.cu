@@ -37,6 +37,9 @@ struct swa_plan_s {
   float* part_o;
   float* part_lse;
   float* delta;        // backward: rowsum(dout * out) [B, Hq, n]
+  void* side_k;        // side keys / values built from k and v (side_from_kv)
+  void* side_v;
+  void* gdo;           // backward: gathered dout rows of the global tokens [B*Hq, gpad, D]
   int last_launches;
   int num_sms;         // persistent grid size
 };
@@ -99,6 +102,17 @@ swa_status swa_plan_create(swa_plan_t* out_plan, const swa_plan_desc* d) {
     o_delta = off;
     off = align_up(off + B * Hq * (size_t)d->seq_len * 4, 256);
   }
+  size_t o_gdo = 0;
+  if (p->gpad > 0 && d->dtype == SWA_BF16) {
+    o_gdo = off;
+    off = align_up(off + B * Hq * (size_t)p->gpad * d->head_dim * 2, 256);
+  }
+  size_t o_side = 0;
+  const size_t side_bytes = swa::side_buffer_bytes(*d);
+  if (side_bytes) {
+    o_side = off;
+    off += 2 * side_bytes;
+  }
   p->ws_bytes = off;
   if (cudaMalloc(&p->ws, p->ws_bytes) != cudaSuccess) {
     cudaGetLastError();
@@ -112,6 +126,11 @@ swa_status swa_plan_create(swa_plan_t* out_plan, const swa_plan_desc* d) {
   }
   p->err = reinterpret_cast<int*>(p->ws);
   if (o_delta) p->delta = reinterpret_cast<float*>(p->ws + o_delta);
+  if (o_gdo) p->gdo = p->ws + o_gdo;
+  if (o_side) {
+    p->side_k = p->ws + o_side;
+    p->side_v = p->ws + o_side + side_bytes;
+  }
   if (gl.end) {
     p->gq = p->ws + gl.gq;
     p->gk = p->ws + gl.gk;
@@ -177,6 +196,9 @@ swa_status swa_forward_ex(swa_plan_t plan, const swa_forward_args* args, void* s
   ws.part_o = plan->part_o;
   ws.part_lse = plan->part_lse;
   ws.nsplit_max = plan->nsplit_max;
+  ws.side_k = plan->side_k;
+  ws.side_v = plan->side_v;
+  ws.agg_count = reinterpret_cast<unsigned*>(plan->ws + 64);   // inside the error-word block
   int launches = 0;
   const swa_status st = swa::enqueue_forward(plan->desc, *args, ws, plan->num_sms,
                                              static_cast<cudaStream_t>(stream), &launches);
@@ -203,7 +225,34 @@ swa_status swa_backward(swa_plan_t plan, const swa_backward_args* a, void* strea
     if (a->dilation && a->dilation[h] < 1) return SWA_ERR_INVALID_ARG;
     if ((long long)a->window[h] * (a->dilation ? a->dilation[h] : 1) > (1LL << 30)) return SWA_ERR_INVALID_ARG;
   }
-  if (d.dtype != SWA_BF16 || d.num_side > 0 || !plan->delta) return SWA_ERR_UNSUPPORTED;
+  if (d.dtype != SWA_BF16 || !plan->delta) return SWA_ERR_UNSUPPORTED;
+  // terms beyond the band (the forward's optional terms)
+  const int num_global = a->num_global;
+  const int32_t* rand_blocks = a->num_rand > 0 ? a->rand_blocks : nullptr;
+  if (num_global < 0 || num_global > d.max_global || (num_global > 0 && !a->global_idx)) return SWA_ERR_INVALID_ARG;
+  if (a->num_rand < 0 || a->num_rand > swa::kMaxRand || (a->num_rand > 0 && !rand_blocks)) return SWA_ERR_INVALID_ARG;
+  if (d.num_side > 0 && (!a->side_k || !a->side_v || !a->dside_k || !a->dside_v || !aligned16(a->side_k) ||
+                         !aligned16(a->side_v) || !aligned16(a->dside_k) || !aligned16(a->dside_v)))
+    return SWA_ERR_INVALID_ARG;
+  if ((a->bias && (reinterpret_cast<uintptr_t>(a->bias) & 3u)) ||
+      (a->local_bias && (reinterpret_cast<uintptr_t>(a->local_bias) & 3u)))
+    return SWA_ERR_INVALID_ARG;
+  if (a->causal && num_global > 0) return SWA_ERR_UNSUPPORTED;
+  if (rand_blocks) {
+    if (a->causal) return SWA_ERR_UNSUPPORTED;
+    for (int h = 0; h < Hq; ++h)
+      if (a->dilation && a->dilation[h] != 1) return SWA_ERR_UNSUPPORTED;
+  }
+  if (a->local_bias) {
+    if (a->local_radius < 0 || a->local_radius > (1 << 30)) return SWA_ERR_INVALID_ARG;
+    for (int h = 0; h < Hq; ++h) {
+      const long long reach = std::min((long long)a->window[h] * (a->dilation ? a->dilation[h] : 1),
+                                       (long long)n - 1);
+      if (a->local_radius < reach) return SWA_ERR_INVALID_ARG;
+    }
+  }
+  if (num_global > 0 && (!plan->gq || !plan->gdo)) return SWA_ERR_UNSUPPORTED;
+  const bool extras = num_global > 0 || d.num_side > 0 || a->local_bias || rand_blocks;
   const int G = Hq / d.num_kv_heads;
   for (int h = 0; h < Hq; ++h) {
     const int h0 = (h / G) * G;
@@ -231,6 +280,20 @@ swa_status swa_backward(swa_plan_t plan, const swa_backward_args* a, void* strea
   p.dk = a->dk;
   p.dv = a->dv;
   p.err = plan->err;
+  p.extras = extras ? 1 : 0;
+  p.global_idx = num_global > 0 ? a->global_idx : nullptr;
+  p.g = num_global;
+  p.gpad = num_global > 0 ? (int)align_up(num_global, kTile) : 0;
+  p.S = d.num_side;
+  p.side_block = d.num_side > 0 ? d.side_block : 1;
+  p.nblk = d.num_side > 0 ? (n + d.side_block - 1) / d.side_block : 0;
+  p.bias = d.num_side > 0 ? a->bias : nullptr;
+  p.local_bias = a->local_bias;
+  p.local_radius = a->local_bias ? a->local_radius : 0;
+  p.rand_blocks = rand_blocks;
+  p.num_rand = rand_blocks ? a->num_rand : 0;
+  p.dsk = d.num_side > 0 ? a->dside_k : nullptr;
+  p.dsv = d.num_side > 0 ? a->dside_v : nullptr;
   // residue classes (as in the forward) and tiles per head
   int nclass = 0;
   swa_status st = SWA_OK;
@@ -261,8 +324,36 @@ swa_status swa_backward(swa_plan_t plan, const swa_backward_args* a, void* strea
     p.max_ktiles = std::max(p.max_ktiles, tiles);
   }
   if (st != SWA_OK) return st;
+  // the non-band jobs walk every position: the (d = 1, c = 0) class
+  if (extras) {
+    p.dense_class = -1;
+    for (int c = 0; c < nclass; ++c)
+      if (p.cls[c].d == 1) p.dense_class = c;
+    if (p.dense_class < 0) {
+      if (nclass + 1 > kMaxClasses) return SWA_ERR_UNSUPPORTED;
+      p.cls[nclass].d = 1;
+      p.cls[nclass].c = 0;
+      p.cls[nclass].n_c = n;
+      p.cls[nclass].nres = 1;
+      p.dense_class = nclass++;
+    }
+  }
   const size_t row = (size_t)D * 2;
   bool ok = true;
+  if (num_global > 0) {
+    const uint64_t gp = (uint64_t)p.gpad;
+    ok = ok && make_map(&p.mgk, plan->gk, D, gp, (uint64_t)p.B * p.Hkv, row, gp * row);
+    ok = ok && make_map(&p.mgv, plan->gv, D, gp, (uint64_t)p.B * p.Hkv, row, gp * row);
+    ok = ok && make_map(&p.mgq, plan->gq, D, gp, (uint64_t)p.B * Hq, row, gp * row);
+    ok = ok && make_map(&p.mgdo, plan->gdo, D, gp, (uint64_t)p.B * Hq, row, gp * row);
+    ok = ok && make_map(&p.mgq64, plan->gq, D, gp, (uint64_t)p.B * Hq, row, gp * row, false, 64);
+    ok = ok && make_map(&p.mgdo64, plan->gdo, D, gp, (uint64_t)p.B * Hq, row, gp * row, false, 64);
+  }
+  if (d.num_side > 0) {
+    const uint64_t S = (uint64_t)d.num_side;
+    ok = ok && make_map(&p.msk, a->side_k, D, S, (uint64_t)p.B * p.Hkv, row, S * row);
+    ok = ok && make_map(&p.msv, a->side_v, D, S, (uint64_t)p.B * p.Hkv, row, S * row);
+  }
   for (int c = 0; c < nclass && ok; ++c) {
     const int dd = p.cls[c].d, cc = p.cls[c].c, nc = p.cls[c].n_c;
     ok = ok && make_map(&p.mq[c], static_cast<const char*>(a->q) + cc * row, D, nc, (uint64_t)p.B * Hq,
@@ -280,17 +371,35 @@ swa_status swa_backward(swa_plan_t plan, const swa_backward_args* a, void* strea
                         (uint64_t)p.B * Hq, dd * row, (uint64_t)n * row, false, 64);
   }
   if (!ok) return SWA_ERR_CUDA;
+  // Launch order: Delta; gathered global rows; dq (band + extra key tiles), then the
+  // global rows' remaining keys added; dk/dv of the band (and the global rows'
+  // remaining keys) written, then the global keys' and random blocks' remaining
+  // rows added; the side keys' gradients.
   int launches = 0;
   cudaError_t ce = swa::launch_bwd_delta(p, s);
   ++launches;
-  if (ce == cudaSuccess) {
-    ce = swa::launch_bwd_dq(p, s);
-    ++launches;
+  auto step = [&](cudaError_t (*fn)(const swa::BwdParams&, cudaStream_t)) {
+    if (ce == cudaSuccess) {
+      ce = fn(p, s);
+      ++launches;
+    }
+  };
+  if (num_global > 0 && ce == cudaSuccess) {
+    ce = swa::launch_gather_rows(a->q, plan->gq, p.global_idx, p.B, Hq, n, num_global, p.gpad, D, 2, s);
+    if (ce == cudaSuccess)
+      ce = swa::launch_gather_rows(a->dout, plan->gdo, p.global_idx, p.B, Hq, n, num_global, p.gpad, D, 2, s);
+    if (ce == cudaSuccess)
+      ce = swa::launch_gather_rows(a->k, plan->gk, p.global_idx, p.B, p.Hkv, n, num_global, p.gpad, D, 2, s);
+    if (ce == cudaSuccess)
+      ce = swa::launch_gather_rows(a->v, plan->gv, p.global_idx, p.B, p.Hkv, n, num_global, p.gpad, D, 2, s);
+    launches += 4;
   }
-  if (ce == cudaSuccess) {
-    ce = swa::launch_bwd_dkv(p, s);
-    ++launches;
-  }
+  step(swa::launch_bwd_dq);
+  if (num_global > 0) step(swa::launch_bwd_dq_global_rows);
+  step(swa::launch_bwd_dkv);
+  if (num_global > 0) step(swa::launch_bwd_dkv_global_keys);
+  if (rand_blocks) step(swa::launch_bwd_dkv_random);
+  if (d.num_side > 0) step(swa::launch_bwd_dkv_side);
   plan->last_launches = launches;
   if (ce != cudaSuccess) return SWA_ERR_CUDA;
   if (d.flags & SWA_DEBUG_CHECKS) return swa_plan_check(plan, stream);
@@ -301,6 +410,11 @@ swa_status swa_selftest_wait_timeout(swa_plan_t plan, uint64_t limit_ns, void* s
   if (!plan || limit_ns == 0 || limit_ns > 5000000000ull) return SWA_ERR_INVALID_ARG;
   plan->last_launches = 1;
   return cuda_status(swa::launch_wait_probe(plan->err, limit_ns, static_cast<cudaStream_t>(stream)));
+}
+
+swa_status swa_selftest_exp2_poly(const float* x, float* y, int n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return SWA_ERR_INVALID_ARG;
+  return cuda_status(swa::launch_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream)));
 }
 
 swa_status swa_side_aggregate(const void* x, void* out, int batch, int heads, int seq_len,

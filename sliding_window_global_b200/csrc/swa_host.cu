@@ -86,6 +86,12 @@ GlobalLayout global_layout(const swa_plan_desc& d, int gpad, int nsplit, size_t 
   return L;
 }
 
+size_t side_buffer_bytes(const swa_plan_desc& d) {
+  if (d.num_side <= 0 || d.side_block < 1 || d.num_side != d.seq_len / d.side_block) return 0;
+  const size_t es = d.dtype == SWA_FP32 ? 4 : 2;
+  return align_up((size_t)d.batch * d.num_kv_heads * d.num_side * d.head_dim * es, 256);
+}
+
 swa_status read_and_clear_error(int* err, cudaStream_t s) {
   if (cudaStreamSynchronize(s) != cudaSuccess) return SWA_ERR_CUDA;
   int h = 0;
@@ -117,6 +123,16 @@ swa_status enqueue_forward(const swa_plan_desc& d, const swa_forward_args& args,
   if (causal != 0 && causal != 1) return SWA_ERR_INVALID_ARG;
   if (num_global < 0 || num_global > d.max_global) return SWA_ERR_INVALID_ARG;
   if (num_global > 0 && !global_idx) return SWA_ERR_INVALID_ARG;
+  if (args.side_from_kv != 0 && args.side_from_kv != 1) return SWA_ERR_INVALID_ARG;
+  const bool build_side = args.side_from_kv == 1;
+  if (build_side) {
+    // side keys / values are the block means of k and v, made here
+    if (side_k || side_v || d.num_side < 1 || d.num_side != d.seq_len / d.side_block)
+      return SWA_ERR_INVALID_ARG;
+    if (!ws.side_k || !ws.side_v) return SWA_ERR_UNSUPPORTED;
+    side_k = ws.side_k;
+    side_v = ws.side_v;
+  }
   if (d.num_side > 0) {
     if (!side_k || !side_v) return SWA_ERR_INVALID_ARG;
     if (!aligned16(side_k) || !aligned16(side_v)) return SWA_ERR_INVALID_ARG;
@@ -218,7 +234,6 @@ swa_status enqueue_forward(const swa_plan_desc& d, const swa_forward_args& args,
   // same rows of two heads that share one KV head; otherwise it is two consecutive
   // row tiles of one head.  (Per-head bias rows are staged once per unit, so a
   // unit keeps one head when either bias is present.)
-  int max_units = 0;
   {
     bool pair = (p.G % 2 == 0) && !(d.num_side > 0 && bias) && !local_bias;
     for (int h = 0; pair && h < Hq; h += 2)
@@ -233,8 +248,13 @@ swa_status enqueue_forward(const swa_plan_desc& d, const swa_forward_args& args,
         units += pair ? tiles : (tiles + 1) / 2;
       }
       p.tiles[h] = units;
-      max_units = std::max(max_units, units);
     }
+    // linear order of band units: batch, head (pair), residue class, row unit
+    p.num_hp = pair ? Hq / 2 : Hq;
+    p.unit_prefix[0] = 0;
+    for (int hp = 0; hp < p.num_hp; ++hp)
+      p.unit_prefix[hp + 1] = p.unit_prefix[hp] + p.tiles[pair ? 2 * hp : hp];
+    p.units_total = (long long)p.B * p.unit_prefix[p.num_hp];
   }
   if (num_global > 0) {
     p.dense_class = -1;
@@ -292,7 +312,6 @@ swa_status enqueue_forward(const swa_plan_desc& d, const swa_forward_args& args,
       p.nsplit = p.nsplit_keys + side_split;
     }
   }
-  p.max_units = max_units;
 
   // ---------------------------------------------------------- launches
   int launches = 0;
@@ -307,6 +326,23 @@ swa_status enqueue_forward(const swa_plan_desc& d, const swa_forward_args& args,
     if (ce != cudaSuccess) return SWA_ERR_CUDA;
     const swa_status st = read_and_clear_error(ws.err, s);
     if (st != SWA_OK) return st;
+  }
+  if (build_side && bf16 && ws.agg_count) {
+    // the band kernel builds the side keys / values in its prologue
+    p.agg_k = k;
+    p.agg_v = v;
+    p.agg_sk = const_cast<void*>(side_k);
+    p.agg_sv = const_cast<void*>(side_v);
+    p.agg_count = ws.agg_count;
+    if (cudaMemsetAsync(ws.agg_count, 0, sizeof(unsigned), s) != cudaSuccess) return SWA_ERR_CUDA;
+  } else if (build_side) {
+    ce = launch_side_aggregate_kv(k, v, const_cast<void*>(side_k), const_cast<void*>(side_v), d.batch,
+                                  d.num_kv_heads, n, D, d.side_block, valid_len, bf16 ? 1 : 0, s);
+    ++launches;
+    if (ce != cudaSuccess) {
+      *launches_out = launches;
+      return SWA_ERR_CUDA;
+    }
   }
   if (!bf16) {
     ce = launch_simt(p, q, k, v, side_k, side_v, 0, s);

@@ -30,7 +30,13 @@ struct ForwardScratch {
   float* part_o = nullptr;       // global-row partials [nsplit, B*Hq, gpad, D] fp32
   float* part_lse = nullptr;     // [nsplit, B*Hq, gpad]
   int nsplit_max = 0;            // splits part_o / part_lse hold (the side-key split included)
+  void* side_k = nullptr;        // side keys / values built from k and v [B*Hkv, S, D] (plan
+  void* side_v = nullptr;        // workspace; null where the caller must pass them)
+  unsigned* agg_count = nullptr; // CTA counter of the band kernel's fused side-key prologue
 };
+
+// Bytes of one side key (or value) buffer a plan reserves for side_from_kv.
+size_t side_buffer_bytes(const swa_plan_desc& d);
 
 // Byte offsets of the global-token scratch for gpad global slots and nsplit
 // splits, laid out from byte `base` (each piece 256-byte aligned).

@@ -56,13 +56,25 @@ struct AttnParams {
   float* part_o;                     // global-row partials [nsplit, B*Hq, gpad, D]
   float* part_lse;                   // [nsplit, B*Hq, gpad]
   int nsplit_keys, split_keys, nsplit;  // global-row key splits (+1 for side keys)
-  int max_units;                     // largest tiles[h]
   int pair_heads;                    // units pair heads 2m, 2m+1 (same rows) instead of row tiles
+  int num_hp;                        // heads (or head pairs) that own work units
+  long long units_total;             // band work units over the batch: B * unit_prefix[num_hp]
   int* err;                          // device error word
+  // Fused Transient-Global prologue (MODE 0): every CTA first builds its share of
+  // the side keys / values (block means of agg_k / agg_v into agg_sk / agg_sv, the
+  // buffers msk / msv map), then counts itself done in *agg_count (zeroed before
+  // the launch); side tiles are loaded once all gridDim.x CTAs are counted.  The
+  // launch is cooperative, so every CTA is resident.  Null agg_count: side keys are inputs.
+  const void* agg_k;
+  const void* agg_v;
+  void* agg_sk;
+  void* agg_sv;
+  unsigned* agg_count;
 
   int window[kMaxHeads];
   int class_base[kMaxHeads];         // class id of (dilation[h], c = 0)
   int tiles[kMaxHeads];              // work units of head h (of head pair h/2 when pairing)
+  int unit_prefix[kMaxHeads + 1];    // units of heads (head pairs) before index hp, one batch
 };
 
 // Launchers (each returns the launch's cudaError_t).
@@ -72,14 +84,23 @@ cudaError_t launch_gather_globals(const AttnParams& p, const void* q, const void
                                   const void* v, void* gq, void* gk, void* gv, int elem_bytes,
                                   cudaStream_t s);
 cudaError_t launch_merge_global_rows(const AttnParams& p, int bf16_out, cudaStream_t s);
+// dst[bh, e, :] = src[bh, gidx[b, e], :] for e < g, zeros up to gpad ([B*H, n, D] -> [B*H, gpad, D]).
+cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* gidx, int B, int H, int n, int g,
+                               int gpad, int D, int elem_bytes, cudaStream_t s);
 cudaError_t launch_simt(const AttnParams& p, const void* q, const void* k, const void* v,
                         const void* side_k, const void* side_v, int bf16, cudaStream_t s);
 // Debug check of the index inputs: global_idx rows strictly increasing inside
 // [0, valid_len), random key blocks inside [0, ceil(n / 128)); sets kDevErrCheck.
 cudaError_t launch_check_inputs(const AttnParams& p, cudaStream_t s);
 cudaError_t launch_wait_probe(int* err, uint64_t limit_ns, cudaStream_t s);
+cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t s);
 cudaError_t launch_side_aggregate(const void* x, void* out, int B, int H, int n, int D, int kb,
                                   const int32_t* valid_len, int bf16, cudaStream_t s);
+// Side keys and values (block means of k and v, as launch_side_aggregate) in one
+// launch; D must be a multiple of 8 (bf16) or 4 (fp32), buffers 16-byte aligned.
+cudaError_t launch_side_aggregate_kv(const void* k, const void* v, void* sk, void* sv, int B, int H,
+                                     int n, int D, int kb, const int32_t* valid_len, int bf16,
+                                     cudaStream_t s);
 size_t band_tc_smem_bytes(int D);
 
 }  // namespace swa

@@ -31,6 +31,7 @@ EXPORTS = (
     "swa_plan_workspace_bytes", "swa_plan_last_launches", "swa_status_string",
     "swa_side_aggregate", "swa_relative_bucket", "swa_expand_side_bias", "swa_forward_noalloc",
     "swa_forward_ex", "swa_bucket_local_bias", "swa_backward", "swa_selftest_wait_timeout",
+    "swa_selftest_exp2_poly",
 )
 
 
@@ -59,6 +60,7 @@ class ForwardArgs(ctypes.Structure):
         ("valid_len", ctypes.c_void_p), ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p),
         ("local_bias", ctypes.c_void_p), ("local_radius", ctypes.c_int),
         ("rand_blocks", ctypes.c_void_p), ("num_rand", ctypes.c_int),
+        ("side_from_kv", ctypes.c_int),
     ]
 
 
@@ -70,6 +72,11 @@ class BackwardArgs(ctypes.Structure):
         ("window", ctypes.c_void_p), ("dilation", ctypes.c_void_p), ("causal", ctypes.c_int),
         ("valid_len", ctypes.c_void_p), ("dq", ctypes.c_void_p), ("dk", ctypes.c_void_p),
         ("dv", ctypes.c_void_p),
+        ("global_idx", ctypes.c_void_p), ("num_global", ctypes.c_int),
+        ("side_k", ctypes.c_void_p), ("side_v", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+        ("local_bias", ctypes.c_void_p), ("local_radius", ctypes.c_int),
+        ("rand_blocks", ctypes.c_void_p), ("num_rand", ctypes.c_int),
+        ("dside_k", ctypes.c_void_p), ("dside_v", ctypes.c_void_p),
     ]
 
 
@@ -118,6 +125,8 @@ def load_library():
         lib.swa_backward.restype = I
         lib.swa_selftest_wait_timeout.argtypes = [P, ctypes.c_uint64, P]
         lib.swa_selftest_wait_timeout.restype = I
+        lib.swa_selftest_exp2_poly.argtypes = [P, P, I, P]
+        lib.swa_selftest_exp2_poly.restype = I
         _lib = lib
         return lib
 
@@ -200,11 +209,14 @@ class Plan:
                 bias: Optional[torch.Tensor] = None, valid_len: Optional[torch.Tensor] = None,
                 out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                 return_lse: bool = True, local_bias: Optional[torch.Tensor] = None,
-                rand_blocks: Optional[torch.Tensor] = None, stream=None):
+                rand_blocks: Optional[torch.Tensor] = None, side_from_kv: bool = False,
+                stream=None):
         """``local_bias``: optional [Hq, 2R+1] fp32 device table of the LongT5 local
         relative-position bias (window keys of non-global rows, column (j - i) + R).
         ``rand_blocks``: optional int32 device tensor [B, Hq, ceil(n/128), r] of
-        BigBird random key blocks (128 keys each) per query block."""
+        BigBird random key blocks (128 keys each) per query block.
+        ``side_from_kv``: build the Transient-Global side keys / values from k and v
+        on the device (block means of ``side_block`` tokens) instead of taking them."""
         d = self.desc
         H = d.num_q_heads
         if out is None:
@@ -214,7 +226,7 @@ class Plan:
         w_arr, _ = _host_i32(window, H, "window")
         d_arr, _ = _host_i32(dilation, H, "dilation")
         g = 0 if global_idx is None else int(global_idx.shape[-1])
-        if local_bias is not None or rand_blocks is not None:
+        if local_bias is not None or rand_blocks is not None or side_from_kv:
             width = 1 if local_bias is None else int(local_bias.shape[-1])
             if local_bias is not None and (local_bias.dim() != 2 or local_bias.shape[0] != H
                                            or width % 2 == 0):
@@ -233,7 +245,8 @@ class Plan:
                 None if d_arr is None else ctypes.cast(d_arr, ctypes.c_void_p), int(bool(causal)),
                 _dev_ptr(valid_len, "valid_len", torch.int32), _dev_ptr(out, "out", self.dtype),
                 _dev_ptr(lse, "lse", torch.float32), _dev_ptr(local_bias, "local_bias", torch.float32),
-                (width - 1) // 2, _dev_ptr(rand_blocks, "rand_blocks", torch.int32), nrand)
+                (width - 1) // 2, _dev_ptr(rand_blocks, "rand_blocks", torch.int32), nrand,
+                int(bool(side_from_kv)))
             st = self._lib.swa_forward_ex(self._h, ctypes.byref(a), _stream_handle(stream))
             if st != 0:
                 raise SwaError(st, "swa_forward_ex")
@@ -253,9 +266,13 @@ class Plan:
                  lse: torch.Tensor, dout: torch.Tensor, *, window, dilation=None,
                  causal: bool = False, valid_len: Optional[torch.Tensor] = None,
                  dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
-                 dv: Optional[torch.Tensor] = None, stream=None):
-        """Gradients (dq, dk, dv), fp32, of the band attention for the upstream gradient
-        ``dout``; ``out`` and ``lse`` are the forward's results."""
+                 dv: Optional[torch.Tensor] = None, global_idx: Optional[torch.Tensor] = None,
+                 side_k: Optional[torch.Tensor] = None, side_v: Optional[torch.Tensor] = None,
+                 bias: Optional[torch.Tensor] = None, local_bias: Optional[torch.Tensor] = None,
+                 rand_blocks: Optional[torch.Tensor] = None, stream=None):
+        """Gradients, fp32, for the upstream gradient ``dout``; ``out`` and ``lse`` are the
+        forward's results, and the optional terms those the forward ran with.  Returns
+        (dq, dk, dv), plus (dside_k, dside_v) when the plan has side keys."""
         d = self.desc
         H, Hkv = d.num_q_heads, d.num_kv_heads
         shape_q = (d.batch, H, d.seq_len, d.head_dim)
@@ -268,16 +285,31 @@ class Plan:
             dv = torch.empty(shape_k, dtype=torch.float32, device=q.device)
         w_arr, _ = _host_i32(window, H, "window")
         d_arr, _ = _host_i32(dilation, H, "dilation")
+        dsk = dsv = None
+        if d.num_side > 0:
+            shape_s = (d.batch, Hkv, d.num_side, d.head_dim)
+            dsk = torch.empty(shape_s, dtype=torch.float32, device=q.device)
+            dsv = torch.empty(shape_s, dtype=torch.float32, device=q.device)
+        g = 0 if global_idx is None else int(global_idx.shape[-1])
+        width = 1 if local_bias is None else int(local_bias.shape[-1])
+        nrand = 0 if rand_blocks is None else int(rand_blocks.shape[-1])
         a = BackwardArgs(
             _dev_ptr(q, "q", self.dtype), _dev_ptr(k, "k", self.dtype), _dev_ptr(v, "v", self.dtype),
             _dev_ptr(out, "out", self.dtype), _dev_ptr(lse, "lse", torch.float32),
             _dev_ptr(dout, "dout", self.dtype), ctypes.cast(w_arr, ctypes.c_void_p),
             None if d_arr is None else ctypes.cast(d_arr, ctypes.c_void_p), int(bool(causal)),
             _dev_ptr(valid_len, "valid_len", torch.int32), _dev_ptr(dq, "dq", torch.float32),
-            _dev_ptr(dk, "dk", torch.float32), _dev_ptr(dv, "dv", torch.float32))
+            _dev_ptr(dk, "dk", torch.float32), _dev_ptr(dv, "dv", torch.float32),
+            _dev_ptr(global_idx, "global_idx", torch.int32), g,
+            _dev_ptr(side_k, "side_k", self.dtype), _dev_ptr(side_v, "side_v", self.dtype),
+            _dev_ptr(bias, "bias", torch.float32), _dev_ptr(local_bias, "local_bias", torch.float32),
+            (width - 1) // 2, _dev_ptr(rand_blocks, "rand_blocks", torch.int32), nrand,
+            _dev_ptr(dsk, "dside_k", torch.float32), _dev_ptr(dsv, "dside_v", torch.float32))
         st = self._lib.swa_backward(self._h, ctypes.byref(a), _stream_handle(stream))
         if st != 0:
             raise SwaError(st, "swa_backward")
+        if dsk is not None:
+            return dq, dk, dv, dsk, dsv
         return dq, dk, dv
 
     def selftest_wait_timeout(self, limit_ns: int, stream=None) -> None:
@@ -342,6 +374,18 @@ def side_aggregate(x: torch.Tensor, block: int, valid_len: Optional[torch.Tensor
     if st != 0:
         raise SwaError(st, "swa_side_aggregate")
     return out
+
+
+def selftest_exp2_poly(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """The band kernel's FMA-pipe 2^x evaluated on a CUDA fp32 tensor (a self test)."""
+    lib = load_library()
+    x = x.contiguous()
+    y = torch.empty_like(x)
+    st = lib.swa_selftest_exp2_poly(_dev_ptr(x, "x", torch.float32), _dev_ptr(y, "y", torch.float32),
+                                    int(x.numel()), _stream_handle(stream))
+    if st != 0:
+        raise SwaError(st, "swa_selftest_exp2_poly")
+    return y
 
 
 def relative_bucket(delta: int) -> int:

@@ -25,7 +25,7 @@ def lib():
 def _declared_functions():
     text = open(os.path.join(ROOT, "include", "swa.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(swa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(swa_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_exports_every_declared_symbol(lib):
@@ -140,6 +140,11 @@ def test_backward_null_arguments(lib):
     assert lib.swa_backward(None, None, None) == 1
     args = binding.BackwardArgs()
     assert lib.swa_backward(None, ctypes.byref(args), None) == 1
+
+
+def test_exp2_selftest_rejects_bad_arguments(lib):
+    assert lib.swa_selftest_exp2_poly(None, None, -1, None) == 1
+    assert lib.swa_selftest_exp2_poly(None, None, 4, None) == 1
 
 
 def test_selftest_rejects_bad_limits(lib):

@@ -1,8 +1,11 @@
 """The bench's multi-rank logic on CPU with two gloo ranks: every rank runs a
 replica, the job time is the slowest rank's (all-reduce MAX), the whole-job
 throughput counts every rank's work, and only rank 0 runs the reference arm."""
+import json
 import os
 import socket
+import subprocess
+import sys
 
 import pytest
 import torch
@@ -60,3 +63,44 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
         workload, steps, warmup = "longformer_tiny", 1, 0
     bench.run_reference(A())
     assert capsys.readouterr().out == ""
+
+
+def test_launch_decision_for_gpus_flag():
+    assert bench.launch_decision(1, {}) == "run"
+    assert bench.launch_decision(2, {}) == "relaunch"
+    assert bench.launch_decision(2, {"WORLD_SIZE": "2"}) == "run"
+    assert bench.launch_decision(2, {"WORLD_SIZE": "4"}) == "error"
+    assert bench.launch_decision(1, {"WORLD_SIZE": "2"}) == "error"
+
+
+def test_torchrun_command_one_rank_per_gpu_on_localhost():
+    cmd = bench.torchrun_command(4, ["--gpus", "4", "--steps", "3"], 29511, 900)
+    assert cmd[:4] == ["timeout", "-k", "60", "900"]
+    assert "--nproc-per-node=4" in cmd and "--nnodes=1" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[cmd.index("--master-port") + 1] == "29511"
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "3"]
+    assert os.path.basename(cmd[-5]) == "bench.py"
+
+
+def test_bench_gpus_two_relaunches_two_ranks_on_cpu():
+    """`bench.py --gpus 2` started without torchrun starts two ranks itself; the
+    reference arm (CPU oracle, rank 0 only) then reports the job's two GPUs."""
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--impl",
+                        "reference", "--workload", "longformer_tiny", "--steps", "1", "--warmup", "0",
+                        "--ref-budget", "0.2"], capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1                               # rank 0 alone prints
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["n_gpus"] == 2
+
+
+def test_bench_rejects_a_rank_count_that_differs_from_gpus():
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="3", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2"],
+                       capture_output=True, text=True, timeout=120, env=env)
+    assert r.returncode != 0

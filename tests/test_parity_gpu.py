@@ -279,6 +279,54 @@ def test_side_aggregate_matches_oracle():
     assert np.all(np.abs(got - ref) <= ulp)
 
 
+@pytest.mark.parametrize("padding,seq_len", [(0, 1024), (45, 1000)], ids=["plain", "padded_ragged"])
+def test_side_keys_built_from_kv(padding, seq_len):
+    """side_from_kv: the band kernel builds the Transient-Global side keys / values in
+    its prologue (one launch in all) -- bit-identical to passing swa_side_aggregate's
+    block means, and within tolerance of the oracle's block means -> attention.  The
+    ragged case has a trailing partial block (n % 16 = 8) and padded tokens."""
+    _need_gpu()
+    import dataclasses
+    from sliding_window_global_b200 import Plan, side_aggregate
+    w = dataclasses.replace(workloads.SMALL["longt5_tglobal"], seq_len=seq_len, padding=padding,
+                            name=f"tglobal_fused_{seq_len}")
+    inp = helpers.host_problem(w)
+    dinp = helpers.to_dev(inp)
+    plan = Plan(w.batch, w.seq_len, w.q_heads, w.kv_heads, w.head_dim, torch.bfloat16,
+                num_side=w.num_side, side_block=w.side_block)
+    kw = dict(window=dinp["window"], dilation=dinp["dilation"], bias=dinp["bias"],
+              valid_len=dinp["valid_len"])
+    out_f, lse_f = plan.forward(dinp["q"], dinp["k"], dinp["v"], side_from_kv=True, **kw)
+    assert plan.last_launches == 1                    # the band kernel builds them in its prologue
+    sk = side_aggregate(dinp["k"], w.side_block, dinp["valid_len"])
+    sv = side_aggregate(dinp["v"], w.side_block, dinp["valid_len"])
+    out_x, lse_x = plan.forward(dinp["q"], dinp["k"], dinp["v"], side_k=sk, side_v=sv, **kw)
+    torch.cuda.synchronize()
+    assert plan.check() == 0
+    assert torch.equal(out_f, out_x) and torch.equal(lse_f, lse_x)
+    ref_o, ref_l, _ = helpers.oracle_problem(w, inp).forward()
+    helpers.compare(out_f.float().cpu().numpy(), lse_f.cpu().numpy(), ref_o, ref_l, "bf16",
+                    "side_from_kv")
+
+
+def test_side_from_kv_argument_checks():
+    _need_gpu()
+    from sliding_window_global_b200 import Plan, SwaError
+    w = workloads.SMALL["longt5_tglobal"]
+    dinp = helpers.to_dev(helpers.host_problem(w))
+    plan = Plan(w.batch, w.seq_len, w.q_heads, w.kv_heads, w.head_dim, torch.bfloat16,
+                num_side=w.num_side, side_block=w.side_block)
+    with pytest.raises(SwaError) as e:          # side keys passed as well
+        plan.forward(dinp["q"], dinp["k"], dinp["v"], window=dinp["window"], side_k=dinp["side_k"],
+                     side_v=dinp["side_v"], side_from_kv=True)
+    assert e.value.status == 1
+    plan2 = Plan(w.batch, w.seq_len, w.q_heads, w.kv_heads, w.head_dim, torch.bfloat16,
+                 num_side=w.num_side - 1, side_block=w.side_block)   # S != n / block
+    with pytest.raises(SwaError) as e:
+        plan2.forward(dinp["q"], dinp["k"], dinp["v"], window=dinp["window"], side_from_kv=True)
+    assert e.value.status == 1
+
+
 def test_debug_mode_flags_bad_global_index():
     """A global index list that is not strictly increasing inside [0, valid_len) is a
     precondition failure.  Debug mode checks it on the device and reads the result
