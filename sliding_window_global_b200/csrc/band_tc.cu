@@ -125,7 +125,10 @@ struct Cfg {
   static constexpr uint32_t kKOff = 2 * kTileBytes;
   static constexpr uint32_t kVOff = kKOff + NS * kTileBytes;
   static constexpr uint32_t kBiasOff = kVOff + NS * kTileBytes;  // 4 shifted copies
-  static constexpr uint32_t kBarOff = kBiasOff + 4 * kBiasCopy * 4;
+  // floats per staged bias copy; the epilogue warpgroup's static state leaves less
+  // room at D = 128
+  static constexpr int kCopy = (D == 128 && kEpiWG) ? 1792 : kBiasCopy;
+  static constexpr uint32_t kBarOff = kBiasOff + 4 * kCopy * 4;
   static constexpr int kNumBars = 2 + 2 + 3 * NS + 2 + 2 + 2 + 2 + 2 + 2 + 2 + 2;
   static constexpr uint32_t kSmemBytes = kBarOff + kNumBars * 8 + 1024;
   // TMEM columns.  D = 128: S_A | S_B | O_A | O_B, P written over S.  D = 64 has
@@ -147,8 +150,10 @@ static_assert(kSoftmaxThreads * kRegsSoftmax + 128 * kRegsControl + (kEpiWG ? 12
               "setmaxnreg split exceeds the launch register budget");
 static_assert(!kEpiWG || (kRegsEpi >= 24 && kRegsEpi % 8 == 0), "epilogue register share");
 static_assert(kRegsSoftmax % 8 == 0 && kRegsControl % 8 == 0, "setmaxnreg takes multiples of 8");
-static_assert(Cfg<64>::kSmemBytes + 2 * kTile * 4 + 16 <= 227 * 1024, "shared memory, D = 64");
-static_assert(Cfg<128>::kSmemBytes + 2 * kTile * 4 + 16 <= 227 * 1024, "shared memory, D = 128");
+// dynamic + static (sGpos, sInv with the epilogue warpgroup, two words) shared memory
+constexpr uint32_t kStaticSmem = 2 * kTile * 4 + (kEpiWG ? 2 * 2 * kTile * 4 : 0) + 16;
+static_assert(Cfg<64>::kSmemBytes + kStaticSmem <= 227 * 1024, "shared memory, D = 64");
+static_assert(Cfg<128>::kSmemBytes + kStaticSmem <= 227 * 1024, "shared memory, D = 128");
 static_assert(emu_per32<64>() % 4 == 0 && emu_per32<64>() <= 32 && emu_per32<128>() % 4 == 0 &&
                   emu_per32<128>() <= 32,
               "polynomial exponentials come in groups of four");
@@ -613,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   // shared bias area: 4 copies of the local-bias row (stride lstride floats), then
   // 4 copies of the side-bias segment (stride side_stride)
   const int lstride = has_local ? p.local_stride : 0;
-  const int side_stride = kBiasCopy - lstride;
+  const int side_stride = C::kCopy - lstride;
   float* sLocal = sBias;
   float* sSide = sBias + 4 * lstride;
 
@@ -1337,6 +1342,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 size_t band_tc_smem_bytes(int D) {
   return D == 64 ? Cfg<64>::kSmemBytes : Cfg<128>::kSmemBytes;
 }
+
+int band_bias_copy(int D) { return D == 64 ? Cfg<64>::kCopy : Cfg<128>::kCopy; }
 
 template <int D, int MODE, bool LOCAL = false, bool RAND = false>
 static cudaError_t launch_one(const AttnParams& p, int units, int num_sms, cudaStream_t s) {

@@ -171,7 +171,7 @@ swa_status enqueue_forward(const swa_plan_desc& d, const swa_forward_args& args,
       r_eff_max = (int)std::max<long long>(r_eff_max, std::min<long long>(window[h], nc));
     }
     local_stride = (int)align_up(2 * (size_t)r_eff_max + 2 * kLocalPad + 4, 32);
-    if (d.dtype == SWA_BF16 && local_stride > kBiasCopy) return SWA_ERR_UNSUPPORTED;
+    if (d.dtype == SWA_BF16 && local_stride > band_bias_copy(d.head_dim)) return SWA_ERR_UNSUPPORTED;
   }
   const bool bf16 = d.dtype == SWA_BF16;
   if (bf16 && num_global > 0 && (!ws.gq || !ws.gk || !ws.gv || !ws.part_o || !ws.part_lse))

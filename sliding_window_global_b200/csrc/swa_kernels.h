@@ -102,5 +102,6 @@ cudaError_t launch_side_aggregate_kv(const void* k, const void* v, void* sk, voi
                                      int n, int D, int kb, const int32_t* valid_len, int bf16,
                                      cudaStream_t s);
 size_t band_tc_smem_bytes(int D);
+int band_bias_copy(int D);           // floats per staged bias copy of the band kernel
 
 }  // namespace swa
