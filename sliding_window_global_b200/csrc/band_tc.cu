@@ -54,8 +54,6 @@
 //               as soon as the softmax has read the current one; the two
 //               issuers share only the K/V ring (read-only) and release each
 //               slot together.  Other warps of the group idle.
-#include <algorithm>
-
 #include "ptx.cuh"
 #include "side_mean.cuh"
 #include "softmax_math.cuh"
@@ -64,27 +62,12 @@
 namespace swa {
 namespace {
 
-#ifndef SWA_EPI_WG
-#define SWA_EPI_WG 0
-#endif
-// A fourth warpgroup drains O from TMEM and stores it, so that the softmax
-// warpgroups go on to the next unit at once.
-constexpr bool kEpiWG = SWA_EPI_WG != 0;
 constexpr int kSoftmaxThreads = 256;
-constexpr int kThreads = kEpiWG ? 512 : 384;  // softmax A, softmax B, control (, epilogue)
-constexpr int kLaunchRegs = kEpiWG ? 128 : 168;   // 65536 / threads, rounded down to 8
-// Registers per thread after reallocation; the sum must fit the launch budget
-// (kThreads * kLaunchRegs).
-#ifndef SWA_REGS_SOFTMAX
-#define SWA_REGS_SOFTMAX (kEpiWG ? 192 : 200)
-#endif
-#ifndef SWA_REGS_CONTROL
-#define SWA_REGS_CONTROL (kEpiWG ? 72 : 104)
-#endif
-constexpr int kRegsSoftmax = SWA_REGS_SOFTMAX;
-constexpr int kRegsControl = SWA_REGS_CONTROL;
-constexpr int kRegsEpi = kEpiWG ? (kThreads * kLaunchRegs - kSoftmaxThreads * kRegsSoftmax - 128 * kRegsControl) / 128
-                                : 0;
+constexpr int kThreads = 384;                 // 3 warpgroups: softmax A, softmax B, control
+// Registers per thread after reallocation: 256 * 200 + 128 * 104 = 384 * 168, the
+// budget the CTA is launched with (168 per thread for 384 threads).
+constexpr int kRegsSoftmax = 200;
+constexpr int kRegsControl = 104;
 constexpr uint32_t kSub = 128 * 128;          // one 128-row x 128-byte swizzle sub-tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -103,12 +86,6 @@ __host__ __device__ constexpr int emu_per32() {
   return D == 128 ? SWA_EMU_PER32_D128 : SWA_EMU_PER32_D64;
 }
 
-#ifndef SWA_EX2_PACKED
-#define SWA_EX2_PACKED 0
-#endif
-// MUFU exponentials on bf16 pairs (ex2.approx.ftz.bf16x2) instead of fp32 singles.
-constexpr bool kEx2Packed = SWA_EX2_PACKED != 0;
-
 // Where the tile max is taken: once after the tile-kind branches (D = 128), or
 // inside each branch (D = 64).  Both compute the same value; the code placement
 // was measured faster for each head size.
@@ -125,11 +102,8 @@ struct Cfg {
   static constexpr uint32_t kKOff = 2 * kTileBytes;
   static constexpr uint32_t kVOff = kKOff + NS * kTileBytes;
   static constexpr uint32_t kBiasOff = kVOff + NS * kTileBytes;  // 4 shifted copies
-  // floats per staged bias copy; the epilogue warpgroup's static state leaves less
-  // room at D = 128
-  static constexpr int kCopy = (D == 128 && kEpiWG) ? 1792 : kBiasCopy;
-  static constexpr uint32_t kBarOff = kBiasOff + 4 * kCopy * 4;
-  static constexpr int kNumBars = 2 + 2 + 3 * NS + 2 + 2 + 2 + 2 + 2 + 2 + 2 + 2;
+  static constexpr uint32_t kBarOff = kBiasOff + 4 * kBiasCopy * 4;
+  static constexpr int kNumBars = 2 + 2 + 3 * NS + 2 + 2 + 2 + 2 + 2 + 2;
   static constexpr uint32_t kSmemBytes = kBarOff + kNumBars * 8 + 1024;
   // TMEM columns.  D = 128: S_A | S_B | O_A | O_B, P written over S.  D = 64 has
   // room for separate P buffers (S_A | S_B | P_A | P_B | O_A | O_B), so the next
@@ -145,15 +119,10 @@ struct Cfg {
 
 // The register split must fit the budget the CTA is launched with (a larger sum
 // would leave setmaxnreg.inc waiting), and the shared memory one CTA per SM.
-static_assert(kSoftmaxThreads * kRegsSoftmax + 128 * kRegsControl + (kEpiWG ? 128 * kRegsEpi : 0) <=
-                  kThreads * kLaunchRegs,
+static_assert(kSoftmaxThreads * kRegsSoftmax + (kThreads - kSoftmaxThreads) * kRegsControl <= kThreads * 168,
               "setmaxnreg split exceeds the launch register budget");
-static_assert(!kEpiWG || (kRegsEpi >= 24 && kRegsEpi % 8 == 0), "epilogue register share");
-static_assert(kRegsSoftmax % 8 == 0 && kRegsControl % 8 == 0, "setmaxnreg takes multiples of 8");
-// dynamic + static (sGpos, sInv with the epilogue warpgroup, two words) shared memory
-constexpr uint32_t kStaticSmem = 2 * kTile * 4 + (kEpiWG ? 2 * 2 * kTile * 4 : 0) + 16;
-static_assert(Cfg<64>::kSmemBytes + kStaticSmem <= 227 * 1024, "shared memory, D = 64");
-static_assert(Cfg<128>::kSmemBytes + kStaticSmem <= 227 * 1024, "shared memory, D = 128");
+static_assert(Cfg<64>::kSmemBytes + 2 * kTile * 4 + 16 <= 227 * 1024, "shared memory, D = 64");
+static_assert(Cfg<128>::kSmemBytes + 2 * kTile * 4 + 16 <= 227 * 1024, "shared memory, D = 128");
 static_assert(emu_per32<64>() % 4 == 0 && emu_per32<64>() <= 32 && emu_per32<128>() % 4 == 0 &&
                   emu_per32<128>() <= 32,
               "polynomial exponentials come in groups of four");
@@ -177,104 +146,49 @@ struct Work {
   int lo[2], hi[2];     // band key range of each query tile (class coordinates)
 };
 
-// Work schedule.  MODE 0: the band units in the linear order (batch, head or head
-// pair, residue class, row unit); each CTA walks one contiguous range of it, so
-// consecutive units of a CTA are usually the next row tiles of the same head (pair):
-// they reuse most of their K/V tiles through L2 and need no fresh decode, only the
-// row offset moves.  MODE 1: global-row units, strided over the CTAs.
-struct Sched {
-  long long id, end;    // current unit, end of this CTA's range (MODE 0); uid, count (MODE 1)
-  int b, hp, c, u;      // batch, head (pair), class offset within the head, unit within the class
-  int uc;               // units of class c
-  int V;                // valid length of batch b
-};
-
-__device__ __forceinline__ int class_units(const AttnParams& p, int cls) {
-  const int tc = (p.cls[cls].n_c + kTile - 1) / kTile;
-  return p.pair_heads ? tc : (tc + 1) / 2;
-}
-
-__device__ __forceinline__ int batch_valid(const AttnParams& p, int b) {
-  return min(p.valid_len ? __ldg(p.valid_len + b) : p.n, p.n);
-}
-
 template <int MODE>
-__device__ __forceinline__ void sched_begin(const AttnParams& p, Sched& s) {
-  if (MODE == 0) {
-    const long long T = p.units_total, G = gridDim.x;
-    s.id = T * blockIdx.x / G;
-    s.end = T * (blockIdx.x + 1) / G;
-    if (s.id >= s.end) return;
-    const int per_b = p.unit_prefix[p.num_hp];
-    s.b = (int)(s.id / per_b);
-    int rem = (int)(s.id - (long long)s.b * per_b);
-    s.hp = 0;
-    while (s.hp + 1 < p.num_hp && p.unit_prefix[s.hp + 1] <= rem) ++s.hp;
-    rem -= p.unit_prefix[s.hp];
-    const int base = p.class_base[p.pair_heads ? 2 * s.hp : s.hp];
-    s.c = 0;
-    s.uc = class_units(p, base);
-    while (rem >= s.uc && s.c + 1 < p.cls[base].nres) {
-      rem -= s.uc;
-      ++s.c;
-      s.uc = class_units(p, base + s.c);
-    }
-    s.u = rem;
-    s.V = batch_valid(p, s.b);
-  } else {
-    s.id = blockIdx.x;
-    s.end = (long long)p.nsplit * (p.gpad / kTile) * p.B * p.Hq;
-  }
-}
-
-template <int MODE>
-__device__ __forceinline__ void sched_next(const AttnParams& p, Sched& s) {
-  if (MODE == 0) {
-    ++s.id;
-    if (s.id >= s.end) return;
-    if (++s.u < s.uc) return;
-    s.u = 0;
-    const int base = p.class_base[p.pair_heads ? 2 * s.hp : s.hp];
-    if (s.c + 1 < p.cls[base].nres) {
-      ++s.c;
-    } else {
-      s.c = 0;
-      if (++s.hp == p.num_hp) {
-        s.hp = 0;
-        ++s.b;
-        s.V = batch_valid(p, s.b);
-      }
-    }
-    const int nb = p.class_base[p.pair_heads ? 2 * s.hp : s.hp];
-    s.uc = class_units(p, nb + s.c);
-  } else {
-    s.id += gridDim.x;
-  }
+__device__ __forceinline__ int total_units(const AttnParams& p) {
+  return MODE == 0 ? p.max_units * p.B * (p.pair_heads ? p.Hq / 2 : p.Hq)
+                   : p.nsplit * (p.gpad / kTile) * p.B * p.Hq;
 }
 
 template <int MODE, bool RAND>
-__device__ __forceinline__ void decode_work(const AttnParams& p, const Sched& sc, Work& w) {
+__device__ __forceinline__ void decode_work(const AttnParams& p, int unit_id, Work& w) {
   if (MODE == 0) {
-    w.valid = true;
-    w.b = sc.b;
-    w.h = p.pair_heads ? 2 * sc.hp : sc.hp;
+    // unit ids run over (unit, batch, head or head pair), heads fastest
+    const int hunits = p.pair_heads ? p.Hq / 2 : p.Hq;
+    const int BH = p.B * hunits;
+    const int bh = unit_id % BH;
+    int unit = unit_id / BH;
+    w.b = bh / hunits;
+    w.h = p.pair_heads ? 2 * (bh % hunits) : bh % hunits;
     w.hx[0] = w.h;
     w.hx[1] = p.pair_heads ? w.h + 1 : w.h;
+    w.valid = unit < p.tiles[w.h];
     w.hk = w.h / p.G;
     w.r = p.window[w.h];
     const int base = p.class_base[w.h];
     w.d = p.cls[base].d;
-    w.c = sc.c;
-    w.cls = base + sc.c;
+    const int nres = p.cls[base].nres;
+    const int per_unit = p.pair_heads ? 1 : 2;           // row tiles per unit and class
+    int c = 0;
+    for (; c < nres - 1; ++c) {
+      const int tc = (p.cls[base + c].n_c + kTile - 1) / kTile;
+      const int uc = (tc + per_unit - 1) / per_unit;
+      if (unit < uc) break;
+      unit -= uc;
+    }
+    w.c = c;
+    w.cls = base + c;
     const int nc = p.cls[w.cls].n_c;
-    const int V = sc.V;
-    w.Vc = V > w.c ? (V - w.c + w.d - 1) / w.d : 0;
+    int V = p.valid_len ? p.valid_len[w.b] : p.n;
+    V = min(V, p.n);
+    w.Vc = V > c ? (V - c + w.d - 1) / w.d : 0;
     w.split = 0;
     w.key_end = 0;
-    const int unit = sc.u;
     for (int x = 0; x < 2; ++x) {
       w.u0[x] = p.pair_heads ? unit * kTile : unit * 2 * kTile + x * kTile;
-      w.rows[x] = max(0, min(kTile, nc - w.u0[x]));
+      w.rows[x] = w.valid ? max(0, min(kTile, nc - w.u0[x])) : 0;
       w.nvalid[x] = max(0, min(w.rows[x], w.Vc - w.u0[x]));
       w.active[x] = w.nvalid[x] > 0;
       w.lo[x] = max(0, w.u0[x] - w.r);
@@ -287,7 +201,6 @@ __device__ __forceinline__ void decode_work(const AttnParams& p, const Sched& sc
     w.ngc = (w.active[0] && p.g > 0) ? (p.g + kTile - 1) / kTile : 0;
     w.nside = (w.active[0] && p.S > 0) ? (p.S + kTile - 1) / kTile : 0;
   } else {
-    const int unit_id = (int)sc.id;
     w.valid = true;
     w.split = unit_id % p.nsplit;
     const int rest = unit_id / p.nsplit;
@@ -459,8 +372,8 @@ __device__ void write_neutral_partial(const AttnParams& p, const Work& w, int ro
   p.part_lse[prow] = -INFINITY;
 }
 
-// Fused Transient-Global prologue: this CTA's share of the side keys and values
-// (16-byte column groups of the side rows of k, then of v), all threads.
+// Fused Transient-Global prologue (AGG): this CTA's share of the side keys and
+// values (16-byte column groups of the side rows of k, then of v), all threads.
 template <int D>
 __device__ __forceinline__ void side_prologue(const AttnParams& p, int tid, int nthreads) {
   constexpr int VEC = 8;                                   // bf16
@@ -483,101 +396,12 @@ __device__ __forceinline__ void side_prologue(const AttnParams& p, int tid, int 
   }
 }
 
-// Epilogue of one query tile: O_x (TMEM) times 1/l -> out (bf16; MODE 0) or the
-// fp32 partials of a global-row split (MODE 1).  Thread `row` owns TMEM lane row.
-// staged: 32-column chunks go through shared memory (two 8 KB buffers at `stage`,
-// 64-byte swizzle) and are written by TMA, the `bar` named barrier (128 threads)
-// ordering the buffer reuse; else each thread stores its row.  o_free: if set, it
-// is arrived at once the last chunk has left TMEM.
-template <int D, int MODE>
-__device__ __forceinline__ void store_o(const AttnParams& p, const Work& w, const TileRows& tr, int row,
-                                        uint32_t o_addr, float inv, bool staged, uint8_t* stage, int bar,
-                                        uint64_t* o_free) {
-  constexpr int NCH = D / 32;
-  if (MODE == 0 && staged) {
-    if (row == 0) tma_store_wait_read<0>();          // previous stores have read the buffers
-    named_barrier_sync(bar, 128);
-#pragma unroll
-    for (int ch = 0; ch < NCH; ++ch) {
-      uint8_t* buf = stage + (ch & 1) * 8192;
-      if (ch >= 2) {
-        if (row == 0) tma_store_wait_read<1>();      // the store of chunk ch-2 has read buf
-        named_barrier_sync(bar, 128);
-      }
-      uint32_t rr[32];
-      tmem_ld32(o_addr + ch * 32, rr);
-      tmem_wait_ld_dep(rr);
-      if (o_free && ch == NCH - 1) {
-        tc_fence_before();
-        mbar_arrive(o_free);
-      }
-      uint8_t* rbase = buf + row * 64;
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint4 v;
-        v.x = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 0]) * inv, __uint_as_float(rr[q4 * 8 + 1]) * inv);
-        v.y = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 2]) * inv, __uint_as_float(rr[q4 * 8 + 3]) * inv);
-        v.z = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 4]) * inv, __uint_as_float(rr[q4 * 8 + 5]) * inv);
-        v.w = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 6]) * inv, __uint_as_float(rr[q4 * 8 + 7]) * inv);
-        *reinterpret_cast<uint4*>(rbase + ((q4 ^ ((row >> 1) & 3)) << 4)) = v;
-      }
-      fence_proxy_async_smem();
-      named_barrier_sync(bar, 128);
-      if (row == 0) {
-        tma_store_3d(&p.mo[w.cls], buf, ch * 32, tr.u0, w.b * p.Hq + tr.head);
-        tma_store_commit();
-      }
-    }
-  } else if (MODE == 0) {
-    const size_t off = out_row(p, w, tr, row);
-    uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + off * D);
-#pragma unroll
-    for (int ch = 0; ch < NCH; ++ch) {
-      uint32_t rr[32];
-      tmem_ld32(o_addr + ch * 32, rr);
-      tmem_wait_ld_dep(rr);
-      if (o_free && ch == NCH - 1) {
-        tc_fence_before();
-        mbar_arrive(o_free);
-      }
-      if (row < tr.rows) {
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 0]) * inv, __uint_as_float(rr[q4 * 8 + 1]) * inv);
-          v.y = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 2]) * inv, __uint_as_float(rr[q4 * 8 + 3]) * inv);
-          v.z = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 4]) * inv, __uint_as_float(rr[q4 * 8 + 5]) * inv);
-          v.w = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 6]) * inv, __uint_as_float(rr[q4 * 8 + 7]) * inv);
-          orow[ch * 4 + q4] = v;
-        }
-      }
-    }
-  } else {
-    const size_t prow = ((size_t)w.split * p.B * p.Hq + (size_t)w.b * p.Hq + w.h) * p.gpad + w.u0[0] + row;
-    float4* po = reinterpret_cast<float4*>(p.part_o + prow * D);
-#pragma unroll
-    for (int ch = 0; ch < NCH; ++ch) {
-      uint32_t rr[32];
-      tmem_ld32(o_addr + ch * 32, rr);
-      tmem_wait_ld_dep(rr);
-      if (o_free && ch == NCH - 1) {
-        tc_fence_before();
-        mbar_arrive(o_free);
-      }
-      if (row < w.rows[0]) {
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4)
-          po[ch * 8 + q4] = make_float4(__uint_as_float(rr[q4 * 4 + 0]) * inv, __uint_as_float(rr[q4 * 4 + 1]) * inv,
-                                        __uint_as_float(rr[q4 * 4 + 2]) * inv, __uint_as_float(rr[q4 * 4 + 3]) * inv);
-      }
-    }
-  }
-}
-
 // LOCAL: band tiles carry the local relative-position bias; RAND: query tiles have
-// random key blocks (MODE 0 only).  They are template parameters so that kernels
-// without them keep their register schedule.
-template <int D, int MODE, bool LOCAL, bool RAND>
+// random key blocks (MODE 0 only); AGG: the CTAs first build the side keys / values
+// from k and v (cooperative launch) and load side tiles once every CTA has counted
+// itself done.  They are template parameters so that kernels without them keep
+// their register schedule.
+template <int D, int MODE, bool LOCAL, bool RAND, bool AGG>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ AttnParams p) {
   using C = Cfg<D>;
   constexpr int NS = C::NS;
@@ -603,22 +427,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   uint64_t* s_free = o_full + 2;          // [2] S read into registers (separate-P layout)
   uint64_t* pv_done = s_free + 2;         // [2] a PV finished: P buffer free, O updated
   uint64_t* p_half = pv_done + 2;         // [2] P of keys 0-63 written (P-over-S layout)
-  uint64_t* epi_in = p_half + 2;          // [2] softmax finished a unit: 1/l of each row staged
-  uint64_t* o_free = epi_in + 2;          // [2] the epilogue has read O_x out of TMEM
   __shared__ uint32_t tmem_slot;
-  __shared__ float sInv[2][2][kTile];     // [unit parity][tile][row] 1/l for the epilogue warpgroup
   __shared__ int abort_flag;
   __shared__ int sGpos[2 * kTile];        // positions of the current global tile, per group
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  const int nunits = total_units<MODE>(p);
   const bool has_bias = p.bias && p.S > 0;
   constexpr bool has_local = LOCAL && MODE == 0;
   // shared bias area: 4 copies of the local-bias row (stride lstride floats), then
   // 4 copies of the side-bias segment (stride side_stride)
   const int lstride = has_local ? p.local_stride : 0;
-  const int side_stride = C::kCopy - lstride;
+  const int side_stride = kBiasCopy - lstride;
   float* sLocal = sBias;
   float* sSide = sBias + 4 * lstride;
 
@@ -632,8 +454,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_init(&s_free[x], kTile);
       mbar_init(&pv_done[x], 1);
       mbar_init(&p_half[x], kTile);
-      mbar_init(&epi_in[x], kTile);
-      mbar_init(&o_free[x], kTile);
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(&k_full[s], 1);
@@ -652,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
   volatile int* abort_v = &abort_flag;
-  if (MODE == 0 && p.agg_count) {
+  if (AGG) {
     side_prologue<D>(p, tid, kThreads);
     fence_proxy_async_global();                // side rows written here are read by TMA
     __threadfence();
@@ -666,12 +486,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       int qloads[2] = {0, 0};
       int kv = 0;                                   // K/V tiles loaded so far (ring position)
       bool ok = true;
-      bool side_ready = false;                      // fused prologue: all CTAs counted
-      Sched sc;
-      sched_begin<MODE>(p, sc);
-      for (; ok && sc.id < sc.end; sched_next<MODE>(p, sc)) {
+      bool side_ready = false;                      // AGG: every CTA counted
+      for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
         Work w;
-        decode_work<MODE, RAND>(p, sc, w);
+        decode_work<MODE, RAND>(p, uid, w);
         if (!w.active[0]) continue;
         const CUtensorMap* mq = (MODE == 0) ? &p.mq[w.cls] : &p.mgq;
         const int kz = w.b * p.Hkv + w.hk;
@@ -696,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             ok = false;
             break;
           }
-          if (MODE == 0 && p.agg_count && !side_ready && j >= w.nband + w.ngc && j < w.rand0) {
+          if (AGG && !side_ready && j >= w.nband + w.ngc && j < w.rand0) {
             // first side tile of this CTA: every CTA must have built its share
             if (!wait_count_bounded(p.agg_count, gridDim.x, abort_v, kWaitLimitNs)) {
               ok = false;
@@ -729,15 +547,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const uint32_t k_base = smem_u32(sK);
       const uint32_t v_base = smem_u32(sV);
       int qwaits[kTilesPerIssuer] = {}, pwaits[kTilesPerIssuer] = {};
-      int ounits[kTilesPerIssuer] = {};                 // units whose O_x was handed to the epilogue
       int nqk[kTilesPerIssuer] = {};                    // QKs issued per tile buffer (kernel-wide)
       int kv = 0;
       bool ok = true;
-      Sched sc;
-      sched_begin<MODE>(p, sc);
-      for (; ok && sc.id < sc.end; sched_next<MODE>(p, sc)) {
+      for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
         Work w;
-        decode_work<MODE, RAND>(p, sc, w);
+        decode_work<MODE, RAND>(p, uid, w);
         if (!w.active[0]) continue;
         const int T = w.total;
         // the tiles' fields as scalars (x0 is a run-time value with two issuers)
@@ -822,13 +637,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const int x = x0 + i;
             if (!ok) break;
             if (!uses(w, tr[i], x, j)) continue;
-            // the first PV of a unit overwrites O_x: the epilogue warpgroup must have
-            // read the previous unit's O_x out of TMEM
-            if (kEpiWG && npv[i] == 0 && ounits[i] > 0 &&
-                !mbar_wait_bounded(&o_free[x], (ounits[i] - 1) & 1, abort_v, kWaitLimitNs)) {
-              ok = false;
-              break;
-            }
             if (!C::kSepP) {
               // P over S: the first half of P (keys 0-63) is published early, so the
               // PV over it overlaps the exponentials of the second half
@@ -848,10 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                       sdesc_sw128(vt + kk * 2048, kSub, 1024), idesc_pv, (npv[i] > 0 || kk > 0) ? 1u : 0u);
             ++npv[i];
             if (C::kSepP) umma_commit(&pv_done[x]);
-            if (j == last[i]) {
-              umma_commit(&o_full[x]);
-              ++ounits[i];
-            }
+            if (j == last[i]) umma_commit(&o_full[x]);
             else if (!C::kSepP && uses(w, tr[i], x, j + 1)) ok = issue_qk(i, j + 1);
           }
           umma_commit(&kv_empty[st]);
@@ -859,9 +664,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         kv += T;
       }
     }
-  } else if (warp >= 10 && warp < 12) {
+  } else if (warp >= 10) {
     setmaxnreg_dec<kRegsControl>();
-  } else if (warp < 8) {
+  } else {
     // ------------------------------------------------------------ softmax warpgroups
     setmaxnreg_inc<kRegsSoftmax>();
     const int x = warp >> 2;                   // 0: tile A, 1: tile B
@@ -875,11 +680,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     int it = 0;                                // S/P tiles handled so far (barrier phase)
     int oc = 0;                                // units finished (o_full phase)
     bool ok = true;
-    Sched sc;
-    sched_begin<MODE>(p, sc);
-    for (; ok && sc.id < sc.end; sched_next<MODE>(p, sc)) {
+    for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
       Work w;
-      decode_work<MODE, RAND>(p, sc, w);
+      decode_work<MODE, RAND>(p, uid, w);
       if (!w.valid) continue;
       const TileRows tr = tile_rows(w, x);
       if (!w.active[0]) {
@@ -1201,18 +1004,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               if (q < emu_per32<D>()) {
                 exp2_poly2(a0, a1, a0, a1);
                 exp2_poly2(a2, a3, a2, a3);
-              } else if (kEx2Packed) {
-                // the exponent rounded to bf16, two exponentials per MUFU operation; P
-                // comes out packed, and l sums exactly the P the PV product reads
-                const uint32_t p01 = ex2_bf16x2(pack_bf16x2(a0, a1));
-                const uint32_t p23 = ex2_bf16x2(pack_bf16x2(a2, a3));
-                pk[q / 2] = p01;
-                pk[q / 2 + 1] = p23;
-                acc0 = add_bf16_lo(p01, acc0);
-                acc1 = add_bf16_hi(p01, acc1);
-                acc2 = add_bf16_lo(p23, acc2);
-                acc3 = add_bf16_hi(p23, acc3);
-                continue;
               } else {
                 a0 = ex2_approx(a0);
                 a1 = ex2_approx(a1);
@@ -1255,68 +1046,93 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       if (!ok) break;
 
       // ---------------------------------------------------------- epilogue
+      // O_x is read out of TMEM before this group's next p_full arrival, which is
+      // what the MMA warp waits for before it overwrites O_x.
+      if (!mbar_wait_bounded(&o_full[x], oc & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+      ++oc;
+      tc_fence_after();
       const bool has = row_valid && l > 0.f;
       const float inv = has ? 1.f / l : 0.f;
       const float lse_v = has ? (m + __log2f(l)) * kLn2 : -INFINITY;
-      if (MODE == 0) {
-        if (row < tr.rows && p.lse) p.lse[out_row(p, w, tr, row)] = lse_v;
-      } else if (row < w.rows[0]) {
-        p.part_lse[((size_t)w.split * p.B * p.Hq + (size_t)w.b * p.Hq + w.h) * p.gpad + w.u0[0] + row] = lse_v;
-      }
-      if (kEpiWG) {
-        // hand the unit to the epilogue warpgroup: 1/l per row, then go on
-        sInv[oc & 1][x][row] = inv;
-        ++oc;
-        mbar_arrive(&epi_in[x]);
-      } else {
-        // O_x is read out of TMEM before this group's next p_full arrival, which is
-        // what the MMA warp waits for before it overwrites O_x.
-        if (!mbar_wait_bounded(&o_full[x], oc & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
-        ++oc;
-        tc_fence_after();
-        store_o<D, MODE>(p, w, tr, row, o_addr, inv, !has_bias && !has_local,
-                         reinterpret_cast<uint8_t*>(sBias) + x * 2 * 8192, 1 + x, nullptr);
-        tc_fence_before();
-      }
-    }
-  }
-
-  if (kEpiWG && warp >= 12) {
-    // ------------------------------------------------------------ epilogue warpgroup
-    // Per unit and query tile: wait for the softmax's 1/l and for the last PV, read
-    // O_x out of TMEM (then release it to the MMA warp), scale and store it.
-    setmaxnreg_dec<kRegsEpi>();
-    const int row = tid & 127;
-    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const bool has_local_e = LOCAL && MODE == 0;
-    int ocx[2] = {0, 0};
-    bool ok = true;
-    Sched sc;
-    sched_begin<MODE>(p, sc);
-    for (; ok && sc.id < sc.end; sched_next<MODE>(p, sc)) {
-      Work w;
-      decode_work<MODE, RAND>(p, sc, w);
-      if (!w.valid || !w.active[0]) continue;
+      if (MODE == 0 && !has_bias && !has_local) {
+        // Coalesced store: 32-column chunks staged in shared memory (the bias area,
+        // unused without biases; two 8 KB buffers per group, 64-byte swizzle)
+        // and written by TMA; rows beyond the class end are clipped by the map.
+        uint8_t* stage = reinterpret_cast<uint8_t*>(sBias) + x * 2 * 8192;
+        if (row == 0) tma_store_wait_read<0>();          // previous unit's stores have read
+        named_barrier_sync(1 + x, 128);
 #pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        if (!ok) break;
-        if (!(x ? w.active[1] : w.active[0])) continue;
-        const int par = ocx[x] & 1;
-        if (!mbar_wait_bounded(&epi_in[x], par, abort_v, kWaitLimitNs) ||
-            !mbar_wait_bounded(&o_full[x], par, abort_v, kWaitLimitNs)) {
-          ok = false;
-          break;
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint8_t* buf = stage + (ch & 1) * 8192;
+          if (ch >= 2) {
+            if (row == 0) tma_store_wait_read<1>();      // the store of chunk ch-2 has read buf
+            named_barrier_sync(1 + x, 128);
+          }
+          uint32_t rr[32];
+          tmem_ld32(o_addr + ch * 32, rr);
+          tmem_wait_ld_dep(rr);
+          uint8_t* rbase = buf + row * 64;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 0]) * inv, __uint_as_float(rr[q4 * 8 + 1]) * inv);
+            v.y = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 2]) * inv, __uint_as_float(rr[q4 * 8 + 3]) * inv);
+            v.z = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 4]) * inv, __uint_as_float(rr[q4 * 8 + 5]) * inv);
+            v.w = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 6]) * inv, __uint_as_float(rr[q4 * 8 + 7]) * inv);
+            *reinterpret_cast<uint4*>(rbase + ((q4 ^ ((row >> 1) & 3)) << 4)) = v;
+          }
+          fence_proxy_async_smem();
+          named_barrier_sync(1 + x, 128);
+          if (row == 0) {
+            tma_store_3d(&p.mo[w.cls], buf, ch * 32, tr.u0, w.b * p.Hq + tr.head);
+            tma_store_commit();
+          }
         }
-        ++ocx[x];
-        tc_fence_after();
-        const TileRows tr = tile_rows(w, x);
-        store_o<D, MODE>(p, w, tr, row, lane_base + C::o_col(x), sInv[par][x][row], !has_bias && !has_local_e,
-                         reinterpret_cast<uint8_t*>(sBias) + x * 2 * 8192, 4, &o_free[x]);
+        if (row < tr.rows && p.lse) p.lse[out_row(p, w, tr, row)] = lse_v;
+      } else if (MODE == 0) {
+        const size_t off = out_row(p, w, tr, row);
+        uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + off * D);
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t rr[32];
+          tmem_ld32(o_addr + ch * 32, rr);
+          tmem_wait_ld_dep(rr);
+          if (row < tr.rows) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 0]) * inv, __uint_as_float(rr[q4 * 8 + 1]) * inv);
+              v.y = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 2]) * inv, __uint_as_float(rr[q4 * 8 + 3]) * inv);
+              v.z = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 4]) * inv, __uint_as_float(rr[q4 * 8 + 5]) * inv);
+              v.w = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 6]) * inv, __uint_as_float(rr[q4 * 8 + 7]) * inv);
+              orow[ch * 4 + q4] = v;
+            }
+          }
+        }
+        if (row < tr.rows && p.lse) p.lse[off] = lse_v;
+      } else {
+        const size_t prow =
+            ((size_t)w.split * p.B * p.Hq + (size_t)w.b * p.Hq + w.h) * p.gpad + w.u0[0] + row;
+        float4* po = reinterpret_cast<float4*>(p.part_o + prow * D);
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t rr[32];
+          tmem_ld32(o_addr + ch * 32, rr);
+          tmem_wait_ld_dep(rr);
+          if (row < w.rows[0]) {
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+              po[ch * 8 + q4] = make_float4(__uint_as_float(rr[q4 * 4 + 0]) * inv, __uint_as_float(rr[q4 * 4 + 1]) * inv,
+                                            __uint_as_float(rr[q4 * 4 + 2]) * inv, __uint_as_float(rr[q4 * 4 + 3]) * inv);
+          }
+        }
+        if (row < w.rows[0]) p.part_lse[prow] = lse_v;
       }
+      tc_fence_before();
     }
   }
 
-  if ((kEpiWG ? warp >= 12 : warp < 8) && (tid & 127) == 0) tma_store_wait_read<0>();   // staged stores have read smem
+  if (warp < 8 && (tid & 127) == 0) tma_store_wait_read<0>();   // staged stores have read smem
   tc_fence_before();
   __syncthreads();
   if (abort_flag) {
@@ -1337,25 +1153,517 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   }
 }
 
+
+// ------------------------------------------------------------------ split-softmax kernel
+// The plain band pattern (window, dilation, causal, padding, GQA pairs; no global
+// tokens, side keys, biases or random blocks) with every query tile's softmax split
+// over two warpgroups: warpgroup (x, h) handles key columns [64h, 64h + 64) of tile
+// x.  Per key tile the two halves exchange their row maxima through shared memory
+// (the reference max m of a row is then the same in both), so P shares one scale
+// and the O accumulator stays whole; each half keeps its own partial row sum, and
+// the halves add them up at the end.  Twice the softmax warps per SM scheduler,
+// each with half the exponentials per tile, against the same MMA chain.
+constexpr int kSplitThreads = 640;             // 4 softmax warpgroups + control
+constexpr int kSplitSoftmaxThreads = 512;
+constexpr int kSplitProducer = 16;             // warp ids of the control warpgroup
+constexpr int kSplitIssuer = 17;
+#ifndef SWA_SPLIT_REGS_SOFTMAX
+#define SWA_SPLIT_REGS_SOFTMAX 104
+#endif
+#ifndef SWA_SPLIT_REGS_CONTROL
+#define SWA_SPLIT_REGS_CONTROL 64
+#endif
+constexpr int kSplitRegsSoftmax = SWA_SPLIT_REGS_SOFTMAX;
+constexpr int kSplitRegsControl = SWA_SPLIT_REGS_CONTROL;
+static_assert(kSplitSoftmaxThreads * kSplitRegsSoftmax + 128 * kSplitRegsControl <= kSplitThreads * 96,
+              "setmaxnreg split exceeds the launch register budget (96 per thread for 640 threads)");
+
+// Row max of 64 values.
+__device__ __forceinline__ float row_max64(const float (&x)[64]) {
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = fmaxf(x[i], x[8 + i]);
+#pragma unroll
+  for (int e = 16; e < 64; e += 16) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = fmax3(m[i], x[e + i], x[e + 8 + i]);
+  }
+  return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSplitThreads, 1) attn_split_kernel(const __grid_constant__ AttnParams p) {
+  using C = Cfg<D>;
+  constexpr int NS = C::NS;
+  constexpr int kIssuers = C::kSepP ? 2 : 1;
+  constexpr int kTilesPerIssuer = 2 / kIssuers;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem + C::kQOff;
+  uint8_t* sK = smem + C::kKOff;
+  uint8_t* sV = smem + C::kVOff;
+  // exchange area (in the bias area, unused here): [parity][tile][half][row] maxima,
+  // then [tile][half][row] partial row sums
+  float* sMax = reinterpret_cast<float*>(smem + C::kBiasOff);
+  float* sSum = sMax + 2 * 2 * 2 * kTile;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* q_full = bars;                // [2]
+  uint64_t* q_empty = bars + 2;           // [2]
+  uint64_t* k_full = bars + 4;            // [NS]
+  uint64_t* v_full = k_full + NS;
+  uint64_t* kv_empty = v_full + NS;
+  uint64_t* s_full = kv_empty + NS;       // [2]
+  uint64_t* p_full = s_full + 2;          // [2]
+  uint64_t* o_full = p_full + 2;          // [2]
+  uint64_t* s_free = o_full + 2;          // [2] both halves read S (separate-P layout)
+  uint64_t* pv_done = s_free + 2;         // [2]
+  uint64_t* p_half = pv_done + 2;         // [2] P over S: half 0 wrote P of keys 0-63, both rescaled O
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int nunits = total_units<0>(p);
+
+  if (tid == 0) {
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&q_full[x], 1);
+      mbar_init(&q_empty[x], 1);
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], C::kSepP ? 2 * kTile : kTile);
+      mbar_init(&o_full[x], 1);
+      mbar_init(&s_free[x], 2 * kTile);
+      mbar_init(&pv_done[x], 1);
+      mbar_init(&p_half[x], 2 * kTile);
+    }
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], kIssuers);
+    }
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kSplitIssuer) {
+    tmem_alloc(&tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  volatile int* abort_v = &abort_flag;
+  if (warp == kSplitProducer) {
+    // ------------------------------------------------------------ TMA producer
+    setmaxnreg_dec<kSplitRegsControl>();
+    if (lane == 0) {
+      int qloads[2] = {0, 0};
+      int kv = 0;                                   // K/V tiles loaded so far (ring position)
+      bool ok = true;
+      for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
+        Work w;
+        decode_work<0, false>(p, uid, w);
+        if (!w.active[0]) continue;
+        const CUtensorMap* mq = &p.mq[w.cls];
+        const int kz = w.b * p.Hkv + w.hk;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (!ok) break;
+          const int qz = w.b * p.Hq + w.hx[x];
+          if (!w.active[x]) continue;
+          if (qloads[x] > 0 &&
+              !mbar_wait_bounded(&q_empty[x], (qloads[x] - 1) & 1, abort_v, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&q_full[x], C::kTileBytes);
+          tma_tile<D>(sQ + x * C::kTileBytes, mq, &q_full[x], w.u0[x], qz);
+          ++qloads[x];
+        }
+        for (int j = 0; ok && j < w.total; ++j, ++kv) {
+          const int st = kv % NS;
+          const int use = kv / NS;
+          if (kv >= NS && !mbar_wait_bounded(&kv_empty[st], (use - 1) & 1, abort_v, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          const CUtensorMap *mk, *mv;
+          int y;
+          tile_source(p, w, j, mk, mv, y);
+          mbar_arrive_expect_tx(&k_full[st], C::kTileBytes);
+          tma_tile<D>(sK + st * C::kTileBytes, mk, &k_full[st], y, kz);
+          mbar_arrive_expect_tx(&v_full[st], C::kTileBytes);
+          tma_tile<D>(sV + st * C::kTileBytes, mv, &v_full[st], y, kz);
+        }
+      }
+    }
+  } else if (warp == kSplitIssuer || (kIssuers == 2 && warp == kSplitIssuer + 1)) {
+    // ------------------------------------------------------------ MMA issuers
+    // P over S (D = 128): warp 9 issues both tiles' MMAs in one fixed order, which
+    // keeps the two softmax groups half a period apart.  Separate P (D = 64): warp
+    // 9 issues tile A's MMAs and warp 10 tile B's, so neither tile's products wait
+    // behind the other tile's barriers.
+    setmaxnreg_dec<kSplitRegsControl>();
+    if (lane == 0) {
+      const int x0 = (kIssuers == 2) ? warp - kSplitIssuer : 0;   // first tile of this issuer
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+      const uint32_t q_base = smem_u32(sQ);
+      const uint32_t k_base = smem_u32(sK);
+      const uint32_t v_base = smem_u32(sV);
+      int qwaits[kTilesPerIssuer] = {}, pwaits[kTilesPerIssuer] = {};
+      int nqk[kTilesPerIssuer] = {};                    // QKs issued per tile buffer (kernel-wide)
+      int kv = 0;
+      bool ok = true;
+      for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
+        Work w;
+        decode_work<0, false>(p, uid, w);
+        if (!w.active[0]) continue;
+        const int T = w.total;
+        // the tiles' fields as scalars (x0 is a run-time value with two issuers)
+        TileRows tr[kTilesPerIssuer];
+        int first[kTilesPerIssuer], last[kTilesPerIssuer], issued[kTilesPerIssuer], npv[kTilesPerIssuer];
+#pragma unroll
+        for (int i = 0; i < kTilesPerIssuer; ++i) {
+          tr[i] = tile_rows(w, x0 + i);
+          first[i] = last[i] = issued[i] = -1;
+          npv[i] = 0;
+          for (int j = 0; j < T; ++j)
+            if (uses(w, tr[i], x0 + i, j)) {
+              if (first[i] < 0) first[i] = j;
+              last[i] = j;
+            }
+        }
+        auto issue_qk = [&](int i, int j) -> bool {
+          const int x = x0 + i;
+          const int g = kv + j;
+          if (!mbar_wait_bounded(&k_full[g % NS], (g / NS) & 1, abort_v, kWaitLimitNs)) return false;
+          // separate-P layout: S_x is rewritten only after the softmax read the last one
+          if (C::kSepP && nqk[i] > 0 &&
+              !mbar_wait_bounded(&s_free[x], (nqk[i] - 1) & 1, abort_v, kWaitLimitNs))
+            return false;
+          ++nqk[i];
+          tc_fence_after();
+          const uint32_t qt = q_base + x * C::kTileBytes;
+          const uint32_t kt = k_base + (g % NS) * C::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
+            umma_ss(tmem + C::s_col(x), sdesc_sw128(qt + off, 16, 1024),
+                    sdesc_sw128(kt + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[x]);
+          if (j == last[i]) umma_commit(&q_empty[x]);   // Q_x may be refilled once this QK is done
+          issued[i] = j;
+          return true;
+        };
+#pragma unroll
+        for (int i = 0; i < kTilesPerIssuer; ++i) {
+          if (!ok) break;
+          if (!tr[i].active) continue;
+          ok = mbar_wait_bounded(&q_full[x0 + i], qwaits[i] & 1, abort_v, kWaitLimitNs);
+          ++qwaits[i];
+          if (ok) ok = issue_qk(i, first[i]);
+        }
+        for (int j = 0; ok && j < T; ++j) {
+          const int g = kv + j;
+          const int st = g % NS;
+          bool any = false;                           // this issuer reads the slot of tile j
+#pragma unroll
+          for (int i = 0; i < kTilesPerIssuer; ++i) {
+            const bool u = uses(w, tr[i], x0 + i, j);
+            any = any || u;
+            if (ok && u && issued[i] < j) ok = issue_qk(i, j);
+          }
+          if (C::kSepP) {
+            // the next S of each tile as soon as its softmax has read the current one
+            // (its next key tile may be j + 2 when random tiles alternate; a tile up
+            // to j + NS - 1 is loadable: its ring slot was freed by tile <= j - 1)
+#pragma unroll
+            for (int i = 0; i < kTilesPerIssuer; ++i) {
+              if (!ok || !uses(w, tr[i], x0 + i, j) || issued[i] != j) continue;
+              int jn = j + 1;
+              while (jn < T && jn < j + NS && !uses(w, tr[i], x0 + i, jn)) ++jn;
+              if (jn < T && jn < j + NS) ok = issue_qk(i, jn);
+            }
+          }
+          if (!ok) break;
+          // With two issuers both wait for V of every tile of the unit, used or not,
+          // before they release its ring slot: the slot's next load needs both
+          // releases, so neither issuer can arrive twice on one phase of kv_empty.
+          if (!mbar_wait_bounded(&v_full[st], (g / NS) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+          if (!any) {
+            mbar_arrive(&kv_empty[st]);               // no MMA of this issuer reads the slot
+            continue;
+          }
+          const uint32_t vt = v_base + st * C::kTileBytes;
+#pragma unroll
+          for (int i = 0; i < kTilesPerIssuer; ++i) {
+            const int x = x0 + i;
+            if (!ok) break;
+            if (!uses(w, tr[i], x, j)) continue;
+            if (!C::kSepP) {
+              // P over S: the first half of P (keys 0-63) is published early, so the
+              // PV over it overlaps the exponentials of the second half
+              if (!mbar_wait_bounded(&p_half[x], pwaits[i] & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < kTile / 32; ++kk)
+                umma_ts(tmem + C::o_col(x), tmem + C::p_col(x) + kk * 8,
+                        sdesc_sw128(vt + kk * 2048, kSub, 1024), idesc_pv, (npv[i] > 0 || kk > 0) ? 1u : 0u);
+            }
+            if (!mbar_wait_bounded(&p_full[x], pwaits[i] & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+            ++pwaits[i];
+            tc_fence_after();
+#pragma unroll
+            for (int kk = C::kSepP ? 0 : kTile / 32; kk < kTile / 16; ++kk)
+              umma_ts(tmem + C::o_col(x), tmem + C::p_col(x) + kk * 8,
+                      sdesc_sw128(vt + kk * 2048, kSub, 1024), idesc_pv, (npv[i] > 0 || kk > 0) ? 1u : 0u);
+            ++npv[i];
+            if (C::kSepP) umma_commit(&pv_done[x]);
+            if (j == last[i]) umma_commit(&o_full[x]);
+            else if (!C::kSepP && uses(w, tr[i], x, j + 1)) ok = issue_qk(i, j + 1);
+          }
+          umma_commit(&kv_empty[st]);
+        }
+        kv += T;
+      }
+    }
+  } else if (warp >= kSplitProducer) {
+    setmaxnreg_dec<kSplitRegsControl>();
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    setmaxnreg_inc<kSplitRegsSoftmax>();
+    const int wg = warp >> 2;
+    const int x = wg >> 1;                     // query tile
+    const int hh = wg & 1;                     // key-column half
+    const int row = tid & 127;                 // TMEM lane == row in the tile
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t s_addr = lane_base + C::s_col(x) + hh * 64;
+    const uint32_t p_addr = lane_base + C::p_col(x) + hh * 32;
+    const uint32_t o_addr = lane_base + C::o_col(x) + hh * (D / 2);
+    const int cbase = hh * 64;
+    int pw = 0;
+    const float sl2 = p.scale_log2;
+    int it = 0;
+    int oc = 0;
+    bool ok = true;
+    for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
+      Work w;
+      decode_work<0, false>(p, uid, w);
+      if (!w.valid) continue;
+      const TileRows tr = tile_rows(w, x);
+      if (!w.active[0] || !tr.active) {
+        if (hh == 0) write_zero_row<D>(p, w, tr, row);
+        continue;
+      }
+      const int T = w.total;
+      const bool row_valid = row < tr.nvalid;
+      const int u = tr.u0 + row;
+      int klo = u - w.r;
+      int khi = min(p.causal ? u : u + w.r, w.Vc - 1) + 1;
+      if (!row_valid) khi = klo;
+      float m = -INFINITY;                     // running reference max (log2 units), shared by both halves
+      float l = 0.f;                           // this half's partial row sum
+      int iu = 0;
+      for (int j = 0; j < T; ++j) {
+        if (!uses(w, tr, x, j)) continue;
+        if (!mbar_wait_bounded(&s_full[x], it & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t xr[64];
+        tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(xr));
+        tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(xr + 32));
+        tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(xr));
+        tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(xr + 32));
+        if (C::kSepP) {
+          tc_fence_before();
+          mbar_arrive(&s_free[x]);
+        }
+        float sc[64];
+#pragma unroll
+        for (int e = 0; e < 64; ++e) sc[e] = __uint_as_float(xr[e]);
+        const int kv0 = w.band_lo + j * kTile + cbase;
+        const int lo_t = klo - kv0, hi_t = khi - kv0;
+        uint32_t live = 0;
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch)
+          if (__any_sync(0xffffffffu, lo_t < 32 * ch + 32 && hi_t > 32 * ch)) live |= 1u << ch;
+        const bool cut_lo = __any_sync(0xffffffffu, lo_t > 0);
+        const bool cut_hi = __any_sync(0xffffffffu, hi_t < 64);
+        if (cut_lo && cut_hi) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) sc[e] = (e >= lo_t && e < hi_t) ? sc[e] : -INFINITY;
+        } else if (cut_lo) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) sc[e] = (e >= lo_t) ? sc[e] : -INFINITY;
+        } else if (cut_hi) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) sc[e] = (e < hi_t) ? sc[e] : -INFINITY;
+        }
+        // this half's row max, exchanged with the other half's through shared memory
+        const float hmax = row_max64(sc) * sl2;
+        float* xm = sMax + ((it & 1) * 4 + x * 2) * kTile;
+        xm[hh * kTile + row] = hmax;
+        named_barrier_sync(1 + x, 2 * kTile);
+        const float tmax = fmaxf(hmax, xm[(1 - hh) * kTile + row]);
+        const float m_new = fmaxf(m, tmax);
+        const bool need = (m == -INFINITY) ? (m_new > -INFINITY) : (m_new > m + kRescaleThreshold);
+        const bool rescale = __any_sync(0xffffffffu, need);
+        float alpha = 1.f;
+        if (rescale) {
+          alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
+          l *= alpha;
+          m = m_new;
+        }
+        const float neg_m = (m == -INFINITY) ? 0.f : -m;
+        if (C::kSepP && pw > 0) {
+          if (!mbar_wait_bounded(&pv_done[x], (pw - 1) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+        }
+        if (!C::kSepP && rescale && iu > 0) {
+          // O_x (this half's columns) must be rescaled before P is published; it is
+          // stable: its previous PV was issued before this S and MMAs complete in order
+#pragma unroll 1
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t rr[16];
+            tmem_ld16(o_addr + ch * 16, rr);
+            tmem_wait_ld_dep16(rr);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
+            tmem_st16(o_addr + ch * 16, rr);
+          }
+        }
+        if (!C::kSepP && hh == 1) {
+          // the PV over keys 0-63 writes every O column: this half's rescale must be in
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&p_half[x]);
+        }
+        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t pk[16];
+          if (!(live & (1u << ch))) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) pk[q] = 0u;
+          } else {
+#pragma unroll
+            for (int q = 0; q < 32; q += 4) {
+              const int e = ch * 32 + q;
+              float a0, a1, a2, a3;
+              ffma2(a0, a1, sc[e], sc[e + 1], sl2, sl2, neg_m, neg_m);
+              ffma2(a2, a3, sc[e + 2], sc[e + 3], sl2, sl2, neg_m, neg_m);
+              if (q < emu_per32<D>()) {
+                exp2_poly2(a0, a1, a0, a1);
+                exp2_poly2(a2, a3, a2, a3);
+              } else {
+                a0 = ex2_approx(a0);
+                a1 = ex2_approx(a1);
+                a2 = ex2_approx(a2);
+                a3 = ex2_approx(a3);
+              }
+              fadd2(acc0, acc1, acc0, acc1, a0, a1);
+              fadd2(acc2, acc3, acc2, acc3, a2, a3);
+              pk[q / 2] = pack_bf16x2(a0, a1);
+              pk[q / 2 + 1] = pack_bf16x2(a2, a3);
+            }
+          }
+          tmem_st16(p_addr + ch * 16, pk);
+        }
+        l += (acc0 + acc1) + (acc2 + acc3);
+        if (C::kSepP && rescale && iu > 0) {
+#pragma unroll
+          for (int ch = 0; ch < D / 64; ++ch) {
+            uint32_t rr[32];
+            tmem_ld32(o_addr + ch * 32, rr);
+            tmem_wait_ld_dep(rr);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
+            tmem_st32(o_addr + ch * 32, rr);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        if (!C::kSepP && hh == 0) mbar_arrive(&p_half[x]);   // P of keys 0-63 (and this half rescaled)
+        else mbar_arrive(&p_full[x]);          // P over S: keys 64-127; separate P: all of P
+        ++pw;
+        ++it;
+        ++iu;
+      }
+      if (!ok) break;
+
+      // ---------------------------------------------------------- epilogue
+      // the two halves' sums, then O / l: each half stores its D/2 output columns
+      float* xs = sSum + x * 2 * kTile;
+      xs[hh * kTile + row] = l;
+      named_barrier_sync(1 + x, 2 * kTile);
+      const float l_all = l + xs[(1 - hh) * kTile + row];
+      if (!mbar_wait_bounded(&o_full[x], oc & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+      ++oc;
+      tc_fence_after();
+      const bool has = row_valid && l_all > 0.f;
+      const float inv = has ? 1.f / l_all : 0.f;
+      const size_t off = out_row(p, w, tr, row);
+      if (hh == 0 && row < tr.rows && p.lse) p.lse[off] = has ? (m + __log2f(l_all)) * kLn2 : -INFINITY;
+      uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + off * D + hh * (D / 2));
+#pragma unroll
+      for (int ch = 0; ch < D / 64; ++ch) {
+        uint32_t rr[32];
+        tmem_ld32(o_addr + ch * 32, rr);
+        tmem_wait_ld_dep(rr);
+        if (row < tr.rows) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 0]) * inv, __uint_as_float(rr[q4 * 8 + 1]) * inv);
+            v.y = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 2]) * inv, __uint_as_float(rr[q4 * 8 + 3]) * inv);
+            v.z = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 4]) * inv, __uint_as_float(rr[q4 * 8 + 5]) * inv);
+            v.w = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 6]) * inv, __uint_as_float(rr[q4 * 8 + 7]) * inv);
+            orow[ch * 4 + q4] = v;
+          }
+        }
+      }
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (abort_flag) {
+    if (tid == 0) {
+      atomicOr(p.err, kDevErrTimeout);
+      const uint64_t t0 = global_timer_ns();
+      while (global_timer_ns() - t0 < 2000000ull) {
+      }
+    }
+    __syncthreads();
+  }
+  if (warp == kSplitIssuer) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
 }  // namespace
 
 size_t band_tc_smem_bytes(int D) {
   return D == 64 ? Cfg<64>::kSmemBytes : Cfg<128>::kSmemBytes;
 }
 
-int band_bias_copy(int D) { return D == 64 ? Cfg<64>::kCopy : Cfg<128>::kCopy; }
-
-template <int D, int MODE, bool LOCAL = false, bool RAND = false>
+template <int D, int MODE, bool LOCAL = false, bool RAND = false, bool AGG = false>
 static cudaError_t launch_one(const AttnParams& p, int units, int num_sms, cudaStream_t s) {
-  auto kern = attn_tc_kernel<D, MODE, LOCAL, RAND>;
+  auto kern = attn_tc_kernel<D, MODE, LOCAL, RAND, AGG>;
   const int smem = static_cast<int>(Cfg<D>::kSmemBytes);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int grid = units < num_sms ? units : num_sms;
   if (grid <= 0) return cudaSuccess;
-  if (MODE == 0 && p.agg_count) {
-    // the fused side-key prologue waits for every CTA: a cooperative launch makes
-    // them all resident at once (one CTA per SM, grid <= SM count)
+  if (AGG) {
+    // the prologue's wait needs every CTA resident at once: a cooperative launch
+    // (one CTA per SM, grid <= SM count)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
@@ -1372,9 +1680,31 @@ static cudaError_t launch_one(const AttnParams& p, int units, int num_sms, cudaS
   return cudaGetLastError();
 }
 
+#ifndef SWA_SPLIT
+#define SWA_SPLIT 1
+#endif
+
+template <int D>
+static cudaError_t launch_split(const AttnParams& p, int units, int num_sms, cudaStream_t s) {
+  auto kern = attn_split_kernel<D>;
+  const int smem = static_cast<int>(Cfg<D>::kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int grid = units < num_sms ? units : num_sms;
+  if (grid <= 0) return cudaSuccess;
+  kern<<<grid, kSplitThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
 // p.tiles[h] holds the number of two-tile units of head h, p.max_units their maximum.
 cudaError_t launch_band_tc(const AttnParams& p, int num_sms, cudaStream_t s) {
-  const int units = (int)std::min<long long>(p.units_total, 1LL << 30);
+  const int units = p.max_units * p.B * p.Hq;
+  if (SWA_SPLIT && p.g == 0 && p.S == 0 && !p.local_bias && p.num_rand == 0 && !p.agg_count)
+    return p.D == 64 ? launch_split<64>(p, units, num_sms, s) : launch_split<128>(p, units, num_sms, s);
+  if (p.agg_count) {      // side keys built in the prologue (no local bias, no random blocks)
+    return p.D == 64 ? launch_one<64, 0, false, false, true>(p, units, num_sms, s)
+                     : launch_one<128, 0, false, false, true>(p, units, num_sms, s);
+  }
   if (p.num_rand > 0) {
     if (p.local_bias)
       return p.D == 64 ? launch_one<64, 0, true, true>(p, units, num_sms, s)
@@ -1392,5 +1722,7 @@ cudaError_t launch_global_rows_tc(const AttnParams& p, int num_sms, cudaStream_t
   const int units = p.nsplit * (p.gpad / kTile) * p.B * p.Hq;
   return p.D == 64 ? launch_one<64, 1>(p, units, num_sms, s) : launch_one<128, 1>(p, units, num_sms, s);
 }
+
+int band_bias_copy(int) { return kBiasCopy; }
 
 }  // namespace swa

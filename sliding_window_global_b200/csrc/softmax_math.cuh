@@ -52,26 +52,4 @@ __device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float a0, float
   y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(r1) << 23));
 }
 
-// Two exponentials 2^x of a bf16 pair in one MUFU operation; the result is the
-// bf16 pair itself (flush-to-zero: -inf and large negative arguments give +0).
-__device__ __forceinline__ uint32_t ex2_bf16x2(uint32_t x) {
-  uint32_t y;
-  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-
-// acc + the low / high bf16 of a packed pair, in fp32.
-__device__ __forceinline__ float add_bf16_lo(uint32_t pair, float acc) {
-  float r;
-  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.bf16 %0, lo, %2;\n\t}"
-      : "=f"(r) : "r"(pair), "f"(acc));
-  return r;
-}
-__device__ __forceinline__ float add_bf16_hi(uint32_t pair, float acc) {
-  float r;
-  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.bf16 %0, hi, %2;\n\t}"
-      : "=f"(r) : "r"(pair), "f"(acc));
-  return r;
-}
-
 }  // namespace swa

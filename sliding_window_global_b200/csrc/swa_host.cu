@@ -249,12 +249,10 @@ swa_status enqueue_forward(const swa_plan_desc& d, const swa_forward_args& args,
       }
       p.tiles[h] = units;
     }
-    // linear order of band units: batch, head (pair), residue class, row unit
-    p.num_hp = pair ? Hq / 2 : Hq;
-    p.unit_prefix[0] = 0;
-    for (int hp = 0; hp < p.num_hp; ++hp)
-      p.unit_prefix[hp + 1] = p.unit_prefix[hp] + p.tiles[pair ? 2 * hp : hp];
-    p.units_total = (long long)p.B * p.unit_prefix[p.num_hp];
+    // unit ids: (row unit, batch, head or head pair), heads fastest; heads with fewer
+    // units than the largest skip the ids beyond theirs
+    p.max_units = 0;
+    for (int h = 0; h < Hq; ++h) p.max_units = std::max(p.max_units, p.tiles[h]);
   }
   if (num_global > 0) {
     p.dense_class = -1;
@@ -327,7 +325,7 @@ swa_status enqueue_forward(const swa_plan_desc& d, const swa_forward_args& args,
     const swa_status st = read_and_clear_error(ws.err, s);
     if (st != SWA_OK) return st;
   }
-  if (build_side && bf16 && ws.agg_count) {
+  if (build_side && bf16 && ws.agg_count && !local_bias && !rand_blocks) {
     // the band kernel builds the side keys / values in its prologue
     p.agg_k = k;
     p.agg_v = v;

@@ -57,8 +57,7 @@ struct AttnParams {
   float* part_lse;                   // [nsplit, B*Hq, gpad]
   int nsplit_keys, split_keys, nsplit;  // global-row key splits (+1 for side keys)
   int pair_heads;                    // units pair heads 2m, 2m+1 (same rows) instead of row tiles
-  int num_hp;                        // heads (or head pairs) that own work units
-  long long units_total;             // band work units over the batch: B * unit_prefix[num_hp]
+  int max_units;                     // largest tiles[h]
   int* err;                          // device error word
   // Fused Transient-Global prologue (MODE 0): every CTA first builds its share of
   // the side keys / values (block means of agg_k / agg_v into agg_sk / agg_sv, the
@@ -74,7 +73,6 @@ struct AttnParams {
   int window[kMaxHeads];
   int class_base[kMaxHeads];         // class id of (dilation[h], c = 0)
   int tiles[kMaxHeads];              // work units of head h (of head pair h/2 when pairing)
-  int unit_prefix[kMaxHeads + 1];    // units of heads (head pairs) before index hp, one batch
 };
 
 // Launchers (each returns the launch's cudaError_t).
