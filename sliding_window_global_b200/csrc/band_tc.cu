@@ -1154,499 +1154,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 }
 
 
-// ------------------------------------------------------------------ split-softmax kernel
-// The plain band pattern (window, dilation, causal, padding, GQA pairs; no global
-// tokens, side keys, biases or random blocks) with every query tile's softmax split
-// over two warpgroups: warpgroup (x, h) handles key columns [64h, 64h + 64) of tile
-// x.  Per key tile the two halves exchange their row maxima through shared memory
-// (the reference max m of a row is then the same in both), so P shares one scale
-// and the O accumulator stays whole; each half keeps its own partial row sum, and
-// the halves add them up at the end.  Twice the softmax warps per SM scheduler,
-// each with half the exponentials per tile, against the same MMA chain.
-constexpr int kSplitThreads = 640;             // 4 softmax warpgroups + control
-constexpr int kSplitSoftmaxThreads = 512;
-constexpr int kSplitProducer = 16;             // warp ids of the control warpgroup
-constexpr int kSplitIssuer = 17;
-#ifndef SWA_SPLIT_REGS_SOFTMAX
-#define SWA_SPLIT_REGS_SOFTMAX 104
-#endif
-#ifndef SWA_SPLIT_REGS_CONTROL
-#define SWA_SPLIT_REGS_CONTROL 64
-#endif
-constexpr int kSplitRegsSoftmax = SWA_SPLIT_REGS_SOFTMAX;
-constexpr int kSplitRegsControl = SWA_SPLIT_REGS_CONTROL;
-static_assert(kSplitSoftmaxThreads * kSplitRegsSoftmax + 128 * kSplitRegsControl <= kSplitThreads * 96,
-              "setmaxnreg split exceeds the launch register budget (96 per thread for 640 threads)");
-
-// Row max of 64 values.
-__device__ __forceinline__ float row_max64(const float (&x)[64]) {
-  float m[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m[i] = fmaxf(x[i], x[8 + i]);
-#pragma unroll
-  for (int e = 16; e < 64; e += 16) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) m[i] = fmax3(m[i], x[e + i], x[e + 8 + i]);
-  }
-  return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
-}
-
-template <int D>
-__global__ void __launch_bounds__(kSplitThreads, 1) attn_split_kernel(const __grid_constant__ AttnParams p) {
-  using C = Cfg<D>;
-  constexpr int NS = C::NS;
-  constexpr int kIssuers = C::kSepP ? 2 : 1;
-  constexpr int kTilesPerIssuer = 2 / kIssuers;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem + C::kQOff;
-  uint8_t* sK = smem + C::kKOff;
-  uint8_t* sV = smem + C::kVOff;
-  // exchange area (in the bias area, unused here): [parity][tile][half][row] maxima,
-  // then [tile][half][row] partial row sums
-  float* sMax = reinterpret_cast<float*>(smem + C::kBiasOff);
-  float* sSum = sMax + 2 * 2 * 2 * kTile;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-  uint64_t* q_full = bars;                // [2]
-  uint64_t* q_empty = bars + 2;           // [2]
-  uint64_t* k_full = bars + 4;            // [NS]
-  uint64_t* v_full = k_full + NS;
-  uint64_t* kv_empty = v_full + NS;
-  uint64_t* s_full = kv_empty + NS;       // [2]
-  uint64_t* p_full = s_full + 2;          // [2]
-  uint64_t* o_full = p_full + 2;          // [2]
-  uint64_t* s_free = o_full + 2;          // [2] both halves read S (separate-P layout)
-  uint64_t* pv_done = s_free + 2;         // [2]
-  uint64_t* p_half = pv_done + 2;         // [2] P over S: half 0 wrote P of keys 0-63, both rescaled O
-  __shared__ uint32_t tmem_slot;
-  __shared__ int abort_flag;
-
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int lane = tid & 31;
-  const int nunits = total_units<0>(p);
-
-  if (tid == 0) {
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(&q_full[x], 1);
-      mbar_init(&q_empty[x], 1);
-      mbar_init(&s_full[x], 1);
-      mbar_init(&p_full[x], C::kSepP ? 2 * kTile : kTile);
-      mbar_init(&o_full[x], 1);
-      mbar_init(&s_free[x], 2 * kTile);
-      mbar_init(&pv_done[x], 1);
-      mbar_init(&p_half[x], 2 * kTile);
-    }
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], kIssuers);
-    }
-    abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == kSplitIssuer) {
-    tmem_alloc(&tmem_slot, C::kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_slot;
-  volatile int* abort_v = &abort_flag;
-  if (warp == kSplitProducer) {
-    // ------------------------------------------------------------ TMA producer
-    setmaxnreg_dec<kSplitRegsControl>();
-    if (lane == 0) {
-      int qloads[2] = {0, 0};
-      int kv = 0;                                   // K/V tiles loaded so far (ring position)
-      bool ok = true;
-      for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
-        Work w;
-        decode_work<0, false>(p, uid, w);
-        if (!w.active[0]) continue;
-        const CUtensorMap* mq = &p.mq[w.cls];
-        const int kz = w.b * p.Hkv + w.hk;
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          if (!ok) break;
-          const int qz = w.b * p.Hq + w.hx[x];
-          if (!w.active[x]) continue;
-          if (qloads[x] > 0 &&
-              !mbar_wait_bounded(&q_empty[x], (qloads[x] - 1) & 1, abort_v, kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&q_full[x], C::kTileBytes);
-          tma_tile<D>(sQ + x * C::kTileBytes, mq, &q_full[x], w.u0[x], qz);
-          ++qloads[x];
-        }
-        for (int j = 0; ok && j < w.total; ++j, ++kv) {
-          const int st = kv % NS;
-          const int use = kv / NS;
-          if (kv >= NS && !mbar_wait_bounded(&kv_empty[st], (use - 1) & 1, abort_v, kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-          const CUtensorMap *mk, *mv;
-          int y;
-          tile_source(p, w, j, mk, mv, y);
-          mbar_arrive_expect_tx(&k_full[st], C::kTileBytes);
-          tma_tile<D>(sK + st * C::kTileBytes, mk, &k_full[st], y, kz);
-          mbar_arrive_expect_tx(&v_full[st], C::kTileBytes);
-          tma_tile<D>(sV + st * C::kTileBytes, mv, &v_full[st], y, kz);
-        }
-      }
-    }
-  } else if (warp == kSplitIssuer || (kIssuers == 2 && warp == kSplitIssuer + 1)) {
-    // ------------------------------------------------------------ MMA issuers
-    // P over S (D = 128): warp 9 issues both tiles' MMAs in one fixed order, which
-    // keeps the two softmax groups half a period apart.  Separate P (D = 64): warp
-    // 9 issues tile A's MMAs and warp 10 tile B's, so neither tile's products wait
-    // behind the other tile's barriers.
-    setmaxnreg_dec<kSplitRegsControl>();
-    if (lane == 0) {
-      const int x0 = (kIssuers == 2) ? warp - kSplitIssuer : 0;   // first tile of this issuer
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-      const uint32_t q_base = smem_u32(sQ);
-      const uint32_t k_base = smem_u32(sK);
-      const uint32_t v_base = smem_u32(sV);
-      int qwaits[kTilesPerIssuer] = {}, pwaits[kTilesPerIssuer] = {};
-      int nqk[kTilesPerIssuer] = {};                    // QKs issued per tile buffer (kernel-wide)
-      int kv = 0;
-      bool ok = true;
-      for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
-        Work w;
-        decode_work<0, false>(p, uid, w);
-        if (!w.active[0]) continue;
-        const int T = w.total;
-        // the tiles' fields as scalars (x0 is a run-time value with two issuers)
-        TileRows tr[kTilesPerIssuer];
-        int first[kTilesPerIssuer], last[kTilesPerIssuer], issued[kTilesPerIssuer], npv[kTilesPerIssuer];
-#pragma unroll
-        for (int i = 0; i < kTilesPerIssuer; ++i) {
-          tr[i] = tile_rows(w, x0 + i);
-          first[i] = last[i] = issued[i] = -1;
-          npv[i] = 0;
-          for (int j = 0; j < T; ++j)
-            if (uses(w, tr[i], x0 + i, j)) {
-              if (first[i] < 0) first[i] = j;
-              last[i] = j;
-            }
-        }
-        auto issue_qk = [&](int i, int j) -> bool {
-          const int x = x0 + i;
-          const int g = kv + j;
-          if (!mbar_wait_bounded(&k_full[g % NS], (g / NS) & 1, abort_v, kWaitLimitNs)) return false;
-          // separate-P layout: S_x is rewritten only after the softmax read the last one
-          if (C::kSepP && nqk[i] > 0 &&
-              !mbar_wait_bounded(&s_free[x], (nqk[i] - 1) & 1, abort_v, kWaitLimitNs))
-            return false;
-          ++nqk[i];
-          tc_fence_after();
-          const uint32_t qt = q_base + x * C::kTileBytes;
-          const uint32_t kt = k_base + (g % NS) * C::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
-            umma_ss(tmem + C::s_col(x), sdesc_sw128(qt + off, 16, 1024),
-                    sdesc_sw128(kt + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&s_full[x]);
-          if (j == last[i]) umma_commit(&q_empty[x]);   // Q_x may be refilled once this QK is done
-          issued[i] = j;
-          return true;
-        };
-#pragma unroll
-        for (int i = 0; i < kTilesPerIssuer; ++i) {
-          if (!ok) break;
-          if (!tr[i].active) continue;
-          ok = mbar_wait_bounded(&q_full[x0 + i], qwaits[i] & 1, abort_v, kWaitLimitNs);
-          ++qwaits[i];
-          if (ok) ok = issue_qk(i, first[i]);
-        }
-        for (int j = 0; ok && j < T; ++j) {
-          const int g = kv + j;
-          const int st = g % NS;
-          bool any = false;                           // this issuer reads the slot of tile j
-#pragma unroll
-          for (int i = 0; i < kTilesPerIssuer; ++i) {
-            const bool u = uses(w, tr[i], x0 + i, j);
-            any = any || u;
-            if (ok && u && issued[i] < j) ok = issue_qk(i, j);
-          }
-          if (C::kSepP) {
-            // the next S of each tile as soon as its softmax has read the current one
-            // (its next key tile may be j + 2 when random tiles alternate; a tile up
-            // to j + NS - 1 is loadable: its ring slot was freed by tile <= j - 1)
-#pragma unroll
-            for (int i = 0; i < kTilesPerIssuer; ++i) {
-              if (!ok || !uses(w, tr[i], x0 + i, j) || issued[i] != j) continue;
-              int jn = j + 1;
-              while (jn < T && jn < j + NS && !uses(w, tr[i], x0 + i, jn)) ++jn;
-              if (jn < T && jn < j + NS) ok = issue_qk(i, jn);
-            }
-          }
-          if (!ok) break;
-          // With two issuers both wait for V of every tile of the unit, used or not,
-          // before they release its ring slot: the slot's next load needs both
-          // releases, so neither issuer can arrive twice on one phase of kv_empty.
-          if (!mbar_wait_bounded(&v_full[st], (g / NS) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
-          if (!any) {
-            mbar_arrive(&kv_empty[st]);               // no MMA of this issuer reads the slot
-            continue;
-          }
-          const uint32_t vt = v_base + st * C::kTileBytes;
-#pragma unroll
-          for (int i = 0; i < kTilesPerIssuer; ++i) {
-            const int x = x0 + i;
-            if (!ok) break;
-            if (!uses(w, tr[i], x, j)) continue;
-            if (!C::kSepP) {
-              // P over S: the first half of P (keys 0-63) is published early, so the
-              // PV over it overlaps the exponentials of the second half
-              if (!mbar_wait_bounded(&p_half[x], pwaits[i] & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
-              tc_fence_after();
-#pragma unroll
-              for (int kk = 0; kk < kTile / 32; ++kk)
-                umma_ts(tmem + C::o_col(x), tmem + C::p_col(x) + kk * 8,
-                        sdesc_sw128(vt + kk * 2048, kSub, 1024), idesc_pv, (npv[i] > 0 || kk > 0) ? 1u : 0u);
-            }
-            if (!mbar_wait_bounded(&p_full[x], pwaits[i] & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
-            ++pwaits[i];
-            tc_fence_after();
-#pragma unroll
-            for (int kk = C::kSepP ? 0 : kTile / 32; kk < kTile / 16; ++kk)
-              umma_ts(tmem + C::o_col(x), tmem + C::p_col(x) + kk * 8,
-                      sdesc_sw128(vt + kk * 2048, kSub, 1024), idesc_pv, (npv[i] > 0 || kk > 0) ? 1u : 0u);
-            ++npv[i];
-            if (C::kSepP) umma_commit(&pv_done[x]);
-            if (j == last[i]) umma_commit(&o_full[x]);
-            else if (!C::kSepP && uses(w, tr[i], x, j + 1)) ok = issue_qk(i, j + 1);
-          }
-          umma_commit(&kv_empty[st]);
-        }
-        kv += T;
-      }
-    }
-  } else if (warp >= kSplitProducer) {
-    setmaxnreg_dec<kSplitRegsControl>();
-  } else {
-    // ------------------------------------------------------------ softmax warpgroups
-    setmaxnreg_inc<kSplitRegsSoftmax>();
-    const int wg = warp >> 2;
-    const int x = wg >> 1;                     // query tile
-    const int hh = wg & 1;                     // key-column half
-    const int row = tid & 127;                 // TMEM lane == row in the tile
-    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const uint32_t s_addr = lane_base + C::s_col(x) + hh * 64;
-    const uint32_t p_addr = lane_base + C::p_col(x) + hh * 32;
-    const uint32_t o_addr = lane_base + C::o_col(x) + hh * (D / 2);
-    const int cbase = hh * 64;
-    int pw = 0;
-    const float sl2 = p.scale_log2;
-    int it = 0;
-    int oc = 0;
-    bool ok = true;
-    for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
-      Work w;
-      decode_work<0, false>(p, uid, w);
-      if (!w.valid) continue;
-      const TileRows tr = tile_rows(w, x);
-      if (!w.active[0] || !tr.active) {
-        if (hh == 0) write_zero_row<D>(p, w, tr, row);
-        continue;
-      }
-      const int T = w.total;
-      const bool row_valid = row < tr.nvalid;
-      const int u = tr.u0 + row;
-      int klo = u - w.r;
-      int khi = min(p.causal ? u : u + w.r, w.Vc - 1) + 1;
-      if (!row_valid) khi = klo;
-      float m = -INFINITY;                     // running reference max (log2 units), shared by both halves
-      float l = 0.f;                           // this half's partial row sum
-      int iu = 0;
-      for (int j = 0; j < T; ++j) {
-        if (!uses(w, tr, x, j)) continue;
-        if (!mbar_wait_bounded(&s_full[x], it & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
-        tc_fence_after();
-        uint32_t xr[64];
-        tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(xr));
-        tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(xr + 32));
-        tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(xr));
-        tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(xr + 32));
-        if (C::kSepP) {
-          tc_fence_before();
-          mbar_arrive(&s_free[x]);
-        }
-        float sc[64];
-#pragma unroll
-        for (int e = 0; e < 64; ++e) sc[e] = __uint_as_float(xr[e]);
-        const int kv0 = w.band_lo + j * kTile + cbase;
-        const int lo_t = klo - kv0, hi_t = khi - kv0;
-        uint32_t live = 0;
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch)
-          if (__any_sync(0xffffffffu, lo_t < 32 * ch + 32 && hi_t > 32 * ch)) live |= 1u << ch;
-        const bool cut_lo = __any_sync(0xffffffffu, lo_t > 0);
-        const bool cut_hi = __any_sync(0xffffffffu, hi_t < 64);
-        if (cut_lo && cut_hi) {
-#pragma unroll
-          for (int e = 0; e < 64; ++e) sc[e] = (e >= lo_t && e < hi_t) ? sc[e] : -INFINITY;
-        } else if (cut_lo) {
-#pragma unroll
-          for (int e = 0; e < 64; ++e) sc[e] = (e >= lo_t) ? sc[e] : -INFINITY;
-        } else if (cut_hi) {
-#pragma unroll
-          for (int e = 0; e < 64; ++e) sc[e] = (e < hi_t) ? sc[e] : -INFINITY;
-        }
-        // this half's row max, exchanged with the other half's through shared memory
-        const float hmax = row_max64(sc) * sl2;
-        float* xm = sMax + ((it & 1) * 4 + x * 2) * kTile;
-        xm[hh * kTile + row] = hmax;
-        named_barrier_sync(1 + x, 2 * kTile);
-        const float tmax = fmaxf(hmax, xm[(1 - hh) * kTile + row]);
-        const float m_new = fmaxf(m, tmax);
-        const bool need = (m == -INFINITY) ? (m_new > -INFINITY) : (m_new > m + kRescaleThreshold);
-        const bool rescale = __any_sync(0xffffffffu, need);
-        float alpha = 1.f;
-        if (rescale) {
-          alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
-          l *= alpha;
-          m = m_new;
-        }
-        const float neg_m = (m == -INFINITY) ? 0.f : -m;
-        if (C::kSepP && pw > 0) {
-          if (!mbar_wait_bounded(&pv_done[x], (pw - 1) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
-          tc_fence_after();
-        }
-        if (!C::kSepP && rescale && iu > 0) {
-          // O_x (this half's columns) must be rescaled before P is published; it is
-          // stable: its previous PV was issued before this S and MMAs complete in order
-#pragma unroll 1
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t rr[16];
-            tmem_ld16(o_addr + ch * 16, rr);
-            tmem_wait_ld_dep16(rr);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
-            tmem_st16(o_addr + ch * 16, rr);
-          }
-        }
-        if (!C::kSepP && hh == 1) {
-          // the PV over keys 0-63 writes every O column: this half's rescale must be in
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(&p_half[x]);
-        }
-        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t pk[16];
-          if (!(live & (1u << ch))) {
-#pragma unroll
-            for (int q = 0; q < 16; ++q) pk[q] = 0u;
-          } else {
-#pragma unroll
-            for (int q = 0; q < 32; q += 4) {
-              const int e = ch * 32 + q;
-              float a0, a1, a2, a3;
-              ffma2(a0, a1, sc[e], sc[e + 1], sl2, sl2, neg_m, neg_m);
-              ffma2(a2, a3, sc[e + 2], sc[e + 3], sl2, sl2, neg_m, neg_m);
-              if (q < emu_per32<D>()) {
-                exp2_poly2(a0, a1, a0, a1);
-                exp2_poly2(a2, a3, a2, a3);
-              } else {
-                a0 = ex2_approx(a0);
-                a1 = ex2_approx(a1);
-                a2 = ex2_approx(a2);
-                a3 = ex2_approx(a3);
-              }
-              fadd2(acc0, acc1, acc0, acc1, a0, a1);
-              fadd2(acc2, acc3, acc2, acc3, a2, a3);
-              pk[q / 2] = pack_bf16x2(a0, a1);
-              pk[q / 2 + 1] = pack_bf16x2(a2, a3);
-            }
-          }
-          tmem_st16(p_addr + ch * 16, pk);
-        }
-        l += (acc0 + acc1) + (acc2 + acc3);
-        if (C::kSepP && rescale && iu > 0) {
-#pragma unroll
-          for (int ch = 0; ch < D / 64; ++ch) {
-            uint32_t rr[32];
-            tmem_ld32(o_addr + ch * 32, rr);
-            tmem_wait_ld_dep(rr);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
-            tmem_st32(o_addr + ch * 32, rr);
-          }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        if (!C::kSepP && hh == 0) mbar_arrive(&p_half[x]);   // P of keys 0-63 (and this half rescaled)
-        else mbar_arrive(&p_full[x]);          // P over S: keys 64-127; separate P: all of P
-        ++pw;
-        ++it;
-        ++iu;
-      }
-      if (!ok) break;
-
-      // ---------------------------------------------------------- epilogue
-      // the two halves' sums, then O / l: each half stores its D/2 output columns
-      float* xs = sSum + x * 2 * kTile;
-      xs[hh * kTile + row] = l;
-      named_barrier_sync(1 + x, 2 * kTile);
-      const float l_all = l + xs[(1 - hh) * kTile + row];
-      if (!mbar_wait_bounded(&o_full[x], oc & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
-      ++oc;
-      tc_fence_after();
-      const bool has = row_valid && l_all > 0.f;
-      const float inv = has ? 1.f / l_all : 0.f;
-      const size_t off = out_row(p, w, tr, row);
-      if (hh == 0 && row < tr.rows && p.lse) p.lse[off] = has ? (m + __log2f(l_all)) * kLn2 : -INFINITY;
-      uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + off * D + hh * (D / 2));
-#pragma unroll
-      for (int ch = 0; ch < D / 64; ++ch) {
-        uint32_t rr[32];
-        tmem_ld32(o_addr + ch * 32, rr);
-        tmem_wait_ld_dep(rr);
-        if (row < tr.rows) {
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 0]) * inv, __uint_as_float(rr[q4 * 8 + 1]) * inv);
-            v.y = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 2]) * inv, __uint_as_float(rr[q4 * 8 + 3]) * inv);
-            v.z = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 4]) * inv, __uint_as_float(rr[q4 * 8 + 5]) * inv);
-            v.w = pack_bf16x2(__uint_as_float(rr[q4 * 8 + 6]) * inv, __uint_as_float(rr[q4 * 8 + 7]) * inv);
-            orow[ch * 4 + q4] = v;
-          }
-        }
-      }
-      tc_fence_before();
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (abort_flag) {
-    if (tid == 0) {
-      atomicOr(p.err, kDevErrTimeout);
-      const uint64_t t0 = global_timer_ns();
-      while (global_timer_ns() - t0 < 2000000ull) {
-      }
-    }
-    __syncthreads();
-  }
-  if (warp == kSplitIssuer) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
-  }
-}
-
 }  // namespace
 
 size_t band_tc_smem_bytes(int D) {
@@ -1680,27 +1187,9 @@ static cudaError_t launch_one(const AttnParams& p, int units, int num_sms, cudaS
   return cudaGetLastError();
 }
 
-#ifndef SWA_SPLIT
-#define SWA_SPLIT 1
-#endif
-
-template <int D>
-static cudaError_t launch_split(const AttnParams& p, int units, int num_sms, cudaStream_t s) {
-  auto kern = attn_split_kernel<D>;
-  const int smem = static_cast<int>(Cfg<D>::kSmemBytes);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  const int grid = units < num_sms ? units : num_sms;
-  if (grid <= 0) return cudaSuccess;
-  kern<<<grid, kSplitThreads, smem, s>>>(p);
-  return cudaGetLastError();
-}
-
 // p.tiles[h] holds the number of two-tile units of head h, p.max_units their maximum.
 cudaError_t launch_band_tc(const AttnParams& p, int num_sms, cudaStream_t s) {
   const int units = p.max_units * p.B * p.Hq;
-  if (SWA_SPLIT && p.g == 0 && p.S == 0 && !p.local_bias && p.num_rand == 0 && !p.agg_count)
-    return p.D == 64 ? launch_split<64>(p, units, num_sms, s) : launch_split<128>(p, units, num_sms, s);
   if (p.agg_count) {      // side keys built in the prologue (no local bias, no random blocks)
     return p.D == 64 ? launch_one<64, 0, false, false, true>(p, units, num_sms, s)
                      : launch_one<128, 0, false, false, true>(p, units, num_sms, s);
