@@ -44,7 +44,7 @@ def _peaks():
 
 def _kernel_hash():
     h = hashlib.sha256()
-    for name in ("band_tc.cu", "ptx.cuh", "swa_kernels.h"):
+    for name in ("band_tc.cu", "ptx.cuh", "swa_kernels.h", "softmax_math.cuh", "side_mean.cuh"):
         with open(os.path.join(ROOT, "sliding_window_global_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
