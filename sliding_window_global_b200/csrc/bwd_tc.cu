@@ -49,8 +49,10 @@ struct BCfg {
   static constexpr uint32_t kBarOff = kStageOff + 4 * kStage * 4;
   static constexpr uint32_t kSmemBytes = kBarOff + 16 * 8 + 1024;
   static constexpr uint32_t kTmemCols = 512;
-  // TMEM columns (dQ pass): S 0-127 with dS written over 0-63, dP 128-255, dQ after.
-  static constexpr uint32_t kS = 0, kDP = 128, kAcc0 = 256;
+  // TMEM columns (dQ pass): S of even key tiles 0-127 and of odd ones 384-511 (dS written
+  // over its first 64 columns), dP 128-255, dQ from 256.
+  static constexpr uint32_t kS = 0, kDP = 128, kAcc0 = 256, kS1 = 384;
+  __host__ __device__ static constexpr uint32_t s_buf(int j) { return (j & 1) ? kS1 : kS; }
 };
 
 // TMA load of one 128 x D bf16 tile (two 64-column boxes when D = 128).
@@ -186,8 +188,12 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
   uint64_t* r_full = bars + 1;      // [2] K, V of a stage loaded
   uint64_t* r_empty = bars + 3;     // [2] the stage's last MMA completed
   uint64_t* s_full = bars + 5;      // S and dP in TMEM
-  uint64_t* ds_full = bars + 6;     // dS written (128 arrivals)
+  uint64_t* ds_full = bars + 9;     // [2] dS of even / odd key tiles written (128 arrivals): with
+                                    // S and dP of tile j+1 issued before the wait for dS(j), the
+                                    // compute warps may finish tile j+1 first; one barrier per parity
+                                    // keeps every wait at most one phase behind
   uint64_t* acc_full = bars + 7;    // dQ complete
+  uint64_t* dp_read = bars + 8;     // dP read into registers (128 arrivals): the next dP may be written
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ int sGpos[kTile];      // key positions of the current global-column tile
@@ -238,8 +244,10 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
       mbar_init(&r_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(ds_full, 128);
+    mbar_init(&ds_full[0], 128);
+    mbar_init(&ds_full[1], 128);
     mbar_init(acc_full, 1);
+    mbar_init(dp_read, 128);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -285,27 +293,41 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
     }
   } else if (warp == 5) {
     if (lane == 0 && T > 0) {
+      // Pipelined: S of tile j+1 is computed into the other S buffer while the compute
+      // warps work on tile j, and dP of tile j+1 as soon as they have read dP of tile j,
+      // so the next tile's products are ready when the compute warps are.  In issue
+      // order (MMAs complete in order): a new S goes into the buffer whose dS the
+      // previous dQ product read; a new dP after dp_read.
       const uint32_t qa = smem_u32(smem + C::kStat0), da = smem_u32(smem + C::kStat1);
+      auto stage = [&](int j) { return smem_u32(smem + C::kRing + (j & 1) * 2 * C::kTileBytes); };
+      auto issue_s = [&](int j) -> bool {           // S(j) = Q K(j)^T
+        if (!mbar_wait_bounded(&r_full[j & 1], (j >> 1) & 1, abort_v, kWaitLimitNs)) return false;
+        tc_fence_after();
+        mma_abt<D>(tmem + C::s_buf(j), qa, stage(j));
+        return true;
+      };
       bool ok = mbar_wait_bounded(a_full, 0, abort_v, kWaitLimitNs);
-      for (int j = 0; ok && j <= T; ++j) {
-        if (j > 0) {
-          // dQ += dS(j-1) K(j-1), then the stage of tile j-1 may be refilled
-          if (!mbar_wait_bounded(ds_full, (j - 1) & 1, abort_v, kWaitLimitNs)) break;
+      if (ok) ok = issue_s(0);
+      if (ok) {
+        mma_abt<D>(tmem + C::kDP, da, stage(0) + C::kTileBytes);     // dP(0) = dO V(0)^T
+        umma_commit(s_full);
+      }
+      if (ok && T > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < T; ++j) {
+        if (j + 1 < T) {
+          // dP(j+1) once the compute warps hold dP(j) in registers
+          if (!mbar_wait_bounded(dp_read, j & 1, abort_v, kWaitLimitNs)) break;
           tc_fence_after();
-          const int sp = (j - 1) & 1;
-          mma_px<D>(tmem + C::kAcc0, tmem + C::kS, smem_u32(smem + C::kRing + sp * 2 * C::kTileBytes), j > 1);
-          umma_commit(&r_empty[sp]);
-          if (j == T) umma_commit(acc_full);
+          mma_abt<D>(tmem + C::kDP, da, stage(j + 1) + C::kTileBytes);
+          umma_commit(s_full);                       // S(j+1) and dP(j+1)
         }
-        if (j < T) {
-          const int st = j & 1;
-          if (!mbar_wait_bounded(&r_full[st], (j >> 1) & 1, abort_v, kWaitLimitNs)) break;
-          tc_fence_after();
-          const uint32_t kb = smem_u32(smem + C::kRing + st * 2 * C::kTileBytes);
-          mma_abt<D>(tmem + C::kS, qa, kb);                          // S = Q K^T
-          mma_abt<D>(tmem + C::kDP, da, kb + C::kTileBytes);         // dP = dO V^T
-          umma_commit(s_full);
-        }
+        // dQ += dS(j) K(j), then the stage of tile j may be refilled
+        if (!mbar_wait_bounded(&ds_full[j & 1], (j >> 1) & 1, abort_v, kWaitLimitNs)) break;
+        tc_fence_after();
+        mma_px<D>(tmem + C::kAcc0, tmem + C::s_buf(j), stage(j), j > 0);
+        umma_commit(&r_empty[j & 1]);
+        if (j == T - 1) umma_commit(acc_full);
+        if (j + 2 < T) ok = issue_s(j + 2);           // into the buffer dQ(j) just read
       }
     }
   } else {
@@ -381,13 +403,21 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
       tc_fence_after();
       const int kv0 = GROWS ? j * kTile : (kind == 3 ? kb * kTile : klo_t + j * kTile);
       const int lo_t = klo - kv0, hi_t = khi - kv0;
+      // dP of the tile into registers, then its TMEM columns go back to the MMA warp
+      uint32_t dpr[kTile];
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) tmem_ld32(lane_base + C::kDP + ch * 32, *reinterpret_cast<uint32_t(*)[32]>(dpr + ch * 32));
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(dpr + ch * 32));
+      tc_fence_before();
+      mbar_arrive(dp_read);
+      const uint32_t sb = lane_base + C::s_buf(j);
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
-        uint32_t sr[32], dr[32];
-        tmem_ld32(lane_base + C::kS + ch * 32, sr);
-        tmem_ld32(lane_base + C::kDP + ch * 32, dr);
+        uint32_t sr[32];
+        tmem_ld32(sb + ch * 32, sr);
         tmem_wait_ld_dep(sr);
-        tmem_wait_ld_dep(dr);
+        const uint32_t* dr = dpr + ch * 32;
         uint32_t pk[16];
 #pragma unroll
         for (int q = 0; q < 32; q += 2) {
@@ -421,11 +451,11 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
           pk[q / 2] = pack_bf16x2(ds[0], ds[1]);
         }
         // dS as bf16 over S: chunk ch writes columns 16ch.. that earlier chunks read
-        tmem_st16(lane_base + C::kS + ch * 16, pk);
+        tmem_st16(sb + ch * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(ds_full);
+      mbar_arrive(&ds_full[j & 1]);
     }
     // epilogue: dQ = scale * (dS K), fp32; padded rows get zeros.  Global rows (GROWS)
     // add their part to what the band pass wrote.

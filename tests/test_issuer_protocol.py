@@ -21,8 +21,9 @@ barrier once the MMAs issued before it have completed.  Checked on every run:
 * every query tile's softmax sees exactly its own key tiles, in order.
 
 Optionally both softmax groups also meet at every unit start, as they do when a side
-or local bias is staged in shared memory.  A second model covers the key-stationary
-dK/dV pass of the backward (csrc/bwd_tc.cu).  Each model has a planted-mistake test.
+or local bias is staged in shared memory.  Two more models cover the backward
+(csrc/bwd_tc.cu): the key-stationary dK/dV pass and the pipelined query-stationary dQ
+pass.  Each model has a planted-mistake test.
 """
 import random
 
@@ -433,6 +434,159 @@ def test_dkv_model_detects_an_early_next_product():
     for seed in range(100):
         try:
             simulate_dkv(seed, 6, early_next=True)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
+
+
+def simulate_dq(seed, T, early_dp=False, early_s=False, per_parity=True):
+    """The query-stationary dQ pass (csrc/bwd_tc.cu): one query tile per CTA, its T key
+    tiles through a two-stage ring; S of tile j in TMEM buffer j & 1, dP in one buffer.
+    The issuer computes S(j+1) while the compute warps work on tile j, dP(j+1) once
+    they hold dP(j) in registers (dp_read), and S(j+2) into the buffer dQ(j) has just
+    read (in issue order).  MMAs complete in issue order.  Checked: the compute warps
+    read S(j) and dP(j) of their own tile, dS(j) is what dQ(j) reads, no ring slot is
+    refilled under a pending reader, no deadlock, no parity-ambiguous wait.
+    per_parity=False models a single dS barrier, which the compute warps can drive two
+    phases past the issuer's wait."""
+    rng = random.Random(seed)
+    a_full = Barrier("a_full", 1)
+    r_full = [Barrier(f"r_full{s}", 1) for s in range(2)]
+    r_empty = [Barrier(f"r_empty{s}", 1) for s in range(2)]
+    s_full = Barrier("s_full", 1)
+    dp_read = Barrier("dp_read", 128)
+    ds_full = [Barrier(f"ds_full{x}", 128) for x in range(2)]   # one per key-tile parity
+    acc_full = Barrier("acc_full", 1)
+    pipe = []
+    pending = {}
+    loads = [0, 0]
+    sbuf = [None, None]                     # what each S buffer holds: ("S", j) or ("dS", j)
+    dpbuf = [None]                          # the tile whose dP the dP buffer holds
+
+    def mma_read(key):
+        pending[key] = pending.get(key, 0) + 1
+        pipe.append(("read", key))
+
+    def producer():
+        a_full.arrive()
+        for j in range(T):
+            st = j & 1
+            if j >= 2:
+                yield from wait(r_empty[st], (j >> 1) - 1)
+            if pending.get(("ring", st, loads[st] - 1), 0):
+                raise ProtocolError(f"ring slot {st} refilled under a pending reader")
+            loads[st] += 1
+            yield
+            r_full[st].arrive()
+
+    def issuer():
+        def issue_s(j):
+            yield from wait(r_full[j & 1], j >> 1)
+            mma_read(("ring", j & 1, loads[j & 1] - 1))
+            pipe.append(("write_s", j))
+
+        def issue_dp(j):
+            mma_read(("ring", j & 1, loads[j & 1] - 1))
+            pipe.append(("write_dp", j))
+
+        yield from wait(a_full, 0)
+        yield from issue_s(0)
+        issue_dp(0)
+        pipe.append(("commit", s_full))
+        if T > 1:
+            yield from issue_s(1)
+        for j in range(T):
+            if j + 1 < T:
+                if not early_dp:
+                    yield from wait(dp_read, j)
+                issue_dp(j + 1)
+                pipe.append(("commit", s_full))
+            yield from wait(ds_full[j & 1] if per_parity else ds_full[0], (j >> 1) if per_parity else j)
+            if early_s and j + 2 < T:              # planted: S(j+2) before dQ(j) read dS(j)
+                yield from issue_s(j + 2)
+            mma_read(("ring", j & 1, loads[j & 1] - 1))
+            pipe.append(("read_ds", j))
+            pipe.append(("commit", r_empty[j & 1]))
+            if j == T - 1:
+                pipe.append(("commit", acc_full))
+            if j + 2 < T and not early_s:
+                yield from issue_s(j + 2)
+
+    def compute():
+        for j in range(T):
+            yield from wait(s_full, j)
+            if dpbuf[0] != j:
+                raise ProtocolError(f"compute of tile {j} read dP of tile {dpbuf[0]}")
+            yield
+            for _ in range(128):
+                dp_read.arrive()
+            if sbuf[j & 1] != ("S", j):
+                raise ProtocolError(f"compute of tile {j} read {sbuf[j & 1]} from S buffer {j & 1}")
+            yield
+            sbuf[j & 1] = ("dS", j)
+            for _ in range(128):
+                (ds_full[j & 1] if per_parity else ds_full[0]).arrive()
+        if T > 0:
+            yield from wait(acc_full, 0)
+
+    agents = [producer(), issuer(), compute()]
+    alive = list(range(len(agents)))
+    stalls = 0
+    while alive or pipe:
+        choices = [("agent", a) for a in alive] + ([("pipe", 0)] if pipe else [])
+        kind, who = rng.choice(choices)
+        if kind == "pipe":
+            k, val = pipe.pop(0)
+            if k == "read":
+                pending[val] -= 1
+            elif k == "write_s":
+                sbuf[val & 1] = ("S", val)
+            elif k == "write_dp":
+                dpbuf[0] = val
+            elif k == "read_ds":
+                if sbuf[val & 1] != ("dS", val):
+                    raise ProtocolError(f"dQ product of tile {val} read {sbuf[val & 1]}")
+            else:
+                val.arrive()
+            stalls = 0
+            continue
+        try:
+            next(agents[who])
+            stalls += 1
+        except StopIteration:
+            alive.remove(who)
+            stalls = 0
+        if stalls > 20000:
+            raise ProtocolError("deadlock: no agent can make progress")
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 4, 5, 9])
+def test_dq_pass_protocol_random_schedules(T):
+    for seed in range(200):
+        simulate_dq(seed, T)
+
+
+def test_dq_model_detects_a_single_ds_barrier():
+    """One dS barrier for every key tile lets the compute warps finish tile j+1 before
+    the issuer waits for tile j: a parity wait two phases behind."""
+    caught = 0
+    for seed in range(200):
+        try:
+            simulate_dq(seed, 5, per_parity=False)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
+
+
+@pytest.mark.parametrize("mistake", ["early_dp", "early_s"])
+def test_dq_model_detects_a_misordered_product(mistake):
+    """dP(j+1) issued before the compute warps hold dP(j), or S(j+2) issued into the
+    buffer before the dQ product has read dS(j) from it, is caught as a wrong buffer
+    content, a parity-ambiguous wait or a deadlock."""
+    caught = 0
+    for seed in range(100):
+        try:
+            simulate_dq(seed, 5, **{mistake: True})
         except AssertionError:
             caught += 1
     assert caught > 0
