@@ -511,8 +511,8 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
 // Key-stationary pass with 64-row query tiles and two compute warpgroups that take
 // alternate query tiles, each with its own S^T / dP^T columns in TMEM (M = 128 keys,
 // N = 64 queries), so one group's exponentials overlap the other group's products.
-// P^T and dS^T go to shared memory (128 keys x 64 queries, K-major with the
-// 128-byte swizzle) and feed dV += P^T dO and dK += dS^T Q as shared-memory operands.
+// P^T and dS^T are written as bf16 over the columns of S^T and dP^T and feed
+// dV += P^T dO and dK += dS^T Q as TMEM operands (A = 128 keys x 64 queries).
 constexpr int kQT = 64;                        // query rows per tile of this pass
 constexpr int kMaxRandList = 2048;             // (query head in group, query block) pairs per key block
 constexpr int kDkvThreads = 320;               // warps 0-3, 4-7 compute; 8 TMA; 9 MMA / TMEM
@@ -524,15 +524,15 @@ struct KCfg {
   static constexpr uint32_t kQSub = kQT * 128u;            // 64-row x 128-byte sub-tile
   static constexpr uint32_t kK = 0, kV = kKVBytes;
   static constexpr uint32_t kRing = 2 * kKVBytes;          // stage s: Q at kRing + 2 s Q, dO after
-  static constexpr uint32_t kPds = kRing + 4 * kQBytes;    // group g: P^T at kPds + 2 g P, dS^T after
-  static constexpr uint32_t kPBytes = 128u * kQT * 2u;     // 16 KB
+  static constexpr uint32_t kFlags = kRing + 4 * kQBytes;  // random job: per-pair flags (set-up only)
   // [group][buffer][lse2 64 | delta 64 | position 64 | row fact 64] (floats, ints)
-  static constexpr uint32_t kStg = kPds + 4 * kPBytes;
+  static constexpr uint32_t kStg = kFlags + kMaxRandList * 4;
   static constexpr uint32_t kList = kStg + 2 * 2 * 256 * 4;  // random job: query blocks drawing the key block
   static constexpr uint32_t kBarOff = kList + kMaxRandList * 4;
   static constexpr uint32_t kSmemBytes = kBarOff + 16 * 8 + 1024;
   static constexpr uint32_t kTmemCols = 512;
-  // TMEM: group g S^T at 128 g, dP^T at 128 g + 64; dV at 256, dK at 256 + D
+  // TMEM: group g S^T at 128 g (P^T over its first 32 columns), dP^T at 128 g + 64
+  // (dS^T over its first 32); dV at 256, dK at 256 + D
   static constexpr uint32_t kAccV = 256, kAccK = 256 + D;
 };
 static_assert(KCfg<128>::kSmemBytes <= 227 * 1024, "shared memory of the dK/dV pass");
@@ -568,8 +568,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
   uint64_t* r_empty = bars + 3;     // [2] that stage's products are done
   uint64_t* s_full = bars + 5;      // [2] S^T, dP^T of group g in TMEM
   uint64_t* p_full = bars + 7;      // [2] group g wrote P^T, dS^T (and read its TMEM), 128 arrivals
-  uint64_t* pds_free = bars + 9;    // [2] group g's P^T / dS^T buffers read by the products
-  uint64_t* acc_full = bars + 11;   // dK, dV complete
+  uint64_t* acc_full = bars + 9;    // dK, dV complete
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ int sCount;
@@ -624,7 +623,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
       // the (head, query block) pairs of the group whose random list names this key
       // block, each counted at its first occurrence; built in a fixed order
       const int pairs = p.G * nqb;
-      int* flags = reinterpret_cast<int*>(smem + C::kPds);     // free until the first tile
+      int* flags = reinterpret_cast<int*>(smem + C::kFlags);
       if (pairs > kMaxRandList) {
         if (tid == 0) atomicOr(p.err, kDevErrCheck);   // more pairs than the list holds: reported
         return;
@@ -681,7 +680,6 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
       mbar_init(&r_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 128);
-      mbar_init(&pds_free[s], 1);
     }
     mbar_init(acc_full, 1);
     abort_flag = 0;
@@ -751,21 +749,21 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
       for (int j = 0; ok && j < T; ++j) {
         const int g = j & 1, st = j & 1;
         if (!mbar_wait_bounded(&p_full[g], (j >> 1) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
-        fence_proxy_async_smem();
         tc_fence_after();
-        const uint32_t pt = smem_u32(smem + C::kPds + g * 2 * C::kPBytes);
         const uint32_t qb = smem_u32(smem + C::kRing + st * 2 * C::kQBytes);
-        // dV += P^T dO, dK += dS^T Q (A: 128 x 64 K-major from shared memory; B: 64 x D MN-major)
+        // dV += P^T dO, dK += dS^T Q (A: 128 x 64 bf16 from the group's TMEM columns,
+        // 16 queries = 8 columns per product; B: 64 x D MN-major from shared memory)
 #pragma unroll
         for (int kk = 0; kk < kQT / 16; ++kk) {
-          umma_ss(tmem + C::kAccV, sdesc_sw128(pt + kk * 32, 16, 1024),
+          umma_ts(tmem + C::kAccV, tmem + 128 * g + kk * 8,
                   sdesc_sw128(qb + C::kQBytes + kk * 2048, C::kQSub, 1024), idesc_a, (j > 0 || kk > 0) ? 1u : 0u);
-          umma_ss(tmem + C::kAccK, sdesc_sw128(pt + C::kPBytes + kk * 32, 16, 1024),
+          umma_ts(tmem + C::kAccK, tmem + 128 * g + 64 + kk * 8,
                   sdesc_sw128(qb + kk * 2048, C::kQSub, 1024), idesc_a, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&pds_free[g]);
         umma_commit(&r_empty[st]);
-        if (j + 2 < T) ok = issue_s(j + 2);     // the group has read its S^T, dP^T of tile j
+        // The group has read its S^T, dP^T of tile j; the next ones overwrite the same
+        // columns only after the products above have read P^T, dS^T (in-order pipe).
+        if (j + 2 < T) ok = issue_s(j + 2);
       }
       if (ok) umma_commit(acc_full);
     }
@@ -781,7 +779,6 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
     int kpos = kBandJob ? u.c + u.d * uk : kpos0 + row;
     if (JOB == kJobGlobalKeys) kpos = key_valid ? __ldg(p.global_idx + (size_t)u.b * p.g + uk) : 0;
     const float sl2 = p.scale_log2;
-    uint8_t* pts = smem + C::kPds + g * 2 * C::kPBytes;   // P^T rows, then dS^T rows
     bool ok = true;
     int nt = 0;                               // tiles handled by this group
     for (int j = g; j < T; j += 2, ++nt) {
@@ -841,14 +838,11 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
       named_barrier_sync(1 + g, 128);
       if (!mbar_wait_bounded(&s_full[g], nt & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
       tc_fence_after();
-      // the products of tile j - 2 have read this group's P^T / dS^T buffers
-      if (nt > 0 && !mbar_wait_bounded(&pds_free[g], (nt - 1) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
       const int d0 = qt.y - uk;                // query - key offset of column 0 (band, class coordinates)
-      uint8_t* prow = pts + row * 128;
-      uint8_t* drow = pts + C::kPBytes + row * 128;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {   // 32 query columns at a time
         uint32_t sr[32], dr[32];
+        uint32_t pk[16], dk[16];               // P^T, dS^T of the 32 columns as bf16 pairs
         tmem_ld32(lane_base + 128 * g + 32 * half, sr);
         tmem_ld32(lane_base + 128 * g + 64 + 32 * half, dr);
         tmem_wait_ld_dep(sr);
@@ -887,21 +881,18 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
             pr[e] = allowed ? ex2_approx(__uint_as_float(sr[c4 * 8 + e]) * sl2 + b2 - lv[e]) : 0.f;
             ds[e] = pr[e] * (__uint_as_float(dr[c4 * 8 + e]) - dv[e]);
           }
-          uint4 pv, dsv;
-          pv.x = pack_bf16x2(pr[0], pr[1]);
-          pv.y = pack_bf16x2(pr[2], pr[3]);
-          pv.z = pack_bf16x2(pr[4], pr[5]);
-          pv.w = pack_bf16x2(pr[6], pr[7]);
-          dsv.x = pack_bf16x2(ds[0], ds[1]);
-          dsv.y = pack_bf16x2(ds[2], ds[3]);
-          dsv.z = pack_bf16x2(ds[4], ds[5]);
-          dsv.w = pack_bf16x2(ds[6], ds[7]);
-          const int sw = (c ^ (row & 7)) << 4; // 128-byte swizzle within the 8-row atom
-          *reinterpret_cast<uint4*>(prow + sw) = pv;
-          *reinterpret_cast<uint4*>(drow + sw) = dsv;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            pk[c4 * 4 + e] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
+            dk[c4 * 4 + e] = pack_bf16x2(ds[2 * e], ds[2 * e + 1]);
+          }
         }
+        // over columns this thread has already read (half 0: S^T 0-15 of 0-31; half 1:
+        // 16-31, read in half 0); the loads of half 1 read columns 32-63
+        tmem_st16(lane_base + 128 * g + 16 * half, pk);
+        tmem_st16(lane_base + 128 * g + 64 + 16 * half, dk);
       }
-      fence_proxy_async_smem();                // generic writes -> tensor-core reads
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[g]);
     }

@@ -321,21 +321,22 @@ def test_model_detects_a_broken_release_count():
 
 def simulate_dkv(seed, T, early_next=False):
     """The key-stationary dK/dV pass (csrc/bwd_tc.cu): one key tile per CTA, its T
-    query tiles through a two-stage ring, compute groups taking alternate tiles, Pᵀ
-    and dSᵀ in one shared-memory buffer per group, the next Sᵀ/dPᵀ of a group issued
-    once its products have read the current ones."""
+    query tiles through a two-stage ring, compute groups taking alternate tiles.  A
+    group writes Pᵀ and dSᵀ as bf16 over the TMEM columns of its Sᵀ and dPᵀ, and the
+    dV / dK products read them from there; the group's next Sᵀ/dPᵀ is issued once
+    those products are issued, so the in-order tensor pipe writes the columns only
+    after the products have read them."""
     rng = random.Random(seed)
     a_full = Barrier("a_full", 1)
     r_full = [Barrier(f"r_full{s}", 1) for s in range(2)]
     r_empty = [Barrier(f"r_empty{s}", 1) for s in range(2)]
     s_full = [Barrier(f"s_full{g}", 1) for g in range(2)]
     p_full = [Barrier(f"p_full{g}", 128) for g in range(2)]
-    pds_free = [Barrier(f"pds_free{g}", 1) for g in range(2)]
     acc_full = Barrier("acc_full", 1)
     pipe = []
     pending = {}
     loads = [0, 0]
-    pbuf_uses = [0, 0]
+    tm_uses = [0, 0]                        # P^T / dS^T written into each group's columns
     consumed = [0, 0]                       # tiles whose S^T/dP^T each group has read
 
     def mma(key):
@@ -361,6 +362,7 @@ def simulate_dkv(seed, T, early_next=False):
             if consumed[g] < (j >> 1):
                 raise ProtocolError(f"S^T of tile {j} written before group {g} read tile {j - 2}")
             mma(("ring", st, loads[st] - 1))
+            pipe.append(("write_tm", g))       # S^T / dP^T land in the group's columns
             pipe.append(("commit", s_full[g]))
 
         yield from wait(a_full, 0)
@@ -373,8 +375,7 @@ def simulate_dkv(seed, T, early_next=False):
                 yield from issue_s(j + 2)
             yield from wait(p_full[g], j >> 1)
             mma(("ring", st, loads[st] - 1))
-            mma(("pbuf", g, pbuf_uses[g] - 1))
-            pipe.append(("commit", pds_free[g]))
+            mma(("tm", g, tm_uses[g] - 1))       # dV, dK read P^T, dS^T from TMEM
             pipe.append(("commit", r_empty[st]))
             if j + 2 < T and not early_next:
                 yield from issue_s(j + 2)
@@ -385,11 +386,9 @@ def simulate_dkv(seed, T, early_next=False):
         for j in range(g, T, 2):
             yield from wait(s_full[g], nt)
             consumed[g] += 1
-            if nt > 0:
-                yield from wait(pds_free[g], nt - 1)
-            if pending.get(("pbuf", g, pbuf_uses[g] - 1), 0):
-                raise ProtocolError(f"P/dS buffer {g} rewritten under a pending reader")
-            pbuf_uses[g] += 1
+            if pending.get(("tm", g, tm_uses[g] - 1), 0):
+                raise ProtocolError(f"P^T of group {g} rewritten under a pending product")
+            tm_uses[g] += 1
             yield
             for _ in range(128):
                 p_full[g].arrive()
@@ -407,6 +406,9 @@ def simulate_dkv(seed, T, early_next=False):
             k, val = pipe.pop(0)
             if k == "mma":
                 pending[val] -= 1
+            elif k == "write_tm":
+                if pending.get(("tm", val, tm_uses[val] - 1), 0):
+                    raise ProtocolError(f"S^T of group {val} written under a pending product")
             else:
                 val.arrive()
             stalls = 0
