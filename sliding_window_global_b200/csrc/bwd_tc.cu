@@ -523,8 +523,11 @@ struct KCfg {
   static constexpr uint32_t kQBytes = kQT * D * 2u;        // a 64 x D tile
   static constexpr uint32_t kQSub = kQT * 128u;            // 64-row x 128-byte sub-tile
   static constexpr uint32_t kK = 0, kV = kKVBytes;
+  // Q / dO ring: a tile's load starts when the products of the tile NR earlier are
+  // done, so with NR > 2 the next S^T of a group need not wait for its load
+  static constexpr int NR = 4;
   static constexpr uint32_t kRing = 2 * kKVBytes;          // stage s: Q at kRing + 2 s Q, dO after
-  static constexpr uint32_t kFlags = kRing + 4 * kQBytes;  // random job: per-pair flags (set-up only)
+  static constexpr uint32_t kFlags = kRing + 2 * NR * kQBytes;  // random job: per-pair flags (set-up only)
   // [group][buffer][lse2 64 | delta 64 | position 64 | row fact 64] (floats, ints)
   static constexpr uint32_t kStg = kFlags + kMaxRandList * 4;
   static constexpr uint32_t kList = kStg + 2 * 2 * 256 * 4;  // random job: query blocks drawing the key block
@@ -563,12 +566,13 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-  uint64_t* a_full = bars;          // K and V loaded
-  uint64_t* r_full = bars + 1;      // [2] Q, dO of a ring stage loaded
-  uint64_t* r_empty = bars + 3;     // [2] that stage's products are done
-  uint64_t* s_full = bars + 5;      // [2] S^T, dP^T of group g in TMEM
-  uint64_t* p_full = bars + 7;      // [2] group g wrote P^T, dS^T (and read its TMEM), 128 arrivals
-  uint64_t* acc_full = bars + 9;    // dK, dV complete
+  constexpr int NR = C::NR;
+  uint64_t* a_full = bars;               // K and V loaded
+  uint64_t* r_full = bars + 1;           // [NR] Q, dO of a ring stage loaded
+  uint64_t* r_empty = r_full + NR;       // [NR] that stage's products are done
+  uint64_t* s_full = r_empty + NR;       // [2] S^T, dP^T of group g in TMEM
+  uint64_t* p_full = s_full + 2;         // [2] group g wrote P^T, dS^T (and read its TMEM), 128 arrivals
+  uint64_t* acc_full = p_full + 2;       // dK, dV complete
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ int sCount;
@@ -675,11 +679,13 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
 
   if (tid == 0) {
     mbar_init(a_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NR; ++s) {
       mbar_init(&r_full[s], 1);
       mbar_init(&r_empty[s], 1);
-      mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
+    }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&s_full[g], 1);
+      mbar_init(&p_full[g], 128);
     }
     mbar_init(acc_full, 1);
     abort_flag = 0;
@@ -705,8 +711,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
       load_tile<D>(smem + C::kK, km, a_full, u.u0, kz);
       load_tile<D>(smem + C::kV, vm, a_full, u.u0, kz);
       for (int j = 0; j < T; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !mbar_wait_bounded(&r_empty[st], ((j >> 1) - 1) & 1, abort_v, kWaitLimitNs)) break;
+        const int st = j % NR;
+        if (j >= NR && !mbar_wait_bounded(&r_empty[st], ((j / NR) - 1) & 1, abort_v, kWaitLimitNs)) break;
         const QTile qt = qtile(j);
         const int qz = u.b * p.Hq + qt.head;
         const CUtensorMap* qm = qt.src == 0 ? &p.mq64[u.cls] : qt.src == 1 ? &p.mgq64 : &p.mq64[p.dense_class];
@@ -727,8 +733,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
       const uint32_t ka = smem_u32(smem + C::kK), va = smem_u32(smem + C::kV);
       // S^T = K Q^T and dP^T = V dO^T of tile j into group (j & 1)'s columns
       auto issue_s = [&](int j) -> bool {
-        const int st = j & 1, g = j & 1;
-        if (!mbar_wait_bounded(&r_full[st], (j >> 1) & 1, abort_v, kWaitLimitNs)) return false;
+        const int st = j % NR, g = j & 1;
+        if (!mbar_wait_bounded(&r_full[st], (j / NR) & 1, abort_v, kWaitLimitNs)) return false;
         tc_fence_after();
         const uint32_t qb = smem_u32(smem + C::kRing + st * 2 * C::kQBytes);
 #pragma unroll
@@ -747,7 +753,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
       if (ok) ok = issue_s(0);
       if (ok && T > 1) ok = issue_s(1);
       for (int j = 0; ok && j < T; ++j) {
-        const int g = j & 1, st = j & 1;
+        const int g = j & 1, st = j % NR;
         if (!mbar_wait_bounded(&p_full[g], (j >> 1) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
         const uint32_t qb = smem_u32(smem + C::kRing + st * 2 * C::kQBytes);

@@ -319,23 +319,23 @@ def test_model_detects_a_broken_release_count():
         Barrier.__init__ = orig
 
 
-def simulate_dkv(seed, T, early_next=False):
+def simulate_dkv(seed, T, early_next=False, NR=4):
     """The key-stationary dK/dV pass (csrc/bwd_tc.cu): one key tile per CTA, its T
-    query tiles through a two-stage ring, compute groups taking alternate tiles.  A
+    query tiles through an NR-stage ring, compute groups taking alternate tiles.  A
     group writes Pᵀ and dSᵀ as bf16 over the TMEM columns of its Sᵀ and dPᵀ, and the
     dV / dK products read them from there; the group's next Sᵀ/dPᵀ is issued once
     those products are issued, so the in-order tensor pipe writes the columns only
     after the products have read them."""
     rng = random.Random(seed)
     a_full = Barrier("a_full", 1)
-    r_full = [Barrier(f"r_full{s}", 1) for s in range(2)]
-    r_empty = [Barrier(f"r_empty{s}", 1) for s in range(2)]
+    r_full = [Barrier(f"r_full{s}", 1) for s in range(NR)]
+    r_empty = [Barrier(f"r_empty{s}", 1) for s in range(NR)]
     s_full = [Barrier(f"s_full{g}", 1) for g in range(2)]
     p_full = [Barrier(f"p_full{g}", 128) for g in range(2)]
     acc_full = Barrier("acc_full", 1)
     pipe = []
     pending = {}
-    loads = [0, 0]
+    loads = [0] * NR
     tm_uses = [0, 0]                        # P^T / dS^T written into each group's columns
     consumed = [0, 0]                       # tiles whose S^T/dP^T each group has read
 
@@ -346,9 +346,9 @@ def simulate_dkv(seed, T, early_next=False):
     def producer():
         a_full.arrive()
         for j in range(T):
-            st = j & 1
-            if j >= 2:
-                yield from wait(r_empty[st], (j >> 1) - 1)
+            st = j % NR
+            if j >= NR:
+                yield from wait(r_empty[st], j // NR - 1)
             if pending.get(("ring", st, loads[st] - 1), 0):
                 raise ProtocolError(f"ring slot {st} refilled under a pending reader")
             loads[st] += 1
@@ -357,8 +357,8 @@ def simulate_dkv(seed, T, early_next=False):
 
     def issuer():
         def issue_s(j):
-            st, g = j & 1, j & 1
-            yield from wait(r_full[st], j >> 1)
+            st, g = j % NR, j & 1
+            yield from wait(r_full[st], j // NR)
             if consumed[g] < (j >> 1):
                 raise ProtocolError(f"S^T of tile {j} written before group {g} read tile {j - 2}")
             mma(("ring", st, loads[st] - 1))
@@ -370,7 +370,7 @@ def simulate_dkv(seed, T, early_next=False):
         if T > 1:
             yield from issue_s(1)
         for j in range(T):
-            g = st = j & 1
+            g, st = j & 1, j % NR
             if early_next and j + 2 < T:         # planted mistake: before the group read S(j)
                 yield from issue_s(j + 2)
             yield from wait(p_full[g], j >> 1)
@@ -423,10 +423,11 @@ def simulate_dkv(seed, T, early_next=False):
             raise ProtocolError("deadlock: no agent can make progress")
 
 
+@pytest.mark.parametrize("NR", [2, 4])
 @pytest.mark.parametrize("T", [1, 2, 3, 4, 7, 12])
-def test_dkv_pass_protocol_random_schedules(T):
+def test_dkv_pass_protocol_random_schedules(T, NR):
     for seed in range(200):
-        simulate_dkv(seed, T)
+        simulate_dkv(seed, T, NR=NR)
 
 
 def test_dkv_model_detects_an_early_next_product():
