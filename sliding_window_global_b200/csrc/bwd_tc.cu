@@ -40,13 +40,15 @@ constexpr float kBLog2e = 1.4426950408889634f;
 template <int D>
 struct BCfg {
   static constexpr uint32_t kTileBytes = 128u * D * 2u;
-  // a stationary pair of tiles, then a two-stage ring of tile pairs
+  // the stationary Q and dO tiles, then a ring of K tiles and a ring of V tiles.  V is
+  // read only by dP and freed early; K, read by S and by dQ, gets one stage more, so
+  // the load of K(j+2) starts while dQ(j) still runs
+  static constexpr int NK = 3, NV = 2;
   static constexpr uint32_t kStat0 = 0;
   static constexpr uint32_t kStat1 = kTileBytes;
-  static constexpr uint32_t kRing = 2 * kTileBytes;   // stage s: first tile at kRing + 2 s T
-  static constexpr uint32_t kStage = 512;             // lse / Delta staging (dKV): 2 x 2 x 128 floats
-  static constexpr uint32_t kStageOff = kRing + 4 * kTileBytes;
-  static constexpr uint32_t kBarOff = kStageOff + 4 * kStage * 4;
+  static constexpr uint32_t kKRing = 2 * kTileBytes;
+  static constexpr uint32_t kVRing = kKRing + NK * kTileBytes;
+  static constexpr uint32_t kBarOff = kVRing + NV * kTileBytes;
   static constexpr uint32_t kSmemBytes = kBarOff + 16 * 8 + 1024;
   static constexpr uint32_t kTmemCols = 512;
   // TMEM columns (dQ pass): S of even key tiles 0-127 and of odd ones 384-511 (dS written
@@ -54,6 +56,9 @@ struct BCfg {
   static constexpr uint32_t kS = 0, kDP = 128, kAcc0 = 256, kS1 = 384;
   __host__ __device__ static constexpr uint32_t s_buf(int j) { return (j & 1) ? kS1 : kS; }
 };
+
+// dynamic shared memory plus the kernel's static arrays (sGpos, TMEM slot, abort flag)
+static_assert(BCfg<128>::kSmemBytes + kTile * 4 + 16 <= 227 * 1024, "shared memory of the dQ pass");
 
 // TMA load of one 128 x D bf16 tile (two 64-column boxes when D = 128).
 template <int D>
@@ -184,16 +189,19 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  constexpr int NK = C::NK, NV = C::NV;
   uint64_t* a_full = bars;          // Q and dO loaded
-  uint64_t* r_full = bars + 1;      // [2] K, V of a stage loaded
-  uint64_t* r_empty = bars + 3;     // [2] the stage's last MMA completed
-  uint64_t* s_full = bars + 5;      // S and dP in TMEM
-  uint64_t* ds_full = bars + 9;     // [2] dS of even / odd key tiles written (128 arrivals): with
+  uint64_t* s_full = bars + 1;      // S and dP in TMEM
+  uint64_t* acc_full = bars + 2;    // dQ complete
+  uint64_t* dp_read = bars + 3;     // dP read into registers (128 arrivals): the next dP may be written
+  uint64_t* ds_full = bars + 4;     // [2] dS of even / odd key tiles written (128 arrivals): with
                                     // S and dP of tile j+1 issued before the wait for dS(j), the
                                     // compute warps may finish tile j+1 first; one barrier per parity
                                     // keeps every wait at most one phase behind
-  uint64_t* acc_full = bars + 7;    // dQ complete
-  uint64_t* dp_read = bars + 8;     // dP read into registers (128 arrivals): the next dP may be written
+  uint64_t* k_full = bars + 6;      // [NK] K tile of a stage loaded
+  uint64_t* k_empty = k_full + NK;  // [NK] its dQ product completed
+  uint64_t* v_full = k_empty + NK;  // [NV] V tile of a stage loaded
+  uint64_t* v_empty = v_full + NV;  // [NV] its dP product completed
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ int sGpos[kTile];      // key positions of the current global-column tile
@@ -239,9 +247,13 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
 
   if (tid == 0) {
     mbar_init(a_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&r_full[s], 1);
-      mbar_init(&r_empty[s], 1);
+    for (int s = 0; s < NK; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(&ds_full[0], 128);
@@ -271,8 +283,8 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
       load_tile<D>(smem + C::kStat0, GROWS ? &p.mgq : &p.mq[u.cls], a_full, u.u0, qz);
       load_tile<D>(smem + C::kStat1, GROWS ? &p.mgdo : &p.mdo[u.cls], a_full, u.u0, qz);
       for (int j = 0; j < T; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !mbar_wait_bounded(&r_empty[st], ((j >> 1) - 1) & 1, abort_v, kWaitLimitNs)) break;
+        const int sk = j % NK, sv = j % NV;
+        if (j >= NK && !mbar_wait_bounded(&k_empty[sk], ((j / NK) - 1) & 1, abort_v, kWaitLimitNs)) break;
         const CUtensorMap *mk = &p.mk[u.cls], *mv = &p.mv[u.cls];
         int y = GROWS ? j * kTile : klo_t + j * kTile;
         if (X && j >= nband) {
@@ -285,10 +297,11 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
             y = __ldg(p.rand_blocks + (((size_t)u.b * p.Hq + u.h) * nqb + qb) * p.num_rand + t) * kTile;
           }
         }
-        uint8_t* dst = smem + C::kRing + st * 2 * C::kTileBytes;
-        mbar_arrive_expect_tx(&r_full[st], 2 * C::kTileBytes);
-        load_tile<D>(dst, mk, &r_full[st], y, kz);
-        load_tile<D>(dst + C::kTileBytes, mv, &r_full[st], y, kz);
+        mbar_arrive_expect_tx(&k_full[sk], C::kTileBytes);
+        load_tile<D>(smem + C::kKRing + sk * C::kTileBytes, mk, &k_full[sk], y, kz);
+        if (j >= NV && !mbar_wait_bounded(&v_empty[sv], ((j / NV) - 1) & 1, abort_v, kWaitLimitNs)) break;
+        mbar_arrive_expect_tx(&v_full[sv], C::kTileBytes);
+        load_tile<D>(smem + C::kVRing + sv * C::kTileBytes, mv, &v_full[sv], y, kz);
       }
     }
   } else if (warp == 5) {
@@ -299,33 +312,37 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
       // order (MMAs complete in order): a new S goes into the buffer whose dS the
       // previous dQ product read; a new dP after dp_read.
       const uint32_t qa = smem_u32(smem + C::kStat0), da = smem_u32(smem + C::kStat1);
-      auto stage = [&](int j) { return smem_u32(smem + C::kRing + (j & 1) * 2 * C::kTileBytes); };
+      auto kstage = [&](int j) { return smem_u32(smem + C::kKRing + (j % NK) * C::kTileBytes); };
       auto issue_s = [&](int j) -> bool {           // S(j) = Q K(j)^T
-        if (!mbar_wait_bounded(&r_full[j & 1], (j >> 1) & 1, abort_v, kWaitLimitNs)) return false;
+        if (!mbar_wait_bounded(&k_full[j % NK], (j / NK) & 1, abort_v, kWaitLimitNs)) return false;
         tc_fence_after();
-        mma_abt<D>(tmem + C::s_buf(j), qa, stage(j));
+        mma_abt<D>(tmem + C::s_buf(j), qa, kstage(j));
+        return true;
+      };
+      auto issue_dp = [&](int j) -> bool {          // dP(j) = dO V(j)^T; V(j) is then free
+        if (!mbar_wait_bounded(&v_full[j % NV], (j / NV) & 1, abort_v, kWaitLimitNs)) return false;
+        tc_fence_after();
+        mma_abt<D>(tmem + C::kDP, da, smem_u32(smem + C::kVRing + (j % NV) * C::kTileBytes));
+        umma_commit(&v_empty[j % NV]);
         return true;
       };
       bool ok = mbar_wait_bounded(a_full, 0, abort_v, kWaitLimitNs);
       if (ok) ok = issue_s(0);
-      if (ok) {
-        mma_abt<D>(tmem + C::kDP, da, stage(0) + C::kTileBytes);     // dP(0) = dO V(0)^T
-        umma_commit(s_full);
-      }
+      if (ok) ok = issue_dp(0);
+      if (ok) umma_commit(s_full);
       if (ok && T > 1) ok = issue_s(1);
       for (int j = 0; ok && j < T; ++j) {
         if (j + 1 < T) {
           // dP(j+1) once the compute warps hold dP(j) in registers
           if (!mbar_wait_bounded(dp_read, j & 1, abort_v, kWaitLimitNs)) break;
-          tc_fence_after();
-          mma_abt<D>(tmem + C::kDP, da, stage(j + 1) + C::kTileBytes);
+          if (!issue_dp(j + 1)) break;
           umma_commit(s_full);                       // S(j+1) and dP(j+1)
         }
         // dQ += dS(j) K(j), then the stage of tile j may be refilled
         if (!mbar_wait_bounded(&ds_full[j & 1], (j >> 1) & 1, abort_v, kWaitLimitNs)) break;
         tc_fence_after();
-        mma_px<D>(tmem + C::kAcc0, tmem + C::s_buf(j), stage(j), j > 0);
-        umma_commit(&r_empty[j & 1]);
+        mma_px<D>(tmem + C::kAcc0, tmem + C::s_buf(j), kstage(j), j > 0);
+        umma_commit(&k_empty[j % NK]);
         if (j == T - 1) umma_commit(acc_full);
         if (j + 2 < T) ok = issue_s(j + 2);           // into the buffer dQ(j) just read
       }

@@ -442,9 +442,10 @@ def test_dkv_model_detects_an_early_next_product():
     assert caught > 0
 
 
-def simulate_dq(seed, T, early_dp=False, early_s=False, per_parity=True):
+def simulate_dq(seed, T, early_dp=False, early_s=False, per_parity=True, NK=3, NV=2):
     """The query-stationary dQ pass (csrc/bwd_tc.cu): one query tile per CTA, its T key
-    tiles through a two-stage ring; S of tile j in TMEM buffer j & 1, dP in one buffer.
+    tiles' K through an NK-stage ring and V through an NV-stage ring (V is released
+    after dP, K after dQ); S of tile j in TMEM buffer j & 1, dP in one buffer.
     The issuer computes S(j+1) while the compute warps work on tile j, dP(j+1) once
     they hold dP(j) in registers (dp_read), and S(j+2) into the buffer dQ(j) has just
     read (in issue order).  MMAs complete in issue order.  Checked: the compute warps
@@ -454,15 +455,16 @@ def simulate_dq(seed, T, early_dp=False, early_s=False, per_parity=True):
     phases past the issuer's wait."""
     rng = random.Random(seed)
     a_full = Barrier("a_full", 1)
-    r_full = [Barrier(f"r_full{s}", 1) for s in range(2)]
-    r_empty = [Barrier(f"r_empty{s}", 1) for s in range(2)]
+    N = {"K": NK, "V": NV}
+    full = {x: [Barrier(f"{x}_full{s}", 1) for s in range(N[x])] for x in "KV"}
+    empty = {x: [Barrier(f"{x}_empty{s}", 1) for s in range(N[x])] for x in "KV"}
     s_full = Barrier("s_full", 1)
     dp_read = Barrier("dp_read", 128)
     ds_full = [Barrier(f"ds_full{x}", 128) for x in range(2)]   # one per key-tile parity
     acc_full = Barrier("acc_full", 1)
     pipe = []
     pending = {}
-    loads = [0, 0]
+    loads = {"K": [0] * NK, "V": [0] * NV}
     sbuf = [None, None]                     # what each S buffer holds: ("S", j) or ("dS", j)
     dpbuf = [None]                          # the tile whose dP the dP buffer holds
 
@@ -473,28 +475,34 @@ def simulate_dq(seed, T, early_dp=False, early_s=False, per_parity=True):
     def producer():
         a_full.arrive()
         for j in range(T):
-            st = j & 1
-            if j >= 2:
-                yield from wait(r_empty[st], (j >> 1) - 1)
-            if pending.get(("ring", st, loads[st] - 1), 0):
-                raise ProtocolError(f"ring slot {st} refilled under a pending reader")
-            loads[st] += 1
-            yield
-            r_full[st].arrive()
+            for x in "KV":
+                st = j % N[x]
+                if j >= N[x]:
+                    yield from wait(empty[x][st], j // N[x] - 1)
+                if pending.get((x, st, loads[x][st] - 1), 0):
+                    raise ProtocolError(f"{x} slot {st} refilled under a pending reader")
+                loads[x][st] += 1
+                yield
+                full[x][st].arrive()
+
+    def ring_read(x, j):
+        mma_read((x, j % N[x], loads[x][j % N[x]] - 1))
 
     def issuer():
         def issue_s(j):
-            yield from wait(r_full[j & 1], j >> 1)
-            mma_read(("ring", j & 1, loads[j & 1] - 1))
+            yield from wait(full["K"][j % NK], j // NK)
+            ring_read("K", j)
             pipe.append(("write_s", j))
 
         def issue_dp(j):
-            mma_read(("ring", j & 1, loads[j & 1] - 1))
+            yield from wait(full["V"][j % NV], j // NV)
+            ring_read("V", j)
             pipe.append(("write_dp", j))
+            pipe.append(("commit", empty["V"][j % NV]))
 
         yield from wait(a_full, 0)
         yield from issue_s(0)
-        issue_dp(0)
+        yield from issue_dp(0)
         pipe.append(("commit", s_full))
         if T > 1:
             yield from issue_s(1)
@@ -502,14 +510,14 @@ def simulate_dq(seed, T, early_dp=False, early_s=False, per_parity=True):
             if j + 1 < T:
                 if not early_dp:
                     yield from wait(dp_read, j)
-                issue_dp(j + 1)
+                yield from issue_dp(j + 1)
                 pipe.append(("commit", s_full))
             yield from wait(ds_full[j & 1] if per_parity else ds_full[0], (j >> 1) if per_parity else j)
             if early_s and j + 2 < T:              # planted: S(j+2) before dQ(j) read dS(j)
                 yield from issue_s(j + 2)
-            mma_read(("ring", j & 1, loads[j & 1] - 1))
+            ring_read("K", j)
             pipe.append(("read_ds", j))
-            pipe.append(("commit", r_empty[j & 1]))
+            pipe.append(("commit", empty["K"][j % NK]))
             if j == T - 1:
                 pipe.append(("commit", acc_full))
             if j + 2 < T and not early_s:
@@ -563,10 +571,11 @@ def simulate_dq(seed, T, early_dp=False, early_s=False, per_parity=True):
             raise ProtocolError("deadlock: no agent can make progress")
 
 
+@pytest.mark.parametrize("rings", [(2, 2), (3, 2)], ids=["kv2", "k3_v2"])
 @pytest.mark.parametrize("T", [1, 2, 3, 4, 5, 9])
-def test_dq_pass_protocol_random_schedules(T):
+def test_dq_pass_protocol_random_schedules(T, rings):
     for seed in range(200):
-        simulate_dq(seed, T)
+        simulate_dq(seed, T, NK=rings[0], NV=rings[1])
 
 
 def test_dq_model_detects_a_single_ds_barrier():
