@@ -27,6 +27,7 @@
 // lane t), warp 4 issues the TMA loads, warp 5 allocates TMEM and issues the MMAs;
 // the dK/dV pass (320 threads) has two compute warpgroups, then the same two.
 #include "ptx.cuh"
+#include "softmax_math.cuh"
 #include "swa_kernels.h"
 #include "bwd_kernels.h"
 
@@ -429,6 +430,13 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
       tc_fence_before();
       mbar_arrive(dp_read);
       const uint32_t sb = lane_base + C::s_buf(j);
+      // Interior band tile: every key of the tile is in the window of every row of this
+      // warp, so no element needs a mask, and pairs of columns take one packed f32x2
+      // instruction per step.
+      // (the condition is warp-uniform outside the vote: kind depends only on j)
+      const bool interior = !GROWS && (!X || kind == 0) &&
+                            __all_sync(0xffffffffu, (!X || !lrow) && lo_t <= 0 && hi_t >= kTile);
+      const float nl2 = -lse2, nd = -delta;
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t sr[32];
@@ -436,6 +444,20 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
         tmem_wait_ld_dep(sr);
         const uint32_t* dr = dpr + ch * 32;
         uint32_t pk[16];
+        if (interior) {
+#pragma unroll
+          for (int q = 0; q < 32; q += 2) {
+            float a0, a1, t0, t1, d0, d1;
+            ffma2(a0, a1, __uint_as_float(sr[q]), __uint_as_float(sr[q + 1]), sl2, sl2, nl2, nl2);
+            a0 = ex2_approx(a0);
+            a1 = ex2_approx(a1);
+            fadd2(t0, t1, __uint_as_float(dr[q]), __uint_as_float(dr[q + 1]), nd, nd);
+            ffma2(d0, d1, a0, a1, t0, t1, 0.f, 0.f);
+            pk[q / 2] = pack_bf16x2(d0, d1);
+          }
+          tmem_st16(sb + ch * 16, pk);
+          continue;
+        }
 #pragma unroll
         for (int q = 0; q < 32; q += 2) {
           float ds[2];
@@ -805,8 +827,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
     bool ok = true;
     int nt = 0;                               // tiles handled by this group
     for (int j = g; j < T; j += 2, ++nt) {
-      // per query row of the tile: lse2 (+inf excludes the row: padded, missing, or
-      // outside the job's rows), Delta, and the row's position or block facts
+      // per query row of the tile: -lse2 (-inf excludes the row: padded, missing, or
+      // outside the job's rows), -Delta, and the row's position or block facts
       const QTile qt = qtile(j);
       float* stg = reinterpret_cast<float*>(smem + C::kStg) + (g * 2 + (nt & 1)) * 256;
       int* stgi = reinterpret_cast<int*>(stg + 2 * kQT);   // [64] positions, [64] extra
@@ -834,8 +856,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
           l2 = p.lse[pr] * kBLog2e;
           dl = p.delta[pr];
         }
-        stg[row] = l2;
-        stg[kQT + row] = dl;
+        stg[row] = -l2;                          // negated: the products below add them
+        stg[kQT + row] = -dl;
         stgi[row] = qp;
         stgi[kQT + row] = ex;
       }
@@ -862,6 +884,16 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
       if (!mbar_wait_bounded(&s_full[g], nt & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
       tc_fence_after();
       const int d0 = qt.y - uk;                // query - key offset of column 0 (band, class coordinates)
+      // Interior tile of the band job: every (key, query) pair of this warp's keys is in
+      // the band, so no element needs a mask (query rows that do not count have
+      // -lse2 = -inf and give p = 0 by themselves).  Pairs of columns then take one
+      // packed f32x2 instruction per step.
+      bool interior = false;
+      if (JOB == kJobBand) {
+        const bool in = key_valid && (p.causal ? (d0 >= 0 && d0 + kQT - 1 <= u.r)
+                                               : (d0 >= -u.r && d0 + kQT - 1 <= u.r));
+        interior = __all_sync(0xffffffffu, in);
+      }
 #pragma unroll
       for (int half = 0; half < 2; ++half) {   // 32 query columns at a time
         uint32_t sr[32], dr[32];
@@ -877,32 +909,45 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
           const float4 lb = *reinterpret_cast<const float4*>(stg + c * 8 + 4);
           const float4 da = *reinterpret_cast<const float4*>(stg + kQT + c * 8);
           const float4 db = *reinterpret_cast<const float4*>(stg + kQT + c * 8 + 4);
-          const float lv[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
-          const float dv[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+          const float lv[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};   // -lse2
+          const float dv[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};   // -Delta
           float pr[8], ds[8];
+          if (interior) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            bool allowed;
-            float b2 = 0.f;
-            if (JOB == kJobBand || (JOB == kJobBandX && qt.src == 0)) {
-              const int off = d0 + c * 8 + e;
-              const bool inband = p.causal ? (off >= 0 && off <= u.r) : (off >= -u.r && off <= u.r);
-              allowed = key_valid && inband;
-              if (JOB == kJobBandX && lrow && allowed && stgi[kQT + c * 8 + e])
-                b2 = __ldg(lrow - u.d * off) * kBLog2e;
-            } else if (JOB == kJobBandX) {
-              // a global query row: keys outside its window (inside it the band tile counts)
-              allowed = key_valid && !in_window(stgi[c * 8 + e], kpos, rd, u.d, p.causal);
-            } else if (JOB == kJobGlobalKeys) {
-              allowed = key_valid && !key_in_rand && !in_window(stgi[c * 8 + e], kpos, rd, u.d, p.causal);
-            } else if (JOB == kJobSide) {
-              allowed = key_valid;
-              if (sbias) b2 = __ldg(sbias - stgi[kQT + c * 8 + e]) * kBLog2e;
-            } else {
-              allowed = key_valid && !in_window(stgi[c * 8 + e], kpos, rd, 1, p.causal);
+            for (int e = 0; e < 8; e += 2) {
+              float a0, a1, t0, t1;
+              ffma2(a0, a1, __uint_as_float(sr[c4 * 8 + e]), __uint_as_float(sr[c4 * 8 + e + 1]), sl2, sl2,
+                    lv[e], lv[e + 1]);
+              pr[e] = ex2_approx(a0);
+              pr[e + 1] = ex2_approx(a1);
+              fadd2(t0, t1, __uint_as_float(dr[c4 * 8 + e]), __uint_as_float(dr[c4 * 8 + e + 1]), dv[e], dv[e + 1]);
+              ffma2(ds[e], ds[e + 1], pr[e], pr[e + 1], t0, t1, 0.f, 0.f);
             }
-            pr[e] = allowed ? ex2_approx(__uint_as_float(sr[c4 * 8 + e]) * sl2 + b2 - lv[e]) : 0.f;
-            ds[e] = pr[e] * (__uint_as_float(dr[c4 * 8 + e]) - dv[e]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              bool allowed;
+              float b2 = 0.f;
+              if (JOB == kJobBand || (JOB == kJobBandX && qt.src == 0)) {
+                const int off = d0 + c * 8 + e;
+                const bool inband = p.causal ? (off >= 0 && off <= u.r) : (off >= -u.r && off <= u.r);
+                allowed = key_valid && inband;
+                if (JOB == kJobBandX && lrow && allowed && stgi[kQT + c * 8 + e])
+                  b2 = __ldg(lrow - u.d * off) * kBLog2e;
+              } else if (JOB == kJobBandX) {
+                // a global query row: keys outside its window (inside it the band tile counts)
+                allowed = key_valid && !in_window(stgi[c * 8 + e], kpos, rd, u.d, p.causal);
+              } else if (JOB == kJobGlobalKeys) {
+                allowed = key_valid && !key_in_rand && !in_window(stgi[c * 8 + e], kpos, rd, u.d, p.causal);
+              } else if (JOB == kJobSide) {
+                allowed = key_valid;
+                if (sbias) b2 = __ldg(sbias - stgi[kQT + c * 8 + e]) * kBLog2e;
+              } else {
+                allowed = key_valid && !in_window(stgi[c * 8 + e], kpos, rd, 1, p.causal);
+              }
+              pr[e] = allowed ? ex2_approx(__uint_as_float(sr[c4 * 8 + e]) * sl2 + b2 + lv[e]) : 0.f;
+              ds[e] = pr[e] * (__uint_as_float(dr[c4 * 8 + e]) + dv[e]);
+            }
           }
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
