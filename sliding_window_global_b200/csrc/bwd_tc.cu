@@ -26,6 +26,8 @@
 // Warp roles of the dQ pass (192 threads): warps 0-3 compute (thread t owns TMEM
 // lane t), warp 4 issues the TMA loads, warp 5 allocates TMEM and issues the MMAs;
 // the dK/dV pass (320 threads) has two compute warpgroups, then the same two.
+#include <type_traits>
+
 #include "ptx.cuh"
 #include "softmax_math.cuh"
 #include "swa_kernels.h"
@@ -133,18 +135,49 @@ __device__ __forceinline__ size_t pos_row(const BwdParams& p, const BUnit& u, in
 }
 
 // ------------------------------------------------------------------ Delta
+// One warp per two rows: every lane loads its D/32 elements of both rows of out and
+// dout with one vector load each before any arithmetic, so four loads per lane are in
+// flight (the pass is bound by HBM bandwidth).
+template <int D>
 __global__ void bwd_delta_kernel(const __grid_constant__ BwdParams p) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  using V = typename std::conditional<D == 128, uint2, uint32_t>::type;   // D / 32 bf16
+  const size_t warp = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const size_t rows = (size_t)p.B * p.Hq * p.n;
-  if ((size_t)warp >= rows) return;
-  const __nv_bfloat16* o = static_cast<const __nv_bfloat16*>(p.out) + (size_t)warp * p.D;
-  const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(p.dout) + (size_t)warp * p.D;
-  float acc = 0.f;
-  for (int x = lane; x < p.D; x += 32) acc = fmaf(__bfloat162float(o[x]), __bfloat162float(g[x]), acc);
+  const size_t r0 = 2 * warp;
+  if (r0 >= rows) return;
+  const bool two = r0 + 1 < rows;
+  const V* o = reinterpret_cast<const V*>(static_cast<const __nv_bfloat16*>(p.out) + r0 * D) + lane;
+  const V* g = reinterpret_cast<const V*>(static_cast<const __nv_bfloat16*>(p.dout) + r0 * D) + lane;
+  constexpr int kPerRow = D / 64;                  // bf16 pairs per lane and row
+  V oa = __ldg(o), ga = __ldg(g), ob = oa, gb = ga;
+  if (two) {
+    ob = __ldg(o + 32);
+    gb = __ldg(g + 32);
+  }
+  float acc[2] = {0.f, 0.f};
+  const V ov[2] = {oa, ob}, gv[2] = {ga, gb};
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) p.delta[warp] = acc;
+  for (int r = 0; r < 2; ++r) {
+    const uint32_t* ow = reinterpret_cast<const uint32_t*>(&ov[r]);
+    const uint32_t* gw = reinterpret_cast<const uint32_t*>(&gv[r]);
+#pragma unroll
+    for (int e = 0; e < kPerRow; ++e) {
+      const float2 of = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ow[e]));
+      const float2 gf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[e]));
+      acc[r] = fmaf(of.x, gf.x, acc[r]);
+      acc[r] = fmaf(of.y, gf.y, acc[r]);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], off);
+    acc[1] += __shfl_xor_sync(0xffffffffu, acc[1], off);
+  }
+  if (lane == 0) {
+    p.delta[r0] = acc[0];
+    if (two) p.delta[r0 + 1] = acc[1];
+  }
 }
 
 // ------------------------------------------------------------------ shared facts
@@ -1043,8 +1076,10 @@ cudaError_t launch_kern(K kern, uint32_t smem, int grid, int threads, const BwdP
 
 cudaError_t launch_bwd_delta(const BwdParams& p, cudaStream_t s) {
   const size_t rows = (size_t)p.B * p.Hq * p.n;
-  const int blocks = (int)((rows * 32 + 255) / 256);
-  bwd_delta_kernel<<<blocks, 256, 0, s>>>(p);
+  const size_t warps = (rows + 1) / 2;
+  const int blocks = (int)((warps * 32 + 255) / 256);
+  if (p.D == 128) bwd_delta_kernel<128><<<blocks, 256, 0, s>>>(p);
+  else bwd_delta_kernel<64><<<blocks, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 
