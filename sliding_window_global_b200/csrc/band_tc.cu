@@ -543,9 +543,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int x0 = (kIssuers == 2) ? warp - 9 : 0;   // first tile of this issuer
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-      const uint32_t q_base = smem_u32(sQ);
-      const uint32_t k_base = smem_u32(sK);
-      const uint32_t v_base = smem_u32(sV);
+      // low descriptor words of tile buffer 0 / ring slot 0 (128-byte swizzle; V is
+      // read MN-major, its 64-column sub-tiles kSub apart); products add offsets
+      const uint32_t q_lo = sdesc_lo(smem_u32(sQ), 16);
+      const uint32_t k_lo = sdesc_lo(smem_u32(sK), 16);
+      const uint32_t v_lo = sdesc_lo(smem_u32(sV), kSub);
       int qwaits[kTilesPerIssuer] = {}, pwaits[kTilesPerIssuer] = {};
       int nqk[kTilesPerIssuer] = {};                    // QKs issued per tile buffer (kernel-wide)
       int kv = 0;
@@ -579,13 +581,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             return false;
           ++nqk[i];
           tc_fence_after();
-          const uint32_t qt = q_base + x * C::kTileBytes;
-          const uint32_t kt = k_base + (g % NS) * C::kTileBytes;
+          const uint32_t qd = q_lo + x * (C::kTileBytes >> 4);
+          const uint32_t kd = k_lo + (g % NS) * (C::kTileBytes >> 4);
+          const uint32_t sd = tmem + C::s_col(x);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
-            umma_ss(tmem + C::s_col(x), sdesc_sw128(qt + off, 16, 1024),
-                    sdesc_sw128(kt + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+            const uint32_t off = ((kk >> 2) * kSub + (kk & 3) * 32) >> 4;
+            umma_ss_lo(sd, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
           }
           umma_commit(&s_full[x]);
           if (j == last[i]) umma_commit(&q_empty[x]);   // Q_x may be refilled once this QK is done
@@ -631,7 +633,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             mbar_arrive(&kv_empty[st]);               // no MMA of this issuer reads the slot
             continue;
           }
-          const uint32_t vt = v_base + st * C::kTileBytes;
+          const uint32_t vd = v_lo + st * (C::kTileBytes >> 4);
 #pragma unroll
           for (int i = 0; i < kTilesPerIssuer; ++i) {
             const int x = x0 + i;
@@ -642,18 +644,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               // PV over it overlaps the exponentials of the second half
               if (!mbar_wait_bounded(&p_half[x], pwaits[i] & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
               tc_fence_after();
+              const uint32_t first = npv[i] > 0 ? 1u : 0u;
 #pragma unroll
               for (int kk = 0; kk < kTile / 32; ++kk)
-                umma_ts(tmem + C::o_col(x), tmem + C::p_col(x) + kk * 8,
-                        sdesc_sw128(vt + kk * 2048, kSub, 1024), idesc_pv, (npv[i] > 0 || kk > 0) ? 1u : 0u);
+                umma_ts_lo(tmem + C::o_col(x), tmem + C::p_col(x) + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv,
+                           kk > 0 ? 1u : first);
             }
             if (!mbar_wait_bounded(&p_full[x], pwaits[i] & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
             ++pwaits[i];
             tc_fence_after();
+            const uint32_t first = npv[i] > 0 ? 1u : 0u;
 #pragma unroll
             for (int kk = C::kSepP ? 0 : kTile / 32; kk < kTile / 16; ++kk)
-              umma_ts(tmem + C::o_col(x), tmem + C::p_col(x) + kk * 8,
-                      sdesc_sw128(vt + kk * 2048, kSub, 1024), idesc_pv, (npv[i] > 0 || kk > 0) ? 1u : 0u);
+              umma_ts_lo(tmem + C::o_col(x), tmem + C::p_col(x) + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv,
+                         kk > 0 ? 1u : first);
             ++npv[i];
             if (C::kSepP) umma_commit(&pv_done[x]);
             if (j == last[i]) umma_commit(&o_full[x]);
