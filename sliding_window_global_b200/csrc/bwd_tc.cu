@@ -75,10 +75,11 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, 
 template <int D>
 __device__ __forceinline__ void mma_abt(uint32_t dst, uint32_t a, uint32_t b) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
+  const uint32_t al = sdesc_lo(a, 16), bl = sdesc_lo(b, 16);   // descriptor low words
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * kBSub + (kk & 3) * 32;
-    umma_ss(dst, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(b + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+    const uint32_t off = ((kk >> 2) * kBSub + (kk & 3) * 32) >> 4;
+    umma_ss_lo(dst, al + off, bl + off, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -87,10 +88,10 @@ __device__ __forceinline__ void mma_abt(uint32_t dst, uint32_t a, uint32_t b) {
 template <int D>
 __device__ __forceinline__ void mma_px(uint32_t dst, uint32_t p_tmem, uint32_t x, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, true);
+  const uint32_t xl = sdesc_lo(x, kBSub);                      // descriptor low word
+  const uint32_t first = accumulate ? 1u : 0u;
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
-    umma_ts(dst, p_tmem + kk * 8, sdesc_sw128(x + kk * 2048, kBSub, 1024), idesc,
-            (accumulate || kk > 0) ? 1u : 0u);
+  for (int kk = 0; kk < 8; ++kk) umma_ts_lo(dst, p_tmem + kk * 8, xl + ((kk * 2048) >> 4), idesc, kk > 0 ? 1u : first);
 }
 
 struct BUnit {
@@ -802,21 +803,20 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
     if (lane == 0 && T > 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kQT, false);    // S^T, dP^T: 128 x 64
       constexpr uint32_t idesc_a = idesc_bf16_f32(128, D, true);       // dV, dK: 128 x D, B MN-major
-      const uint32_t ka = smem_u32(smem + C::kK), va = smem_u32(smem + C::kV);
+      const uint32_t ka = sdesc_lo(smem_u32(smem + C::kK), 16), va = sdesc_lo(smem_u32(smem + C::kV), 16);
       // S^T = K Q^T and dP^T = V dO^T of tile j into group (j & 1)'s columns
       auto issue_s = [&](int j) -> bool {
         const int st = j % NR, g = j & 1;
         if (!mbar_wait_bounded(&r_full[st], (j / NR) & 1, abort_v, kWaitLimitNs)) return false;
         tc_fence_after();
-        const uint32_t qb = smem_u32(smem + C::kRing + st * 2 * C::kQBytes);
+        const uint32_t qb = sdesc_lo(smem_u32(smem + C::kRing + st * 2 * C::kQBytes), 16);
+        const uint32_t db = qb + (C::kQBytes >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t offa = (kk >> 2) * kBSub + (kk & 3) * 32;
-          const uint32_t offb = (kk >> 2) * C::kQSub + (kk & 3) * 32;
-          umma_ss(tmem + 128 * g, sdesc_sw128(ka + offa, 16, 1024), sdesc_sw128(qb + offb, 16, 1024),
-                  idesc_s, kk > 0 ? 1u : 0u);
-          umma_ss(tmem + 128 * g + 64, sdesc_sw128(va + offa, 16, 1024),
-                  sdesc_sw128(qb + C::kQBytes + offb, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          const uint32_t offa = ((kk >> 2) * kBSub + (kk & 3) * 32) >> 4;
+          const uint32_t offb = ((kk >> 2) * C::kQSub + (kk & 3) * 32) >> 4;
+          umma_ss_lo(tmem + 128 * g, ka + offa, qb + offb, idesc_s, kk > 0 ? 1u : 0u);
+          umma_ss_lo(tmem + 128 * g + 64, va + offa, db + offb, idesc_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[g]);
         return true;
@@ -828,15 +828,17 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
         const int g = j & 1, st = j % NR;
         if (!mbar_wait_bounded(&p_full[g], (j >> 1) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t qb = smem_u32(smem + C::kRing + st * 2 * C::kQBytes);
+        const uint32_t qb = sdesc_lo(smem_u32(smem + C::kRing + st * 2 * C::kQBytes), C::kQSub);
+        const uint32_t db = qb + (C::kQBytes >> 4);
+        const uint32_t first = j > 0 ? 1u : 0u;
         // dV += P^T dO, dK += dS^T Q (A: 128 x 64 bf16 from the group's TMEM columns,
         // 16 queries = 8 columns per product; B: 64 x D MN-major from shared memory)
 #pragma unroll
         for (int kk = 0; kk < kQT / 16; ++kk) {
-          umma_ts(tmem + C::kAccV, tmem + 128 * g + kk * 8,
-                  sdesc_sw128(qb + C::kQBytes + kk * 2048, C::kQSub, 1024), idesc_a, (j > 0 || kk > 0) ? 1u : 0u);
-          umma_ts(tmem + C::kAccK, tmem + 128 * g + 64 + kk * 8,
-                  sdesc_sw128(qb + kk * 2048, C::kQSub, 1024), idesc_a, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_ts_lo(tmem + C::kAccV, tmem + 128 * g + kk * 8, db + ((kk * 2048) >> 4), idesc_a,
+                     kk > 0 ? 1u : first);
+          umma_ts_lo(tmem + C::kAccK, tmem + 128 * g + 64 + kk * 8, qb + ((kk * 2048) >> 4), idesc_a,
+                     kk > 0 ? 1u : first);
         }
         umma_commit(&r_empty[st]);
         // The group has read its S^T, dP^T of tile j; the next ones overwrite the same
