@@ -35,25 +35,29 @@ __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return
 
 // ------------------------------------------------------------------ gather
 // dst[bh, e, :] = src[bh', global_idx[b, e], :] for e < g, zeros for g <= e < gpad.
-__global__ void gather_rows_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
-                                   const int32_t* __restrict__ gidx, int H, int n, int g, int gpad,
+// Every array of a GatherSet in one launch: the index range is the concatenation
+// of the arrays' [B*H, gpad, row_vecs] ranges (job j ends at end[j]).
+__global__ void gather_rows_kernel(const GatherSet gs, const int32_t* __restrict__ gidx, int n, int g, int gpad,
                                    int row_vecs, int B) {
-  const size_t total = (size_t)B * H * gpad * row_vecs;
+  const size_t total = gs.end[gs.count - 1];
   for (size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x; t < total;
        t += (size_t)gridDim.x * blockDim.x) {
-    int x = (int)(t % row_vecs);
-    size_t r = t / row_vecs;
-    int e = (int)(r % gpad);
-    size_t bh = r / gpad;
-    int b = (int)(bh / H);
+    int jb = 0;
+    while (jb + 1 < gs.count && t >= gs.end[jb]) ++jb;
+    const size_t lt = t - (jb > 0 ? gs.end[jb - 1] : 0);
+    const int x = (int)(lt % row_vecs);
+    const size_t r = lt / row_vecs;
+    const int e = (int)(r % gpad);
+    const size_t bh = r / gpad;
+    const int b = (int)(bh / gs.heads[jb]);
     uint4 v = make_uint4(0, 0, 0, 0);
     if (e < g) {
       // a position outside the sequence (a broken precondition) gathers zeros
       // instead of reading out of bounds
       const int pos = gidx[(size_t)b * g + e];
-      if (pos >= 0 && pos < n) v = src[(bh * n + pos) * row_vecs + x];
+      if (pos >= 0 && pos < n) v = static_cast<const uint4*>(gs.src[jb])[(bh * n + pos) * row_vecs + x];
     }
-    dst[t] = v;
+    static_cast<uint4*>(gs.dst[jb])[lt] = v;
   }
 }
 
@@ -356,31 +360,20 @@ cudaError_t launch_wait_probe(int* err, uint64_t limit_ns, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather_globals(const AttnParams& p, const void* q, const void* k, const void* v,
-                                  void* gq, void* gk, void* gv, int elem_bytes, cudaStream_t s) {
-  const int row_vecs = p.D * elem_bytes / 16;
-  const int threads = 256;
-  auto blocks = [&](size_t total) { return (int)min((total + threads - 1) / threads, (size_t)4096); };
-  size_t tq = (size_t)p.B * p.Hq * p.gpad * row_vecs;
-  size_t tk = (size_t)p.B * p.Hkv * p.gpad * row_vecs;
-  gather_rows_kernel<<<blocks(tq), threads, 0, s>>>(static_cast<const uint4*>(q), static_cast<uint4*>(gq),
-                                                    p.global_idx, p.Hq, p.n, p.g, p.gpad, row_vecs, p.B);
-  gather_rows_kernel<<<blocks(tk), threads, 0, s>>>(static_cast<const uint4*>(k), static_cast<uint4*>(gk),
-                                                    p.global_idx, p.Hkv, p.n, p.g, p.gpad, row_vecs, p.B);
-  gather_rows_kernel<<<blocks(tk), threads, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(gv),
-                                                    p.global_idx, p.Hkv, p.n, p.g, p.gpad, row_vecs, p.B);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* gidx, int B, int H, int n, int g,
-                               int gpad, int D, int elem_bytes, cudaStream_t s) {
+cudaError_t launch_gather_rows(const GatherSet& set, const int32_t* gidx, int B, int n, int g, int gpad, int D,
+                               int elem_bytes, cudaStream_t s) {
+  if (set.count < 1 || set.count > kMaxGather) return cudaErrorInvalidValue;
   const int row_vecs = D * elem_bytes / 16;
-  const size_t total = (size_t)B * H * gpad * row_vecs;
+  GatherSet gs = set;
+  size_t total = 0;
+  for (int j = 0; j < gs.count; ++j) {
+    total += (size_t)B * gs.heads[j] * gpad * row_vecs;
+    gs.end[j] = total;
+  }
   if (total == 0) return cudaSuccess;
   const int threads = 256;
   const int blocks = (int)min((total + threads - 1) / threads, (size_t)4096);
-  gather_rows_kernel<<<blocks, threads, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), gidx,
-                                                H, n, g, gpad, row_vecs, B);
+  gather_rows_kernel<<<blocks, threads, 0, s>>>(gs, gidx, n, g, gpad, row_vecs, B);
   return cudaGetLastError();
 }
 

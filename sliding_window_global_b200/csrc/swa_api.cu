@@ -385,14 +385,10 @@ swa_status swa_backward(swa_plan_t plan, const swa_backward_args* a, void* strea
     }
   };
   if (num_global > 0 && ce == cudaSuccess) {
-    ce = swa::launch_gather_rows(a->q, plan->gq, p.global_idx, p.B, Hq, n, num_global, p.gpad, D, 2, s);
-    if (ce == cudaSuccess)
-      ce = swa::launch_gather_rows(a->dout, plan->gdo, p.global_idx, p.B, Hq, n, num_global, p.gpad, D, 2, s);
-    if (ce == cudaSuccess)
-      ce = swa::launch_gather_rows(a->k, plan->gk, p.global_idx, p.B, p.Hkv, n, num_global, p.gpad, D, 2, s);
-    if (ce == cudaSuccess)
-      ce = swa::launch_gather_rows(a->v, plan->gv, p.global_idx, p.B, p.Hkv, n, num_global, p.gpad, D, 2, s);
-    launches += 4;
+    const swa::GatherSet gs = {{a->q, a->dout, a->k, a->v}, {plan->gq, plan->gdo, plan->gk, plan->gv},
+                               {Hq, Hq, p.Hkv, p.Hkv}, {}, 4};
+    ce = swa::launch_gather_rows(gs, p.global_idx, p.B, n, num_global, p.gpad, D, 2, s);
+    ++launches;
   }
   step(swa::launch_bwd_dq);
   if (num_global > 0) step(swa::launch_bwd_dq_global_rows);

@@ -347,8 +347,9 @@ swa_status enqueue_forward(const swa_plan_desc& d, const swa_forward_args& args,
     ++launches;
   } else {
     if (num_global > 0) {
-      ce = launch_gather_globals(p, q, k, v, ws.gq, ws.gk, ws.gv, 2, s);
-      launches += 3;
+      GatherSet gs = {{q, k, v}, {ws.gq, ws.gk, ws.gv}, {p.Hq, p.Hkv, p.Hkv}, {}, 3};
+      ce = launch_gather_rows(gs, p.global_idx, p.B, p.n, p.g, p.gpad, p.D, 2, s);
+      ++launches;
     }
     if (ce == cudaSuccess) {
       ce = launch_band_tc(p, num_sms, s);

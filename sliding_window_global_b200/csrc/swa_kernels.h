@@ -78,13 +78,20 @@ struct AttnParams {
 // Launchers (each returns the launch's cudaError_t).
 cudaError_t launch_band_tc(const AttnParams& p, int num_sms, cudaStream_t s);
 cudaError_t launch_global_rows_tc(const AttnParams& p, int num_sms, cudaStream_t s);
-cudaError_t launch_gather_globals(const AttnParams& p, const void* q, const void* k,
-                                  const void* v, void* gq, void* gk, void* gv, int elem_bytes,
-                                  cudaStream_t s);
 cudaError_t launch_merge_global_rows(const AttnParams& p, int bf16_out, cudaStream_t s);
-// dst[bh, e, :] = src[bh, gidx[b, e], :] for e < g, zeros up to gpad ([B*H, n, D] -> [B*H, gpad, D]).
-cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* gidx, int B, int H, int n, int g,
-                               int gpad, int D, int elem_bytes, cudaStream_t s);
+// Up to kMaxGather arrays gathered by one launch; `end` is filled by the launcher.
+constexpr int kMaxGather = 4;
+struct GatherSet {
+  const void* src[kMaxGather];
+  void* dst[kMaxGather];
+  int heads[kMaxGather];
+  size_t end[kMaxGather];
+  int count;
+};
+// For every array of the set: dst[bh, e, :] = src[bh, gidx[b, e], :] for e < g, zeros up
+// to gpad ([B*H, n, D] -> [B*H, gpad, D]); one launch for all of them.
+cudaError_t launch_gather_rows(const GatherSet& set, const int32_t* gidx, int B, int n, int g, int gpad, int D,
+                               int elem_bytes, cudaStream_t s);
 cudaError_t launch_simt(const AttnParams& p, const void* q, const void* k, const void* v,
                         const void* side_k, const void* side_v, int bf16, cudaStream_t s);
 // Debug check of the index inputs: global_idx rows strictly increasing inside

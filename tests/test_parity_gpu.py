@@ -386,7 +386,7 @@ def test_repeat_calls_deterministic_and_launch_count():
     o1, l1, plan = helpers.run_gpu(w, dinp)
     o2, l2, _ = helpers.run_gpu(w, dinp, plan=plan)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
-    assert plan.last_launches == 6   # gather x3, band, global rows, merge
+    assert plan.last_launches == 4   # gather (q, k, v in one launch), band, global rows, merge
 
 
 def test_bounded_wait_expires_into_a_status_and_the_context_survives():
