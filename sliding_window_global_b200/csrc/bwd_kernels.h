@@ -27,6 +27,7 @@ struct BwdParams {
   float* dv;                         // [B, Hkv, n, D] fp32
   int* err;
   int max_qtiles;                    // largest qtiles[h]
+  int num_sms;                       // grid of the persistent dq pass
   int max_ktiles;                    // largest ktiles[hk]
   // Terms beyond the band (all optional; see swa_backward_args).
   int extras;                        // any of the terms below is present

@@ -217,6 +217,59 @@ __device__ __forceinline__ int batch_valid_len(const BwdParams& p, int b) {
 // only their window and side keys here.  GROWS: the stationary tile is 128 gathered
 // global query rows, the key tiles are every tile of the sequence, and the mask keeps
 // the keys outside each row's window; the result is added to dq.
+// Units of the dQ pass: band, a 128-row query tile of one head's class (heads fastest);
+// GROWS, a tile of 128 global slots of one head.  The kernel is persistent: CTA c takes
+// units c, c + grid, ...
+template <bool GROWS>
+__device__ __forceinline__ int dq_units(const BwdParams& p) {
+  return GROWS ? p.B * p.Hq * (p.gpad / kTile) : p.max_qtiles * p.B * p.Hq;
+}
+
+// Unit uid of the dQ pass and its key tiles: band tiles from klo_t (class
+// coordinates), then (X) global-column, side and random tiles.  false: the unit has
+// no rows (every role skips it).
+template <bool X, bool GROWS>
+__device__ __forceinline__ bool dq_unit(const BwdParams& p, int uid, BUnit& u, int& klo_t, int& T, int& nband,
+                                        int& ngc, int& nside, int& nrand) {
+  klo_t = T = nband = ngc = nside = nrand = 0;
+  if (!GROWS) {
+    decode_bunit(p, uid, false, u);
+    if (!u.valid) return false;
+    // band key range of the tile: [klo_t, khi_t) in class coordinates
+    const int last = u.u0 + u.nvalid - 1;
+    klo_t = max(0, u.u0 - u.r);
+    const int khi_t = u.nvalid > 0 ? (p.causal ? min(u.Vc, last + 1) : min(u.Vc, last + u.r + 1)) : klo_t;
+    nband = khi_t > klo_t ? (khi_t - klo_t + kTile - 1) / kTile : 0;
+    if (X && u.nvalid > 0) {
+      ngc = p.g > 0 ? (p.g + kTile - 1) / kTile : 0;
+      nside = p.S > 0 ? (p.S + kTile - 1) / kTile : 0;
+      nrand = p.rand_blocks ? p.num_rand : 0;
+    }
+    T = nband + ngc + nside + nrand;
+  } else {
+    // global rows: unit = (batch, query head, tile of 128 global slots)
+    const int gtiles = p.gpad / kTile;
+    const int bh = uid / gtiles, gt = uid % gtiles;
+    u.valid = true;
+    u.b = bh / p.Hq;
+    u.h = bh % p.Hq;
+    u.hk = u.h / p.G;
+    u.cls = p.dense_class;
+    u.c = 0;
+    u.d = p.cls[p.class_base[u.h]].d;             // the head's own dilation, for its window
+    u.r = p.window[u.h];
+    u.nc = p.n;
+    u.Vc = batch_valid_len(p, u.b);
+    u.u0 = gt * kTile;
+    u.rows = min(kTile, p.gpad - u.u0);
+    u.nvalid = max(0, min(u.rows, p.g - u.u0));
+    if (u.nvalid == 0) return false;
+    T = (u.Vc + kTile - 1) / kTile;
+    nband = T;
+  }
+  return true;
+}
+
 template <int D, bool X, bool GROWS>
 __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_constant__ BwdParams p) {
   using C = BCfg<D>;
@@ -237,48 +290,13 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
   uint64_t* k_empty = k_full + NK;  // [NK] its dQ product completed
   uint64_t* v_full = k_empty + NK;  // [NV] V tile of a stage loaded
   uint64_t* v_empty = v_full + NV;  // [NV] its dP product completed
+  uint64_t* stat_empty = v_empty + NV;  // the unit's last S and dP done: Q, dO may be replaced
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ int sGpos[kTile];      // key positions of the current global-column tile
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  BUnit u;
-  int klo_t = 0, T = 0, nband = 0, ngc = 0, nside = 0, nrand = 0;
-  if (!GROWS) {
-    decode_bunit(p, blockIdx.x, false, u);
-    if (!u.valid) return;
-    // band key range of the tile: [klo_t, khi_t) in class coordinates
-    const int last = u.u0 + u.nvalid - 1;
-    klo_t = max(0, u.u0 - u.r);
-    const int khi_t = u.nvalid > 0 ? (p.causal ? min(u.Vc, last + 1) : min(u.Vc, last + u.r + 1)) : klo_t;
-    nband = khi_t > klo_t ? (khi_t - klo_t + kTile - 1) / kTile : 0;
-    if (X && u.nvalid > 0) {
-      ngc = p.g > 0 ? (p.g + kTile - 1) / kTile : 0;
-      nside = p.S > 0 ? (p.S + kTile - 1) / kTile : 0;
-      nrand = p.rand_blocks ? p.num_rand : 0;
-    }
-    T = nband + ngc + nside + nrand;
-  } else {
-    // global rows: unit = (batch, query head, tile of 128 global slots)
-    const int gtiles = p.gpad / kTile;
-    const int bh = blockIdx.x / gtiles, gt = blockIdx.x % gtiles;
-    u.valid = true;
-    u.b = bh / p.Hq;
-    u.h = bh % p.Hq;
-    u.hk = u.h / p.G;
-    u.cls = p.dense_class;
-    u.c = 0;
-    u.d = p.cls[p.class_base[u.h]].d;             // the head's own dilation, for its window
-    u.r = p.window[u.h];
-    u.nc = p.n;
-    u.Vc = batch_valid_len(p, u.b);
-    u.u0 = gt * kTile;
-    u.rows = min(kTile, p.gpad - u.u0);
-    u.nvalid = max(0, min(u.rows, p.g - u.u0));
-    if (u.nvalid == 0) return;
-    T = (u.Vc + kTile - 1) / kTile;
-    nband = T;
-  }
+  const int nunits = dq_units<GROWS>(p);
 
   if (tid == 0) {
     mbar_init(a_full, 1);
@@ -295,6 +313,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
     mbar_init(&ds_full[1], 128);
     mbar_init(acc_full, 1);
     mbar_init(dp_read, 128);
+    mbar_init(stat_empty, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -307,19 +326,37 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
   volatile int* abort_v = &abort_flag;
-  const int qz = u.b * p.Hq + u.h;
-  const int kz = u.b * p.Hkv + u.hk;
-  const int qb = u.u0 / kTile;                     // query block of the tile (random blocks: d = 1)
   const int nqb = (p.n + kTile - 1) / kTile;
+  // Every role walks the same units in the same order and keeps the same counters:
+  // ka, units with key tiles so far (phases of a_full, stat_empty, acc_full), and jg,
+  // key tiles so far (ring stages, S buffers and the per-tile barriers' phases).
+  BUnit u;
+  int klo_t, T, nband, ngc, nside, nrand;
 
   if (warp == 4) {
-    if (lane == 0 && T > 0) {
+    if (lane == 0) {
+      bool ok = true;
+      int ka = 0, jg = 0;
+      for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
+      if (!dq_unit<X, GROWS>(p, uid, u, klo_t, T, nband, ngc, nside, nrand) || T == 0) continue;
+      const int qz = u.b * p.Hq + u.h;
+      const int kz = u.b * p.Hkv + u.hk;
+      const int qb = u.u0 / kTile;                 // query block of the tile (random blocks: d = 1)
+      // Q and dO of this unit replace the last unit's once its last S and dP are done
+      if (ka > 0 && !mbar_wait_bounded(stat_empty, (ka - 1) & 1, abort_v, kWaitLimitNs)) {
+        ok = false;
+        break;
+      }
       mbar_arrive_expect_tx(a_full, 2 * C::kTileBytes);
       load_tile<D>(smem + C::kStat0, GROWS ? &p.mgq : &p.mq[u.cls], a_full, u.u0, qz);
       load_tile<D>(smem + C::kStat1, GROWS ? &p.mgdo : &p.mdo[u.cls], a_full, u.u0, qz);
       for (int j = 0; j < T; ++j) {
-        const int sk = j % NK, sv = j % NV;
-        if (j >= NK && !mbar_wait_bounded(&k_empty[sk], ((j / NK) - 1) & 1, abort_v, kWaitLimitNs)) break;
+        const int jj = jg + j;                     // ring position
+        const int sk = jj % NK, sv = jj % NV;
+        if (jj >= NK && !mbar_wait_bounded(&k_empty[sk], ((jj / NK) - 1) & 1, abort_v, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
         const CUtensorMap *mk = &p.mk[u.cls], *mv = &p.mv[u.cls];
         int y = GROWS ? j * kTile : klo_t + j * kTile;
         if (X && j >= nband) {
@@ -334,18 +371,28 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
         }
         mbar_arrive_expect_tx(&k_full[sk], C::kTileBytes);
         load_tile<D>(smem + C::kKRing + sk * C::kTileBytes, mk, &k_full[sk], y, kz);
-        if (j >= NV && !mbar_wait_bounded(&v_empty[sv], ((j / NV) - 1) & 1, abort_v, kWaitLimitNs)) break;
+        if (jj >= NV && !mbar_wait_bounded(&v_empty[sv], ((jj / NV) - 1) & 1, abort_v, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
         mbar_arrive_expect_tx(&v_full[sv], C::kTileBytes);
         load_tile<D>(smem + C::kVRing + sv * C::kTileBytes, mv, &v_full[sv], y, kz);
       }
+      ++ka;
+      jg += T;
+      }
     }
   } else if (warp == 5) {
-    if (lane == 0 && T > 0) {
+    if (lane == 0) {
       // Pipelined: S of tile j+1 is computed into the other S buffer while the compute
       // warps work on tile j, and dP of tile j+1 as soon as they have read dP of tile j,
       // so the next tile's products are ready when the compute warps are.  In issue
       // order (MMAs complete in order): a new S goes into the buffer whose dS the
-      // previous dQ product read; a new dP after dp_read.
+      // previous dQ product read; a new dP after dp_read.  Indices are CTA-wide (jg +
+      // j), so a unit's first S and dP follow the last unit's products at once and
+      // overlap its last dS and its epilogue; the first dQ product of a unit, which
+      // overwrites the accumulator, waits for the compute warps' dS of its first tile,
+      // which they write after their epilogue has read the accumulator.
       const uint32_t qa = smem_u32(smem + C::kStat0), da = smem_u32(smem + C::kStat1);
       auto kstage = [&](int j) { return smem_u32(smem + C::kKRing + (j % NK) * C::kTileBytes); };
       auto issue_s = [&](int j) -> bool {           // S(j) = Q K(j)^T
@@ -361,31 +408,50 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
         umma_commit(&v_empty[j % NV]);
         return true;
       };
-      bool ok = mbar_wait_bounded(a_full, 0, abort_v, kWaitLimitNs);
-      if (ok) ok = issue_s(0);
-      if (ok) ok = issue_dp(0);
-      if (ok) umma_commit(s_full);
-      if (ok && T > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < T; ++j) {
-        if (j + 1 < T) {
-          // dP(j+1) once the compute warps hold dP(j) in registers
-          if (!mbar_wait_bounded(dp_read, j & 1, abort_v, kWaitLimitNs)) break;
-          if (!issue_dp(j + 1)) break;
-          umma_commit(s_full);                       // S(j+1) and dP(j+1)
+      bool ok = true;
+      int ka = 0, jg = 0;
+      for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
+        if (!dq_unit<X, GROWS>(p, uid, u, klo_t, T, nband, ngc, nside, nrand) || T == 0) continue;
+        ok = mbar_wait_bounded(a_full, ka & 1, abort_v, kWaitLimitNs);
+        if (ok) ok = issue_s(jg);
+        // dP of the first tile replaces the last unit's last dP once it is in registers
+        if (ok && jg > 0) ok = mbar_wait_bounded(dp_read, (jg - 1) & 1, abort_v, kWaitLimitNs);
+        if (ok) ok = issue_dp(jg);
+        if (ok) {
+          umma_commit(s_full);
+          if (T == 1) umma_commit(stat_empty);       // the unit's last S and dP
         }
-        // dQ += dS(j) K(j), then the stage of tile j may be refilled
-        if (!mbar_wait_bounded(&ds_full[j & 1], (j >> 1) & 1, abort_v, kWaitLimitNs)) break;
-        tc_fence_after();
-        mma_px<D>(tmem + C::kAcc0, tmem + C::s_buf(j), kstage(j), j > 0);
-        umma_commit(&k_empty[j % NK]);
-        if (j == T - 1) umma_commit(acc_full);
-        if (j + 2 < T) ok = issue_s(j + 2);           // into the buffer dQ(j) just read
+        if (ok && T > 1) ok = issue_s(jg + 1);
+        for (int j = 0; ok && j < T; ++j) {
+          const int jj = jg + j;
+          if (j + 1 < T) {
+            // dP(j+1) once the compute warps hold dP(j) in registers
+            if (!mbar_wait_bounded(dp_read, jj & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+            if (!issue_dp(jj + 1)) { ok = false; break; }
+            umma_commit(s_full);                     // S(j+1) and dP(j+1)
+            if (j + 2 == T) umma_commit(stat_empty); // the unit's last S and dP
+          }
+          // dQ += dS(j) K(j), then the stage of tile j may be refilled
+          if (!mbar_wait_bounded(&ds_full[jj & 1], (jj >> 1) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          mma_px<D>(tmem + C::kAcc0, tmem + C::s_buf(jj), kstage(jj), j > 0);
+          umma_commit(&k_empty[jj % NK]);
+          if (j == T - 1) umma_commit(acc_full);
+          if (j + 2 < T) ok = issue_s(jj + 2);         // into the buffer dQ(j) just read
+        }
+        ++ka;
+        jg += T;
       }
     }
   } else {
     // ------------------------------------------------------------ compute
     const int row = tid;                       // TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    bool ok = true;
+    int ka = 0, jg = 0;
+    for (int uid = blockIdx.x; ok && uid < nunits; uid += gridDim.x) {
+    if (!dq_unit<X, GROWS>(p, uid, u, klo_t, T, nband, ngc, nside, nrand)) continue;
+    const int qb = u.u0 / kTile;               // query block of the tile (random blocks: d = 1)
     const bool row_valid = row < u.nvalid;
     const int uq = u.u0 + row;
     const int rd = u.r * u.d;
@@ -421,8 +487,8 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
         if (t < nrand) rbl[t] = __ldg(p.rand_blocks + (((size_t)u.b * p.Hq + u.h) * nqb + qb) * p.num_rand + t);
     }
     const float sl2 = p.scale_log2;
-    bool ok = true;
     for (int j = 0; j < T; ++j) {
+      const int jj = jg + j;                   // CTA-wide tile index: barrier phases, S buffer
       // tile kind: 0 band (or every key, GROWS), 1 global columns, 2 side, 3 random
       int kind = 0, base = 0, t_rand = 0;
       if (X && j >= nband) {
@@ -451,7 +517,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
         for (int t = 0; t < kMaxRand; ++t) dup = dup || (t < t_rand && rbl[t] == kb);
         dup = dup || kb < 0 || kb >= nqb;
       }
-      if (!mbar_wait_bounded(s_full, j & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+      if (!mbar_wait_bounded(s_full, jj & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
       tc_fence_after();
       const int kv0 = GROWS ? j * kTile : (kind == 3 ? kb * kTile : klo_t + j * kTile);
       const int lo_t = klo - kv0, hi_t = khi - kv0;
@@ -463,7 +529,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
       for (int ch = 0; ch < 4; ++ch) tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(dpr + ch * 32));
       tc_fence_before();
       mbar_arrive(dp_read);
-      const uint32_t sb = lane_base + C::s_buf(j);
+      const uint32_t sb = lane_base + C::s_buf(jj);
       // Interior band tile: every key of the tile is in the window of every row of this
       // warp, so no element needs a mask, and pairs of columns take one packed f32x2
       // instruction per step.
@@ -528,11 +594,11 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&ds_full[j & 1]);
+      mbar_arrive(&ds_full[jj & 1]);
     }
     // epilogue: dQ = scale * (dS K), fp32; padded rows get zeros.  Global rows (GROWS)
     // add their part to what the band pass wrote.
-    if (ok && T > 0) ok = mbar_wait_bounded(acc_full, 0, abort_v, kWaitLimitNs);
+    if (ok && T > 0) ok = mbar_wait_bounded(acc_full, ka & 1, abort_v, kWaitLimitNs);
     if (ok) {
       tc_fence_after();
       float* dst = p.dq + prow * D;
@@ -559,6 +625,9 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
           }
         }
       }
+    }
+    if (T > 0) ++ka;
+    jg += T;
     }
   }
 
@@ -1086,7 +1155,7 @@ cudaError_t launch_bwd_delta(const BwdParams& p, cudaStream_t s) {
 }
 
 cudaError_t launch_bwd_dq(const BwdParams& p, cudaStream_t s) {
-  const int grid = p.max_qtiles * p.B * p.Hq;
+  const int grid = min(p.max_qtiles * p.B * p.Hq, p.num_sms);       // persistent
   if (p.extras)
     return p.D == 64 ? launch_kern(bwd_dq_kernel<64, true, false>, BCfg<64>::kSmemBytes, grid, kBThreads, p, s)
                      : launch_kern(bwd_dq_kernel<128, true, false>, BCfg<128>::kSmemBytes, grid, kBThreads, p, s);
@@ -1096,7 +1165,7 @@ cudaError_t launch_bwd_dq(const BwdParams& p, cudaStream_t s) {
 
 cudaError_t launch_bwd_dq_global_rows(const BwdParams& p, cudaStream_t s) {
   if (p.g == 0) return cudaSuccess;
-  const int grid = p.B * p.Hq * (p.gpad / kTile);
+  const int grid = min(p.B * p.Hq * (p.gpad / kTile), p.num_sms);   // persistent
   return p.D == 64 ? launch_kern(bwd_dq_kernel<64, false, true>, BCfg<64>::kSmemBytes, grid, kBThreads, p, s)
                    : launch_kern(bwd_dq_kernel<128, false, true>, BCfg<128>::kSmemBytes, grid, kBThreads, p, s);
 }

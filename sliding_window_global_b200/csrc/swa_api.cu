@@ -262,6 +262,7 @@ swa_status swa_backward(swa_plan_t plan, const swa_backward_args* a, void* strea
 
   swa::BwdParams p;   // on the stack: the call allocates nothing
   memset(&p, 0, sizeof(p));
+  p.num_sms = plan->num_sms;
   p.B = d.batch;
   p.Hq = Hq;
   p.Hkv = d.num_kv_heads;

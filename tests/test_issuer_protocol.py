@@ -442,19 +442,29 @@ def test_dkv_model_detects_an_early_next_product():
     assert caught > 0
 
 
-def simulate_dq(seed, T, early_dp=False, early_s=False, per_parity=True, NK=3, NV=2):
-    """The query-stationary dQ pass (csrc/bwd_tc.cu): one query tile per CTA, its T key
-    tiles' K through an NK-stage ring and V through an NV-stage ring (V is released
-    after dP, K after dQ); S of tile j in TMEM buffer j & 1, dP in one buffer.
-    The issuer computes S(j+1) while the compute warps work on tile j, dP(j+1) once
-    they hold dP(j) in registers (dp_read), and S(j+2) into the buffer dQ(j) has just
-    read (in issue order).  MMAs complete in issue order.  Checked: the compute warps
-    read S(j) and dP(j) of their own tile, dS(j) is what dQ(j) reads, no ring slot is
-    refilled under a pending reader, no deadlock, no parity-ambiguous wait.
-    per_parity=False models a single dS barrier, which the compute warps can drive two
-    phases past the issuer's wait."""
+def simulate_dq(seed, Ts, early_dp=False, early_s=False, per_parity=True, NK=3, NV=2, stat_early=False):
+    """The query-stationary dQ pass (csrc/bwd_tc.cu), persistent: one CTA walks units
+    of Ts[u] key tiles each (a unit without key tiles only writes zeros).  Q and dO of
+    a unit are loaded once the last unit's last S and dP are done (stat_empty); K
+    through an NK-stage ring and V through an NV-stage ring (V released after dP, K
+    after dQ), with CTA-wide tile indices; S of tile j in TMEM buffer j & 1, dP in one
+    buffer.  The issuer computes S(j+1) while the compute warps work on tile j, dP(j+1)
+    once they hold dP(j) in registers (dp_read), and S(j+2) into the buffer dQ(j) has
+    just read; a unit's first S and dP follow the last unit's products at once (its
+    first dP after the last unit's last dP was read), and its first dQ product, which
+    overwrites the accumulator, after the compute warps' dS of its first tile, which
+    they write after their epilogue has read the accumulator.  MMAs complete in issue
+    order.  Checked: the compute warps read S(j) and dP(j) of their own tile, dS(j) is
+    what dQ(j) reads, the epilogue reads its own unit's accumulator, no ring slot or
+    Q/dO buffer is refilled under a pending reader, no deadlock, no parity-ambiguous
+    wait.  per_parity=False models a single dS barrier, which the compute warps can
+    drive two phases past the issuer's wait; stat_early releases Q/dO one product too
+    early."""
+    if isinstance(Ts, int):
+        Ts = [Ts]
     rng = random.Random(seed)
     a_full = Barrier("a_full", 1)
+    stat_empty = Barrier("stat_empty", 1)
     N = {"K": NK, "V": NV}
     full = {x: [Barrier(f"{x}_full{s}", 1) for s in range(N[x])] for x in "KV"}
     empty = {x: [Barrier(f"{x}_empty{s}", 1) for s in range(N[x])] for x in "KV"}
@@ -465,80 +475,123 @@ def simulate_dq(seed, T, early_dp=False, early_s=False, per_parity=True, NK=3, N
     pipe = []
     pending = {}
     loads = {"K": [0] * NK, "V": [0] * NV}
+    stat_loads = [0]
     sbuf = [None, None]                     # what each S buffer holds: ("S", j) or ("dS", j)
     dpbuf = [None]                          # the tile whose dP the dP buffer holds
+    acc = [None]                            # the unit whose dQ products the accumulator holds
 
     def mma_read(key):
         pending[key] = pending.get(key, 0) + 1
         pipe.append(("read", key))
 
-    def producer():
-        a_full.arrive()
-        for j in range(T):
-            for x in "KV":
-                st = j % N[x]
-                if j >= N[x]:
-                    yield from wait(empty[x][st], j // N[x] - 1)
-                if pending.get((x, st, loads[x][st] - 1), 0):
-                    raise ProtocolError(f"{x} slot {st} refilled under a pending reader")
-                loads[x][st] += 1
-                yield
-                full[x][st].arrive()
-
     def ring_read(x, j):
         mma_read((x, j % N[x], loads[x][j % N[x]] - 1))
+
+    def producer():
+        ka = jg = 0
+        for T in Ts:
+            if T == 0:
+                continue
+            if ka > 0:
+                yield from wait(stat_empty, ka - 1)
+            if pending.get(("stat", stat_loads[0] - 1), 0):
+                raise ProtocolError("Q/dO replaced while an S or dP product still reads them")
+            stat_loads[0] += 1
+            yield
+            a_full.arrive()
+            for j in range(T):
+                jj = jg + j
+                for x in "KV":
+                    st = jj % N[x]
+                    if jj >= N[x]:
+                        yield from wait(empty[x][st], jj // N[x] - 1)
+                    if pending.get((x, st, loads[x][st] - 1), 0):
+                        raise ProtocolError(f"{x} slot {st} refilled under a pending reader")
+                    loads[x][st] += 1
+                    yield
+                    full[x][st].arrive()
+            ka += 1
+            jg += T
 
     def issuer():
         def issue_s(j):
             yield from wait(full["K"][j % NK], j // NK)
             ring_read("K", j)
+            mma_read(("stat", stat_loads[0] - 1))
             pipe.append(("write_s", j))
 
         def issue_dp(j):
             yield from wait(full["V"][j % NV], j // NV)
             ring_read("V", j)
+            mma_read(("stat", stat_loads[0] - 1))
             pipe.append(("write_dp", j))
             pipe.append(("commit", empty["V"][j % NV]))
 
-        yield from wait(a_full, 0)
-        yield from issue_s(0)
-        yield from issue_dp(0)
-        pipe.append(("commit", s_full))
-        if T > 1:
-            yield from issue_s(1)
-        for j in range(T):
-            if j + 1 < T:
-                if not early_dp:
-                    yield from wait(dp_read, j)
-                yield from issue_dp(j + 1)
-                pipe.append(("commit", s_full))
-            yield from wait(ds_full[j & 1] if per_parity else ds_full[0], (j >> 1) if per_parity else j)
-            if early_s and j + 2 < T:              # planted: S(j+2) before dQ(j) read dS(j)
-                yield from issue_s(j + 2)
-            ring_read("K", j)
-            pipe.append(("read_ds", j))
-            pipe.append(("commit", empty["K"][j % NK]))
-            if j == T - 1:
-                pipe.append(("commit", acc_full))
-            if j + 2 < T and not early_s:
-                yield from issue_s(j + 2)
+        ka = jg = 0
+        for u, T in enumerate(Ts):
+            if T == 0:
+                continue
+            yield from wait(a_full, ka)
+            yield from issue_s(jg)
+            if jg > 0:
+                yield from wait(dp_read, jg - 1)
+            if stat_early and T == 1:
+                pipe.append(("commit", stat_empty))
+            yield from issue_dp(jg)
+            pipe.append(("commit", s_full))
+            if T == 1 and not stat_early:
+                pipe.append(("commit", stat_empty))
+            if T > 1:
+                yield from issue_s(jg + 1)
+            for j in range(T):
+                jj = jg + j
+                if j + 1 < T:
+                    if not early_dp:
+                        yield from wait(dp_read, jj)
+                    if stat_early and j + 2 == T:
+                        pipe.append(("commit", stat_empty))
+                    yield from issue_dp(jj + 1)
+                    pipe.append(("commit", s_full))
+                    if j + 2 == T and not stat_early:
+                        pipe.append(("commit", stat_empty))
+                yield from wait(ds_full[jj & 1] if per_parity else ds_full[0], (jj >> 1) if per_parity else jj)
+                if early_s and j + 2 < T:              # planted: S(j+2) before dQ(j) read dS(j)
+                    yield from issue_s(jj + 2)
+                ring_read("K", jj)
+                pipe.append(("read_ds", jj))
+                pipe.append(("dq", u))
+                pipe.append(("commit", empty["K"][jj % NK]))
+                if j == T - 1:
+                    pipe.append(("commit", acc_full))
+                if j + 2 < T and not early_s:
+                    yield from issue_s(jj + 2)
+            ka += 1
+            jg += T
 
     def compute():
-        for j in range(T):
-            yield from wait(s_full, j)
-            if dpbuf[0] != j:
-                raise ProtocolError(f"compute of tile {j} read dP of tile {dpbuf[0]}")
-            yield
-            for _ in range(128):
-                dp_read.arrive()
-            if sbuf[j & 1] != ("S", j):
-                raise ProtocolError(f"compute of tile {j} read {sbuf[j & 1]} from S buffer {j & 1}")
-            yield
-            sbuf[j & 1] = ("dS", j)
-            for _ in range(128):
-                (ds_full[j & 1] if per_parity else ds_full[0]).arrive()
-        if T > 0:
-            yield from wait(acc_full, 0)
+        ka = jg = 0
+        for u, T in enumerate(Ts):
+            for j in range(T):
+                jj = jg + j
+                yield from wait(s_full, jj)
+                if dpbuf[0] != jj:
+                    raise ProtocolError(f"compute of tile {jj} read dP of tile {dpbuf[0]}")
+                yield
+                for _ in range(128):
+                    dp_read.arrive()
+                if sbuf[jj & 1] != ("S", jj):
+                    raise ProtocolError(f"compute of tile {jj} read {sbuf[jj & 1]} from S buffer {jj & 1}")
+                yield
+                sbuf[jj & 1] = ("dS", jj)
+                for _ in range(128):
+                    (ds_full[jj & 1] if per_parity else ds_full[0]).arrive()
+            if T > 0:
+                yield from wait(acc_full, ka)
+                if acc[0] != u:
+                    raise ProtocolError(f"epilogue of unit {u} read the accumulator of unit {acc[0]}")
+                yield
+                ka += 1
+            jg += T
 
     agents = [producer(), issuer(), compute()]
     alive = list(range(len(agents)))
@@ -557,6 +610,8 @@ def simulate_dq(seed, T, early_dp=False, early_s=False, per_parity=True, NK=3, N
             elif k == "read_ds":
                 if sbuf[val & 1] != ("dS", val):
                     raise ProtocolError(f"dQ product of tile {val} read {sbuf[val & 1]}")
+            elif k == "dq":
+                acc[0] = val
             else:
                 val.arrive()
             stalls = 0
@@ -569,6 +624,27 @@ def simulate_dq(seed, T, early_dp=False, early_s=False, per_parity=True, NK=3, N
             stalls = 0
         if stalls > 20000:
             raise ProtocolError("deadlock: no agent can make progress")
+
+
+@pytest.mark.parametrize("seed0", [0, 1000])
+def test_dq_persistent_units_random_schedules(seed0):
+    """Several units per CTA, some without key tiles, with random tile counts."""
+    for seed in range(seed0, seed0 + 150):
+        r = random.Random(seed)
+        Ts = [r.choice([0, 1, 2, 3, 5]) for _ in range(r.randint(1, 5))]
+        simulate_dq(seed, Ts)
+
+
+def test_dq_model_detects_an_early_stat_release():
+    """Releasing Q/dO before the unit's last dP product is issued lets the next
+    unit's load replace them under that product on some schedule."""
+    caught = 0
+    for seed in range(300):
+        try:
+            simulate_dq(seed, [2, 3, 1, 2], stat_early=True)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
 
 
 @pytest.mark.parametrize("rings", [(2, 2), (3, 2)], ids=["kv2", "k3_v2"])
