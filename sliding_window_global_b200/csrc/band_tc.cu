@@ -119,8 +119,13 @@ struct Cfg {
 
 // The register split must fit the budget the CTA is launched with (a larger sum
 // would leave setmaxnreg.inc waiting), and the shared memory one CTA per SM.
+// setmaxnreg moves registers only between the warps of one SM sub-partition (warp
+// w runs on sub-partition w % 4), so the split must also fit each sub-partition's
+// share: here one warp of each softmax group and one control warp.
 static_assert(kSoftmaxThreads * kRegsSoftmax + (kThreads - kSoftmaxThreads) * kRegsControl <= kThreads * 168,
               "setmaxnreg split exceeds the launch register budget");
+static_assert(kThreads == 12 * 32 && kSoftmaxThreads == 8 * 32 && 2 * kRegsSoftmax + kRegsControl <= 3 * 168,
+              "setmaxnreg split exceeds a sub-partition's registers");
 static_assert(Cfg<64>::kSmemBytes + 2 * kTile * 4 + 16 <= 227 * 1024, "shared memory, D = 64");
 static_assert(Cfg<128>::kSmemBytes + 2 * kTile * 4 + 16 <= 227 * 1024, "shared memory, D = 128");
 static_assert(emu_per32<64>() % 4 == 0 && emu_per32<64>() <= 32 && emu_per32<128>() % 4 == 0 &&
