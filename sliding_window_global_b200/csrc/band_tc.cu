@@ -404,9 +404,10 @@ __device__ __forceinline__ void side_prologue(const AttnParams& p, int tid, int 
 // LOCAL: band tiles carry the local relative-position bias; RAND: query tiles have
 // random key blocks (MODE 0 only); AGG: the CTAs first build the side keys / values
 // from k and v (cooperative launch) and load side tiles once every CTA has counted
-// itself done.  They are template parameters so that kernels without them keep
-// their register schedule.
-template <int D, int MODE, bool LOCAL, bool RAND, bool AGG>
+// itself done; GLOB: the tile lists hold global-column tiles (launches with global
+// tokens).  They are template parameters so that kernels without them keep their
+// register schedule.
+template <int D, int MODE, bool LOCAL, bool RAND, bool AGG, bool GLOB>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ AttnParams p) {
   using C = Cfg<D>;
   constexpr int NS = C::NS;
@@ -434,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   uint64_t* p_half = pv_done + 2;         // [2] P of keys 0-63 written (P-over-S layout)
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
-  __shared__ int sGpos[2 * kTile];        // positions of the current global tile, per group
+  __shared__ __align__(16) int sGpos[2 * kTile];   // the current global tile's keys, per group
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -786,7 +787,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       for (int t = 0; t < kRandRegs; ++t)
         rbl[t] = (has_rand && t < p.num_rand) ? rand_block(p, w.b, tr.head, tr.u0, t) : -1;
       // this thread's position of the unit's first global-column tile, loaded early
-      const int gpos0 = (w.ngc > 0 && row < p.g) ? __ldg(p.global_idx + (size_t)w.b * p.g + row) : -1;
+      const int gpos0 = (GLOB && w.ngc > 0 && row < p.g) ? __ldg(p.global_idx + (size_t)w.b * p.g + row) : -1;
       int klo, khi;                            // band keys [klo, khi) of this row
       if (MODE == 0) {
         klo = u - w.r;
@@ -868,7 +869,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (!kMaxAfter) tmax = row_max128(s) * sl2;
             raw = true;
           }
-        } else if (j < w.nband + w.ngc) {
+        } else if (GLOB && j < w.nband + w.ngc) {
           // global-column tile: stage its 128 positions in shared memory (one per
           // thread of the group), each with the per-key facts every row shares:
           // -1 for no key (or a key a random block of this tile already counts),
@@ -887,16 +888,53 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (in_rand) code = -1;
             else if (w.d > 1 && code % w.d != w.c) code |= 1 << 30;
           }
-          named_barrier_sync(1 + x, 128);      // the previous tile's readers are done
-          sGpos[x * kTile + row] = code;
-          named_barrier_sync(1 + x, 128);
+          if constexpr (has_rand) {
+            named_barrier_sync(1 + x, 128);      // the previous tile's readers are done
+            sGpos[x * kTile + row] = code;
+            named_barrier_sync(1 + x, 128);
 #pragma unroll
-          for (int e = 0; e < kTile; ++e) {
-            const int cv = sGpos[x * kTile + e];
-            const int diff = pos - (cv & ~(1 << 30));
-            const bool inwin = !(cv & (1 << 30)) && (p.causal ? (diff >= 0 && diff <= rd) : (abs(diff) <= rd));
-            const bool allowed = row_valid && cv >= 0 && !inwin;
-            s[e] = allowed ? s[e] * sl2 : -INFINITY;
+            for (int e = 0; e < kTile; ++e) {
+              const int cv = sGpos[x * kTile + e];
+              const int diff = pos - (cv & ~(1 << 30));
+              const bool inwin =
+                  !(cv & (1 << 30)) && (p.causal ? (diff >= 0 && diff <= rd) : (abs(diff) <= rd));
+              const bool allowed = row_valid && cv >= 0 && !inwin;
+              s[e] = allowed ? s[e] * sl2 : -INFINITY;
+            }
+          } else {
+            // Without random blocks and without the causal cut (global tokens never come
+            // with it), a key is masked iff it lies beyond the g global slots or inside the
+            // row's window, |pos - key| <= rd: one unsigned compare, (unsigned)(pos + rd -
+            // key) <= 2 rd.  A key of another residue class is staged as a position no
+            // window reaches.
+            const bool fast = !p.causal;
+            if (fast && code >= 0) code = (code & (1 << 30)) ? -(1 << 29) : code;
+            named_barrier_sync(1 + x, 128);    // the previous tile's readers are done
+            sGpos[x * kTile + row] = code;
+            named_barrier_sync(1 + x, 128);
+            if (fast) {
+              const int posr = pos + rd;
+              const unsigned span = 2u * (unsigned)rd;
+              const int glim = row_valid ? p.g - e0 : 0;   // slots of this tile that hold a key
+#pragma unroll
+              for (int e = 0; e < kTile; e += 4) {
+                const int4 kp = *reinterpret_cast<const int4*>(&sGpos[x * kTile + e]);
+                s[e] = (e < glim && (unsigned)(posr - kp.x) > span) ? s[e] * sl2 : -INFINITY;
+                s[e + 1] = (e + 1 < glim && (unsigned)(posr - kp.y) > span) ? s[e + 1] * sl2 : -INFINITY;
+                s[e + 2] = (e + 2 < glim && (unsigned)(posr - kp.z) > span) ? s[e + 2] * sl2 : -INFINITY;
+                s[e + 3] = (e + 3 < glim && (unsigned)(posr - kp.w) > span) ? s[e + 3] * sl2 : -INFINITY;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < kTile; ++e) {
+                const int cv = sGpos[x * kTile + e];
+                const int diff = pos - (cv & ~(1 << 30));
+                const bool inwin =
+                    !(cv & (1 << 30)) && (p.causal ? (diff >= 0 && diff <= rd) : (abs(diff) <= rd));
+                const bool allowed = row_valid && cv >= 0 && !inwin;
+                s[e] = allowed ? s[e] * sl2 : -INFINITY;
+              }
+            }
           }
           if (!kMaxAfter) tmax = row_max128(s);
         } else if (has_rand && j >= w.rand0) {
@@ -1169,9 +1207,9 @@ size_t band_tc_smem_bytes(int D) {
   return D == 64 ? Cfg<64>::kSmemBytes : Cfg<128>::kSmemBytes;
 }
 
-template <int D, int MODE, bool LOCAL = false, bool RAND = false, bool AGG = false>
+template <int D, int MODE, bool LOCAL = false, bool RAND = false, bool AGG = false, bool GLOB = true>
 static cudaError_t launch_one(const AttnParams& p, int units, int num_sms, cudaStream_t s) {
-  auto kern = attn_tc_kernel<D, MODE, LOCAL, RAND, AGG>;
+  auto kern = attn_tc_kernel<D, MODE, LOCAL, RAND, AGG, GLOB>;
   const int smem = static_cast<int>(Cfg<D>::kSmemBytes);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -1197,23 +1235,31 @@ static cudaError_t launch_one(const AttnParams& p, int units, int num_sms, cudaS
 }
 
 // p.tiles[h] holds the number of two-tile units of head h, p.max_units their maximum.
-cudaError_t launch_band_tc(const AttnParams& p, int num_sms, cudaStream_t s) {
-  const int units = p.max_units * p.B * p.Hq;
+// The band kernel for one value of GLOB (global-column tiles present or not).
+template <bool GLOB>
+static cudaError_t launch_band_variant(const AttnParams& p, int units, int num_sms, cudaStream_t s) {
   if (p.agg_count) {      // side keys built in the prologue (no local bias, no random blocks)
-    return p.D == 64 ? launch_one<64, 0, false, false, true>(p, units, num_sms, s)
-                     : launch_one<128, 0, false, false, true>(p, units, num_sms, s);
+    return p.D == 64 ? launch_one<64, 0, false, false, true, GLOB>(p, units, num_sms, s)
+                     : launch_one<128, 0, false, false, true, GLOB>(p, units, num_sms, s);
   }
   if (p.num_rand > 0) {
     if (p.local_bias)
-      return p.D == 64 ? launch_one<64, 0, true, true>(p, units, num_sms, s)
-                       : launch_one<128, 0, true, true>(p, units, num_sms, s);
-    return p.D == 64 ? launch_one<64, 0, false, true>(p, units, num_sms, s)
-                     : launch_one<128, 0, false, true>(p, units, num_sms, s);
+      return p.D == 64 ? launch_one<64, 0, true, true, false, GLOB>(p, units, num_sms, s)
+                       : launch_one<128, 0, true, true, false, GLOB>(p, units, num_sms, s);
+    return p.D == 64 ? launch_one<64, 0, false, true, false, GLOB>(p, units, num_sms, s)
+                     : launch_one<128, 0, false, true, false, GLOB>(p, units, num_sms, s);
   }
   if (p.local_bias)
-    return p.D == 64 ? launch_one<64, 0, true>(p, units, num_sms, s)
-                     : launch_one<128, 0, true>(p, units, num_sms, s);
-  return p.D == 64 ? launch_one<64, 0>(p, units, num_sms, s) : launch_one<128, 0>(p, units, num_sms, s);
+    return p.D == 64 ? launch_one<64, 0, true, false, false, GLOB>(p, units, num_sms, s)
+                     : launch_one<128, 0, true, false, false, GLOB>(p, units, num_sms, s);
+  return p.D == 64 ? launch_one<64, 0, false, false, false, GLOB>(p, units, num_sms, s)
+                   : launch_one<128, 0, false, false, false, GLOB>(p, units, num_sms, s);
+}
+
+cudaError_t launch_band_tc(const AttnParams& p, int num_sms, cudaStream_t s) {
+  const int units = p.max_units * p.B * p.Hq;
+  return p.g > 0 ? launch_band_variant<true>(p, units, num_sms, s)
+                 : launch_band_variant<false>(p, units, num_sms, s);
 }
 
 cudaError_t launch_global_rows_tc(const AttnParams& p, int num_sms, cudaStream_t s) {

@@ -26,7 +26,8 @@ from tests import helpers
 
 pytestmark = pytest.mark.gpu
 
-SWA_OK, SWA_ERR_UNSUPPORTED = 0, 2
+SWA_OK, SWA_ERR_UNSUPPORTED, SWA_ERR_DEVICE_CHECK = 0, 2, 6
+SWA_DEBUG_CHECKS = 1
 
 
 def _need_gpu():
@@ -38,11 +39,11 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _noalloc(w, dinp, out, lse, max_global):
+def _noalloc(w, dinp, out, lse, max_global, flags=0):
     lib = load_library()
     S = 0 if dinp.get("side_k") is None else int(dinp["side_k"].shape[2])
     desc = PlanDesc(w.batch, w.seq_len, w.q_heads, w.kv_heads, w.head_dim,
-                    0 if w.dtype == "bf16" else 1, max_global, S, w.side_block if S else 0, 0.0, 0)
+                    0 if w.dtype == "bf16" else 1, max_global, S, w.side_block if S else 0, 0.0, flags)
     H = w.q_heads
     win = (ctypes.c_int32 * H)(*[int(x) for x in dinp["window"].tolist()])
     dil = (ctypes.c_int32 * H)(*[int(x) for x in dinp["dilation"].tolist()])
@@ -113,3 +114,30 @@ def test_noalloc_rejects_problems_beyond_the_scratch_limit():
     assert _noalloc(w, dinp, out, lse, max_global=w.num_global) == SWA_ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert bool((out == 0).all())                     # nothing was launched
+
+
+def test_noalloc_debug_mode_reports_device_checks():
+    """With SWA_DEBUG_CHECKS the allocation-free entry point synchronises and returns
+    what the device error word says: a global index list that breaks its
+    precondition (not increasing, beyond the sequence, negative) gives
+    SWA_ERR_DEVICE_CHECK before any kernel that indexes with it runs, so out stays
+    untouched; the next call with a valid list returns SWA_OK (the word was cleared)
+    and matches the plan-based forward."""
+    _need_gpu()
+    w = workloads.SMALL["longformer_base"]
+    dinp = helpers.to_dev(helpers.host_problem(w))
+    n = w.seq_len
+    out = torch.full((w.batch, w.q_heads, n, w.head_dim), 7.0, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((w.batch, w.q_heads, n), dtype=torch.float32, device="cuda")
+    for bad in ([3, 2, 5, 9], [2, 3, 5, n + 40], [-1, 3, 5, 9]):
+        d = dict(dinp, global_idx=torch.tensor([bad], dtype=torch.int32, device="cuda"))
+        st = _noalloc(w, d, out, lse, max_global=4, flags=SWA_DEBUG_CHECKS)
+        torch.cuda.synchronize()
+        assert st == SWA_ERR_DEVICE_CHECK, bad
+        assert bool((out == 7.0).all()), bad
+    good = torch.tensor([[2, 3, 5, 9]], dtype=torch.int32, device="cuda")
+    d = dict(dinp, global_idx=good)
+    assert _noalloc(w, d, out, lse, max_global=4, flags=SWA_DEBUG_CHECKS) == SWA_OK
+    torch.cuda.synchronize()
+    ref_out, ref_lse, _ = helpers.run_gpu(w, d)
+    _compare(w, out, lse, ref_out, ref_lse)
