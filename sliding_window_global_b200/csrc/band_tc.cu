@@ -952,11 +952,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           for (int t2 = 0; t2 < kRandRegs; ++t2) dup = dup || (t2 < t && rbl[t2] == kb);
           const int kv0 = kb * kTile;
           const int lo_t = klo - kv0, hi_t = khi - kv0, v_t = w.Vc - kv0;
+          // key e counts iff e < vlim (the valid keys of a live row and block) and it lies
+          // outside the row's window [lo_t, hi_t): (unsigned)(e - lo_t) >= hi_t - lo_t
+          const int vlim = (row_valid && !dup) ? v_t : 0;
+          const unsigned span = (unsigned)max(hi_t - lo_t, 0);
 #pragma unroll
-          for (int e = 0; e < kTile; ++e) {
-            const bool allowed = row_valid && !dup && e < v_t && (e < lo_t || e >= hi_t);
-            s[e] = allowed ? s[e] * sl2 : -INFINITY;
-          }
+          for (int e = 0; e < kTile; ++e)
+            s[e] = (e < vlim && (unsigned)(e - lo_t) >= span) ? s[e] * sl2 : -INFINITY;
           live = 0;
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch)
