@@ -888,10 +888,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (in_rand) code = -1;
             else if (w.d > 1 && code % w.d != w.c) code |= 1 << 30;
           }
-          if constexpr (has_rand) {
-            named_barrier_sync(1 + x, 128);      // the previous tile's readers are done
-            sGpos[x * kTile + row] = code;
-            named_barrier_sync(1 + x, 128);
+          // Without the causal cut (global tokens never come with it), a key is masked iff it
+          // lies beyond the g global slots or inside the row's window, |pos - key| <= rd:
+          // one unsigned compare, (unsigned)(pos + rd - key) <= 2 rd.  A key of another
+          // residue class is staged as a position no window reaches.  A key that a random
+          // block of this tile already counts (dilation 1 there) is staged as the position
+          // of the tile's middle row, which every row's window holds when r >= 64.
+          const bool fast = !p.causal && (!has_rand || w.r >= kTile / 2);
+          if (fast) {
+            if (code >= 0) code = (code & (1 << 30)) ? -(1 << 29) : code;
+            else if (has_rand) code = w.c + w.d * (tr.u0 + kTile / 2);
+          }
+          named_barrier_sync(1 + x, 128);      // the previous tile's readers are done
+          sGpos[x * kTile + row] = code;
+          named_barrier_sync(1 + x, 128);
+          if (fast) {
+            const int posr = pos + rd;
+            const unsigned span = 2u * (unsigned)rd;
+            const int glim = row_valid ? p.g - e0 : 0;     // slots of this tile that hold a key
+#pragma unroll
+            for (int e = 0; e < kTile; e += 4) {
+              const int4 kp = *reinterpret_cast<const int4*>(&sGpos[x * kTile + e]);
+              s[e] = (e < glim && (unsigned)(posr - kp.x) > span) ? s[e] * sl2 : -INFINITY;
+              s[e + 1] = (e + 1 < glim && (unsigned)(posr - kp.y) > span) ? s[e + 1] * sl2 : -INFINITY;
+              s[e + 2] = (e + 2 < glim && (unsigned)(posr - kp.z) > span) ? s[e + 2] * sl2 : -INFINITY;
+              s[e + 3] = (e + 3 < glim && (unsigned)(posr - kp.w) > span) ? s[e + 3] * sl2 : -INFINITY;
+            }
+          } else {
 #pragma unroll
             for (int e = 0; e < kTile; ++e) {
               const int cv = sGpos[x * kTile + e];
@@ -900,40 +923,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                   !(cv & (1 << 30)) && (p.causal ? (diff >= 0 && diff <= rd) : (abs(diff) <= rd));
               const bool allowed = row_valid && cv >= 0 && !inwin;
               s[e] = allowed ? s[e] * sl2 : -INFINITY;
-            }
-          } else {
-            // Without random blocks and without the causal cut (global tokens never come
-            // with it), a key is masked iff it lies beyond the g global slots or inside the
-            // row's window, |pos - key| <= rd: one unsigned compare, (unsigned)(pos + rd -
-            // key) <= 2 rd.  A key of another residue class is staged as a position no
-            // window reaches.
-            const bool fast = !p.causal;
-            if (fast && code >= 0) code = (code & (1 << 30)) ? -(1 << 29) : code;
-            named_barrier_sync(1 + x, 128);    // the previous tile's readers are done
-            sGpos[x * kTile + row] = code;
-            named_barrier_sync(1 + x, 128);
-            if (fast) {
-              const int posr = pos + rd;
-              const unsigned span = 2u * (unsigned)rd;
-              const int glim = row_valid ? p.g - e0 : 0;   // slots of this tile that hold a key
-#pragma unroll
-              for (int e = 0; e < kTile; e += 4) {
-                const int4 kp = *reinterpret_cast<const int4*>(&sGpos[x * kTile + e]);
-                s[e] = (e < glim && (unsigned)(posr - kp.x) > span) ? s[e] * sl2 : -INFINITY;
-                s[e + 1] = (e + 1 < glim && (unsigned)(posr - kp.y) > span) ? s[e + 1] * sl2 : -INFINITY;
-                s[e + 2] = (e + 2 < glim && (unsigned)(posr - kp.z) > span) ? s[e + 2] * sl2 : -INFINITY;
-                s[e + 3] = (e + 3 < glim && (unsigned)(posr - kp.w) > span) ? s[e + 3] * sl2 : -INFINITY;
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < kTile; ++e) {
-                const int cv = sGpos[x * kTile + e];
-                const int diff = pos - (cv & ~(1 << 30));
-                const bool inwin =
-                    !(cv & (1 << 30)) && (p.causal ? (diff >= 0 && diff <= rd) : (abs(diff) <= rd));
-                const bool allowed = row_valid && cv >= 0 && !inwin;
-                s[e] = allowed ? s[e] * sl2 : -INFINITY;
-              }
             }
           }
           if (!kMaxAfter) tmax = row_max128(s);

@@ -201,6 +201,9 @@ RANDOM = [
     ("rand_window_covers_seq", _small("bigbird_itc", window=(3000,) * 4, num_global=0,
                                       global_mode="none")),
     ("rand_tiny_seq", _small("bigbird_itc", seq_len=100, num_global=3, padding=7)),
+    # windows on both sides of r = 64, where a global key that a random block of the
+    # tile already counts switches from a per-key test to the one-compare mask
+    ("rand_globals_windows_around_64", _small("bigbird_itc", window=(40, 63, 64, 100))),
     ("rand_fp32", dataclasses.replace(workloads.SMALL["bigbird_itc"], dtype="fp32", seq_len=500,
                                       num_global=5)),
 ]
@@ -212,12 +215,15 @@ def test_random_blocks(name, w):
     _check_workload(w)
 
 
-def test_random_blocks_with_repeats_and_overlaps():
+@pytest.mark.parametrize("window", [None, (40, 63, 64, 100)], ids=["r100", "r40_63_64_100"])
+def test_random_blocks_with_repeats_and_overlaps(window):
     """Hand-written draws: a block repeated in the list, the query block itself, its
     neighbours (overlapping the window), a block holding global keys and the block
     holding the padded tail -- each key must still count once."""
     _need_gpu()
     w = _small("bigbird_itc", seq_len=1000, num_rand=5, padding=60)
+    if window is not None:
+        w = dataclasses.replace(w, window=window)
     inp = workloads.make_inputs(w)
     nqb = (w.seq_len + 127) // 128
     rb = torch.empty((1, w.q_heads, nqb, 5), dtype=torch.int32)
