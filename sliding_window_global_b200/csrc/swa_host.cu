@@ -172,6 +172,12 @@ swa_status enqueue_forward(const swa_plan_desc& d, const swa_forward_args& args,
     }
     local_stride = (int)align_up(2 * (size_t)r_eff_max + 2 * kLocalPad + 4, 32);
     if (d.dtype == SWA_BF16 && local_stride > band_bias_copy(d.head_dim)) return SWA_ERR_UNSUPPORTED;
+    // The band kernel keeps four copies of the row, shifted by 0..3 floats, local_stride
+    // apart, and a 16-byte read takes copy (key offset & 3) at the offset rounded down
+    // to 4.  Four consecutive rows (one quarter-warp step of that read) use the four
+    // copies at one rounded offset: copies 8 floats past a multiple of 32 apart put
+    // them on different shared-memory banks, where a multiple of 32 would stack them.
+    if (local_stride + 8 <= band_bias_copy(d.head_dim)) local_stride += 8;
   }
   const bool bf16 = d.dtype == SWA_BF16;
   if (bf16 && num_global > 0 && (!ws.gq || !ws.gk || !ws.gv || !ws.part_o || !ws.part_lse))
