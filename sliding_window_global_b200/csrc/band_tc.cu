@@ -64,10 +64,19 @@ namespace {
 
 constexpr int kSoftmaxThreads = 256;
 constexpr int kThreads = 384;                 // 3 warpgroups: softmax A, softmax B, control
-// Registers per thread after reallocation: 256 * 200 + 128 * 104 = 384 * 168, the
-// budget the CTA is launched with (168 per thread for 384 threads).
-constexpr int kRegsSoftmax = 200;
-constexpr int kRegsControl = 104;
+// Registers per thread after reallocation, per head size: the softmax warps get 200
+// at D = 128 and 216 at D = 64, the control warps 104 and 72 (256 * 200 + 128 * 104 =
+// 256 * 216 + 128 * 72 = 384 * 168, the budget the CTA is launched with).  The split
+// was chosen by the compiler's spill counts: at D = 64 the wider softmax budget
+// removes most spills, at D = 128 the control warps need the 104.
+template <int D>
+__host__ __device__ constexpr int regs_softmax() {
+  return D == 64 ? 216 : 200;
+}
+template <int D>
+__host__ __device__ constexpr int regs_control() {
+  return D == 64 ? 72 : 104;
+}
 constexpr uint32_t kSub = 128 * 128;          // one 128-row x 128-byte swizzle sub-tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -122,10 +131,13 @@ struct Cfg {
 // setmaxnreg moves registers only between the warps of one SM sub-partition (warp
 // w runs on sub-partition w % 4), so the split must also fit each sub-partition's
 // share: here one warp of each softmax group and one control warp.
-static_assert(kSoftmaxThreads * kRegsSoftmax + (kThreads - kSoftmaxThreads) * kRegsControl <= kThreads * 168,
-              "setmaxnreg split exceeds the launch register budget");
-static_assert(kThreads == 12 * 32 && kSoftmaxThreads == 8 * 32 && 2 * kRegsSoftmax + kRegsControl <= 3 * 168,
-              "setmaxnreg split exceeds a sub-partition's registers");
+template <int D>
+constexpr bool split_fits() {
+  return kSoftmaxThreads * regs_softmax<D>() + (kThreads - kSoftmaxThreads) * regs_control<D>() <= kThreads * 168 &&
+         2 * regs_softmax<D>() + regs_control<D>() <= 3 * 168;
+}
+static_assert(kThreads == 12 * 32 && kSoftmaxThreads == 8 * 32 && split_fits<64>() && split_fits<128>(),
+              "setmaxnreg split exceeds the launch budget or a sub-partition's registers");
 static_assert(Cfg<64>::kSmemBytes + 2 * kTile * 4 + 16 <= 227 * 1024, "shared memory, D = 64");
 static_assert(Cfg<128>::kSmemBytes + 2 * kTile * 4 + 16 <= 227 * 1024, "shared memory, D = 128");
 static_assert(emu_per32<64>() % 4 == 0 && emu_per32<64>() <= 32 && emu_per32<128>() % 4 == 0 &&
@@ -487,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   }
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
-    setmaxnreg_dec<kRegsControl>();
+    setmaxnreg_dec<regs_control<D>()>();
     if (lane == 0) {
       int qloads[2] = {0, 0};
       int kv = 0;                                   // K/V tiles loaded so far (ring position)
@@ -544,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // keeps the two softmax groups half a period apart.  Separate P (D = 64): warp
     // 9 issues tile A's MMAs and warp 10 tile B's, so neither tile's products wait
     // behind the other tile's barriers.
-    setmaxnreg_dec<kRegsControl>();
+    setmaxnreg_dec<regs_control<D>()>();
     if (lane == 0) {
       const int x0 = (kIssuers == 2) ? warp - 9 : 0;   // first tile of this issuer
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
@@ -675,10 +687,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
     }
   } else if (warp >= 10) {
-    setmaxnreg_dec<kRegsControl>();
+    setmaxnreg_dec<regs_control<D>()>();
   } else {
     // ------------------------------------------------------------ softmax warpgroups
-    setmaxnreg_inc<kRegsSoftmax>();
+    setmaxnreg_inc<regs_softmax<D>()>();
     const int x = warp >> 2;                   // 0: tile A, 1: tile B
     const int row = tid & 127;                 // TMEM lane == row in the tile
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
