@@ -558,36 +558,53 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
           tmem_st16(sb + ch * 16, pk);
           continue;
         }
+        if constexpr (!GROWS && !X) {
+          // band boundary tile: the same packed steps, then keys outside the row's
+          // window [lo_t, hi_t) (one unsigned compare each) give p = 0
+          const unsigned span = (unsigned)max(hi_t - lo_t, 0);
 #pragma unroll
-        for (int q = 0; q < 32; q += 2) {
-          float ds[2];
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int e = ch * 32 + q + h2;
-            bool allowed;
-            float b2 = 0.f;                    // bias in log2 units
-            if (GROWS) {
-              const int key = kv0 + e;
-              allowed = row_valid && key < u.Vc && !in_window(qpos, key, rd, u.d, p.causal);
-            } else if (!X || kind == 0) {
-              allowed = e >= lo_t && e < hi_t;
-              if (X && lrow && allowed) b2 = __ldg(lrow + u.d * (kv0 + e - uq)) * kBLog2e;
-            } else if (kind == 1) {
-              const int cv = sGpos[e];
-              allowed = row_valid && !row_global && cv >= 0 && !in_window(qpos, cv, rd, u.d, p.causal);
-            } else if (kind == 2) {
-              const int sg = base + e;
-              allowed = row_valid && sg < p.S;
-              if (srow && allowed) b2 = __ldg(srow + sg) * kBLog2e;
-            } else {
-              const int key = kv0 + e;
-              allowed = row_valid && !row_global && !dup && key < u.Vc &&
-                        !in_window(qpos, key, rd, 1, p.causal);
-            }
-            const float pr = allowed ? ex2_approx(__uint_as_float(sr[q + h2]) * sl2 + b2 - lse2) : 0.f;
-            ds[h2] = pr * (__uint_as_float(dr[q + h2]) - delta);
+          for (int q = 0; q < 32; q += 2) {
+            const int e = ch * 32 + q;
+            float a0, a1, t0, t1, d0, d1;
+            ffma2(a0, a1, __uint_as_float(sr[q]), __uint_as_float(sr[q + 1]), sl2, sl2, nl2, nl2);
+            a0 = ((unsigned)(e - lo_t) < span) ? ex2_approx(a0) : 0.f;
+            a1 = ((unsigned)(e + 1 - lo_t) < span) ? ex2_approx(a1) : 0.f;
+            fadd2(t0, t1, __uint_as_float(dr[q]), __uint_as_float(dr[q + 1]), nd, nd);
+            ffma2(d0, d1, a0, a1, t0, t1, 0.f, 0.f);
+            pk[q / 2] = pack_bf16x2(d0, d1);
           }
-          pk[q / 2] = pack_bf16x2(ds[0], ds[1]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; q += 2) {
+            float ds[2];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int e = ch * 32 + q + h2;
+              bool allowed;
+              float b2 = 0.f;                    // bias in log2 units
+              if (GROWS) {
+                const int key = kv0 + e;
+                allowed = row_valid && key < u.Vc && !in_window(qpos, key, rd, u.d, p.causal);
+              } else if (!X || kind == 0) {
+                allowed = e >= lo_t && e < hi_t;
+                if (X && lrow && allowed) b2 = __ldg(lrow + u.d * (kv0 + e - uq)) * kBLog2e;
+              } else if (kind == 1) {
+                const int cv = sGpos[e];
+                allowed = row_valid && !row_global && cv >= 0 && !in_window(qpos, cv, rd, u.d, p.causal);
+              } else if (kind == 2) {
+                const int sg = base + e;
+                allowed = row_valid && sg < p.S;
+                if (srow && allowed) b2 = __ldg(srow + sg) * kBLog2e;
+              } else {
+                const int key = kv0 + e;
+                allowed = row_valid && !row_global && !dup && key < u.Vc &&
+                          !in_window(qpos, key, rd, 1, p.causal);
+              }
+              const float pr = allowed ? ex2_approx(__uint_as_float(sr[q + h2]) * sl2 + b2 - lse2) : 0.f;
+              ds[h2] = pr * (__uint_as_float(dr[q + h2]) - delta);
+            }
+            pk[q / 2] = pack_bf16x2(ds[0], ds[1]);
+          }
         }
         // dS as bf16 over S: chunk ch writes columns 16ch.. that earlier chunks read
         tmem_st16(sb + ch * 16, pk);
@@ -1024,6 +1041,23 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
                     lv[e], lv[e + 1]);
               pr[e] = ex2_approx(a0);
               pr[e + 1] = ex2_approx(a1);
+              fadd2(t0, t1, __uint_as_float(dr[c4 * 8 + e]), __uint_as_float(dr[c4 * 8 + e + 1]), dv[e], dv[e + 1]);
+              ffma2(ds[e], ds[e + 1], pr[e], pr[e + 1], t0, t1, 0.f, 0.f);
+            }
+          } else if (JOB == kJobBand) {
+            // band boundary tile: the packed steps of the interior, then pairs outside
+            // the band (offset outside [lo, lo + span), one unsigned compare each; a
+            // padded key has span 0) give p = 0
+            const int lo = p.causal ? 0 : -u.r;
+            const unsigned span = key_valid ? (unsigned)(p.causal ? u.r + 1 : 2 * u.r + 1) : 0u;
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              const int off = d0 + c * 8 + e;
+              float a0, a1, t0, t1;
+              ffma2(a0, a1, __uint_as_float(sr[c4 * 8 + e]), __uint_as_float(sr[c4 * 8 + e + 1]), sl2, sl2,
+                    lv[e], lv[e + 1]);
+              pr[e] = ((unsigned)(off - lo) < span) ? ex2_approx(a0) : 0.f;
+              pr[e + 1] = ((unsigned)(off + 1 - lo) < span) ? ex2_approx(a1) : 0.f;
               fadd2(t0, t1, __uint_as_float(dr[c4 * 8 + e]), __uint_as_float(dr[c4 * 8 + e + 1]), dv[e], dv[e + 1]);
               ffma2(ds[e], ds[e + 1], pr[e], pr[e + 1], t0, t1, 0.f, 0.f);
             }
