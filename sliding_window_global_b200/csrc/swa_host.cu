@@ -302,12 +302,13 @@ swa_status enqueue_forward(const swa_plan_desc& d, const swa_forward_args& args,
                           (uint64_t)d.num_side * row);
     }
     if (!ok) return SWA_ERR_CUDA;
-    // global-row split: about two waves of CTAs over the key tiles
+    // global-row split: at most one wave of CTAs over the key tiles (measured against
+    // two waves and half a wave: fewer, longer units and fewer partials to merge)
     if (num_global > 0) {
       const int ntiles = (n + kTile - 1) / kTile;
       const int side_split = d.num_side > 0 ? 1 : 0;
       const long long units = (long long)p.B * Hq * (p.gpad / kTile);
-      int want = (int)std::max(1LL, (2LL * num_sms + units - 1) / units);
+      int want = (int)std::max(1LL, (long long)num_sms / units);
       want = std::min(want, std::min(ntiles, ws.nsplit_max - side_split));
       if (want < 1) return SWA_ERR_INVALID_ARG;
       const int tiles_per = (ntiles + want - 1) / want;
