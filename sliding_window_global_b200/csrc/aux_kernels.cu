@@ -65,6 +65,7 @@ __global__ void gather_rows_kernel(const GatherSet gs, const int32_t* __restrict
 // One warp per global row: o = sum_s w_s o_s / sum_s w_s, w_s = exp(lse_s - max).
 template <typename T, int D>
 __global__ void merge_global_rows_kernel(AttnParams p) {
+  grid_dependency_wait();               // the partials of the global-row kernel before it
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int rows = p.B * p.Hq * p.g;
@@ -381,14 +382,21 @@ cudaError_t launch_merge_global_rows(const AttnParams& p, int bf16_out, cudaStre
   const int rows = p.B * p.Hq * p.g;
   const int threads = 256;
   const int blocks = (rows * 32 + threads - 1) / threads;
-  if (bf16_out) {
-    if (p.D == 64) merge_global_rows_kernel<__nv_bfloat16, 64><<<blocks, threads, 0, s>>>(p);
-    else merge_global_rows_kernel<__nv_bfloat16, 128><<<blocks, threads, 0, s>>>(p);
-  } else {
-    if (p.D == 64) merge_global_rows_kernel<float, 64><<<blocks, threads, 0, s>>>(p);
-    else merge_global_rows_kernel<float, 128><<<blocks, threads, 0, s>>>(p);
-  }
-  return cudaGetLastError();
+  // programmatic dependent launch behind the global-row kernel (the kernel waits)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(threads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (bf16_out)
+    return p.D == 64 ? cudaLaunchKernelEx(&cfg, merge_global_rows_kernel<__nv_bfloat16, 64>, p)
+                     : cudaLaunchKernelEx(&cfg, merge_global_rows_kernel<__nv_bfloat16, 128>, p);
+  return p.D == 64 ? cudaLaunchKernelEx(&cfg, merge_global_rows_kernel<float, 64>, p)
+                   : cudaLaunchKernelEx(&cfg, merge_global_rows_kernel<float, 128>, p);
 }
 
 cudaError_t launch_simt(const AttnParams& p, const void* q, const void* k, const void* v,

@@ -490,6 +490,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
   volatile int* abort_v = &abort_flag;
+  // Launched right behind the kernel that produces its inputs (the gathered global
+  // rows, the band output the global rows follow), this kernel has set up its
+  // barriers and TMEM meanwhile; nothing before this point reads global memory.
+  grid_dependency_wait();
   if (AGG) {
     side_prologue<D>(p, tid, kThreads);
     fence_proxy_async_global();                // side rows written here are read by TMA
@@ -1211,7 +1215,7 @@ size_t band_tc_smem_bytes(int D) {
 }
 
 template <int D, int MODE, bool LOCAL = false, bool RAND = false, bool AGG = false, bool GLOB = true>
-static cudaError_t launch_one(const AttnParams& p, int units, int num_sms, cudaStream_t s) {
+static cudaError_t launch_one(const AttnParams& p, int units, int num_sms, cudaStream_t s, bool pdl = false) {
   auto kern = attn_tc_kernel<D, MODE, LOCAL, RAND, AGG, GLOB>;
   const int smem = static_cast<int>(Cfg<D>::kSmemBytes);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1233,6 +1237,20 @@ static cudaError_t launch_one(const AttnParams& p, int units, int num_sms, cudaS
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, p);
   }
+  if (pdl) {
+    // programmatic dependent launch: scheduled while the previous kernel drains
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
+  }
   kern<<<grid, kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
@@ -1247,16 +1265,16 @@ static cudaError_t launch_band_variant(const AttnParams& p, int units, int num_s
   }
   if (p.num_rand > 0) {
     if (p.local_bias)
-      return p.D == 64 ? launch_one<64, 0, true, true, false, GLOB>(p, units, num_sms, s)
-                       : launch_one<128, 0, true, true, false, GLOB>(p, units, num_sms, s);
-    return p.D == 64 ? launch_one<64, 0, false, true, false, GLOB>(p, units, num_sms, s)
-                     : launch_one<128, 0, false, true, false, GLOB>(p, units, num_sms, s);
+      return p.D == 64 ? launch_one<64, 0, true, true, false, GLOB>(p, units, num_sms, s, GLOB)
+                       : launch_one<128, 0, true, true, false, GLOB>(p, units, num_sms, s, GLOB);
+    return p.D == 64 ? launch_one<64, 0, false, true, false, GLOB>(p, units, num_sms, s, GLOB)
+                     : launch_one<128, 0, false, true, false, GLOB>(p, units, num_sms, s, GLOB);
   }
   if (p.local_bias)
-    return p.D == 64 ? launch_one<64, 0, true, false, false, GLOB>(p, units, num_sms, s)
-                     : launch_one<128, 0, true, false, false, GLOB>(p, units, num_sms, s);
-  return p.D == 64 ? launch_one<64, 0, false, false, false, GLOB>(p, units, num_sms, s)
-                   : launch_one<128, 0, false, false, false, GLOB>(p, units, num_sms, s);
+    return p.D == 64 ? launch_one<64, 0, true, false, false, GLOB>(p, units, num_sms, s, GLOB)
+                     : launch_one<128, 0, true, false, false, GLOB>(p, units, num_sms, s, GLOB);
+  return p.D == 64 ? launch_one<64, 0, false, false, false, GLOB>(p, units, num_sms, s, GLOB)
+                   : launch_one<128, 0, false, false, false, GLOB>(p, units, num_sms, s, GLOB);
 }
 
 cudaError_t launch_band_tc(const AttnParams& p, int num_sms, cudaStream_t s) {
@@ -1267,7 +1285,7 @@ cudaError_t launch_band_tc(const AttnParams& p, int num_sms, cudaStream_t s) {
 
 cudaError_t launch_global_rows_tc(const AttnParams& p, int num_sms, cudaStream_t s) {
   const int units = p.nsplit * (p.gpad / kTile) * p.B * p.Hq;
-  return p.D == 64 ? launch_one<64, 1>(p, units, num_sms, s) : launch_one<128, 1>(p, units, num_sms, s);
+  return p.D == 64 ? launch_one<64, 1>(p, units, num_sms, s, true) : launch_one<128, 1>(p, units, num_sms, s, true);
 }
 
 int band_bias_copy(int) { return kBiasCopy; }
