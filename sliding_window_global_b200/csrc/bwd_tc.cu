@@ -326,6 +326,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
   volatile int* abort_v = &abort_flag;
+  grid_dependency_wait();           // Delta (and the gathered rows) of the kernels before
   const int nqb = (p.n + kTile - 1) / kTile;
   // Every role walks the same units in the same order and keeps the same counters:
   // ka, units with key tiles so far (phases of a_full, stat_empty, acc_full), and jg,
@@ -859,6 +860,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
   volatile int* abort_v = &abort_flag;
+  grid_dependency_wait();           // the passes before: Delta, dq, and dk/dv that this job adds to
   const int kz = u.b * p.Hkv + u.hk;
 
   if (warp == 8) {
@@ -1168,13 +1170,25 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
   }
 }
 
+// Every dQ and dK/dV launch follows the Delta pass (and the gather) of the same
+// backward, so it is a programmatic dependent launch: scheduled while the kernel
+// before it drains, it sets up its barriers and TMEM and then waits for it.
 template <typename K>
 cudaError_t launch_kern(K kern, uint32_t smem, int grid, int threads, const BwdParams& p, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, threads, smem, s>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 }  // namespace
