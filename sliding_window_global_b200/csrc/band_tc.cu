@@ -490,10 +490,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
   volatile int* abort_v = &abort_flag;
-  // Launched right behind the kernel that produces its inputs (the gathered global
-  // rows, the band output the global rows follow), this kernel has set up its
-  // barriers and TMEM meanwhile; nothing before this point reads global memory.
-  grid_dependency_wait();
+  // Launched right behind the kernel before it, this kernel has set up its barriers
+  // and TMEM meanwhile; nothing before this point reads global memory.  The band
+  // kernel (MODE 0) waits here for the gathered global rows, then lets the
+  // global-row kernel after it start on SMs its CTAs leave: that kernel reads only
+  // the gathered rows, which are complete now, and waits for this grid only at its
+  // end, before the merge that overwrites the band's global rows.
+  if (MODE == 0) {
+    grid_dependency_wait();
+    if (GLOB) grid_launch_dependents();
+  }
   if (AGG) {
     side_prologue<D>(p, tid, kThreads);
     fence_proxy_async_global();                // side rows written here are read by TMA
@@ -1187,6 +1193,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   }
 
   if (warp < 8 && (tid & 127) == 0) tma_store_wait_read<0>();   // staged stores have read smem
+  if (MODE == 1) grid_dependency_wait();    // the band grid, before the merge behind this one
   tc_fence_before();
   __syncthreads();
   if (abort_flag) {
