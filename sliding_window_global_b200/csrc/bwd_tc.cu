@@ -559,9 +559,9 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
           tmem_st16(sb + ch * 16, pk);
           continue;
         }
-        if constexpr (!GROWS && !X) {
-          // band boundary tile: the same packed steps, then keys outside the row's
-          // window [lo_t, hi_t) (one unsigned compare each) give p = 0
+        // band boundary tile: the packed steps of the interior, then keys outside the
+        // row's window [lo_t, hi_t) (one unsigned compare each) give p = 0
+        auto band_packed = [&]() {
           const unsigned span = (unsigned)max(hi_t - lo_t, 0);
 #pragma unroll
           for (int q = 0; q < 32; q += 2) {
@@ -574,7 +574,9 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
             ffma2(d0, d1, a0, a1, t0, t1, 0.f, 0.f);
             pk[q / 2] = pack_bf16x2(d0, d1);
           }
-        } else {
+        };
+        // per-element path: every tile kind, with its masks and biases
+        auto generic_path = [&]() {
 #pragma unroll
           for (int q = 0; q < 32; q += 2) {
             float ds[2];
@@ -606,6 +608,37 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
             }
             pk[q / 2] = pack_bf16x2(ds[0], ds[1]);
           }
+        };
+        if constexpr (GROWS) {
+          generic_path();
+        } else if constexpr (!X) {
+          band_packed();
+        } else if (kind == 0 && !p.local_bias) {
+          band_packed();
+        } else if (kind == 2) {
+          // side tile: p = 2^(s scale log2e + bias log2e - lse log2e) for side keys below
+          // S (every valid row attends them), packed steps; the bias of each key is read
+          // from the row's side-bias row
+          const int lim = row_valid ? p.S - base : 0;
+#pragma unroll
+          for (int q = 0; q < 32; q += 2) {
+            const int e = ch * 32 + q;
+            float b0 = 0.f, b1 = 0.f;
+            if (srow) {
+              b0 = e < lim ? __ldg(srow + base + e) : 0.f;
+              b1 = e + 1 < lim ? __ldg(srow + base + e + 1) : 0.f;
+            }
+            float a0, a1, t0, t1, d0, d1;
+            ffma2(a0, a1, b0, b1, kBLog2e, kBLog2e, nl2, nl2);
+            ffma2(a0, a1, __uint_as_float(sr[q]), __uint_as_float(sr[q + 1]), sl2, sl2, a0, a1);
+            a0 = e < lim ? ex2_approx(a0) : 0.f;
+            a1 = e + 1 < lim ? ex2_approx(a1) : 0.f;
+            fadd2(t0, t1, __uint_as_float(dr[q]), __uint_as_float(dr[q + 1]), nd, nd);
+            ffma2(d0, d1, a0, a1, t0, t1, 0.f, 0.f);
+            pk[q / 2] = pack_bf16x2(d0, d1);
+          }
+        } else {
+          generic_path();
         }
         // dS as bf16 over S: chunk ch writes columns 16ch.. that earlier chunks read
         tmem_st16(sb + ch * 16, pk);
