@@ -559,22 +559,29 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
           tmem_st16(sb + ch * 16, pk);
           continue;
         }
-        // band boundary tile: the packed steps of the interior, then keys outside the
-        // row's window [lo_t, hi_t) (one unsigned compare each) give p = 0
-        auto band_packed = [&]() {
-          const unsigned span = (unsigned)max(hi_t - lo_t, 0);
+        // the packed steps of the interior; keys the predicate rejects give p = 0
+        auto masked_packed = [&](auto allow) {
 #pragma unroll
           for (int q = 0; q < 32; q += 2) {
             const int e = ch * 32 + q;
             float a0, a1, t0, t1, d0, d1;
             ffma2(a0, a1, __uint_as_float(sr[q]), __uint_as_float(sr[q + 1]), sl2, sl2, nl2, nl2);
-            a0 = ((unsigned)(e - lo_t) < span) ? ex2_approx(a0) : 0.f;
-            a1 = ((unsigned)(e + 1 - lo_t) < span) ? ex2_approx(a1) : 0.f;
+            a0 = allow(e) ? ex2_approx(a0) : 0.f;
+            a1 = allow(e + 1) ? ex2_approx(a1) : 0.f;
             fadd2(t0, t1, __uint_as_float(dr[q]), __uint_as_float(dr[q + 1]), nd, nd);
             ffma2(d0, d1, a0, a1, t0, t1, 0.f, 0.f);
             pk[q / 2] = pack_bf16x2(d0, d1);
           }
         };
+        // band boundary tile: keys outside the row's window [lo_t, hi_t), one unsigned
+        // compare each
+        auto band_packed = [&]() {
+          const unsigned span = (unsigned)max(hi_t - lo_t, 0);
+          masked_packed([&](int e) { return (unsigned)(e - lo_t) < span; });
+        };
+        // Without dilation and the causal cut, "outside the row's window" is one unsigned
+        // compare: (unsigned)(qpos + rd - key) > 2 rd.
+        const unsigned span2 = 2u * (unsigned)rd;
         // per-element path: every tile kind, with its masks and biases
         auto generic_path = [&]() {
 #pragma unroll
@@ -610,7 +617,14 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
           }
         };
         if constexpr (GROWS) {
-          generic_path();
+          if (u.d == 1 && !p.causal) {
+            // a global row over every key tile: valid keys outside its window
+            const int vlim = row_valid ? u.Vc - kv0 : 0;
+            const int br = qpos + rd - kv0;
+            masked_packed([&](int e) { return e < vlim && (unsigned)(br - e) > span2; });
+          } else {
+            generic_path();
+          }
         } else if constexpr (!X) {
           band_packed();
         } else if (kind == 0 && !p.local_bias) {
@@ -637,6 +651,21 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
             ffma2(d0, d1, a0, a1, t0, t1, 0.f, 0.f);
             pk[q / 2] = pack_bf16x2(d0, d1);
           }
+        } else if (kind == 1 && u.d == 1 && !p.causal) {
+          // global-column tile: staged keys (-1: none, or counted by a random block)
+          // outside the row's window, for rows that are not global themselves
+          const bool row_ok = row_valid && !row_global;
+          const int qr = qpos + rd;
+          masked_packed([&](int e) {
+            const int cv = sGpos[e];
+            return row_ok && cv >= 0 && (unsigned)(qr - cv) > span2;
+          });
+        } else if (kind == 3 && !p.causal) {
+          // random tile (dilation 1): valid keys of a first occurrence of the block,
+          // outside the row's window, for rows that are not global
+          const int vlim = (row_valid && !row_global && !dup) ? u.Vc - kv0 : 0;
+          const int br = qpos + rd - kv0;
+          masked_packed([&](int e) { return e < vlim && (unsigned)(br - e) > span2; });
         } else {
           generic_path();
         }
