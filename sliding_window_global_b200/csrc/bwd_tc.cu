@@ -1034,7 +1034,9 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
           take = uq < u.Vc;
           qp = uq;
           if (JOB == kJobGlobalKeys || JOB == kJobRandom) take = take && !is_global_pos(p, u.b, qp);
-          if (JOB == kJobSide) ex = qp / p.side_block;                 // query block of the side bias
+          // query block of the side bias (block 0 for rows that do not count, so that the
+          // bias read of every column stays inside the table)
+          if (JOB == kJobSide) ex = take ? qp / p.side_block : 0;
         }
         if (take) {
           const size_t pr = ((size_t)u.b * p.Hq + qt.head) * p.n + qp;
@@ -1108,7 +1110,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
               fadd2(t0, t1, __uint_as_float(dr[c4 * 8 + e]), __uint_as_float(dr[c4 * 8 + e + 1]), dv[e], dv[e + 1]);
               ffma2(ds[e], ds[e + 1], pr[e], pr[e + 1], t0, t1, 0.f, 0.f);
             }
-          } else if (JOB == kJobBand) {
+          } else if (JOB == kJobBand || (JOB == kJobBandX && qt.src == 0 && !p.local_bias)) {
             // band boundary tile: the packed steps of the interior, then pairs outside
             // the band (offset outside [lo, lo + span), one unsigned compare each; a
             // padded key has span 0) give p = 0
@@ -1122,6 +1124,42 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
                     lv[e], lv[e + 1]);
               pr[e] = ((unsigned)(off - lo) < span) ? ex2_approx(a0) : 0.f;
               pr[e + 1] = ((unsigned)(off + 1 - lo) < span) ? ex2_approx(a1) : 0.f;
+              fadd2(t0, t1, __uint_as_float(dr[c4 * 8 + e]), __uint_as_float(dr[c4 * 8 + e + 1]), dv[e], dv[e + 1]);
+              ffma2(ds[e], ds[e + 1], pr[e], pr[e + 1], t0, t1, 0.f, 0.f);
+            }
+          } else if (((JOB == kJobBandX && qt.src != 0) || JOB == kJobGlobalKeys || JOB == kJobRandom) &&
+                     !p.causal && (JOB == kJobRandom || u.d == 1)) {
+            // query rows whose window misses the key (global query rows of the band job,
+            // the global-key job, the random job; dilation 1): one unsigned compare on
+            // the staged query position, (unsigned)(qpos - kpos + rd) > 2 rd.  Rows that
+            // do not count have -lse = -inf and give p = 0 by themselves.
+            const bool kok = key_valid && !(JOB == kJobGlobalKeys && key_in_rand);
+            const int kr = rd - kpos;
+            const unsigned span2 = 2u * (unsigned)rd;
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              float a0, a1, t0, t1;
+              ffma2(a0, a1, __uint_as_float(sr[c4 * 8 + e]), __uint_as_float(sr[c4 * 8 + e + 1]), sl2, sl2,
+                    lv[e], lv[e + 1]);
+              pr[e] = (kok && (unsigned)(stgi[c * 8 + e] + kr) > span2) ? ex2_approx(a0) : 0.f;
+              pr[e + 1] = (kok && (unsigned)(stgi[c * 8 + e + 1] + kr) > span2) ? ex2_approx(a1) : 0.f;
+              fadd2(t0, t1, __uint_as_float(dr[c4 * 8 + e]), __uint_as_float(dr[c4 * 8 + e + 1]), dv[e], dv[e + 1]);
+              ffma2(ds[e], ds[e + 1], pr[e], pr[e + 1], t0, t1, 0.f, 0.f);
+            }
+          } else if (JOB == kJobSide) {
+            // side tile: every valid query row, with the side bias of its query block
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              float b0 = 0.f, b1 = 0.f;
+              if (sbias) {
+                b0 = __ldg(sbias - stgi[kQT + c * 8 + e]);
+                b1 = __ldg(sbias - stgi[kQT + c * 8 + e + 1]);
+              }
+              float a0, a1, t0, t1;
+              ffma2(a0, a1, b0, b1, kBLog2e, kBLog2e, lv[e], lv[e + 1]);
+              ffma2(a0, a1, __uint_as_float(sr[c4 * 8 + e]), __uint_as_float(sr[c4 * 8 + e + 1]), sl2, sl2, a0, a1);
+              pr[e] = key_valid ? ex2_approx(a0) : 0.f;
+              pr[e + 1] = key_valid ? ex2_approx(a1) : 0.f;
               fadd2(t0, t1, __uint_as_float(dr[c4 * 8 + e]), __uint_as_float(dr[c4 * 8 + e + 1]), dv[e], dv[e + 1]);
               ffma2(ds[e], ds[e + 1], pr[e], pr[e + 1], t0, t1, 0.f, 0.f);
             }
