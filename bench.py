@@ -222,16 +222,17 @@ def time_device(w, plan, dev, steps, warmup, device):
 
 
 def time_backward(w, plan, dev, steps, warmup, device):
-    """Per-step CUDA-event time of one backward (dq, dk, dv) from the forward's out and
-    lse and a seeded upstream gradient, L2 flushed before each step."""
+    """Per-step CUDA-event time of one backward (dq, dk, dv, and the side keys' gradients
+    when the workload has side keys) from the forward's out and lse and a seeded
+    upstream gradient, with every term of the workload's pattern, L2 flushed before
+    each step."""
     import torch
     from sliding_window_global_b200.profile_case import forward_kwargs
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
     out, lse = plan.forward(dev["q"], dev["k"], dev["v"], **forward_kwargs(w, dev))
     g = torch.Generator(device=device).manual_seed(11)
     dout = torch.randn(out.shape, generator=g, device=device).to(out.dtype)
-    kw = dict(window=list(w.window), dilation=list(w.dilation), causal=w.causal,
-              valid_len=dev["valid_len"])
+    kw = forward_kwargs(w, dev)
     grads = plan.backward(dev["q"], dev["k"], dev["v"], out, lse, dout, **kw)
     for _ in range(warmup):
         flush.fill_(1.0)
@@ -420,6 +421,13 @@ def run_ours(args):
                                    "useful_gflop_per_step": bflop / 1e9, "gpu_launches": blaunch,
                                    "frac_of_peak": bflop / (bms * 1e-3) / 1e12 / peaks["bf16_tflops"],
                                    "kernels": "bwd_delta + bwd_dq_kernel<D> + bwd_dkv_kernel<D>"}
+        elif not args.no_backward:
+            # secondary workloads: the backward of their full pattern
+            bms, blaunch = time_backward(w, plan, dev, args.steps, args.warmup, device)
+            bms = _max_over_ranks(dist, bms, device)
+            bflop = 2.5 * flop
+            res["backward"] = {"value": replica_throughput(bflop, world, bms), "unit": "TFLOP/s",
+                               "ms_per_step": bms, "gpu_launches": blaunch}
         plan.close()
         del dev
         torch.cuda.empty_cache()
@@ -456,12 +464,15 @@ def run_ours(args):
             line["secondary"] = []
             for sec in secs:
                 sw = sec.pop("w")
-                line["secondary"].append({
+                entry = {
                     "workload": sw.name, "value": sec["value"], "unit": "TFLOP/s",
                     "ms_per_step": sec["ms_per_step"],
                     "frac_of_peak": sec["value"] / world / peaks["bf16_tflops"],
                     "useful_gflop_per_step": sec["useful_gflop_per_step"],
-                    "gpu_launches": sec["gpu_launches"], "clocks": sec["clocks"]})
+                    "gpu_launches": sec["gpu_launches"], "clocks": sec["clocks"]}
+                if "backward" in sec:
+                    entry["backward"] = sec["backward"]
+                line["secondary"].append(entry)
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
