@@ -629,6 +629,28 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
           band_packed();
         } else if (kind == 0 && !p.local_bias) {
           band_packed();
+        } else if (kind == 0) {
+          // band tile with the local bias: keys of the row's window [lo_t, hi_t), each
+          // with the bias of its offset (none for a global row, lrow = null)
+          const unsigned span = (unsigned)max(hi_t - lo_t, 0);
+#pragma unroll
+          for (int q = 0; q < 32; q += 2) {
+            const int e = ch * 32 + q;
+            const bool in0 = (unsigned)(e - lo_t) < span, in1 = (unsigned)(e + 1 - lo_t) < span;
+            float b0 = 0.f, b1 = 0.f;
+            if (lrow) {
+              b0 = in0 ? __ldg(lrow + u.d * (kv0 + e - uq)) : 0.f;
+              b1 = in1 ? __ldg(lrow + u.d * (kv0 + e + 1 - uq)) : 0.f;
+            }
+            float a0, a1, t0, t1, d0, d1;
+            ffma2(a0, a1, b0, b1, kBLog2e, kBLog2e, nl2, nl2);
+            ffma2(a0, a1, __uint_as_float(sr[q]), __uint_as_float(sr[q + 1]), sl2, sl2, a0, a1);
+            a0 = in0 ? ex2_approx(a0) : 0.f;
+            a1 = in1 ? ex2_approx(a1) : 0.f;
+            fadd2(t0, t1, __uint_as_float(dr[q]), __uint_as_float(dr[q + 1]), nd, nd);
+            ffma2(d0, d1, a0, a1, t0, t1, 0.f, 0.f);
+            pk[q / 2] = pack_bf16x2(d0, d1);
+          }
         } else if (kind == 2) {
           // side tile: p = 2^(s scale log2e + bias log2e - lse log2e) for side keys below
           // S (every valid row attends them), packed steps; the bias of each key is read
@@ -1124,6 +1146,28 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
                     lv[e], lv[e + 1]);
               pr[e] = ((unsigned)(off - lo) < span) ? ex2_approx(a0) : 0.f;
               pr[e + 1] = ((unsigned)(off + 1 - lo) < span) ? ex2_approx(a1) : 0.f;
+              fadd2(t0, t1, __uint_as_float(dr[c4 * 8 + e]), __uint_as_float(dr[c4 * 8 + e + 1]), dv[e], dv[e + 1]);
+              ffma2(ds[e], ds[e + 1], pr[e], pr[e + 1], t0, t1, 0.f, 0.f);
+            }
+          } else if (JOB == kJobBandX && qt.src == 0) {
+            // band query tile with the local bias: pairs inside the band, each with the
+            // bias of its offset for query rows that are not global (staged flag)
+            const int lo = p.causal ? 0 : -u.r;
+            const unsigned span = key_valid ? (unsigned)(p.causal ? u.r + 1 : 2 * u.r + 1) : 0u;
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              const int off = d0 + c * 8 + e;
+              const bool in0 = (unsigned)(off - lo) < span, in1 = (unsigned)(off + 1 - lo) < span;
+              float b0 = 0.f, b1 = 0.f;
+              if (lrow) {
+                b0 = (in0 && stgi[kQT + c * 8 + e]) ? __ldg(lrow - u.d * off) : 0.f;
+                b1 = (in1 && stgi[kQT + c * 8 + e + 1]) ? __ldg(lrow - u.d * (off + 1)) : 0.f;
+              }
+              float a0, a1, t0, t1;
+              ffma2(a0, a1, b0, b1, kBLog2e, kBLog2e, lv[e], lv[e + 1]);
+              ffma2(a0, a1, __uint_as_float(sr[c4 * 8 + e]), __uint_as_float(sr[c4 * 8 + e + 1]), sl2, sl2, a0, a1);
+              pr[e] = in0 ? ex2_approx(a0) : 0.f;
+              pr[e + 1] = in1 ? ex2_approx(a1) : 0.f;
               fadd2(t0, t1, __uint_as_float(dr[c4 * 8 + e]), __uint_as_float(dr[c4 * 8 + e + 1]), dv[e], dv[e + 1]);
               ffma2(ds[e], ds[e + 1], pr[e], pr[e + 1], t0, t1, 0.f, 0.f);
             }
