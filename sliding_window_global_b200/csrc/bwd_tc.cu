@@ -617,11 +617,15 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
           }
         };
         if constexpr (GROWS) {
-          if (u.d == 1 && !p.causal) {
-            // a global row over every key tile: valid keys outside its window
+          if (!p.causal && (u.d & (u.d - 1)) == 0) {
+            // a global row over every key tile: valid keys outside its window, i.e. not
+            // within rd of the row or (dilation a power of two) of another residue class
             const int vlim = row_valid ? u.Vc - kv0 : 0;
             const int br = qpos + rd - kv0;
-            masked_packed([&](int e) { return e < vlim && (unsigned)(br - e) > span2; });
+            const unsigned dm = (unsigned)u.d - 1u;
+            masked_packed([&](int e) {
+              return e < vlim && ((unsigned)(br - e) > span2 || ((unsigned)(br - e) & dm) != 0u);
+            });
           } else {
             generic_path();
           }
@@ -673,14 +677,16 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_dq_kernel(const __grid_const
             ffma2(d0, d1, a0, a1, t0, t1, 0.f, 0.f);
             pk[q / 2] = pack_bf16x2(d0, d1);
           }
-        } else if (kind == 1 && u.d == 1 && !p.causal) {
+        } else if (kind == 1 && !p.causal && (u.d & (u.d - 1)) == 0) {
           // global-column tile: staged keys (-1: none, or counted by a random block)
-          // outside the row's window, for rows that are not global themselves
+          // outside the row's window (not within rd, or of another residue class when
+          // the dilation is a power of two), for rows that are not global themselves
           const bool row_ok = row_valid && !row_global;
           const int qr = qpos + rd;
+          const unsigned dm = (unsigned)u.d - 1u;
           masked_packed([&](int e) {
             const int cv = sGpos[e];
-            return row_ok && cv >= 0 && (unsigned)(qr - cv) > span2;
+            return row_ok && cv >= 0 && ((unsigned)(qr - cv) > span2 || ((unsigned)(qr - cv) & dm) != 0u);
           });
         } else if (kind == 3 && !p.causal) {
           // random tile (dilation 1): valid keys of a first occurrence of the block,
