@@ -1178,21 +1178,24 @@ __global__ void __launch_bounds__(kDkvThreads, 1) bwd_dkv_kernel(const __grid_co
               ffma2(ds[e], ds[e + 1], pr[e], pr[e + 1], t0, t1, 0.f, 0.f);
             }
           } else if (((JOB == kJobBandX && qt.src != 0) || JOB == kJobGlobalKeys || JOB == kJobRandom) &&
-                     !p.causal && (JOB == kJobRandom || u.d == 1)) {
+                     !p.causal && (JOB == kJobRandom || (u.d & (u.d - 1)) == 0)) {
             // query rows whose window misses the key (global query rows of the band job,
-            // the global-key job, the random job; dilation 1): one unsigned compare on
-            // the staged query position, (unsigned)(qpos - kpos + rd) > 2 rd.  Rows that
-            // do not count have -lse = -inf and give p = 0 by themselves.
+            // the global-key job, the random job): on the staged query position,
+            // (unsigned)(qpos - kpos + rd) > 2 rd, or with a power-of-two dilation a query
+            // of another residue class.  Rows that do not count have -lse = -inf and give
+            // p = 0 by themselves.
             const bool kok = key_valid && !(JOB == kJobGlobalKeys && key_in_rand);
             const int kr = rd - kpos;
             const unsigned span2 = 2u * (unsigned)rd;
+            const unsigned dm = JOB == kJobRandom ? 0u : (unsigned)u.d - 1u;
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
               float a0, a1, t0, t1;
               ffma2(a0, a1, __uint_as_float(sr[c4 * 8 + e]), __uint_as_float(sr[c4 * 8 + e + 1]), sl2, sl2,
                     lv[e], lv[e + 1]);
-              pr[e] = (kok && (unsigned)(stgi[c * 8 + e] + kr) > span2) ? ex2_approx(a0) : 0.f;
-              pr[e + 1] = (kok && (unsigned)(stgi[c * 8 + e + 1] + kr) > span2) ? ex2_approx(a1) : 0.f;
+              const unsigned x0 = (unsigned)(stgi[c * 8 + e] + kr), x1 = (unsigned)(stgi[c * 8 + e + 1] + kr);
+              pr[e] = (kok && (x0 > span2 || (x0 & dm) != 0u)) ? ex2_approx(a0) : 0.f;
+              pr[e + 1] = (kok && (x1 > span2 || (x1 & dm) != 0u)) ? ex2_approx(a1) : 0.f;
               fadd2(t0, t1, __uint_as_float(dr[c4 * 8 + e]), __uint_as_float(dr[c4 * 8 + e + 1]), dv[e], dv[e + 1]);
               ffma2(ds[e], ds[e + 1], pr[e], pr[e + 1], t0, t1, 0.f, 0.f);
             }
